@@ -1,0 +1,169 @@
+"""ctypes wrapper of the fp64 CPU oracle (liboracle.so, built from qlora_oracle.cpp).
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline leg
+import this module.  It shares no code with the CUDA path: it takes numpy arrays of the raw
+stored bytes (bf16 bit patterns as uint16, packed 4-bit codes as uint8, scales as float32/uint8)
+and returns fp64 numpy arrays of the exact definition, or uint16 bf16 bit patterns for the
+decoded weight.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build_oracle
+
+FORMATS = {"nf4": 0, "mxfp4": 1, "nvfp4": 2}
+BLOCK = {0: 64, 1: 32, 2: 16}
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = build_oracle.build()
+        L = ctypes.CDLL(path)
+        c = ctypes
+        L.oracle_nf4_levels_spec.argtypes = [c.c_void_p]
+        L.oracle_nf4_levels_as241.argtypes = [c.c_void_p]
+        L.oracle_norm_ppf.argtypes = [c.c_double]
+        L.oracle_norm_ppf.restype = c.c_double
+        for name in ("oracle_decode_e2m1", "oracle_decode_e8m0", "oracle_decode_e4m3"):
+            getattr(L, name).argtypes = [c.c_uint32]
+            getattr(L, name).restype = c.c_float
+        L.oracle_f32_to_bf16.argtypes = [c.c_float]
+        L.oracle_f32_to_bf16.restype = c.c_uint16
+        L.oracle_bf16_to_f32.argtypes = [c.c_uint16]
+        L.oracle_bf16_to_f32.restype = c.c_float
+        L.oracle_weight_bytes.argtypes = [c.c_int, c.c_int64, c.c_int64]
+        L.oracle_weight_bytes.restype = c.c_int64
+        L.oracle_dequant.argtypes = [c.c_int, c.c_int64, c.c_int64, c.c_void_p, c.c_void_p,
+                                     c.c_float, c.c_int, c.c_void_p]
+        L.oracle_dequant.restype = c.c_int
+        L.oracle_layer.argtypes = [c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_int, c.c_double,
+                                   c.c_void_p, c.c_void_p, c.c_float,
+                                   c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
+                                   c.c_void_p, c.c_int64,
+                                   c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
+                                   c.c_void_p, c.c_void_p]
+        L.oracle_layer.restype = c.c_int
+        L.oracle_num_threads.restype = c.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _fmt(fmt):
+    return FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def nf4_levels_spec():
+    out = np.zeros(16, np.float32)
+    lib().oracle_nf4_levels_spec(_ptr(out))
+    return out
+
+
+def nf4_levels_as241():
+    out = np.zeros(16, np.float64)
+    lib().oracle_nf4_levels_as241(_ptr(out))
+    return out
+
+
+def norm_ppf(p):
+    return lib().oracle_norm_ppf(float(p))
+
+
+def decode_e2m1(code):
+    return lib().oracle_decode_e2m1(int(code))
+
+
+def decode_e8m0(code):
+    return lib().oracle_decode_e8m0(int(code))
+
+
+def decode_e4m3(code):
+    return lib().oracle_decode_e4m3(int(code))
+
+
+def f32_to_bf16(x):
+    return lib().oracle_f32_to_bf16(float(np.float32(x)))
+
+
+def bf16_to_f32(h):
+    return lib().oracle_bf16_to_f32(int(h))
+
+
+def weight_bytes(fmt, N, K):
+    return lib().oracle_weight_bytes(_fmt(fmt), int(N), int(K))
+
+
+def dequant(fmt, N, K, codes, scales, tensor_scale=1.0, with_tensor_scale=True):
+    """Decoded weight [N,K] as bf16 bit patterns (uint16)."""
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales)
+    out = np.zeros((N, K), np.uint16)
+    rc = lib().oracle_dequant(_fmt(fmt), N, K, _ptr(codes), _ptr(scales), float(tensor_scale),
+                              1 if with_tensor_scale else 0, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_dequant rejected its arguments")
+    return out
+
+
+def layer(fmt, M, N, K, r, s, codes, scales, tensor_scale, X, A, B, dY=None, rows=None,
+          want=("Y", "dX", "T", "U", "dA", "dB")):
+    """fp64 layer forward + backward.  X/A/B/dY are uint16 bf16 bit patterns.
+
+    rows: optional int64 array of the rows of Y and dX to produce (None: all rows).
+    Returns a dict of fp64 arrays for the names in `want`.
+    """
+    X = np.ascontiguousarray(X, np.uint16)
+    A = np.ascontiguousarray(A, np.uint16)
+    B = np.ascontiguousarray(B, np.uint16)
+    dY = None if dY is None else np.ascontiguousarray(dY, np.uint16)
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales)
+    rows_arr = None if rows is None else np.ascontiguousarray(rows, np.int64)
+    nrows = M if rows_arr is None else len(rows_arr)
+    out = {}
+    out["Y"] = np.zeros((nrows, N)) if "Y" in want else None
+    out["dX"] = np.zeros((nrows, K)) if ("dX" in want and dY is not None) else None
+    out["T"] = np.zeros((M, r)) if "T" in want else None
+    out["U"] = np.zeros((M, r)) if ("U" in want and dY is not None) else None
+    out["dA"] = np.zeros((r, K)) if ("dA" in want and dY is not None) else None
+    out["dB"] = np.zeros((N, r)) if ("dB" in want and dY is not None) else None
+    rc = lib().oracle_layer(_fmt(fmt), M, N, K, r, float(s), _ptr(codes), _ptr(scales),
+                            float(tensor_scale), _ptr(X), _ptr(A), _ptr(B), _ptr(dY),
+                            _ptr(rows_arr), nrows,
+                            _ptr(out["Y"]), _ptr(out["dX"]), _ptr(out["T"]), _ptr(out["U"]),
+                            _ptr(out["dA"]), _ptr(out["dB"]))
+    if rc != 0:
+        raise ValueError("oracle_layer rejected its arguments")
+    return {k: v for k, v in out.items() if v is not None}
+
+
+def grouped_layer(fmt, offsets, N, K, r, s, codes, scales, tensor_scales, X, A, B, dY=None,
+                  rows_per_expert=None, want=("Y", "dX", "T", "U", "dA", "dB")):
+    """The grouped (MoE) layer: the single layer above applied to each expert e on its rows
+    [offsets[e], offsets[e+1]) of the packed X / dY with that expert's own weight and adapters.
+
+    codes [E, N, K/2], scales [E, N, K/bs], tensor_scales [E] (NVFP4) or None, A [E, r, K],
+    B [E, N, r].  rows_per_expert: optional list of local row indices per expert.
+    Returns a list of per-expert dicts (row indices in each are local to the expert).
+    """
+    E = len(offsets) - 1
+    res = []
+    for e in range(E):
+        m0, m1 = int(offsets[e]), int(offsets[e + 1])
+        ts = 1.0 if tensor_scales is None else float(tensor_scales[e])
+        rows = None if rows_per_expert is None else rows_per_expert[e]
+        res.append(layer(fmt, m1 - m0, N, K, r, s, codes[e], scales[e], ts, X[m0:m1], A[e], B[e],
+                         None if dY is None else dY[m0:m1], rows=rows, want=want))
+    return res
+
+
+def num_threads():
+    return lib().oracle_num_threads()
