@@ -1,0 +1,449 @@
+// qlora.cu -- host side of the library: argument validation, workspace layout, TMA tensor maps,
+// kernel launches and the extern "C" entry points declared in include/qlora.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "qlora.h"
+#include "qlora_debug.cuh"
+#include "qlora_fused.cuh"
+#include "qlora_lora.cuh"
+
+namespace qlora {
+namespace {
+
+// ------------------------------------------------------------------------------------ helpers
+constexpr size_t kHeaderBytes = 256;        // [0]: device status word
+constexpr int kMaxCounters = 16384;         // reduction tile counters
+constexpr size_t kCounterBytes = size_t(kMaxCounters) * 4;
+constexpr int kMaxDevices = 64;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int rank_pad(int r) { return (r + 15) / 16 * 16; }
+bool rank_ok(int r) { return r == 8 || r == 16 || r == 32 || r == 64; }
+
+int block_size(int fmt) { return fmt == QLORA_FMT_NF4 ? 64 : (fmt == QLORA_FMT_MXFP4 ? 32 : 16); }
+
+int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return d;
+}
+
+int num_sms() {
+  static int cache[kMaxDevices] = {0};
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return 148;
+  if (cache[d] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || v <= 0) v = 148;
+    cache[d] = v;
+  }
+  return cache[d];
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [outer, inner] (inner contiguous, row pitch in bytes), box {bi, bo}.
+bool tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+             uint64_t outer, uint64_t pitch_bytes, uint32_t bi, uint32_t bo, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {bi, bo};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+CUtensorMapSwizzle swizzle_for_bytes(uint32_t b) {
+  return b == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                  : (b == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
+template <typename K>
+bool set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(bytes)) == cudaSuccess;
+}
+
+qlora_status_t check_weight(const qlora_weight_t* W) {
+  if (!W) return QLORA_ERR_INVALID_ARG;
+  if (W->fmt < QLORA_FMT_NF4 || W->fmt > QLORA_FMT_NVFP4) return QLORA_ERR_INVALID_ARG;
+  if (W->N < 16 || W->N % 16 != 0 || W->K < 64 || W->K % 64 != 0) return QLORA_ERR_INVALID_ARG;
+  if (W->N > (int64_t(1) << 30) || W->K > (int64_t(1) << 30)) return QLORA_ERR_INVALID_ARG;
+  if (!W->codes || !W->scales || !aligned16(W->codes) || !aligned16(W->scales))
+    return QLORA_ERR_INVALID_ARG;
+  if (W->fmt == QLORA_FMT_NVFP4 &&
+      (!W->tensor_scale || (reinterpret_cast<uintptr_t>(W->tensor_scale) & 3u)))
+    return QLORA_ERR_INVALID_ARG;
+  return QLORA_OK;
+}
+
+bool ptr_ok(const void* p) { return p && aligned16(p); }
+
+// ------------------------------------------------------------------------------- workspace
+// Reduction plan of the dA/dB kernel: tiles of 128 rows of N (dB) and of K (dA), M split into
+// S ranges of whole 64-row steps.
+struct WgradPlan {
+  int tiles0, tiles1, S, sps, total_steps;
+};
+
+WgradPlan wgrad_plan(int64_t N, int64_t K, int64_t M, int sms) {
+  WgradPlan p{};
+  p.tiles0 = int((N + 127) / 128);
+  p.tiles1 = int((K + 127) / 128);
+  p.total_steps = int((M + 63) / 64);
+  const int tiles = p.tiles0 + p.tiles1;
+  int S = (2 * sms + tiles - 1) / tiles;
+  S = S < 1 ? 1 : (S > 16 ? 16 : S);
+  if (S > p.total_steps) S = p.total_steps > 0 ? p.total_steps : 1;
+  p.sps = (p.total_steps + S - 1) / S;
+  if (p.sps < 1) p.sps = 1;
+  p.S = p.total_steps > 0 ? (p.total_steps + p.sps - 1) / p.sps : 1;
+  return p;
+}
+
+struct WsLayout {
+  size_t zs, t, u, partial, total;
+};
+
+WsLayout ws_layout(int64_t N, int64_t K, int64_t M, int r, bool bwd, int sms) {
+  WsLayout L{};
+  size_t off = kHeaderBytes + kCounterBytes;
+  const size_t mr = align_up(size_t(M > 0 ? M : 0) * size_t(r) * 2, 256);
+  L.zs = off; off += mr;
+  L.t = off; off += mr;
+  L.u = off; off += bwd ? mr : 0;
+  L.partial = off;
+  if (bwd) {
+    const WgradPlan wp = wgrad_plan(N, K, M, sms);
+    if (wp.S > 1) off += align_up(size_t(wp.S) * size_t(N + K) * size_t(rank_pad(r)) * 4, 256);
+  }
+  L.total = off;
+  return L;
+}
+
+int* ws_status(void* ws) { return reinterpret_cast<int*>(ws); }
+int* ws_counters(void* ws) { return reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + kHeaderBytes); }
+
+// ---------------------------------------------------------------------------------- launches
+qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t Kc, const void* R,
+                                int64_t R_rows, int r, float s, const float* ts, void* z, void* zs,
+                                int* status, cudaStream_t st) {
+  DownParams p{};
+  const int rpad = rank_pad(r);
+  if (!tmap_2d(&p.tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, uint64_t(Kc), uint64_t(M),
+               uint64_t(Kc) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return QLORA_ERR_CUDA;
+  if (!r_mn) {  // R = A [r, K]: K-major rows, box {64, rpad}
+    if (!tmap_2d(&p.tm_r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, uint64_t(Kc), uint64_t(r),
+                 uint64_t(Kc) * 2, 64, uint32_t(rpad), CU_TENSOR_MAP_SWIZZLE_128B))
+      return QLORA_ERR_CUDA;
+  } else {      // R = B [N, r]: MN-major, box {rpad, 64}
+    if (!tmap_2d(&p.tm_r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, uint64_t(r), uint64_t(R_rows),
+                 uint64_t(r) * 2, uint32_t(rpad), 64, swizzle_for_bytes(uint32_t(rpad) * 2)))
+      return QLORA_ERR_CUDA;
+  }
+  p.tensor_scale = ts;
+  p.z = static_cast<__nv_bfloat16*>(z);
+  p.zs = static_cast<__nv_bfloat16*>(zs);
+  p.status = status;
+  p.M = int(M);
+  p.r = r;
+  p.rpad = rpad;
+  p.num_k = int((Kc + 63) / 64);
+  p.s = s;
+  const dim3 grid(unsigned((M + 127) / 128));
+  if (r_mn) {
+    if (!set_smem(qlora_lora_down_kernel<true>, lora::kSmemBytes)) return QLORA_ERR_CUDA;
+    qlora_lora_down_kernel<true><<<grid, lora::kThreads, lora::kSmemBytes, st>>>(p);
+  } else {
+    if (!set_smem(qlora_lora_down_kernel<false>, lora::kSmemBytes)) return QLORA_ERR_CUDA;
+    qlora_lora_down_kernel<false><<<grid, lora::kThreads, lora::kSmemBytes, st>>>(p);
+  }
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+template <int FMT, bool DX>
+qlora_status_t launch_fused_t(const FusedParams& p, int grid, cudaStream_t st) {
+  if (!set_smem(qlora_fused_gemm_kernel<FMT, DX>, fused::kSmemBytes)) return QLORA_ERR_CUDA;
+  qlora_fused_gemm_kernel<FMT, DX><<<grid, fused::kThreads, fused::kSmemBytes, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status_t launch_fused(const qlora_weight_t* W, bool dx, const void* act, const void* zs,
+                            const void* lora_up, void* out, int64_t M, int r, int* status,
+                            cudaStream_t st) {
+  FusedParams p{};
+  const int64_t N = W->N, K = W->K;
+  const int64_t Kc = dx ? N : K;
+  if (!tmap_2d(&p.tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, uint64_t(Kc), uint64_t(M),
+               uint64_t(Kc) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return QLORA_ERR_CUDA;
+  if (!dx) {
+    if (!tmap_2d(&p.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, uint64_t(K / 2),
+                 uint64_t(N), uint64_t(K / 2), 32, 128, CU_TENSOR_MAP_SWIZZLE_32B))
+      return QLORA_ERR_CUDA;
+  } else {
+    if (!tmap_2d(&p.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, uint64_t(K / 2),
+                 uint64_t(N), uint64_t(K / 2), 64, 64, CU_TENSOR_MAP_SWIZZLE_64B))
+      return QLORA_ERR_CUDA;
+  }
+  if (!tmap_2d(&p.tm_zs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, zs, uint64_t(r), uint64_t(M),
+               uint64_t(r) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return QLORA_ERR_CUDA;
+  p.scales = W->scales;
+  p.tensor_scale = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
+  p.lora_up = static_cast<const __nv_bfloat16*>(lora_up);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.status = status;
+  p.M = int(M);
+  p.N = int(N);
+  p.K = int(K);
+  p.r = r;
+  p.num_m = int((M + fused::BM - 1) / fused::BM);
+  p.num_n = int(((dx ? K : N) + fused::BN - 1) / fused::BN);
+  p.num_k = int((Kc + fused::BK - 1) / fused::BK);
+  const int tiles = p.num_m * p.num_n;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  switch (W->fmt * 2 + (dx ? 1 : 0)) {
+    case 0: return launch_fused_t<kFmtNF4, false>(p, grid, st);
+    case 1: return launch_fused_t<kFmtNF4, true>(p, grid, st);
+    case 2: return launch_fused_t<kFmtMXFP4, false>(p, grid, st);
+    case 3: return launch_fused_t<kFmtMXFP4, true>(p, grid, st);
+    case 4: return launch_fused_t<kFmtNVFP4, false>(p, grid, st);
+    default: return launch_fused_t<kFmtNVFP4, true>(p, grid, st);
+  }
+}
+
+qlora_status_t launch_wgrad(const void* X, const void* dY, const void* T, const void* U, int64_t M,
+                            int64_t N, int64_t K, int r, float s, void* dA, void* dB, void* ws,
+                            const WsLayout& L, cudaStream_t st) {
+  WgradParams p{};
+  const int rpad = rank_pad(r);
+  const WgradPlan wp = wgrad_plan(N, K, M, num_sms());
+  const CUtensorMapSwizzle rsw = swizzle_for_bytes(uint32_t(rpad) * 2);
+  if (!tmap_2d(&p.tm_l[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, uint64_t(N), uint64_t(M),
+               uint64_t(N) * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tmap_2d(&p.tm_l[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, uint64_t(K), uint64_t(M),
+               uint64_t(K) * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tmap_2d(&p.tm_r[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, uint64_t(r), uint64_t(M),
+               uint64_t(r) * 2, uint32_t(rpad), 64, rsw) ||
+      !tmap_2d(&p.tm_r[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U, uint64_t(r), uint64_t(M),
+               uint64_t(r) * 2, uint32_t(rpad), 64, rsw))
+    return QLORA_ERR_CUDA;
+  p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.partial);
+  p.counters = ws_counters(ws);
+  p.out0 = static_cast<__nv_bfloat16*>(dB);
+  p.out1 = static_cast<__nv_bfloat16*>(dA);
+  p.status = ws_status(ws);
+  p.M = int(M);
+  p.P0 = int(N);
+  p.P1 = int(K);
+  p.r = r;
+  p.rpad = rpad;
+  p.S = wp.S;
+  p.tiles0 = wp.tiles0;
+  p.tiles1 = wp.tiles1;
+  p.steps_per_split = wp.sps;
+  p.total_steps = wp.total_steps;
+  p.s = s;
+  if (wp.tiles0 + wp.tiles1 > kMaxCounters) return QLORA_ERR_UNSUPPORTED;
+  if (!set_smem(qlora_lora_wgrad_kernel, lora::kSmemBytes)) return QLORA_ERR_CUDA;
+  const unsigned grid = unsigned((wp.tiles0 + wp.tiles1) * wp.S);
+  qlora_lora_wgrad_kernel<<<grid, lora::kThreads, lora::kSmemBytes, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" {
+
+size_t qlora_workspace_size(int op, const qlora_weight_t* W, int64_t M, int r, int E) {
+  (void)E;
+  if (check_weight(W) != QLORA_OK || M < 0 || !rank_ok(r)) return 0;
+  if (op != QLORA_OP_FWD && op != QLORA_OP_BWD) return 0;
+  return ws_layout(W->N, W->K, M, r, op == QLORA_OP_BWD, num_sms()).total;
+}
+
+qlora_status_t qlora_workspace_init(void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!ws || !aligned16(ws) || ws_bytes < kHeaderBytes + kCounterBytes) return QLORA_ERR_WORKSPACE;
+  return cudaMemsetAsync(ws, 0, kHeaderBytes + kCounterBytes, reinterpret_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? QLORA_OK
+             : QLORA_ERR_CUDA;
+}
+
+qlora_status_t qlora_linear_fwd(const qlora_weight_t* W, const void* X, const void* A,
+                                const void* B, void* Y, void* T_save, int64_t M, int r,
+                                float scale, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  qlora_status_t st = check_weight(W);
+  if (st != QLORA_OK) return st;
+  if (M < 0 || M > (int64_t(1) << 31) - 512) return QLORA_ERR_INVALID_ARG;
+  if (!rank_ok(r)) return (r > 0 && r <= 256) ? QLORA_ERR_UNSUPPORTED : QLORA_ERR_INVALID_ARG;
+  if (!ptr_ok(X) || !ptr_ok(A) || !ptr_ok(B) || !ptr_ok(Y) || (T_save && !aligned16(T_save)))
+    return QLORA_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(W->N, W->K, M, r, false, num_sms());
+  if (!ws || !aligned16(ws) || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (M == 0) return QLORA_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  void* T = T_save ? T_save : w + L.t;
+  void* Zs = w + L.zs;
+  const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
+  st = launch_lora_down(false, X, M, W->K, A, r, r, scale, ts, T, Zs, ws_status(ws), s);
+  if (st != QLORA_OK) return st;
+  return launch_fused(W, false, X, Zs, B, Y, M, r, ws_status(ws), s);
+}
+
+qlora_status_t qlora_linear_bwd(const qlora_weight_t* W, const void* X, const void* A,
+                                const void* B, const void* T, const void* dY, void* dX, void* dA,
+                                void* dB, int64_t M, int r, float scale, void* ws, size_t ws_bytes,
+                                qlora_stream_t stream) {
+  qlora_status_t st = check_weight(W);
+  if (st != QLORA_OK) return st;
+  if (M < 0 || M > (int64_t(1) << 31) - 512) return QLORA_ERR_INVALID_ARG;
+  if (!rank_ok(r)) return (r > 0 && r <= 256) ? QLORA_ERR_UNSUPPORTED : QLORA_ERR_INVALID_ARG;
+  if (!ptr_ok(X) || !ptr_ok(A) || !ptr_ok(B) || !ptr_ok(dY) || !ptr_ok(dA) || !ptr_ok(dB) ||
+      (T && !aligned16(T)) || (dX && !aligned16(dX)))
+    return QLORA_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(W->N, W->K, M, r, true, num_sms());
+  if (!ws || !aligned16(ws) || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    if (cudaMemsetAsync(dA, 0, size_t(r) * W->K * 2, s) != cudaSuccess ||
+        cudaMemsetAsync(dB, 0, size_t(W->N) * r * 2, s) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
+  void* Zs = w + L.zs;
+  void* U = w + L.u;
+  if (!T) {  // recompute T = X A^T (its scaled copy lands in Zs and is overwritten below)
+    st = launch_lora_down(false, X, M, W->K, A, r, r, scale, ts, w + L.t, Zs, ws_status(ws), s);
+    if (st != QLORA_OK) return st;
+    T = w + L.t;
+  }
+  st = launch_lora_down(true, dY, M, W->N, B, W->N, r, scale, ts, U, Zs, ws_status(ws), s);
+  if (st != QLORA_OK) return st;
+  if (dX) {
+    st = launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), s);
+    if (st != QLORA_OK) return st;
+  }
+  return launch_wgrad(X, dY, T, U, M, W->N, W->K, r, scale, dA, dB, ws, L, s);
+}
+
+qlora_status_t qlora_grouped_fwd(const qlora_weight_t* W, int E, const int32_t* d_offsets,
+                                 int64_t M_total, const void* X, const void* A, const void* B,
+                                 void* Y, void* T_save, int r, float scale, void* ws,
+                                 size_t ws_bytes, qlora_stream_t stream) {
+  (void)W; (void)E; (void)d_offsets; (void)M_total; (void)X; (void)A; (void)B; (void)Y;
+  (void)T_save; (void)r; (void)scale; (void)ws; (void)ws_bytes; (void)stream;
+  return QLORA_ERR_UNSUPPORTED;
+}
+
+qlora_status_t qlora_grouped_bwd(const qlora_weight_t* W, int E, const int32_t* d_offsets,
+                                 int64_t M_total, const void* X, const void* A, const void* B,
+                                 const void* T, const void* dY, void* dX, void* dA, void* dB,
+                                 int r, float scale, void* ws, size_t ws_bytes,
+                                 qlora_stream_t stream) {
+  (void)W; (void)E; (void)d_offsets; (void)M_total; (void)X; (void)A; (void)B; (void)T; (void)dY;
+  (void)dX; (void)dA; (void)dB; (void)r; (void)scale; (void)ws; (void)ws_bytes; (void)stream;
+  return QLORA_ERR_UNSUPPORTED;
+}
+
+qlora_status_t qlora_get_device_status(void* ws, qlora_stream_t stream) {
+  if (!ws || !aligned16(ws)) return QLORA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return static_cast<qlora_status_t>(v);
+}
+
+qlora_status_t qlora_debug_dequant(const qlora_weight_t* W, int transposed, void* out,
+                                   qlora_stream_t stream) {
+  qlora_status_t st = check_weight(W);
+  if (st != QLORA_OK) return st;
+  if (!ptr_ok(out)) return QLORA_ERR_INVALID_ARG;
+  DebugDequantParams p{};
+  const bool dx = transposed != 0;
+  const int64_t N = W->N, K = W->K;
+  if (!tmap_2d(&p.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, uint64_t(K / 2), uint64_t(N),
+               uint64_t(K / 2), dx ? 64 : 32, dx ? 64 : 128,
+               dx ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B))
+    return QLORA_ERR_CUDA;
+  p.scales = W->scales;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.status = nullptr;
+  p.N = int(N);
+  p.K = int(K);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid = dx ? dim3(unsigned((K + 127) / 128), unsigned((N + 63) / 64))
+                       : dim3(unsigned((N + 127) / 128), unsigned(K / 64));
+  switch (W->fmt * 2 + (dx ? 1 : 0)) {
+    case 0: qlora_debug_dequant_kernel<kFmtNF4, false><<<grid, 128, 0, s>>>(p); break;
+    case 1: qlora_debug_dequant_kernel<kFmtNF4, true><<<grid, 128, 0, s>>>(p); break;
+    case 2: qlora_debug_dequant_kernel<kFmtMXFP4, false><<<grid, 128, 0, s>>>(p); break;
+    case 3: qlora_debug_dequant_kernel<kFmtMXFP4, true><<<grid, 128, 0, s>>>(p); break;
+    case 4: qlora_debug_dequant_kernel<kFmtNVFP4, false><<<grid, 128, 0, s>>>(p); break;
+    default: qlora_debug_dequant_kernel<kFmtNVFP4, true><<<grid, 128, 0, s>>>(p); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status_t qlora_debug_wait_timeout(void* ws, size_t ws_bytes, int limit_us,
+                                        qlora_stream_t stream) {
+  if (!ws || !aligned16(ws) || ws_bytes < kHeaderBytes) return QLORA_ERR_WORKSPACE;
+  if (limit_us <= 0 || limit_us > 1000000) return QLORA_ERR_INVALID_ARG;
+  int clk_khz = 0;
+  if (cudaDeviceGetAttribute(&clk_khz, cudaDevAttrClockRate, current_device()) != cudaSuccess ||
+      clk_khz <= 0)
+    clk_khz = 2000000;
+  const unsigned long long cycles = (unsigned long long)limit_us * (unsigned long long)clk_khz / 1000ull;
+  qlora_debug_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(ws_status(ws), cycles);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+const char* qlora_status_string(qlora_status_t status) {
+  switch (status) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument (pointer, alignment or shape)";
+    case QLORA_ERR_UNSUPPORTED: return "unsupported by this build (e.g. rank not in {8,16,32,64})";
+    case QLORA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case QLORA_ERR_CUDA: return "a CUDA call failed (launch or tensor map)";
+    case QLORA_ERR_DEVICE_TIMEOUT: return "a device-side pipeline wait gave up";
+  }
+  return "unknown status";
+}
+
+const char* qlora_build_info(void) { return "qlora-b200 0.1 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,85 @@
+// qlora_debug.cuh -- test-only kernels: the dequant stage run on its own (decoded tiles written
+// back un-swizzled), and a bounded wait that is meant to run out.
+#pragma once
+#include <cuda_bf16.h>
+#include "qlora_fused.cuh"
+
+namespace qlora {
+
+struct DebugDequantParams {
+  CUtensorMap tm_codes;  // same tensor map shape as the fused kernel's
+  const void* scales;
+  __nv_bfloat16* out;    // [N, K]
+  int* status;
+  int N, K;
+};
+
+// One CTA = one pipeline step of the fused kernel's weight operand: forward tiling = 128 weight
+// rows x 64 columns (K-major tile), dX tiling = 64 weight rows x 128 columns (MN-major tile).
+// 128 threads, one 64-element item each, exactly as in the fused kernel's dequant group.
+template <int FMT, bool DX>
+__global__ void __launch_bounds__(128)
+qlora_debug_dequant_kernel(const __grid_constant__ DebugDequantParams p) {
+  __shared__ __align__(1024) uint8_t wtile[fused::W_BYTES];
+  __shared__ __align__(1024) uint8_t ctile[fused::C_BYTES];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const int tg = threadIdx.x;
+  const int c0 = blockIdx.x * fused::BN;    // forward: first weight row; dX: first column
+  const int ks = blockIdx.y;                 // forward: column step;     dX: row step
+  const uint32_t b = ptx::smem_u32(&bar);
+  if (tg == 0) {
+    ptx::mbar_init(b, 1);
+    abort_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (tg == 0) {
+    ptx::mbar_arrive_expect_tx(b, fused::C_BYTES);
+    if (!DX) ptx::tma_load_2d(ptx::smem_u32(ctile), &p.tm_codes, b, ks * (fused::BK / 2), c0);
+    else ptx::tma_load_2d(ptx::smem_u32(ctile), &p.tm_codes, b, c0 / 2, ks * fused::BK);
+  }
+  const ItemGeom<DX> geo(tg);
+  const int n = DX ? ks * fused::BK + geo.row : c0 + geo.row;
+  const int kcol = DX ? c0 + geo.chunk * 64 : ks * fused::BK;
+  const bool valid = n < p.N && kcol < p.K;
+  ItemScale sc{0u};
+  if (valid) sc = load_item_scale<FMT>(p.scales, n, kcol, p.K);
+  if (!ptx::mbar_wait(b, 0, p.status, &abort_flag)) return;
+  const uint32_t cb = ptx::smem_u32(ctile);
+  const uint4 lo = ptx::ld_shared_v4(cb + geo.code_off(0));
+  const uint4 hi = ptx::ld_shared_v4(cb + geo.code_off(1));
+  const uint32_t cw[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  const uint32_t rb = geo.op_row_base(ptx::smem_u32(wtile));
+  if (valid) dequant_item_store<FMT>(cw, sc, rb, geo.swz());
+  else zero_item_store(rb);
+  __syncthreads();
+  // read back a DIFFERENT thread's item (the next row of the same chunk) through the swizzle
+  const ItemGeom<DX> g2((tg & ~63) | ((tg + 1) & 63));
+  const int n2 = DX ? ks * fused::BK + g2.row : c0 + g2.row;
+  const int k2 = DX ? c0 + g2.chunk * 64 : ks * fused::BK;
+  if (n2 < p.N && k2 < p.K) {
+    const uint32_t rb2 = g2.op_row_base(ptx::smem_u32(wtile));
+    for (int j = 0; j < 8; ++j) {
+      const uint4 v = ptx::ld_shared_v4(rb2 + ((uint32_t(j) ^ g2.swz()) << 4));
+      *reinterpret_cast<uint4*>(p.out + size_t(n2) * p.K + k2 + j * 8) = v;
+    }
+  }
+}
+
+__global__ void qlora_debug_wait_kernel(int* status, unsigned long long limit_cycles) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(ptx::smem_u32(&bar), 1);
+    abort_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // nothing ever arrives on this barrier: the wait must give up and record the timeout
+    ptx::mbar_wait(ptx::smem_u32(&bar), 0, status, &abort_flag, limit_cycles);
+  }
+}
+
+}  // namespace qlora

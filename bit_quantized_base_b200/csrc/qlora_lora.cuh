@@ -1,0 +1,315 @@
+// qlora_lora.cuh -- the rank-r side path of the layer on tcgen05.
+//
+// lora_down: Z[M, r] = Act[M, Kc] . R, one 128-row tile per CTA.
+//   forward : Z = T = X A^T   (R = A^T: A [r, K] is a K-major operand)
+//   backward: Z = U = dY B    (R = B:   B [N, r] is an MN-major operand)
+//   It writes Z (bf16) and Zs = bf16(Z * s / ts), the operand of the fused GEMM's LoRA step.
+//   ("Training LLMs on a Budget: LoRA, QLoRA, and LoftQ", §2 "Initialization matters": z = A x
+//   and dL/dz = B^T dL/dy.)
+//
+// lora_wgrad: the adapter gradients, reductions over the M rows:
+//   dB[N, r] = s . dY^T T     and     dA^T[K, r] = s . X^T U   (dA written as [r, K])
+//   ("Training LLMs on a Budget", §2 "Initialization matters": dL/dB = dL/dy z^T,
+//   dL/dA = (B^T dL/dy) x^T, with the layer's scale s.)  Both are out[P, r] = s . L^T R with L
+//   [M, P] and R [M, r]: an M=128 x N=rpad tcgen05 GEMM per 128-row tile of P whose operands are
+//   both MN-major (M is the contraction).  M is split over S CTAs per tile when there are too few
+//   tiles to fill the GPU; each split stores an fp32 partial, and the last split to finish (an
+//   atomic counter) adds the S partials in split order 0..S-1 and writes bf16, so the result is
+//   bitwise deterministic.
+#pragma once
+#include <cuda_bf16.h>
+#include "qlora_ptx.cuh"
+
+namespace qlora {
+namespace lora {
+constexpr int BM = 128, BK = 64, NS = 6;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB
+constexpr int R_BYTES = 64 * 128;     // up to 64 x 128 B
+constexpr int kThreads = 6 * 32;      // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kTmemCols = 64;
+constexpr size_t kSmemBytes = 1024 + size_t(NS) * (A_BYTES + R_BYTES) + 512;
+}  // namespace lora
+
+__device__ __forceinline__ uint32_t swz_mode_for_row_bytes(uint32_t rowb) {
+  return rowb == 128 ? ptx::kSw128 : (rowb == 64 ? ptx::kSw64 : ptx::kSw32);
+}
+
+struct DownParams {
+  CUtensorMap tm_act;  // X [M, K] or dY [M, N] bf16, box {64, 128}, SW128
+  CUtensorMap tm_r;    // T: A [r, K] box {64, rpad} SW128; U: B [N, r] box {rpad, 64} SW(2 rpad)
+  const float* tensor_scale;
+  __nv_bfloat16* z;    // [M, r]
+  __nv_bfloat16* zs;   // [M, r]
+  int* status;
+  int M, r, rpad, num_k;
+  float s;
+};
+
+template <bool R_MN>
+__global__ void __launch_bounds__(lora::kThreads, 1)
+qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
+  using namespace lora;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* as = smem;
+  uint8_t* rs = as + NS * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rs + NS * R_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t b0 = ptx::smem_u32(bars);
+  auto full = [&](uint32_t s) { return b0 + 8u * s; };
+  auto empty = [&](uint32_t s) { return b0 + 8u * (NS + s); };
+  const uint32_t acc_full = b0 + 8u * (2 * NS);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) { ptx::mbar_init(full(s), 1); ptx::mbar_init(empty(s), 1); }
+    ptx::mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int m0 = blockIdx.x * BM;
+  const uint32_t rowb = uint32_t(p.rpad) * 2u;
+  const uint32_t r_bytes = uint32_t(p.rpad) * 128u;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int ks = 0; ks < p.num_k; ++ks) {
+        const uint32_t s = ks % NS, ph = (ks / NS) & 1;
+        if (!ptx::mbar_wait(empty(s), ph ^ 1u, p.status, abort_flag)) break;
+        ptx::mbar_arrive_expect_tx(full(s), A_BYTES + r_bytes);
+        ptx::tma_load_2d(ptx::smem_u32(as + s * A_BYTES), &p.tm_act, full(s), ks * BK, m0);
+        if (!R_MN) ptx::tma_load_2d(ptx::smem_u32(rs + s * R_BYTES), &p.tm_r, full(s), ks * BK, 0);
+        else ptx::tma_load_2d(ptx::smem_u32(rs + s * R_BYTES), &p.tm_r, full(s), 0, ks * BK);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = ptx::idesc_bf16(128, uint32_t(p.rpad), 0, R_MN ? 1u : 0u);
+      bool ok = true;
+      for (int ks = 0; ks < p.num_k; ++ks) {
+        const uint32_t s = ks % NS, ph = (ks / NS) & 1;
+        if (!ptx::mbar_wait(full(s), ph, p.status, abort_flag)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint32_t a = ptx::smem_u32(as + s * A_BYTES), b = ptx::smem_u32(rs + s * R_BYTES);
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t ad = ptx::smem_desc(a + kk * 32, 16, 1024, ptx::kSw128);
+          const uint64_t bd = R_MN ? ptx::smem_desc(b + kk * 16 * rowb, 64 * rowb, 8 * rowb,
+                                                    swz_mode_for_row_bytes(rowb))
+                                   : ptx::smem_desc(b + kk * 32, 16, 1024, ptx::kSw128);
+          ptx::mma_bf16(tmem, ad, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+        }
+        ptx::mma_commit(empty(s));
+      }
+      if (ok) ptx::mma_commit(acc_full);
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = m0 + q * 32 + lane;
+    if (ptx::mbar_wait(acc_full, 0, p.status, abort_flag)) {
+      ptx::tc_fence_after();
+      const float ts = p.tensor_scale ? __ldg(p.tensor_scale) : 1.0f;
+      const float zscale = p.s / ts;
+#pragma unroll 1
+      for (int c = 0; c < p.rpad; c += 16) {
+        uint32_t v[16];
+        ptx::tmem_ld_32x32b_x16(tmem + (uint32_t(q * 32) << 16) + c, v);
+        ptx::tmem_ld_wait();
+        if (row < p.M) {
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            const int col = c + g * 8;
+            if (col < p.r) {
+              uint4 z, zs;
+              const float* f = reinterpret_cast<const float*>(v + g * 8);
+              z.x = ptx::cvt_bf16x2(f[0], f[1]); z.y = ptx::cvt_bf16x2(f[2], f[3]);
+              z.z = ptx::cvt_bf16x2(f[4], f[5]); z.w = ptx::cvt_bf16x2(f[6], f[7]);
+              zs.x = ptx::cvt_bf16x2(f[0] * zscale, f[1] * zscale);
+              zs.y = ptx::cvt_bf16x2(f[2] * zscale, f[3] * zscale);
+              zs.z = ptx::cvt_bf16x2(f[4] * zscale, f[5] * zscale);
+              zs.w = ptx::cvt_bf16x2(f[6] * zscale, f[7] * zscale);
+              *reinterpret_cast<uint4*>(p.z + size_t(row) * p.r + col) = z;
+              *reinterpret_cast<uint4*>(p.zs + size_t(row) * p.r + col) = zs;
+            }
+          }
+        }
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 1) ptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+struct WgradParams {
+  CUtensorMap tm_l[2];  // L: dY [M, N] (problem 0, dB) / X [M, K] (problem 1, dA); box {64, 64} SW128
+  CUtensorMap tm_r[2];  // R: T [M, r] / U [M, r]; box {rpad, 64} SW(2 rpad)
+  float* partial;       // [S, P0 + P1, rpad] fp32 (S > 1)
+  int* counters;        // [tiles0 + tiles1], zero between calls
+  __nv_bfloat16* out0;  // dB [N, r]: (p, j) at p * r + j
+  __nv_bfloat16* out1;  // dA [r, K]: (p, j) at j * K + p
+  int* status;
+  int M, P0, P1, r, rpad, S, tiles0, tiles1, steps_per_split, total_steps;
+  float s;
+};
+
+__global__ void __launch_bounds__(lora::kThreads, 1)
+qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
+  using namespace lora;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* as = smem;
+  uint8_t* rs = as + NS * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rs + NS * R_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  const uint32_t b0 = ptx::smem_u32(bars);
+  auto full = [&](uint32_t s) { return b0 + 8u * s; };
+  auto empty = [&](uint32_t s) { return b0 + 8u * (NS + s); };
+  const uint32_t acc_full = b0 + 8u * (2 * NS);
+
+  const int tile = blockIdx.x / p.S, split = blockIdx.x % p.S;
+  const int prob = tile < p.tiles0 ? 0 : 1;
+  const int p0 = (tile - (prob ? p.tiles0 : 0)) * BM;
+  const int P = prob ? p.P1 : p.P0;
+  const int ks0 = split * p.steps_per_split;
+  const int ks1 = min(ks0 + p.steps_per_split, p.total_steps);
+  const CUtensorMap* tml = &p.tm_l[prob];
+  const CUtensorMap* tmr = &p.tm_r[prob];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) { ptx::mbar_init(full(s), 1); ptx::mbar_init(empty(s), 1); }
+    ptx::mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t rowb = uint32_t(p.rpad) * 2u;
+  const uint32_t r_bytes = 64u * rowb;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int ks = ks0; ks < ks1; ++ks) {
+        const int it = ks - ks0;
+        const uint32_t s = it % NS, ph = (it / NS) & 1;
+        if (!ptx::mbar_wait(empty(s), ph ^ 1u, p.status, abort_flag)) break;
+        ptx::mbar_arrive_expect_tx(full(s), A_BYTES + r_bytes);
+        const uint32_t ad = ptx::smem_u32(as + s * A_BYTES);
+        ptx::tma_load_2d(ad, tml, full(s), p0, ks * BK);
+        ptx::tma_load_2d(ad + A_BYTES / 2, tml, full(s), p0 + 64, ks * BK);
+        ptx::tma_load_2d(ptx::smem_u32(rs + s * R_BYTES), tmr, full(s), 0, ks * BK);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && ks1 > ks0) {
+      const uint32_t idesc = ptx::idesc_bf16(128, uint32_t(p.rpad), 1u, 1u);
+      const uint32_t rsw = swz_mode_for_row_bytes(rowb);
+      bool ok = true;
+      for (int ks = ks0; ks < ks1; ++ks) {
+        const int it = ks - ks0;
+        const uint32_t s = it % NS, ph = (it / NS) & 1;
+        if (!ptx::mbar_wait(full(s), ph, p.status, abort_flag)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint32_t a = ptx::smem_u32(as + s * A_BYTES), b = ptx::smem_u32(rs + s * R_BYTES);
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t ad = ptx::smem_desc(a + kk * 2048, 8192, 1024, ptx::kSw128);
+          const uint64_t bd = ptx::smem_desc(b + kk * 16 * rowb, 64 * rowb, 8 * rowb, rsw);
+          ptx::mma_bf16(tmem, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        ptx::mma_commit(empty(s));
+      }
+      if (ok) ptx::mma_commit(acc_full);
+    }
+  } else {
+    const int q = warp & 3;
+    const int et = threadIdx.x - 64;   // 0..127
+    const int prow = p0 + q * 32 + lane;
+    const bool have = ks1 > ks0;
+    if (have) ptx::mbar_wait(acc_full, 0, p.status, abort_flag);
+    // every epilogue thread takes the same branch below: a thread whose wait gave up set
+    // abort_flag before this barrier
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const bool ok = *abort_flag == 0;
+    if (ok && have) ptx::tc_fence_after();
+    const int Ptot = p.P0 + p.P1;
+    const int poff = prob ? p.P0 : 0;
+    auto write_out = [&](int j, float v) {
+      const __nv_bfloat16 b = __float2bfloat16_rn(v * p.s);
+      if (prob == 0) p.out0[size_t(prow) * p.r + j] = b;
+      else p.out1[size_t(j) * p.P1 + prow] = b;
+    };
+    if (ok) {
+#pragma unroll 1
+      for (int c = 0; c < p.rpad; c += 16) {
+        uint32_t v[16];
+        if (have) {
+          ptx::tmem_ld_32x32b_x16(tmem + (uint32_t(q * 32) << 16) + c, v);
+          ptx::tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int g = 0; g < 16; ++g) v[g] = 0u;
+        }
+        if (prow < P) {
+          if (p.S == 1) {
+            for (int g = 0; g < 16 && c + g < p.r; ++g) write_out(c + g, __uint_as_float(v[g]));
+          } else {
+            float* dst = p.partial + (size_t(split) * Ptot + poff + prow) * p.rpad + c;
+#pragma unroll
+            for (int g = 0; g < 16; g += 4)
+              __stcg(reinterpret_cast<float4*>(dst + g),
+                     make_float4(__uint_as_float(v[g]), __uint_as_float(v[g + 1]),
+                                 __uint_as_float(v[g + 2]), __uint_as_float(v[g + 3])));
+          }
+        }
+      }
+      if (p.S > 1) {
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (et == 0) {
+          const int old = atomicAdd(&p.counters[tile], 1);
+          *last_flag = (old == p.S - 1) ? 1 : 0;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (*last_flag) {
+          __threadfence();
+          if (prow < P) {
+            for (int j = 0; j < p.r; ++j) {
+              float acc = 0.0f;
+              for (int sp = 0; sp < p.S; ++sp)
+                acc += __ldcg(p.partial + (size_t(sp) * Ptot + poff + prow) * p.rpad + j);
+              write_out(j, acc);
+            }
+          }
+          if (et == 0) p.counters[tile] = 0;
+        }
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 1) ptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace qlora

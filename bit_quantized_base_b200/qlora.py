@@ -1,0 +1,203 @@
+"""Python binding of libqlora.so (include/qlora.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls and takes torch tensors already on
+the GPU (PyTorch provides device memory and streams; all computation happens in the library's
+CUDA kernels).  A non-OK status raises QLoraError.  If libqlora.so is missing the import fails:
+there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqlora.so")
+
+FMT = {"nf4": 0, "mxfp4": 1, "nvfp4": 2}
+BLOCK = {"nf4": 64, "mxfp4": 32, "nvfp4": 16}
+OP_FWD, OP_BWD, OP_GROUPED_FWD, OP_GROUPED_BWD = 0, 1, 2, 3
+
+STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED",
+          3: "QLORA_ERR_WORKSPACE", 4: "QLORA_ERR_CUDA", 5: "QLORA_ERR_DEVICE_TIMEOUT"}
+
+# every symbol include/qlora.h declares
+EXPORTS = ("qlora_workspace_size", "qlora_workspace_init", "qlora_linear_fwd", "qlora_linear_bwd",
+           "qlora_grouped_fwd", "qlora_grouped_bwd", "qlora_get_device_status",
+           "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_status_string",
+           "qlora_build_info")
+
+
+class QLoraError(RuntimeError):
+    def __init__(self, status, where=""):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS.get(self.status, self.status)} "
+                         f"({_status_string(self.status)})")
+
+
+class qlora_weight_t(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("tensor_scale", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python bit_quantized_base_b200/build.py` (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    c = ctypes
+    P = c.c_void_p
+    W = c.POINTER(qlora_weight_t)
+    L.qlora_workspace_size.argtypes = [c.c_int, W, c.c_int64, c.c_int, c.c_int]
+    L.qlora_workspace_size.restype = c.c_size_t
+    L.qlora_workspace_init.argtypes = [P, c.c_size_t, P]
+    L.qlora_linear_fwd.argtypes = [W, P, P, P, P, P, c.c_int64, c.c_int, c.c_float, P, c.c_size_t, P]
+    L.qlora_linear_bwd.argtypes = [W, P, P, P, P, P, P, P, P, c.c_int64, c.c_int, c.c_float, P,
+                                   c.c_size_t, P]
+    L.qlora_grouped_fwd.argtypes = [W, c.c_int, P, c.c_int64, P, P, P, P, P, c.c_int, c.c_float,
+                                    P, c.c_size_t, P]
+    L.qlora_grouped_bwd.argtypes = [W, c.c_int, P, c.c_int64, P, P, P, P, P, P, P, P, c.c_int,
+                                    c.c_float, P, c.c_size_t, P]
+    L.qlora_get_device_status.argtypes = [P, P]
+    L.qlora_debug_dequant.argtypes = [W, c.c_int, P, P]
+    L.qlora_debug_wait_timeout.argtypes = [P, c.c_size_t, c.c_int, P]
+    L.qlora_status_string.argtypes = [c.c_int]
+    L.qlora_status_string.restype = c.c_char_p
+    L.qlora_build_info.restype = c.c_char_p
+    for name in ("qlora_workspace_init", "qlora_linear_fwd", "qlora_linear_bwd",
+                 "qlora_grouped_fwd", "qlora_grouped_bwd", "qlora_get_device_status",
+                 "qlora_debug_dequant", "qlora_debug_wait_timeout"):
+        getattr(L, name).restype = c.c_int
+    return L
+
+
+lib = _load()
+
+
+def _status_string(s):
+    return lib.qlora_status_string(int(s)).decode()
+
+
+def _check(status, where):
+    if status != 0:
+        raise QLoraError(status, where)
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+class Weight:
+    """A frozen 4-bit weight resident on the GPU (codes [.., N, K/2] uint8, scales, and for NVFP4
+    the tensor scale as a float32 device tensor)."""
+
+    def __init__(self, fmt, N, K, codes, scales, tensor_scale=None):
+        self.fmt, self.N, self.K = fmt, int(N), int(K)
+        self.codes, self.scales, self.tensor_scale = codes, scales, tensor_scale
+        self.c = qlora_weight_t(FMT[fmt], 0, self.N, self.K, _p(codes), _p(scales),
+                                _p(tensor_scale))
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+    def nbytes(self):
+        n = self.codes.numel() * self.codes.element_size() + self.scales.numel() * self.scales.element_size()
+        if self.tensor_scale is not None:
+            n += self.tensor_scale.numel() * 4
+        return n
+
+
+def qlora_workspace_size(op, W: Weight, M, r, E=0):
+    return int(lib.qlora_workspace_size(int(op), W.ref, int(M), int(r), int(E)))
+
+
+def qlora_workspace_init(ws, stream=None):
+    _check(lib.qlora_workspace_init(_p(ws), ws.numel(), _stream(stream)), "qlora_workspace_init")
+
+
+def qlora_linear_fwd(W: Weight, X, A, B, Y, T_save, M, r, scale, ws, stream=None):
+    _check(lib.qlora_linear_fwd(W.ref, _p(X), _p(A), _p(B), _p(Y), _p(T_save), int(M), int(r),
+                                float(scale), _p(ws), 0 if ws is None else ws.numel(),
+                                _stream(stream)), "qlora_linear_fwd")
+
+
+def qlora_linear_bwd(W: Weight, X, A, B, T, dY, dX, dA, dB, M, r, scale, ws, stream=None):
+    _check(lib.qlora_linear_bwd(W.ref, _p(X), _p(A), _p(B), _p(T), _p(dY), _p(dX), _p(dA), _p(dB),
+                                int(M), int(r), float(scale), _p(ws),
+                                0 if ws is None else ws.numel(), _stream(stream)),
+           "qlora_linear_bwd")
+
+
+def qlora_grouped_fwd(W: Weight, E, offsets, M_total, X, A, B, Y, T_save, r, scale, ws,
+                      stream=None):
+    _check(lib.qlora_grouped_fwd(W.ref, int(E), _p(offsets), int(M_total), _p(X), _p(A), _p(B),
+                                 _p(Y), _p(T_save), int(r), float(scale), _p(ws),
+                                 0 if ws is None else ws.numel(), _stream(stream)),
+           "qlora_grouped_fwd")
+
+
+def qlora_grouped_bwd(W: Weight, E, offsets, M_total, X, A, B, T, dY, dX, dA, dB, r, scale, ws,
+                      stream=None):
+    _check(lib.qlora_grouped_bwd(W.ref, int(E), _p(offsets), int(M_total), _p(X), _p(A), _p(B),
+                                 _p(T), _p(dY), _p(dX), _p(dA), _p(dB), int(r), float(scale),
+                                 _p(ws), 0 if ws is None else ws.numel(), _stream(stream)),
+           "qlora_grouped_bwd")
+
+
+def qlora_get_device_status(ws, stream=None):
+    return int(lib.qlora_get_device_status(_p(ws), _stream(stream)))
+
+
+def qlora_debug_dequant(W: Weight, transposed, out, stream=None):
+    _check(lib.qlora_debug_dequant(W.ref, int(transposed), _p(out), _stream(stream)),
+           "qlora_debug_dequant")
+
+
+def qlora_debug_wait_timeout(ws, limit_us, stream=None):
+    _check(lib.qlora_debug_wait_timeout(_p(ws), ws.numel(), int(limit_us), _stream(stream)),
+           "qlora_debug_wait_timeout")
+
+
+def qlora_build_info():
+    return lib.qlora_build_info().decode()
+
+
+# ------------------------------------------------------------------------------ convenience
+def alloc_workspace(op, W: Weight, M, r, E=0, device="cuda"):
+    """A zero-initialised workspace for `op` (uint8 tensor)."""
+    n = qlora_workspace_size(op, W, M, r, E)
+    if n == 0:
+        raise QLoraError(1, "qlora_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def bf16_from_bits(a, device="cuda"):
+    """numpy uint16 bf16 bit patterns -> torch bfloat16 tensor on `device`."""
+    return torch.from_numpy(a.view("int16")).view(torch.bfloat16).to(device)
+
+
+def weight_from_numpy(fmt, codes, scales, tensor_scale=None, device="cuda"):
+    """Upload a stored weight (numpy arrays as made by synth) to the GPU."""
+    N = codes.shape[-2]
+    K = codes.shape[-1] * 2
+    c = torch.from_numpy(codes).to(device)
+    s = torch.from_numpy(scales).to(device)
+    ts = None
+    if fmt == "nvfp4":
+        import numpy as np
+        ts = torch.from_numpy(np.atleast_1d(np.asarray(tensor_scale, np.float32))).to(device)
+    return Weight(fmt, N, K, c, s, ts)

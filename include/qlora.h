@@ -1,0 +1,179 @@
+/* qlora.h -- C ABI of the B200 (sm_100a) library for the forward and backward pass of an
+ * unmerged-LoRA linear layer whose frozen base weight stays in 4-bit storage.
+ *
+ * The layer ("Training LLMs on a Budget: LoRA, QLoRA, and LoftQ", §2 "The math":
+ * y = W x + (alpha/r) B A x, the scaling "part of the layer" wherever BA appears; §3 "The setup":
+ * the 4-bit base is dequantised to bf16 on the fly, the matmul computed and the dequantised tensor
+ * discarded), written for a batch of M rows with s = alpha/r (or alpha/sqrt(r)):
+ *
+ *   T  = X A^T                    Y  = X deq(W)^T + s T B^T
+ *   U  = dY B                     dX = dY deq(W) + s U A
+ *   dA = s U^T X                  dB = s dY^T T
+ *
+ * dA and dB follow "Training LLMs on a Budget", §2 "Initialization matters" (dL/dA = B^T dL/dy x^T,
+ * dL/dB = dL/dy x^T A^T); there is no dW: the base is frozen ("Quantized weights, full precision:
+ * The math behind 75% cheaper fine-tuning", "Backward pass and optimizer step in training").
+ * deq(W) is computed inside the GEMM kernels; no bf16 copy of W is ever written to device memory.
+ *
+ * Shapes and layouts (row-major, last index contiguous):
+ *   X [M,K], Y [M,N], dY [M,N], dX [M,K], A [r,K], B [N,r], T/U [M,r], dA [r,K], dB [N,r]: bf16
+ *   (PyTorch's nn.Linear convention: W is [N = out, K = in]).
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers are device pointers unless stated otherwise; the caller owns every buffer.  The
+ *     library never allocates, frees or synchronises on the compute path; all work is enqueued
+ *     on `stream`.
+ *   - Arguments are validated before anything is enqueued; a failed check returns
+ *     QLORA_ERR_INVALID_ARG / QLORA_ERR_UNSUPPORTED / QLORA_ERR_WORKSPACE and enqueues nothing.
+ *     A failed launch returns QLORA_ERR_CUDA.  Device-side pipeline waits are bounded: if one ever
+ *     gives up, the kernel records QLORA_ERR_DEVICE_TIMEOUT in the workspace and ends, and
+ *     qlora_get_device_status() reports it.
+ *   - Shape limits: K % 64 == 0, N % 16 == 0, K >= 64, N >= 16, M >= 0 (M == 0 is a no-op that
+ *     still overwrites dA and dB with zeros), r in {8, 16, 32, 64}; every pointer 16-byte aligned.
+ *   - Outputs are overwritten, never accumulated (gradient accumulation across micro-batches is the
+ *     caller's job).  Results are deterministic: the same inputs give bitwise-identical outputs.
+ *   - Calls that share a workspace must be ordered on one stream.
+ */
+#ifndef QLORA_H_
+#define QLORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* qlora_stream_t; /* a cudaStream_t; NULL = the legacy default stream */
+
+typedef enum {
+  /* NF4: 16 normal-quantile levels times one fp32 absmax per 64 weights along K
+   * ("Training LLMs on a Budget", §3 "The three QLoRA tricks", items 1 and 2). */
+  QLORA_FMT_NF4 = 0,
+  /* MXFP4: E2M1 elements times one E8M0 scale 2^(e-127) per 32 along K
+   * ("Fine-Tuning 4-Bit Models: Adapting a Base That Only Ships Quantized", "Case 2: An NVFP4
+   * deployment checkpoint is what you were handed"). */
+  QLORA_FMT_MXFP4 = 1,
+  /* NVFP4: E2M1 elements times one E4M3 scale per 16 along K, times one fp32 tensor scale
+   * (same page and section: "a per-block FP8 scale over 16-element micro-blocks"). */
+  QLORA_FMT_NVFP4 = 2
+} qlora_format_t;
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1,    /* a NULL/misaligned pointer or a shape outside the limits */
+  QLORA_ERR_UNSUPPORTED = 2,    /* a valid request this build does not implement (e.g. rank) */
+  QLORA_ERR_WORKSPACE = 3,      /* workspace NULL or smaller than qlora_workspace_size() */
+  QLORA_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed (launch, tensor map) */
+  QLORA_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait gave up (kernel ended early) */
+} qlora_status_t;
+
+/* One frozen 4-bit weight W [N,K] (row n = output feature, K contiguous).
+ *   codes  [N, K/2] uint8: element 2j of a row in the low nibble of byte j, 2j+1 in the high.
+ *   scales NF4: float [N, K/64]; MXFP4: uint8 E8M0 [N, K/32]; NVFP4: uint8 E4M3 [N, K/16].
+ *          Block b of row n covers k in [b*bs, (b+1)*bs).
+ *   tensor_scale NVFP4: device float* holding the decode multiplier (grouped: [E] values);
+ *          NULL for NF4 and MXFP4.  It must be finite and non-zero.
+ * Decode of element (n,k) with code c: NF4 bf16(fp32(level[c] * absmax)); MXFP4
+ * bf16(e2m1(c) * 2^(e-127)); NVFP4 bf16(fp32(fp32(e2m1(c) * e4m3(s)) * tensor_scale)), every
+ * multiply binary32 round-to-nearest-even without flush-to-zero.  The kernels apply the NVFP4
+ * tensor scale to the fp32 accumulator rather than to each element (it is uniform over W); the
+ * per-element micro-block decode is exact.
+ * For the grouped entry points codes/scales are stacked [E, N, ...]. */
+typedef struct {
+  int32_t fmt; /* qlora_format_t */
+  int32_t reserved;
+  int64_t N, K;
+  const uint8_t* codes;
+  const void* scales;
+  const float* tensor_scale;
+} qlora_weight_t;
+
+typedef enum {
+  QLORA_OP_FWD = 0,
+  QLORA_OP_BWD = 1,
+  QLORA_OP_GROUPED_FWD = 2,
+  QLORA_OP_GROUPED_BWD = 3
+} qlora_op_t;
+
+/* Bytes of device workspace `op` needs for these shapes (E = number of experts for the grouped
+ * ops, ignored otherwise; for the grouped ops M is the total row count).  Returns 0 for invalid
+ * arguments.  A workspace sized for an op and shapes also serves smaller M. */
+QLORA_API size_t qlora_workspace_size(int op, const qlora_weight_t* W, int64_t M, int r, int E);
+
+/* Zero the workspace's status word and reduction counters.  Call once after allocating a
+ * workspace (or zero it yourself), and again after a QLORA_ERR_DEVICE_TIMEOUT.  Async on stream. */
+QLORA_API qlora_status_t qlora_workspace_init(void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* Forward: Y = X deq(W)^T + s (X A^T) B^T.  Two launches: T = X A^T (written to T_save when not
+ * NULL, for the backward pass), then the fused dequant-GEMM whose epilogue adds s T B^T.
+ *   W: frozen weight (host struct, device arrays); X [M,K], A [r,K], B [N,r]; Y [M,N] out;
+ *   T_save [M,r] out or NULL; scale = s; ws/ws_bytes: workspace (>= qlora_workspace_size(FWD)). */
+QLORA_API qlora_status_t qlora_linear_fwd(const qlora_weight_t* W, const void* X, const void* A,
+                                const void* B, void* Y, void* T_save, int64_t M, int r,
+                                float scale, void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* Backward: dX = dY deq(W) + s (dY B) A, dA = s (dY B)^T X, dB = s dY^T T.
+ *   T [M,r]: the forward's T_save, or NULL to recompute it from X and A.
+ *   dX [M,K] out or NULL (skip the input gradient); dA [r,K] and dB [N,r] out (overwritten). */
+QLORA_API qlora_status_t qlora_linear_bwd(const qlora_weight_t* W, const void* X, const void* A,
+                                const void* B, const void* T, const void* dY, void* dX, void* dA,
+                                void* dB, int64_t M, int r, float scale, void* ws, size_t ws_bytes,
+                                qlora_stream_t stream);
+
+/* Grouped (mixture-of-experts) forward: expert e applies its own W_e, A_e, B_e to rows
+ * [offsets[e], offsets[e+1]) of the expert-packed X ("Quantized weights, full precision", "LoRA
+ * operations and quantization": LoRA on the mxfp4 experts of an MoE model).
+ *   W: one struct describing the stacked weights (codes [E,N,K/2], scales [E,N,K/bs],
+ *   tensor_scale [E] for NVFP4); d_offsets: device int32 [E+1], exclusive prefix sum,
+ *   offsets[0] = 0, offsets[E] = M_total, non-decreasing (checked on the device: a violation is
+ *   reported as QLORA_ERR_INVALID_ARG by qlora_get_device_status); A [E,r,K], B [E,N,r];
+ *   X [M_total,K]; Y [M_total,N]; T_save [M_total,r] or NULL. */
+QLORA_API qlora_status_t qlora_grouped_fwd(const qlora_weight_t* W, int E, const int32_t* d_offsets,
+                                 int64_t M_total, const void* X, const void* A, const void* B,
+                                 void* Y, void* T_save, int r, float scale, void* ws,
+                                 size_t ws_bytes, qlora_stream_t stream);
+
+/* Grouped backward: per expert as qlora_linear_bwd; dA [E,r,K], dB [E,N,r] (experts with no rows
+ * get zeros); dX [M_total,K] or NULL; T [M_total,r] or NULL (recompute). */
+QLORA_API qlora_status_t qlora_grouped_bwd(const qlora_weight_t* W, int E, const int32_t* d_offsets,
+                                 int64_t M_total, const void* X, const void* A, const void* B,
+                                 const void* T, const void* dY, void* dX, void* dA, void* dB,
+                                 int r, float scale, void* ws, size_t ws_bytes,
+                                 qlora_stream_t stream);
+
+/* Synchronise `stream` and read the workspace's device status word (QLORA_OK or the first
+ * device-side error recorded since qlora_workspace_init).  Not for the compute path. */
+QLORA_API qlora_status_t qlora_get_device_status(void* ws, qlora_stream_t stream);
+
+/* Test-only: decode the whole weight through the kernels' own dequant stage (TMA code loads,
+ * register decode, swizzled shared-memory tile) and write it un-swizzled as bf16 [N,K] to `out`
+ * (N*K*2 bytes).  transposed = 0 uses the forward tiling (K-major operand tile), 1 the dX tiling
+ * (MN-major operand tile).  NVFP4 is written WITHOUT the tensor scale (the kernels apply it in the
+ * epilogue).  This is the one call that writes a bf16 weight to memory: it exists to check the
+ * decode bit for bit and is never used by the layer. */
+QLORA_API qlora_status_t qlora_debug_dequant(const qlora_weight_t* W, int transposed, void* out,
+                                   qlora_stream_t stream);
+
+/* Test-only: run a kernel that waits on a barrier nothing ever completes, with a wait limit of
+ * about limit_us microseconds, to check that bounded waits end with QLORA_ERR_DEVICE_TIMEOUT
+ * recorded in the workspace instead of hanging. */
+QLORA_API qlora_status_t qlora_debug_wait_timeout(void* ws, size_t ws_bytes, int limit_us,
+                                        qlora_stream_t stream);
+
+/* A short English description of a status code (static storage). */
+QLORA_API const char* qlora_status_string(qlora_status_t status);
+
+/* Build identification: "<version> sm_100a". */
+QLORA_API const char* qlora_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_H_ */

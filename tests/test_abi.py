@@ -1,0 +1,112 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments with the documented status before touching CUDA."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def Q():
+    from bit_quantized_base_b200 import build
+    build.build()
+    from bit_quantized_base_b200 import qlora
+    return qlora
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "qlora.h")).read()
+    return sorted(set(re.findall(r"QLORA_API\s+[\w\s\*]+?\b(qlora_\w+)\s*\(", src)))
+
+
+def test_header_declarations_are_exported(Q):
+    names = _declared()
+    assert len(names) >= 11
+    for n in names:
+        getattr(Q.lib, n)                     # raises AttributeError if not exported
+    assert sorted(Q.EXPORTS) == names
+
+
+def test_status_strings(Q):
+    for s in range(6):
+        assert Q.lib.qlora_status_string(s)
+    assert b"sm_100a" in Q.lib.qlora_build_info()
+
+
+class FakeT:
+    """Stands in for a device tensor: only data_ptr() / numel() are used by the binding."""
+
+    def __init__(self, ptr, n=1 << 30):
+        self.ptr, self.n = ptr, n
+
+    def data_ptr(self):
+        return self.ptr
+
+    def numel(self):
+        return self.n
+
+
+def _w(Q, fmt="nf4", N=256, K=512, codes=0x1000, scales=0x2000, ts=None):
+    W = Q.Weight.__new__(Q.Weight)
+    W.fmt, W.N, W.K = fmt, N, K
+    W.codes, W.scales, W.tensor_scale = None, None, None
+    W.c = Q.qlora_weight_t(Q.FMT[fmt], 0, N, K, codes, scales, ts)
+    return W
+
+
+def test_workspace_size_rules(Q):
+    W = _w(Q)
+    assert Q.qlora_workspace_size(Q.OP_FWD, W, 1024, 16) > 0
+    assert Q.qlora_workspace_size(Q.OP_BWD, W, 1024, 16) >= Q.qlora_workspace_size(Q.OP_FWD, W, 1024, 16)
+    assert Q.qlora_workspace_size(Q.OP_FWD, W, 1024, 12) == 0          # rank not supported
+    assert Q.qlora_workspace_size(Q.OP_FWD, _w(Q, K=96), 16, 16) == 0  # K % 64
+    assert Q.qlora_workspace_size(Q.OP_FWD, _w(Q, N=40), 16, 16) == 0  # N % 16
+    assert Q.qlora_workspace_size(Q.OP_FWD, _w(Q, fmt="nvfp4"), 16, 16) == 0   # NVFP4 needs tensor scale
+    assert Q.qlora_workspace_size(Q.OP_FWD, _w(Q, codes=0x1008), 16, 16) == 0  # misaligned codes
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(M=-1), "QLORA_ERR_INVALID_ARG"),
+    (dict(r=12), "QLORA_ERR_UNSUPPORTED"),
+    (dict(r=0), "QLORA_ERR_INVALID_ARG"),
+    (dict(X=0x1004), "QLORA_ERR_INVALID_ARG"),
+    (dict(Y=0), "QLORA_ERR_INVALID_ARG"),
+    (dict(ws=0), "QLORA_ERR_WORKSPACE"),
+    (dict(ws_bytes=64), "QLORA_ERR_WORKSPACE"),
+    (dict(W=dict(K=100)), "QLORA_ERR_INVALID_ARG"),
+    (dict(W=dict(fmt="nvfp4")), "QLORA_ERR_INVALID_ARG"),
+])
+def test_forward_rejects_bad_arguments(Q, bad, status):
+    W = _w(Q, **bad.get("W", {}))
+    args = dict(X=0x10000, A=0x20000, B=0x30000, Y=0x40000, T=0, M=64, r=16, ws=0x50000,
+                ws_bytes=1 << 30)
+    args.update({k: v for k, v in bad.items() if k != "W"})
+    rc = Q.lib.qlora_linear_fwd(W.ref, args["X"], args["A"], args["B"], args["Y"],
+                                args["T"] or None, args["M"], args["r"], 2.0,
+                                args["ws"] or None, args["ws_bytes"], None)
+    assert Q.STATUS[rc] == status
+
+
+def test_backward_rejects_bad_arguments(Q):
+    W = _w(Q)
+    ok = dict(X=0x10000, A=0x20000, B=0x30000, T=None, dY=0x60000, dX=None, dA=0x70000,
+              dB=0x80000)
+    for key in ("X", "A", "B", "dY", "dA", "dB"):
+        a = dict(ok)
+        a[key] = None
+        rc = Q.lib.qlora_linear_bwd(W.ref, a["X"], a["A"], a["B"], a["T"], a["dY"], a["dX"],
+                                    a["dA"], a["dB"], 64, 16, 2.0, 0x50000, 1 << 30, None)
+        assert Q.STATUS[rc] == "QLORA_ERR_INVALID_ARG", key
+    a = dict(ok, dX=0x90008)   # misaligned optional output
+    rc = Q.lib.qlora_linear_bwd(W.ref, a["X"], a["A"], a["B"], a["T"], a["dY"], a["dX"], a["dA"],
+                                a["dB"], 64, 16, 2.0, 0x50000, 1 << 30, None)
+    assert Q.STATUS[rc] == "QLORA_ERR_INVALID_ARG"
+
+
+def test_workspace_init_and_status_reject_null(Q):
+    assert Q.STATUS[Q.lib.qlora_workspace_init(None, 1 << 20, None)] == "QLORA_ERR_WORKSPACE"
+    assert Q.STATUS[Q.lib.qlora_get_device_status(None, None)] == "QLORA_ERR_WORKSPACE"
+    assert Q.STATUS[Q.lib.qlora_debug_wait_timeout(0x1000, 1 << 20, 0, None)] == "QLORA_ERR_INVALID_ARG"
