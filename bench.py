@@ -1,0 +1,452 @@
+#!/usr/bin/env python3
+"""Benchmark: forward + backward of one unmerged-LoRA linear on a frozen 4-bit base (B200).
+
+A step is one pass of the whole hot path over one batch: T = X A^T, the fused dequant-GEMM
+Y = X deq(W)^T + s T B^T, U = dY B, the fused dX = dY deq(W) + s U A, and dA, dB -- five kernel
+launches through the library's C ABI (qlora_linear_fwd + qlora_linear_bwd).
+
+Workload (one GPU): Llama-3-8B-shaped MLP up-projection, NF4 base: X [4096, 4096], W [14336, 4096]
+(NF4, absmax per 64 along K), LoRA rank 64, alpha 128, synthetic seeded inputs.  Throughput counts
+the algorithmic flops 4MNK + 6Mr(K+N) per step.  Every step reads a different device copy of W, X
+and dY (3 copies, 546 MB > 2x the 126 MB L2), so no input is served from L2 across steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl own|reference]
+
+N > 1 (launched with torch.distributed.run): each rank runs its own replica of the workload (the
+layer has no cross-GPU exchange in this benchmark), timing is the max over ranks of the device time
+of the K steps.  --impl reference times the CPU oracle instead (rank 0 only).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fwd+bwd TFLOP/s per 4-bit-base LoRA linear; weight-stream GB/s at small M"
+WORKLOAD = "Llama-3-8B-shaped MLP up-proj, NF4 base: M=4096 tokens, N=14336, K=4096, r=64, alpha=128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# device sources of the fused dequant-GEMM kernel: a traffic figure taken on other sources is stale
+KERNEL_SOURCES = ["qlora_fused.cuh", "qlora_dequant.cuh", "qlora_ptx.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["own", "reference"], default="own")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the small-M weight-stream sweep")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def flops(M, N, K, r):
+    return 4.0 * M * N * K + 6.0 * M * r * (K + N)
+
+
+def weight_bytes(fmt, N, K):
+    bs = {"nf4": 64, "mxfp4": 32, "nvfp4": 16}[fmt]
+    per_scale = 4 if fmt == "nf4" else 1
+    return N * K // 2 + N * (K // bs) * per_scale + (4 if fmt == "nvfp4" else 0)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "bit_quantized_base_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel):
+    """dram bytes per launch of `kernel` from the committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                    power.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        # samples taken while the GPU was busy: the upper half by power draw
+        if sm:
+            pairs = sorted(zip(power, sm))
+            busy = [s for p, s in pairs[len(pairs) // 2:]] or sm
+            return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(smax),
+                    "reasons": sorted(reasons), "samples": len(sm),
+                    "power_w_max": max(power)}
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+# ------------------------------------------------------------------------------- own arm
+def dist_setup(args):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(ws, x):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_own(args):
+    import numpy as np
+    import torch
+    from bit_quantized_base_b200 import qlora as Q
+    from bit_quantized_base_b200 import synth
+
+    ws_n, rank, local = dist_setup(args)
+    cfg = synth.CONFIGS[2]
+    p = synth.layer_inputs(2)
+    fmt, M, N, K, r, s = p["fmt"], p["M"], p["N"], p["K"], p["r"], p["s"]
+    ncopy = 3
+    Ws = [Q.weight_from_numpy(fmt, p["codes"], p["scales"], p["tensor_scale"]) for _ in range(ncopy)]
+    Xs = [Q.bf16_from_bits(p["X"]) for _ in range(ncopy)]
+    dYs = [Q.bf16_from_bits(p["dY"]) for _ in range(ncopy)]
+    A = Q.bf16_from_bits(p["A"])
+    B = Q.bf16_from_bits(p["B"])
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    T = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty((r, K), dtype=torch.bfloat16, device="cuda")
+    dB = torch.empty((N, r), dtype=torch.bfloat16, device="cuda")
+    ws = Q.alloc_workspace(Q.OP_BWD, Ws[0], M, r)
+    Q.qlora_workspace_init(ws)
+    in_bytes = ncopy * (Ws[0].nbytes() + Xs[0].numel() * 2 + dYs[0].numel() * 2)
+
+    def step(i):
+        c = i % ncopy
+        Q.qlora_linear_fwd(Ws[c], Xs[c], A, B, Y, T, M, r, s, ws)
+        Q.qlora_linear_bwd(Ws[c], Xs[c], A, B, T, dYs[c], dX, dA, dB, M, r, s, ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if Q.qlora_get_device_status(ws) != 0:
+        raise RuntimeError("device status after warm-up: %d" % Q.qlora_get_device_status(ws))
+
+    # ---- timed region (device time, CUDA events on the launching stream)
+    Q.qlora_profile_enable(True)
+    Q.qlora_profile_reset()
+    clk = ClockSampler(local)
+    clk.start()
+    barrier(ws_n)
+    torch.cuda.synchronize()
+    launches0 = Q.qlora_launch_count()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    ev1.record()
+    ev1.synchronize()
+    torch.cuda.synchronize()
+    barrier(ws_n)
+    launches = Q.qlora_launch_count() - launches0
+    clocks = clk.stop()
+    ms_local = ev0.elapsed_time(ev1)
+    prof = Q.qlora_profile_read()
+    Q.qlora_profile_enable(False)
+    ms_total = max_over_ranks(ws_n, ms_local)
+    ms_step = ms_total / args.steps
+    fl = flops(M, N, K, r)
+    value = ws_n * fl * args.steps / (ms_total * 1e-3) / 1e12
+
+    if Q.qlora_get_device_status(ws) != 0:
+        raise RuntimeError("device status after the timed region: %d" % Q.qlora_get_device_status(ws))
+
+    # ---- dominant kernel and its roofline
+    peaks, peak_src = load_peaks()
+    kflops = {"fused_fwd": 2.0 * M * N * K + 2.0 * M * N * r,
+              "fused_dx": 2.0 * M * N * K + 2.0 * M * K * r,
+              "lora_down_T": 2.0 * M * K * r, "lora_down_U": 2.0 * M * N * r,
+              "lora_wgrad": 2.0 * M * N * r + 2.0 * M * K * r}
+    dom = max(prof, key=lambda k: prof[k][1])
+    cnt, tot = prof[dom]
+    avg_ms = tot / cnt
+    achieved = kflops[dom] / (avg_ms * 1e-3) / 1e12
+    long_region = ms_local > 1000.0
+    peak = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
+    roofline = {
+        "kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+        "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+        "peak_source": f"{'sustained' if long_region else 'burst'} bf16, {peak_src}",
+        "frac_of_nominal_2250": round(achieved / 2250.0, 4),
+        "traffic": load_traffic(dom),
+        "avg_launch_ms": round(avg_ms, 4),
+    }
+    breakdown = {k: {"launches": c, "total_ms": round(t, 3), "avg_ms": round(t / c, 4),
+                     "share": round(t / sum(v[1] for v in prof.values()), 4)}
+                 for k, (c, t) in sorted(prof.items())}
+
+    # ---- end to end through the public API with host buffers
+    hX = torch.from_numpy(p["X"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hdY = torch.from_numpy(p["dY"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hdA = torch.empty((r, K), dtype=torch.bfloat16).pin_memory()
+    hdB = torch.empty((N, r), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 30))
+
+    def e2e_step(i):
+        c = i % ncopy
+        Xs[c].copy_(hX, non_blocking=True)
+        dYs[c].copy_(hdY, non_blocking=True)
+        Q.qlora_linear_fwd(Ws[c], Xs[c], A, B, Y, T, M, r, s, ws)
+        Q.qlora_linear_bwd(Ws[c], Xs[c], A, B, T, dYs[c], dX, dA, dB, M, r, s, ws)
+        hdA.copy_(dA, non_blocking=True)
+        hdB.copy_(dB, non_blocking=True)
+
+    for i in range(2):
+        e2e_step(i)
+    barrier(ws_n)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record()
+    e1.synchronize()
+    e2e_ms = max_over_ranks(ws_n, e0.elapsed_time(e1))
+    e2e = {"value": round(ws_n * fl * e2e_steps / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int((hX.numel() + hdY.numel()) * 2),
+           "d2h_bytes_per_step": int((hdA.numel() + hdB.numel()) * 2),
+           "ms_per_step": round(e2e_ms / e2e_steps, 4)}
+
+    # ---- small-M weight-stream sweep on the same weight
+    sweep = None
+    if not args.no_sweep:
+        sweep = {}
+        wbytes = weight_bytes(fmt, N, K)
+        nw = int(math.ceil(3 * 126e6 / wbytes)) + 1
+        Wsw = Ws + [Q.weight_from_numpy(fmt, p["codes"], p["scales"], p["tensor_scale"])
+                    for _ in range(max(0, nw - ncopy))]
+        for Ms in (16, 32, 64, 128, 256):
+            Xm, dYm = Xs[0][:Ms], dYs[0][:Ms]
+            Ym, Tm, dXm = Y[:Ms], T[:Ms], dX[:Ms]
+            wsm = Q.alloc_workspace(Q.OP_BWD, Wsw[0], Ms, r)
+            Q.qlora_workspace_init(wsm)
+
+            def sstep(i):
+                w = Wsw[i % len(Wsw)]
+                Q.qlora_linear_fwd(w, Xm, A, B, Ym, Tm, Ms, r, s, wsm)
+                Q.qlora_linear_bwd(w, Xm, A, B, Tm, dYm, dXm, dA, dB, Ms, r, s, wsm)
+
+            for i in range(5):
+                sstep(i)
+            torch.cuda.synchronize()
+            n_it = 60
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record()
+            for i in range(n_it):
+                sstep(i)
+            a1.record()
+            a1.synchronize()
+            t = a0.elapsed_time(a1) / n_it * 1e-3
+            sweep[str(Ms)] = {"us_per_step": round(t * 1e6, 1),
+                              "weight_gbs": round(2 * wbytes / t / 1e9, 1),
+                              "tflops": round(flops(Ms, N, K, r) / t / 1e12, 1)}
+
+    # ---- CPU baseline: the oracle on a bounded sample of the same workload
+    cpu = None
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(p, args.cpu_seconds)
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws_n,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded numpy PCG64; W ~ N(0, 0.02) quantised to NF4)",
+        "config": {"workload": WORKLOAD, "fmt": fmt, "M": M, "N": N, "K": K, "r": r,
+                   "alpha": cfg.alpha, "flops_per_step": fl,
+                   "l2": f"inputs larger than L2: {ncopy} rotating device copies of W, X, dY "
+                         f"({in_bytes / 1e6:.0f} MB)",
+                   "parallelism": f"replicas x{ws_n} (no data-path collective)"},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "roofline": roofline,
+        "kernel_breakdown": breakdown,
+        "e2e": e2e,
+        "weight_stream_small_m": sweep,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if ws_n > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------------------- CPU oracle
+def _oracle_sample(p, rows):
+    """Time the oracle on the layer restricted to the first `rows` rows of the batch."""
+    from oracle import oracle as O
+    t0 = time.perf_counter()
+    O.layer(p["fmt"], rows, p["N"], p["K"], p["r"], p["s"], p["codes"], p["scales"],
+            p["tensor_scale"], p["X"][:rows], p["A"], p["B"], p["dY"][:rows])
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(p, target_s):
+    from oracle import oracle as O
+    N, K, r = p["N"], p["K"], p["r"]
+    t1 = _oracle_sample(p, 1)
+    t8 = _oracle_sample(p, 8)
+    per_row = max((t8 - t1) / 7, 1e-4)
+    rows = int(max(8, min(p["M"], (target_s - t1) / per_row)))
+    t = _oracle_sample(p, rows)
+    v = flops(rows, N, K, r) / t / 1e12
+    return {"value": round(v, 6), "unit": "TFLOP/s", "cores": O.num_threads(), "kind": "oracle",
+            "seconds": round(t, 2),
+            "sample": f"full fp64 fwd+bwd of the same layer on the first {rows} of the "
+                      f"{p['M']} rows (W decode included), OpenMP"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    ws_n = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from bit_quantized_base_b200 import synth
+    from oracle import oracle as O
+    p = synth.layer_inputs(2)
+    N, K, r = p["N"], p["K"], p["r"]
+    # each step: the oracle on a bounded sample of the batch, sized so that warm-up + steps stay
+    # within a few minutes
+    budget_s = 150.0
+    t1 = _oracle_sample(p, 1)
+    per_step = budget_s / max(1, args.steps + args.warmup)
+    rows = 1
+    if per_step > t1:
+        t4 = _oracle_sample(p, 4)
+        per_row = max((t4 - t1) / 3, 1e-4)
+        rows = int(max(1, min(p["M"], 1 + (per_step - t1) / per_row)))
+    for _ in range(args.warmup):
+        _oracle_sample(p, rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_sample(p, rows)
+    dt = time.perf_counter() - t0
+    v = flops(rows, N, K, r) * args.steps / dt / 1e12
+    sample = (f"per step: full fp64 fwd+bwd of the same layer on the first {rows} of the "
+              f"{p['M']} rows (W decode included), OpenMP")
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s",
+        "n_gpus": ws_n, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "fmt": p["fmt"], "M": p["M"], "N": N, "K": K, "r": r},
+        "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": O.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_own(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -3,9 +3,11 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "qlora.h"
 #include "qlora_debug.cuh"
@@ -148,6 +150,42 @@ WsLayout ws_layout(int64_t N, int64_t K, int64_t M, int r, bool bwd, int sms) {
 int* ws_status(void* ws) { return reinterpret_cast<int*>(ws); }
 int* ws_counters(void* ws) { return reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + kHeaderBytes); }
 
+// ---------------------------------------------------------------------------------- profiling
+enum Kind : int {
+  kKindFusedFwd = 0, kKindFusedDx, kKindDownT, kKindDownU, kKindWgrad,
+  kKindGFusedFwd, kKindGFusedDx, kKindGDownT, kKindGDownU, kKindGWgrad, kNumKinds
+};
+const char* const kKindNames[kNumKinds] = {
+    "fused_fwd", "fused_dx", "lora_down_T", "lora_down_U", "lora_wgrad",
+    "grouped_fused_fwd", "grouped_fused_dx", "grouped_lora_down_T", "grouped_lora_down_U",
+    "grouped_lora_wgrad"};
+constexpr int kMaxProfiled = 65536;
+
+std::atomic<int64_t> g_launches{0};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<cudaEvent_t> g_ev;          // 2 per record
+std::vector<int> g_rec_kind;
+
+// Brackets one kernel launch: counts it, and records start/end events while profiling is on.
+struct LaunchScope {
+  int slot = -1;
+  cudaStream_t st;
+  LaunchScope(int kind, cudaStream_t s) : st(s) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (!g_prof_on) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    const int n = int(g_rec_kind.size());
+    if (!g_prof_on || 2 * (n + 1) > int(g_ev.size())) return;
+    slot = n;
+    g_rec_kind.push_back(kind);
+    cudaEventRecord(g_ev[2 * n], st);
+  }
+  ~LaunchScope() {
+    if (slot >= 0) cudaEventRecord(g_ev[2 * slot + 1], st);
+  }
+};
+
 // ---------------------------------------------------------------------------------- launches
 qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t Kc, const void* R,
                                 int64_t R_rows, int r, float s, const float* ts, void* z, void* zs,
@@ -176,6 +214,7 @@ qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t K
   p.num_k = int((Kc + 63) / 64);
   p.s = s;
   const dim3 grid(unsigned((M + 127) / 128));
+  LaunchScope scope(r_mn ? kKindDownU : kKindDownT, st);
   if (r_mn) {
     if (!set_smem(qlora_lora_down_kernel<true>, lora::kSmemBytes)) return QLORA_ERR_CUDA;
     qlora_lora_down_kernel<true><<<grid, lora::kThreads, lora::kSmemBytes, st>>>(p);
@@ -189,6 +228,7 @@ qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t K
 template <int FMT, bool DX>
 qlora_status_t launch_fused_t(const FusedParams& p, int grid, cudaStream_t st) {
   if (!set_smem(qlora_fused_gemm_kernel<FMT, DX>, fused::kSmemBytes)) return QLORA_ERR_CUDA;
+  LaunchScope scope(DX ? kKindFusedDx : kKindFusedFwd, st);
   qlora_fused_gemm_kernel<FMT, DX><<<grid, fused::kThreads, fused::kSmemBytes, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
@@ -273,6 +313,7 @@ qlora_status_t launch_wgrad(const void* X, const void* dY, const void* T, const 
   if (wp.tiles0 + wp.tiles1 > kMaxCounters) return QLORA_ERR_UNSUPPORTED;
   if (!set_smem(qlora_lora_wgrad_kernel, lora::kSmemBytes)) return QLORA_ERR_CUDA;
   const unsigned grid = unsigned((wp.tiles0 + wp.tiles1) * wp.S);
+  LaunchScope scope(kKindWgrad, st);
   qlora_lora_wgrad_kernel<<<grid, lora::kThreads, lora::kSmemBytes, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
@@ -445,5 +486,55 @@ const char* qlora_status_string(qlora_status_t status) {
 }
 
 const char* qlora_build_info(void) { return "qlora-b200 0.1 sm_100a"; }
+
+int64_t qlora_launch_count(void) { return g_launches.load(); }
+
+qlora_status_t qlora_profile_enable(int enable) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (enable && g_ev.empty()) {
+    g_ev.resize(2 * size_t(kMaxProfiled));
+    for (auto& e : g_ev)
+      if (cudaEventCreate(&e) != cudaSuccess) {
+        g_ev.clear();
+        return QLORA_ERR_CUDA;
+      }
+  }
+  g_prof_on = enable != 0;
+  return QLORA_OK;
+}
+
+qlora_status_t qlora_profile_reset(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_rec_kind.clear();
+  return QLORA_OK;
+}
+
+qlora_status_t qlora_profile_read(int max_kinds, int* n_kinds, const char** names, int* counts,
+                                  double* total_ms) {
+  if (!n_kinds || max_kinds < 0 || (max_kinds > 0 && (!names || !counts || !total_ms)))
+    return QLORA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  int cnt[kNumKinds] = {0};
+  double ms[kNumKinds] = {0.0};
+  for (size_t i = 0; i < g_rec_kind.size(); ++i) {
+    if (cudaEventSynchronize(g_ev[2 * i + 1]) != cudaSuccess) return QLORA_ERR_CUDA;
+    float t = 0.0f;
+    if (cudaEventElapsedTime(&t, g_ev[2 * i], g_ev[2 * i + 1]) != cudaSuccess) return QLORA_ERR_CUDA;
+    cnt[g_rec_kind[i]] += 1;
+    ms[g_rec_kind[i]] += t;
+  }
+  int n = 0;
+  for (int k = 0; k < kNumKinds; ++k) {
+    if (cnt[k] == 0) continue;
+    if (n < max_kinds) {
+      names[n] = kKindNames[k];
+      counts[n] = cnt[k];
+      total_ms[n] = ms[k];
+    }
+    ++n;
+  }
+  *n_kinds = n;
+  return QLORA_OK;
+}
 
 }  // extern "C"

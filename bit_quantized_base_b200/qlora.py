@@ -26,7 +26,8 @@ STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED",
 EXPORTS = ("qlora_workspace_size", "qlora_workspace_init", "qlora_linear_fwd", "qlora_linear_bwd",
            "qlora_grouped_fwd", "qlora_grouped_bwd", "qlora_get_device_status",
            "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_status_string",
-           "qlora_build_info")
+           "qlora_build_info", "qlora_launch_count", "qlora_profile_enable",
+           "qlora_profile_reset", "qlora_profile_read")
 
 
 class QLoraError(RuntimeError):
@@ -67,9 +68,14 @@ def _load():
     L.qlora_status_string.argtypes = [c.c_int]
     L.qlora_status_string.restype = c.c_char_p
     L.qlora_build_info.restype = c.c_char_p
+    L.qlora_launch_count.restype = c.c_int64
+    L.qlora_profile_enable.argtypes = [c.c_int]
+    L.qlora_profile_read.argtypes = [c.c_int, c.POINTER(c.c_int), c.POINTER(c.c_char_p),
+                                     c.POINTER(c.c_int), c.POINTER(c.c_double)]
     for name in ("qlora_workspace_init", "qlora_linear_fwd", "qlora_linear_bwd",
                  "qlora_grouped_fwd", "qlora_grouped_bwd", "qlora_get_device_status",
-                 "qlora_debug_dequant", "qlora_debug_wait_timeout"):
+                 "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_profile_enable",
+                 "qlora_profile_reset", "qlora_profile_read"):
         getattr(L, name).restype = c.c_int
     return L
 
@@ -174,6 +180,29 @@ def qlora_debug_wait_timeout(ws, limit_us, stream=None):
 
 def qlora_build_info():
     return lib.qlora_build_info().decode()
+
+
+def qlora_launch_count():
+    return int(lib.qlora_launch_count())
+
+
+def qlora_profile_enable(enable=True):
+    _check(lib.qlora_profile_enable(1 if enable else 0), "qlora_profile_enable")
+
+
+def qlora_profile_reset():
+    _check(lib.qlora_profile_reset(), "qlora_profile_reset")
+
+
+def qlora_profile_read():
+    """{kind: (launches, total_ms)} of the launches recorded since the last reset."""
+    n = ctypes.c_int(0)
+    cap = 16
+    names = (ctypes.c_char_p * cap)()
+    counts = (ctypes.c_int * cap)()
+    ms = (ctypes.c_double * cap)()
+    _check(lib.qlora_profile_read(cap, ctypes.byref(n), names, counts, ms), "qlora_profile_read")
+    return {names[i].decode(): (int(counts[i]), float(ms[i])) for i in range(min(n.value, cap))}
 
 
 # ------------------------------------------------------------------------------ convenience

@@ -167,6 +167,20 @@ QLORA_API qlora_status_t qlora_debug_dequant(const qlora_weight_t* W, int transp
 QLORA_API qlora_status_t qlora_debug_wait_timeout(void* ws, size_t ws_bytes, int limit_us,
                                         qlora_stream_t stream);
 
+/* Profiling support for benchmarks.  qlora_launch_count() is the number of kernels this library
+ * has launched in the process (always counted).  While profiling is enabled, every launch is also
+ * bracketed by two CUDA events recorded on its stream (up to 65536 launches; events are created by
+ * qlora_profile_enable, never on the compute path); qlora_profile_read synchronises on them and
+ * returns, per kernel kind, the launch count and total milliseconds.  Kinds: "fused_fwd",
+ * "fused_dx", "lora_down_T", "lora_down_U", "lora_wgrad" (grouped variants add "grouped_").
+ * Host-side bookkeeping only; the compute path is unchanged when profiling is off. */
+QLORA_API int64_t qlora_launch_count(void);
+QLORA_API qlora_status_t qlora_profile_enable(int enable);
+QLORA_API qlora_status_t qlora_profile_reset(void);
+/* Fills up to max_kinds entries; returns the number of kinds through *n_kinds. */
+QLORA_API qlora_status_t qlora_profile_read(int max_kinds, int* n_kinds, const char** names,
+                                            int* counts, double* total_ms);
+
 /* A short English description of a status code (static storage). */
 QLORA_API const char* qlora_status_string(qlora_status_t status);
 
