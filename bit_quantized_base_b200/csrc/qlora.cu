@@ -318,6 +318,29 @@ qlora_status_t launch_wgrad(const void* X, const void* dY, const void* T, const 
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------- fixed scratch (no alloc)
+// Scratch of qlora_linear_fwd_noalloc: a file-scope device array, present on every GPU that loads
+// the library.  Host code must not pass the symbol itself to a kernel (on the host it names a
+// stand-in, not device memory): its device address is looked up once per device.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+void* g_noalloc_addr[kMaxDevices] = {nullptr};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch on the current device, or nullptr if it cannot be resolved.
+void* noalloc_scratch_address() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[d]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return nullptr;
+    g_noalloc_addr[d] = ptr;
+  }
+  return g_noalloc_addr[d];
+}
+
 }  // namespace
 }  // namespace qlora
 
@@ -360,6 +383,32 @@ qlora_status_t qlora_linear_fwd(const qlora_weight_t* W, const void* X, const vo
   st = launch_lora_down(false, X, M, W->K, A, r, r, scale, ts, T, Zs, ws_status(ws), s);
   if (st != QLORA_OK) return st;
   return launch_fused(W, false, X, Zs, B, Y, M, r, ws_status(ws), s);
+}
+
+qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const void* X, const void* A,
+                                        const void* B, void* Y, void* T_save, int64_t M, int r,
+                                        float scale, qlora_stream_t stream) {
+  qlora_status_t st = check_weight(W);
+  if (st != QLORA_OK) return st;
+  if (M < 0 || M > (int64_t(1) << 31) - 512) return QLORA_ERR_INVALID_ARG;
+  if (!rank_ok(r)) return (r > 0 && r <= 256) ? QLORA_ERR_UNSUPPORTED : QLORA_ERR_INVALID_ARG;
+  if (!ptr_ok(X) || !ptr_ok(A) || !ptr_ok(B) || !ptr_ok(Y) || (T_save && !aligned16(T_save)))
+    return QLORA_ERR_INVALID_ARG;
+  const size_t mr = align_up(size_t(M) * size_t(r) * 2, 256);
+  const size_t need = kHeaderBytes + mr + (T_save ? 0 : mr);
+  if (need > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
+  if (M == 0) return QLORA_OK;
+  uint8_t* w = static_cast<uint8_t*>(noalloc_scratch_address());
+  if (!w) return QLORA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(w, 0, kHeaderBytes, s) != cudaSuccess) return QLORA_ERR_CUDA;
+  int* status = reinterpret_cast<int*>(w);
+  void* Zs = w + kHeaderBytes;
+  void* T = T_save ? T_save : w + kHeaderBytes + mr;
+  const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
+  st = launch_lora_down(false, X, M, W->K, A, r, r, scale, ts, T, Zs, status, s);
+  if (st != QLORA_OK) return st;
+  return launch_fused(W, false, X, Zs, B, Y, M, r, status, s);
 }
 
 qlora_status_t qlora_linear_bwd(const qlora_weight_t* W, const void* X, const void* A,

@@ -27,7 +27,7 @@ EXPORTS = ("qlora_workspace_size", "qlora_workspace_init", "qlora_linear_fwd", "
            "qlora_grouped_fwd", "qlora_grouped_bwd", "qlora_get_device_status",
            "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_status_string",
            "qlora_build_info", "qlora_launch_count", "qlora_profile_enable",
-           "qlora_profile_reset", "qlora_profile_read")
+           "qlora_profile_reset", "qlora_profile_read", "qlora_linear_fwd_noalloc")
 
 
 class QLoraError(RuntimeError):
@@ -69,6 +69,8 @@ def _load():
     L.qlora_status_string.restype = c.c_char_p
     L.qlora_build_info.restype = c.c_char_p
     L.qlora_launch_count.restype = c.c_int64
+    L.qlora_linear_fwd_noalloc.argtypes = [W, P, P, P, P, P, c.c_int64, c.c_int, c.c_float, P]
+    L.qlora_linear_fwd_noalloc.restype = c.c_int
     L.qlora_profile_enable.argtypes = [c.c_int]
     L.qlora_profile_read.argtypes = [c.c_int, c.POINTER(c.c_int), c.POINTER(c.c_char_p),
                                      c.POINTER(c.c_int), c.POINTER(c.c_double)]
@@ -139,6 +141,13 @@ def qlora_linear_fwd(W: Weight, X, A, B, Y, T_save, M, r, scale, ws, stream=None
     _check(lib.qlora_linear_fwd(W.ref, _p(X), _p(A), _p(B), _p(Y), _p(T_save), int(M), int(r),
                                 float(scale), _p(ws), 0 if ws is None else ws.numel(),
                                 _stream(stream)), "qlora_linear_fwd")
+
+
+def qlora_linear_fwd_noalloc(W: Weight, X, A, B, Y, T_save, M, r, scale, stream=None):
+    """Forward with the library's fixed internal scratch instead of a caller workspace."""
+    _check(lib.qlora_linear_fwd_noalloc(W.ref, _p(X), _p(A), _p(B), _p(Y), _p(T_save), int(M),
+                                        int(r), float(scale), _stream(stream)),
+           "qlora_linear_fwd_noalloc")
 
 
 def qlora_linear_bwd(W: Weight, X, A, B, T, dY, dX, dA, dB, M, r, scale, ws, stream=None):

@@ -148,6 +148,29 @@ QLORA_API qlora_status_t qlora_grouped_bwd(const qlora_weight_t* W, int E, const
                                  int r, float scale, void* ws, size_t ws_bytes,
                                  qlora_stream_t stream);
 
+/* Forward without a workspace: the same computation and kernels as qlora_linear_fwd, for callers
+ * that cannot allocate device memory where they run the layer -- for example runtimes that
+ * allocate everything at start-up and forbid allocation on the step path (an allocation can
+ * synchronise the device and fragment its memory), or plain C callers with no allocator of their
+ * own.  The paper has no counterpart of this entry point; it only changes who provides scratch.
+ *   Scratch is a fixed 4 MiB array inside the library (every GPU that loads the library holds it
+ *   until the process exits): 256 bytes of status, the [M,r] bf16 operand Zs and, when T_save is
+ *   NULL, an [M,r] bf16 T.  Sizes that do not fit -- M*r > 2,097,024 with T_save, or
+ *   M*r > 1,048,512 without -- are rejected with QLORA_ERR_WORKSPACE before anything is enqueued.
+ *   The call allocates nothing (no cudaMalloc/cudaFree, no allocating library routine); it clears
+ *   the status word on `stream` each call.
+ *   The first call on each device looks up the array's device address (cudaGetSymbolAddress) with
+ *   that device current; make that first call before any stream capture.
+ *   Every call uses the same array and leaves its contents behind: calls whose work overlaps on
+ *   the GPU (other streams, other threads) race on it, so order them on one stream.
+ *   A device-side wait that gives up ends the kernel early; its status word lives in the array and
+ *   is not visible through qlora_get_device_status.
+ * Arguments and their checks are those of qlora_linear_fwd, minus the workspace. */
+QLORA_API qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const void* X,
+                                                  const void* A, const void* B, void* Y,
+                                                  void* T_save, int64_t M, int r, float scale,
+                                                  qlora_stream_t stream);
+
 /* Synchronise `stream` and read the workspace's device status word (QLORA_OK or the first
  * device-side error recorded since qlora_workspace_init).  Not for the compute path. */
 QLORA_API qlora_status_t qlora_get_device_status(void* ws, qlora_stream_t stream);
