@@ -266,8 +266,10 @@ qlora_status_t launch_fused(const qlora_weight_t* W, bool dx, const void* act, c
   p.num_m = int((M + fused::BM - 1) / fused::BM);
   p.num_n = int(((dx ? K : N) + fused::BN - 1) / fused::BN);
   p.num_k = int((Kc + fused::BK - 1) / fused::BK);
+  // one CTA pair per pair tile, at most one pair per two SMs (persistent beyond that)
   const int tiles = p.num_m * p.num_n;
-  const int grid = tiles < num_sms() ? tiles : num_sms();
+  const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
+  const int grid = 2 * (pairs > 0 ? pairs : 1);
   switch (W->fmt * 2 + (dx ? 1 : 0)) {
     case 0: return launch_fused_t<kFmtNF4, false>(p, grid, st);
     case 1: return launch_fused_t<kFmtNF4, true>(p, grid, st);

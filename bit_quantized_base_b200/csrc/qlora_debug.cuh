@@ -25,7 +25,7 @@ qlora_debug_dequant_kernel(const __grid_constant__ DebugDequantParams p) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
   const int tg = threadIdx.x;
-  const int c0 = blockIdx.x * fused::BN;    // forward: first weight row; dX: first column
+  const int c0 = blockIdx.x * fused::HN;    // forward: first weight row; dX: first column
   const int ks = blockIdx.y;                 // forward: column step;     dX: row step
   const uint32_t b = ptx::smem_u32(&bar);
   if (tg == 0) {

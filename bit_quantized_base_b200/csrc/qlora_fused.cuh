@@ -8,13 +8,34 @@
 // lora_down kernel), its B operand the rows of B (forward) or A (backward), so it accumulates into
 // the same fp32 tensor-memory accumulator as the base product and the epilogue only scales by ts.
 //
-// Per CTA tile: 256 rows (two M=128 UMMA halves sharing one B operand) x 128 output columns,
-// 64-deep contraction steps.  Warp roles (448 threads, one CTA per SM, persistent over tiles):
+// The kernel runs on CTA pairs (clusters of 2) sharing one tcgen05.mma.cta_group::2 of M=256,
+// N=256 per 16-deep step.  A pair tile is 256 rows x 256 output columns; CTA rank r holds rows
+// [128r, 128r+128) of the activation operand and output columns [128r, 128r+128) of the
+// dequantised weight operand, and receives rows [128r, 128r+128) x all 256 columns of the fp32
+// accumulator in its own tensor memory (double buffered: 2 x 256 columns).  Each weight element is
+// decoded once per 256 rows, and each activation tile is fetched once per 256 output columns.
+//
+// Warp roles per CTA (480 threads, one CTA per SM, persistent over pair tiles):
 //   warps 0-3   epilogue: tensor memory -> registers -> * ts -> bf16 -> global
-//   warp  4     TMA producer: activation tiles (SW128, K-major) and packed-code tiles
-//   warp  5     tensor-memory allocation and the single thread that issues tcgen05.mma
-//   warps 6-13  dequant: two groups of 4 warps taking alternate steps; each thread decodes one
-//               64-element item of W per step into the swizzled operand tile
+//   warp  4     TMA producer of this CTA's activation half (completion counted on the leader's
+//               barrier)
+//   warp  6     TMA producer of this CTA's packed-code tiles, running ahead of the activation
+//               stream on its own deeper ring so the decode never waits for codes
+//   warp  5     tensor-memory allocation; in the leader CTA the single thread that issues the
+//               pair MMA and commits (arriving on both CTAs' barriers); in the other CTA one
+//               thread that forwards "weight half ready" to the leader, one cluster-scope arrive
+//               per step (the dequant warps themselves only arrive on their own CTA's barrier)
+// An operand stage holds this CTA's activation half and weight half of one 64-deep step.  The
+// leader's stage-full barrier collects everything the pair MMA needs -- the activation bytes of
+// both CTAs (TMA transaction count), the leader's 4 dequant warps and the other CTA's relayed
+// arrive -- so the MMA thread waits once and commits once per step (a commit plus several waits
+// per step cost the tensor pipe up to a third of its rate).
+//   warps 7-14  dequant: two groups of 4 warps taking alternate steps; each thread decodes one
+//               64-element item of its CTA's weight half per step into the swizzled operand tile;
+//               its block scale is loaded from global memory two of its own steps ahead
+// Barriers that only the pair's tensor core (commit) or local threads complete are waited on with
+// CTA-scope acquire; the two that threads of the other CTA arrive on (the leader's stage-full and
+// accumulator-empty barriers) are waited on with cluster-scope acquire.
 // The weight tile is K-major for the forward pass (rows of W are rows of the operand) and
 // MN-major for dX (rows of W run along the contraction); in both cases a 64-element item is one
 // 128-byte swizzled row, so the decode stage is the same code.
@@ -25,18 +46,19 @@
 
 namespace qlora {
 namespace fused {
-constexpr int BM = 256, BN = 128, BK = 64;
-constexpr int NX = 4, NW = 4, NC = 6;
-constexpr int X_BYTES = BM * BK * 2;   // 32 KB: two 128-row boxes
-constexpr int W_BYTES = BN * BK * 2;   // 16 KB
-constexpr int C_BYTES = BN * BK / 2;   // 4 KB of packed codes
-constexpr int kEpiWarps = 4, kTmaWarp = 4, kMmaWarp = 5, kDqWarp0 = 6, kDqWarps = 8;
+constexpr int BM = 256, BN = 256;      // pair tile
+constexpr int HM = 128, HN = 128;      // per-CTA halves
+constexpr int BK = 64;
+constexpr int NS = 6, NC = 8;         // operand stages (activation + weight halves), code stages
+constexpr int X_BYTES = HM * BK * 2;   // 16 KB
+constexpr int W_BYTES = HN * BK * 2;   // 16 KB
+constexpr int C_BYTES = HN * BK / 2;   // 4 KB of packed codes
+constexpr int kEpiWarps = 4, kTmaWarp = 4, kMmaWarp = 5, kCodeWarp = 6, kDqWarp0 = 7, kDqWarps = 8;
 constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;
-constexpr int kTmemCols = 512;         // 2 buffers x 2 halves x 128 columns
+constexpr int kTmemCols = 512;         // 2 buffers x 256 columns
 constexpr int GM = 8;                  // m-tiles per raster group
-constexpr int kNumBars = 2 * NX + 2 * NW + 2 * NC + 4;
-constexpr size_t kSmemBytes = 1024 + size_t(NX) * X_BYTES + size_t(NW) * W_BYTES +
-                              size_t(NC) * C_BYTES + 1024;
+constexpr int kNumBars = 2 * NS + 2 * NC + 4;
+constexpr size_t kSmemBytes = 1024 + size_t(NS) * (X_BYTES + W_BYTES) + size_t(NC) * C_BYTES + 1024;
 }  // namespace fused
 
 struct FusedParams {
@@ -49,7 +71,7 @@ struct FusedParams {
   __nv_bfloat16* out;                // fwd: Y [M, N]; dX: dX [M, K]
   int* status;
   int M, N, K, r;
-  int num_m, num_n, num_k;           // tiles over rows, over output columns; contraction steps
+  int num_m, num_n, num_k;           // pair tiles over rows, over output columns; contraction steps
 };
 
 __device__ __forceinline__ void fused_tile_coords(int t, int num_m, int num_n, int& mt, int& nt) {
@@ -76,10 +98,11 @@ __device__ __forceinline__ ItemScale load_item_scale(const void* scales, int n, 
   return s;
 }
 
-// Shared-memory geometry of one dequant item (thread tg = 0..127 of a dequant group).
-//   forward: item = weight row (c0 + tg), columns [ks*64, ks*64+64): operand row tg of the
+// Shared-memory geometry of one dequant item (thread tg = 0..127 of a dequant group) in a CTA's
+// 128-column weight half whose first weight row (forward) or column (dX) is h0:
+//   forward: item = weight row (h0 + tg), columns [ks*64, ks*64+64): operand row tg of the
 //            K-major tile; code bytes: row tg of a 128 x 32-byte SW32 tile.
-//   dX     : item = weight row (ks*64 + tg%64), columns [c0 + 64*(tg/64), +64): row tg%64 of
+//   dX     : item = weight row (ks*64 + tg%64), columns [h0 + 64*(tg/64), +64): row tg%64 of
 //            operand block tg/64 of the MN-major tile; code bytes: row tg%64, bytes
 //            32*(tg/64).. of a 64 x 64-byte SW64 tile.
 template <bool DX>
@@ -105,49 +128,54 @@ struct ItemGeom {
 };
 
 template <int FMT, bool DX>
-__global__ void __launch_bounds__(fused::kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fused::kThreads, 1)
 qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
   using namespace fused;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* xs = smem;
-  uint8_t* wsm = xs + NX * X_BYTES;
-  uint8_t* cs = wsm + NW * W_BYTES;
+  uint8_t* xs = smem;                      // NS activation halves
+  uint8_t* wsm = xs + NS * X_BYTES;        // NS weight halves
+  uint8_t* cs = wsm + NS * W_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(cs + NC * C_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t b0 = ptx::smem_u32(bars);
-  auto full_x = [&](uint32_t s) { return b0 + 8u * s; };
-  auto empty_x = [&](uint32_t s) { return b0 + 8u * (NX + s); };
-  auto full_w = [&](uint32_t s) { return b0 + 8u * (2 * NX + s); };
-  auto empty_w = [&](uint32_t s) { return b0 + 8u * (2 * NX + NW + s); };
-  auto full_c = [&](uint32_t s) { return b0 + 8u * (2 * NX + 2 * NW + s); };
-  auto empty_c = [&](uint32_t s) { return b0 + 8u * (2 * NX + 2 * NW + NC + s); };
-  auto acc_full = [&](uint32_t b) { return b0 + 8u * (2 * NX + 2 * NW + 2 * NC + b); };
-  auto acc_empty = [&](uint32_t b) { return b0 + 8u * (2 * NX + 2 * NW + 2 * NC + 2 + b); };
+  auto full_s = [&](uint32_t s) { return b0 + 8u * s; };
+  auto empty_s = [&](uint32_t s) { return b0 + 8u * (NS + s); };
+  auto full_c = [&](uint32_t s) { return b0 + 8u * (2 * NS + s); };
+  auto empty_c = [&](uint32_t s) { return b0 + 8u * (2 * NS + NC + s); };
+  auto acc_full = [&](uint32_t b) { return b0 + 8u * (2 * NS + 2 * NC + b); };
+  auto acc_empty = [&](uint32_t b) { return b0 + 8u * (2 * NS + 2 * NC + 2 + b); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const int pair = int(blockIdx.x >> 1), npairs = int(gridDim.x >> 1);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NX; ++s) { ptx::mbar_init(full_x(s), 1); ptx::mbar_init(empty_x(s), 1); }
-    for (int s = 0; s < NW; ++s) { ptx::mbar_init(full_w(s), kDqWarps / 2); ptx::mbar_init(empty_w(s), 1); }
+    // stage full: leader = producer's expect-tx arrive + 4 dequant warps + 1 relayed arrive;
+    // other CTA = its 4 dequant warps (waited on by its relay).  acc_empty is used in the leader.
+    for (int s = 0; s < NS; ++s) {
+      ptx::mbar_init(full_s(s), rank == 0 ? 2 + kDqWarps / 2 : kDqWarps / 2);
+      ptx::mbar_init(empty_s(s), 1);
+    }
     for (int s = 0; s < NC; ++s) { ptx::mbar_init(full_c(s), 1); ptx::mbar_init(empty_c(s), kDqWarps / 2); }
-    for (int b = 0; b < 2; ++b) { ptx::mbar_init(acc_full(b), 1); ptx::mbar_init(acc_empty(b), kEpiWarps); }
+    for (int b = 0; b < 2; ++b) { ptx::mbar_init(acc_full(b), 1); ptx::mbar_init(acc_empty(b), 2 * kEpiWarps); }
     *abort_flag = 0;
     ptx::fence_mbarrier_init();
   }
   if (warp == kTmaWarp && lane == 0) {
     ptx::prefetch_tmap(&p.tm_act);
-    ptx::prefetch_tmap(&p.tm_codes);
     ptx::prefetch_tmap(&p.tm_zs);
   }
+  if (warp == kCodeWarp && lane == 0) ptx::prefetch_tmap(&p.tm_codes);
   if (warp == kMmaWarp) {
-    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
-    ptx::tmem_relinquish();
+    ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), kTmemCols);
+    ptx::tmem_relinquish_pair();
   }
   ptx::tc_fence_before();
   __syncthreads();
+  ptx::cluster_sync();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -155,72 +183,88 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
   const int nk = p.num_k;
 
   if (warp == kTmaWarp) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ activation producer
     if (lane == 0) {
-      uint32_t i = 0, j = 0;
-      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      uint32_t i = 0;
+      for (int t = pair; t < num_tiles; t += npairs) {
         int mt, nt;
         fused_tile_coords(t, p.num_m, p.num_n, mt, nt);
-        const int m0 = mt * BM, c0 = nt * BN;
-        for (int ks = 0; ks <= nk; ++ks, ++i) {
-          const uint32_t sx = i % NX, px = (i / NX) & 1u;
-          if (!ptx::mbar_wait(empty_x(sx), px ^ 1u, p.status, abort_flag)) goto producer_done;
-          ptx::mbar_arrive_expect_tx(full_x(sx), X_BYTES);
-          const uint32_t xd = ptx::smem_u32(xs + sx * X_BYTES);
-          if (ks < nk) {
-            ptx::tma_load_2d(xd, &p.tm_act, full_x(sx), ks * BK, m0);
-            ptx::tma_load_2d(xd + X_BYTES / 2, &p.tm_act, full_x(sx), ks * BK, m0 + 128);
-          } else {
-            ptx::tma_load_2d(xd, &p.tm_zs, full_x(sx), 0, m0);
-            ptx::tma_load_2d(xd + X_BYTES / 2, &p.tm_zs, full_x(sx), 0, m0 + 128);
-          }
-          if (ks < nk) {
-            const uint32_t sc = j % NC, pc = (j / NC) & 1u;
-            if (!ptx::mbar_wait(empty_c(sc), pc ^ 1u, p.status, abort_flag)) goto producer_done;
-            ptx::mbar_arrive_expect_tx(full_c(sc), C_BYTES);
-            const uint32_t cd = ptx::smem_u32(cs + sc * C_BYTES);
-            if (!DX) ptx::tma_load_2d(cd, &p.tm_codes, full_c(sc), ks * (BK / 2), c0);
-            else ptx::tma_load_2d(cd, &p.tm_codes, full_c(sc), c0 / 2, ks * BK);
-            ++j;
-          }
-        }
-      }
-    producer_done:;
-    }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = ptx::idesc_bf16(128, BN, 0, DX ? 1u : 0u);
-      const int lora_kk = (p.r + 15) / 16;
-      uint32_t i = 0, tc = 0;
-      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tc) {
-        const uint32_t buf = tc & 1u;
-        if (!ptx::mbar_wait(acc_empty(buf), ((tc >> 1) & 1u) ^ 1u, p.status, abort_flag)) break;
-        ptx::tc_fence_after();
-        const uint32_t d0 = tmem + buf * 2u * BN, d1 = d0 + BN;
+        const int m0 = mt * BM + int(rank) * HM;      // this CTA's activation rows
         bool ok = true;
         for (int ks = 0; ks <= nk; ++ks, ++i) {
-          const uint32_t sx = i % NX, sw = i % NW;
-          if (!ptx::mbar_wait(full_x(sx), (i / NX) & 1u, p.status, abort_flag) ||
-              !ptx::mbar_wait(full_w(sw), (i / NW) & 1u, p.status, abort_flag)) { ok = false; break; }
-          ptx::tc_fence_after();
-          const uint32_t xa = ptx::smem_u32(xs + sx * X_BYTES);
-          const uint32_t wb = ptx::smem_u32(wsm + sw * W_BYTES);
-          const int nkk = ks < nk ? BK / 16 : lora_kk;
-          for (int kk = 0; kk < nkk; ++kk) {
-            const uint64_t a0 = ptx::smem_desc(xa + kk * 32, 16, 1024, ptx::kSw128);
-            const uint64_t a1 = ptx::smem_desc(xa + X_BYTES / 2 + kk * 32, 16, 1024, ptx::kSw128);
-            const uint64_t bd = DX ? ptx::smem_desc(wb + kk * 2048, 8192, 1024, ptx::kSw128)
-                                   : ptx::smem_desc(wb + kk * 32, 16, 1024, ptx::kSw128);
-            const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
-            ptx::mma_bf16(d0, a0, bd, idesc, acc);
-            ptx::mma_bf16(d1, a1, bd, idesc, acc);
-          }
-          ptx::mma_commit(empty_x(sx));
-          ptx::mma_commit(empty_w(sw));
+          const uint32_t sx = i % NS, px = (i / NS) & 1u;
+          if (!ptx::mbar_wait(empty_s(sx), px ^ 1u, p.status, abort_flag)) { ok = false; break; }
+          if (rank == 0) ptx::mbar_arrive_expect_tx(full_s(sx), 2 * X_BYTES);
+          const uint32_t xd = ptx::smem_u32(xs + sx * X_BYTES);
+          const uint32_t fx = ptx::mapa(full_s(sx), 0);
+          if (ks < nk) ptx::tma_load_2d_pair(xd, &p.tm_act, fx, ks * BK, m0);
+          else ptx::tma_load_2d_pair(xd, &p.tm_zs, fx, 0, m0);
         }
         if (!ok) break;
-        ptx::mma_commit(acc_full(buf));
+      }
+    }
+  } else if (warp == kCodeWarp) {
+    // ------------------------------------------------------------------ code producer
+    if (lane == 0) {
+      uint32_t j = 0;
+      for (int t = pair; t < num_tiles; t += npairs) {
+        int mt, nt;
+        fused_tile_coords(t, p.num_m, p.num_n, mt, nt);
+        const int h0 = nt * BN + int(rank) * HN;      // this CTA's weight half
+        bool ok = true;
+        for (int ks = 0; ks < nk; ++ks, ++j) {
+          const uint32_t sc = j % NC, pc = (j / NC) & 1u;
+          if (!ptx::mbar_wait(empty_c(sc), pc ^ 1u, p.status, abort_flag)) { ok = false; break; }
+          ptx::mbar_arrive_expect_tx(full_c(sc), C_BYTES);
+          const uint32_t cd = ptx::smem_u32(cs + sc * C_BYTES);
+          if (!DX) ptx::tma_load_2d(cd, &p.tm_codes, full_c(sc), ks * (BK / 2), h0);
+          else ptx::tma_load_2d(cd, &p.tm_codes, full_c(sc), h0 / 2, ks * BK);
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = ptx::idesc_bf16(256, BN, 0, DX ? 1u : 0u);
+      const int lora_kk = (p.r + 15) / 16;
+      uint32_t i = 0, tc = 0;
+      for (int t = pair; t < num_tiles; t += npairs, ++tc) {
+        const uint32_t buf = tc & 1u;
+        if (!ptx::mbar_wait_cluster(acc_empty(buf), ((tc >> 1) & 1u) ^ 1u, p.status, abort_flag)) break;
+        ptx::tc_fence_after();
+        const uint32_t d = tmem + buf * BN;
+        bool ok = true;
+        for (int ks = 0; ks <= nk; ++ks, ++i) {
+          const uint32_t st = i % NS;
+          if (!ptx::mbar_wait_cluster(full_s(st), (i / NS) & 1u, p.status, abort_flag)) { ok = false; break; }
+          ptx::tc_fence_after();
+          const uint32_t xa = ptx::smem_u32(xs + st * X_BYTES);
+          const uint32_t wb = ptx::smem_u32(wsm + st * W_BYTES);
+          const int nkk = ks < nk ? BK / 16 : lora_kk;
+          for (int kk = 0; kk < nkk; ++kk) {
+            const uint64_t ad = ptx::smem_desc(xa + kk * 32, 16, 1024, ptx::kSw128);
+            const uint64_t bd = DX ? ptx::smem_desc(wb + kk * 2048, 8192, 1024, ptx::kSw128)
+                                   : ptx::smem_desc(wb + kk * 32, 16, 1024, ptx::kSw128);
+            ptx::mma_bf16_pair(d, ad, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+          }
+          ptx::mma_commit_pair(empty_s(st), 3);
+        }
+        if (!ok) break;
+        ptx::mma_commit_pair(acc_full(buf), 3);
+      }
+    } else if (lane == 0) {
+      // relay (other CTA): this CTA's weight half of step i is complete -> tell the leader
+      const uint32_t full_leader0 = ptx::mapa(full_s(0), 0);
+      uint32_t i = 0;
+      for (int t = pair; t < num_tiles; t += npairs) {
+        bool ok = true;
+        for (int ks = 0; ks <= nk; ++ks, ++i) {
+          const uint32_t st = i % NS;
+          if (!ptx::mbar_wait(full_s(st), (i / NS) & 1u, p.status, abort_flag)) { ok = false; break; }
+          ptx::mbar_arrive_remote(full_leader0 + 8u * st);
+        }
+        if (!ok) break;
       }
     }
   } else if (warp < kEpiWarps) {
@@ -228,42 +272,40 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     const int q = warp;  // tensor-memory lanes 32q .. 32q+31
     const float ts = (FMT == kFmtNVFP4 && p.tensor_scale) ? __ldg(p.tensor_scale) : 1.0f;
     const int ncols = DX ? p.K : p.N;
+    const uint32_t acc_empty_leader0 = ptx::mapa(acc_empty(0), 0);
     uint32_t tc = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tc) {
+    for (int t = pair; t < num_tiles; t += npairs, ++tc) {
       int mt, nt;
       fused_tile_coords(t, p.num_m, p.num_n, mt, nt);
-      const int m0 = mt * BM, c0 = nt * BN;
+      const int row = mt * BM + int(rank) * HM + q * 32 + lane;
+      const int c0 = nt * BN;
       const uint32_t buf = tc & 1u;
       if (!ptx::mbar_wait(acc_full(buf), (tc >> 1) & 1u, p.status, abort_flag)) break;
       ptx::tc_fence_after();
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const int row = m0 + h * 128 + q * 32 + lane;
-#pragma unroll 1
-        for (int cb = 0; cb < BN / 32; ++cb) {
-          uint32_t v[32];
-          ptx::tmem_ld_32x32b_x32(tmem + (uint32_t(q * 32) << 16) + (buf * 2u + h) * BN + cb * 32, v);
-          ptx::tmem_ld_wait();
-          if (row < p.M) {
-            __nv_bfloat16* orow = p.out + size_t(row) * ncols;
+      for (int cb = 0; cb < BN / 32; ++cb) {
+        uint32_t v[32];
+        ptx::tmem_ld_32x32b_x32(tmem + (uint32_t(q * 32) << 16) + buf * BN + cb * 32, v);
+        ptx::tmem_ld_wait();
+        if (row < p.M) {
+          __nv_bfloat16* orow = p.out + size_t(row) * ncols;
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const int col = c0 + cb * 32 + g * 8;
-              if (col < ncols) {
-                uint4 o;
-                o.x = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 0]) * ts, __uint_as_float(v[g * 8 + 1]) * ts);
-                o.y = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 2]) * ts, __uint_as_float(v[g * 8 + 3]) * ts);
-                o.z = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 4]) * ts, __uint_as_float(v[g * 8 + 5]) * ts);
-                o.w = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 6]) * ts, __uint_as_float(v[g * 8 + 7]) * ts);
-                *reinterpret_cast<uint4*>(orow + col) = o;
-              }
+          for (int g = 0; g < 4; ++g) {
+            const int col = c0 + cb * 32 + g * 8;
+            if (col < ncols) {
+              uint4 o;
+              o.x = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 0]) * ts, __uint_as_float(v[g * 8 + 1]) * ts);
+              o.y = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 2]) * ts, __uint_as_float(v[g * 8 + 3]) * ts);
+              o.z = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 4]) * ts, __uint_as_float(v[g * 8 + 5]) * ts);
+              o.w = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 6]) * ts, __uint_as_float(v[g * 8 + 7]) * ts);
+              *reinterpret_cast<uint4*>(orow + col) = o;
             }
           }
         }
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(acc_empty(buf));
+      if (lane == 0) ptx::mbar_arrive_remote(acc_empty_leader0 + 8u * buf);
     }
   } else {
     // ------------------------------------------------------------------ dequant
@@ -271,70 +313,103 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     const int grp = dw >> 2;
     const int tg = (dw & 3) * 32 + lane;
     const ItemGeom<DX> geo(tg);
-    uint32_t i = 0, j = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+    // Cursor over this group's steps (every other step of the CTA's pipeline): tile t (the lt-th
+    // of this pair), step ks of the tile (ks == nk is the LoRA step), weight-half origin h0.
+    struct Cursor {
+      int t, lt, ks, h0;
+    };
+    auto tile_h0 = [&](int t) {
       int mt, nt;
       fused_tile_coords(t, p.num_m, p.num_n, mt, nt);
-      const int c0 = nt * BN;
-      for (int ks = 0; ks <= nk; ++ks, ++i) {
-        const bool real = ks < nk;
-        if (int(i & 1u) == grp) {
-          const uint32_t sw = i % NW, pw = (i / NW) & 1u;
-          const uint32_t rb = geo.op_row_base(ptx::smem_u32(wsm + sw * W_BYTES));
-          if (real) {
-            const int n = DX ? ks * BK + geo.row : c0 + geo.row;
-            const int kcol = DX ? c0 + geo.chunk * 64 : ks * BK;
-            const bool valid = n < p.N && kcol < p.K;
-            ItemScale sc{0u};
-            if (valid) sc = load_item_scale<FMT>(p.scales, n, kcol, p.K);
-            const uint32_t scs = j % NC;
-            if (!ptx::mbar_wait(full_c(scs), (j / NC) & 1u, p.status, abort_flag)) { ok = false; break; }
-            const uint32_t cb = ptx::smem_u32(cs + scs * C_BYTES);
-            const uint4 c_lo = ptx::ld_shared_v4(cb + geo.code_off(0));
-            const uint4 c_hi = ptx::ld_shared_v4(cb + geo.code_off(1));
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(empty_c(scs));
-            const uint32_t cw[8] = {c_lo.x, c_lo.y, c_lo.z, c_lo.w, c_hi.x, c_hi.y, c_hi.z, c_hi.w};
-            if (!ptx::mbar_wait(empty_w(sw), pw ^ 1u, p.status, abort_flag)) { ok = false; break; }
-            if (valid) dequant_item_store<FMT>(cw, sc, rb, geo.swz());
-            else zero_item_store(rb);
-          } else {
-            // LoRA step: rows of B (forward, K-major) or of A (dX, MN-major), zero padded.
-            uint4 v[8];
-            if (!DX) {
-              const int n = c0 + geo.row;
-#pragma unroll
-              for (int jj = 0; jj < 8; ++jj)
-                v[jj] = (n < p.N && jj * 8 < p.r)
-                            ? __ldg(reinterpret_cast<const uint4*>(p.lora_up + size_t(n) * p.r + jj * 8))
-                            : make_uint4(0, 0, 0, 0);
-            } else {
-              const int rj = geo.row, kc = c0 + geo.chunk * 64;
-#pragma unroll
-              for (int jj = 0; jj < 8; ++jj)
-                v[jj] = (rj < p.r && kc < p.K)
-                            ? __ldg(reinterpret_cast<const uint4*>(p.lora_up + size_t(rj) * p.K + kc + jj * 8))
-                            : make_uint4(0, 0, 0, 0);
-            }
-            if (!ptx::mbar_wait(empty_w(sw), pw ^ 1u, p.status, abort_flag)) { ok = false; break; }
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-              ptx::st_shared_v4(rb + ((uint32_t(jj) ^ geo.swz()) << 4), v[jj].x, v[jj].y, v[jj].z, v[jj].w);
-          }
-          ptx::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(full_w(sw));
-        }
-        if (real) ++j;
+      return nt * BN + int(rank) * HN;
+    };
+    auto advance2 = [&](Cursor& c) {
+      c.ks += 2;
+      if (c.ks > nk) {
+        c.ks -= nk + 1;
+        c.t += npairs;
+        ++c.lt;
+        if (c.t < num_tiles) c.h0 = tile_h0(c.t);
       }
+    };
+    auto scale_for = [&](const Cursor& c) {
+      ItemScale sc{0u};
+      if (c.t < num_tiles && c.ks < nk) {
+        const int n = DX ? c.ks * BK + geo.row : c.h0 + geo.row;
+        const int kcol = DX ? c.h0 + geo.chunk * 64 : c.ks * BK;
+        if (n < p.N && kcol < p.K) sc = load_item_scale<FMT>(p.scales, n, kcol, p.K);
+      }
+      return sc;
+    };
+    Cursor cur{pair, 0, grp, pair < num_tiles ? tile_h0(pair) : 0};
+    Cursor pf = cur;
+    advance2(pf);
+    ItemScale s_cur = scale_for(cur), s_next = scale_for(pf);
+    advance2(pf);
+    while (cur.t < num_tiles) {
+      const ItemScale s_pref = scale_for(pf);   // two own steps ahead
+      advance2(pf);
+      const uint32_t i = uint32_t(cur.lt * (nk + 1) + cur.ks);     // pipeline step
+      const uint32_t sw = i % NS, pw = (i / NS) & 1u;
+      const uint32_t rb = geo.op_row_base(ptx::smem_u32(wsm + sw * W_BYTES));
+      if (cur.ks < nk) {
+        const int n = DX ? cur.ks * BK + geo.row : cur.h0 + geo.row;
+        const int kcol = DX ? cur.h0 + geo.chunk * 64 : cur.ks * BK;
+        const bool valid = n < p.N && kcol < p.K;
+        const uint32_t j = uint32_t(cur.lt * nk + cur.ks);          // code step
+        const uint32_t scs = j % NC;
+        if (!ptx::mbar_wait(full_c(scs), (j / NC) & 1u, p.status, abort_flag)) break;
+        const uint32_t cb = ptx::smem_u32(cs + scs * C_BYTES);
+        const uint4 c_lo = ptx::ld_shared_v4(cb + geo.code_off(0));
+        const uint4 c_hi = ptx::ld_shared_v4(cb + geo.code_off(1));
+        const uint32_t cw[8] = {c_lo.x, c_lo.y, c_lo.z, c_lo.w, c_hi.x, c_hi.y, c_hi.z, c_hi.w};
+        if (!ptx::mbar_wait(empty_s(sw), pw ^ 1u, p.status, abort_flag)) break;
+        if (valid) dequant_item_store<FMT>(cw, s_cur, rb, geo.swz());
+        else zero_item_store(rb);
+        // release the code stage only once the loaded code words have been consumed: the
+        // producer's next TMA into this stage must not overtake the loads above
+        const uint32_t used = (c_lo.x ^ c_lo.y ^ c_lo.z ^ c_lo.w) ^ (c_hi.x ^ c_hi.y ^ c_hi.z ^ c_hi.w);
+        uint32_t dep;
+        asm volatile("and.b32 %0, %1, 0;" : "=r"(dep) : "r"(used));
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(empty_c(scs) + dep);
+      } else {
+        // LoRA step: rows of B (forward, K-major) or of A (dX, MN-major), zero padded.
+        uint4 v[8];
+        if (!DX) {
+          const int n = cur.h0 + geo.row;
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj)
+            v[jj] = (n < p.N && jj * 8 < p.r)
+                        ? __ldg(reinterpret_cast<const uint4*>(p.lora_up + size_t(n) * p.r + jj * 8))
+                        : make_uint4(0, 0, 0, 0);
+        } else {
+          const int rj = geo.row, kc = cur.h0 + geo.chunk * 64;
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj)
+            v[jj] = (rj < p.r && kc < p.K)
+                        ? __ldg(reinterpret_cast<const uint4*>(p.lora_up + size_t(rj) * p.K + kc + jj * 8))
+                        : make_uint4(0, 0, 0, 0);
+        }
+        if (!ptx::mbar_wait(empty_s(sw), pw ^ 1u, p.status, abort_flag)) break;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+          ptx::st_shared_v4(rb + ((uint32_t(jj) ^ geo.swz()) << 4), v[jj].x, v[jj].y, v[jj].z, v[jj].w);
+      }
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(full_s(sw));
+      s_cur = s_next;
+      s_next = s_pref;
+      advance2(cur);
     }
   }
 
   ptx::tc_fence_before();
   __syncthreads();
+  ptx::cluster_sync();
   ptx::tc_fence_after();
-  if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) ptx::tmem_dealloc_pair(tmem, kTmemCols);
 }
 
 }  // namespace qlora
