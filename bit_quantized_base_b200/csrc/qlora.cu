@@ -118,7 +118,7 @@ WgradPlan wgrad_plan(int64_t N, int64_t K, int64_t M, int sms) {
   p.tiles1 = int((K + 127) / 128);
   p.total_steps = int((M + 63) / 64);
   const int tiles = p.tiles0 + p.tiles1;
-  int S = (2 * sms + tiles - 1) / tiles;
+  int S = (sms + tiles - 1) / tiles;                         // about one wave of long splits
   S = S < 1 ? 1 : (S > 16 ? 16 : S);
   if (S > p.total_steps) S = p.total_steps > 0 ? p.total_steps : 1;
   p.sps = (p.total_steps + S - 1) / S;
@@ -127,8 +127,32 @@ WgradPlan wgrad_plan(int64_t N, int64_t K, int64_t M, int sms) {
   return p;
 }
 
+// Split plan of the lora_down kernel: 128-row tiles, the contraction (Kc) split into S ranges of
+// whole 64-deep steps, at least 2 steps per split.
+struct DownPlan {
+  int tiles, S, sps, num_k;
+};
+
+DownPlan down_plan(int64_t M, int64_t Kc, int sms) {
+  DownPlan p{};
+  p.tiles = int((M + 127) / 128);
+  p.num_k = int((Kc + 63) / 64);
+  int S = p.tiles > 0 ? (sms + p.tiles - 1) / p.tiles : 1;   // about one wave of long splits
+  S = S < 1 ? 1 : (S > 16 ? 16 : S);
+  const int max_s = p.num_k / 2 > 0 ? p.num_k / 2 : 1;
+  if (S > max_s) S = max_s;
+  p.sps = (p.num_k + S - 1) / S;
+  p.S = (p.num_k + p.sps - 1) / p.sps;
+  return p;
+}
+
+size_t down_partial_bytes(int64_t M, int64_t Kc, int r, int sms) {
+  const DownPlan dp = down_plan(M, Kc, sms);
+  return dp.S > 1 ? size_t(dp.S) * size_t(M) * size_t(rank_pad(r)) * 4 : 0;
+}
+
 struct WsLayout {
-  size_t zs, t, u, partial, total;
+  size_t zs, t, u, partial, partial_bytes, total;
 };
 
 WsLayout ws_layout(int64_t N, int64_t K, int64_t M, int r, bool bwd, int sms) {
@@ -139,10 +163,17 @@ WsLayout ws_layout(int64_t N, int64_t K, int64_t M, int r, bool bwd, int sms) {
   L.t = off; off += mr;
   L.u = off; off += bwd ? mr : 0;
   L.partial = off;
+  // fp32 split partials, shared by the (sequential) lora_down and lora_wgrad launches
+  size_t pb = down_partial_bytes(M, K, r, sms);
   if (bwd) {
+    const size_t pu = down_partial_bytes(M, N, r, sms);
+    pb = pu > pb ? pu : pb;
     const WgradPlan wp = wgrad_plan(N, K, M, sms);
-    if (wp.S > 1) off += align_up(size_t(wp.S) * size_t(N + K) * size_t(rank_pad(r)) * 4, 256);
+    const size_t pw = wp.S > 1 ? size_t(wp.S) * size_t(N + K) * size_t(rank_pad(r)) * 4 : 0;
+    pb = pw > pb ? pw : pb;
   }
+  L.partial_bytes = align_up(pb, 256);
+  off += L.partial_bytes;
   L.total = off;
   return L;
 }
@@ -187,11 +218,20 @@ struct LaunchScope {
 };
 
 // ---------------------------------------------------------------------------------- launches
+// partial / partial_bytes: fp32 scratch for the split contraction (the split count is reduced
+// until its partials fit); counters: one zeroed int per 128-row tile.
 qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t Kc, const void* R,
                                 int64_t R_rows, int r, float s, const float* ts, void* z, void* zs,
-                                int* status, cudaStream_t st) {
+                                int* status, float* partial, size_t partial_bytes, int* counters,
+                                cudaStream_t st) {
   DownParams p{};
   const int rpad = rank_pad(r);
+  DownPlan dp = down_plan(M, Kc, num_sms());
+  while (dp.S > 1 && size_t(dp.S) * size_t(M) * size_t(rpad) * 4 > partial_bytes) {
+    dp.sps = (dp.num_k + dp.S - 2) / (dp.S - 1);
+    dp.S = (dp.num_k + dp.sps - 1) / dp.sps;
+  }
+  if (dp.tiles > kMaxCounters) return QLORA_ERR_UNSUPPORTED;
   if (!tmap_2d(&p.tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, uint64_t(Kc), uint64_t(M),
                uint64_t(Kc) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
@@ -208,12 +248,16 @@ qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t K
   p.z = static_cast<__nv_bfloat16*>(z);
   p.zs = static_cast<__nv_bfloat16*>(zs);
   p.status = status;
+  p.partial = partial;
+  p.counters = counters;
   p.M = int(M);
   p.r = r;
   p.rpad = rpad;
-  p.num_k = int((Kc + 63) / 64);
+  p.num_k = dp.num_k;
+  p.S = dp.S;
+  p.steps_per_split = dp.sps;
   p.s = s;
-  const dim3 grid(unsigned((M + 127) / 128));
+  const dim3 grid(unsigned(dp.tiles * dp.S));
   LaunchScope scope(r_mn ? kKindDownU : kKindDownT, st);
   if (r_mn) {
     if (!set_smem(qlora_lora_down_kernel<true>, lora::kSmemBytes)) return QLORA_ERR_CUDA;
@@ -382,7 +426,8 @@ qlora_status_t qlora_linear_fwd(const qlora_weight_t* W, const void* X, const vo
   void* T = T_save ? T_save : w + L.t;
   void* Zs = w + L.zs;
   const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
-  st = launch_lora_down(false, X, M, W->K, A, r, r, scale, ts, T, Zs, ws_status(ws), s);
+  st = launch_lora_down(false, X, M, W->K, A, r, r, scale, ts, T, Zs, ws_status(ws),
+                        reinterpret_cast<float*>(w + L.partial), L.partial_bytes, ws_counters(ws), s);
   if (st != QLORA_OK) return st;
   return launch_fused(W, false, X, Zs, B, Y, M, r, ws_status(ws), s);
 }
@@ -408,7 +453,13 @@ qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const void* X, 
   void* Zs = w + kHeaderBytes;
   void* T = T_save ? T_save : w + kHeaderBytes + mr;
   const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
-  st = launch_lora_down(false, X, M, W->K, A, r, r, scale, ts, T, Zs, status, s);
+  // the rest of the array holds the lora_down split partials (fewer splits if it is short)
+  const size_t used = kHeaderBytes + 256 + mr + (T_save ? 0 : mr);
+  float* part = reinterpret_cast<float*>(w + used);
+  const size_t part_bytes = kNoAllocScratchBytes - used;
+  int* counters = reinterpret_cast<int*>(w + 128);   // 32 tile counters inside the header
+  st = launch_lora_down(false, X, M, W->K, A, r, r, scale, ts, T, Zs, status, part,
+                        (M + 127) / 128 <= 32 ? part_bytes : 0, counters, s);
   if (st != QLORA_OK) return st;
   return launch_fused(W, false, X, Zs, B, Y, M, r, status, s);
 }
@@ -437,12 +488,15 @@ qlora_status_t qlora_linear_bwd(const qlora_weight_t* W, const void* X, const vo
   const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
   void* Zs = w + L.zs;
   void* U = w + L.u;
+  float* part = reinterpret_cast<float*>(w + L.partial);
   if (!T) {  // recompute T = X A^T (its scaled copy lands in Zs and is overwritten below)
-    st = launch_lora_down(false, X, M, W->K, A, r, r, scale, ts, w + L.t, Zs, ws_status(ws), s);
+    st = launch_lora_down(false, X, M, W->K, A, r, r, scale, ts, w + L.t, Zs, ws_status(ws), part,
+                          L.partial_bytes, ws_counters(ws), s);
     if (st != QLORA_OK) return st;
     T = w + L.t;
   }
-  st = launch_lora_down(true, dY, M, W->N, B, W->N, r, scale, ts, U, Zs, ws_status(ws), s);
+  st = launch_lora_down(true, dY, M, W->N, B, W->N, r, scale, ts, U, Zs, ws_status(ws), part,
+                        L.partial_bytes, ws_counters(ws), s);
   if (st != QLORA_OK) return st;
   if (dX) {
     st = launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), s);

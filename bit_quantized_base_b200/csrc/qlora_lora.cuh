@@ -1,6 +1,6 @@
 // qlora_lora.cuh -- the rank-r side path of the layer on tcgen05.
 //
-// lora_down: Z[M, r] = Act[M, Kc] . R, one 128-row tile per CTA.
+// lora_down: Z[M, r] = Act[M, Kc] . R, 128-row tiles, the contraction split over S CTAs per tile.
 //   forward : Z = T = X A^T   (R = A^T: A [r, K] is a K-major operand)
 //   backward: Z = U = dY B    (R = B:   B [N, r] is an MN-major operand)
 //   It writes Z (bf16) and Zs = bf16(Z * s / ts), the operand of the fused GEMM's LoRA step.
@@ -12,10 +12,12 @@
 //   ("Training LLMs on a Budget", §2 "Initialization matters": dL/dB = dL/dy z^T,
 //   dL/dA = (B^T dL/dy) x^T, with the layer's scale s.)  Both are out[P, r] = s . L^T R with L
 //   [M, P] and R [M, r]: an M=128 x N=rpad tcgen05 GEMM per 128-row tile of P whose operands are
-//   both MN-major (M is the contraction).  M is split over S CTAs per tile when there are too few
-//   tiles to fill the GPU; each split stores an fp32 partial, and the last split to finish (an
-//   atomic counter) adds the S partials in split order 0..S-1 and writes bf16, so the result is
-//   bitwise deterministic.
+//   both MN-major (M is the contraction), M split over S CTAs per tile.
+//
+// Both kernels are memory bound (they stream an activation once) and have few output tiles, so
+// the contraction is split to fill the GPU.  Each split stores its fp32 partial tile; the last
+// split to finish (an atomic counter per tile, reset by that CTA for the next call) adds the S
+// partials in split order 0..S-1, so the result is bitwise deterministic.
 #pragma once
 #include <cuda_bf16.h>
 #include "qlora_ptx.cuh"
@@ -34,14 +36,78 @@ __device__ __forceinline__ uint32_t swz_mode_for_row_bytes(uint32_t rowb) {
   return rowb == 128 ? ptx::kSw128 : (rowb == 64 ? ptx::kSw64 : ptx::kSw32);
 }
 
+// Epilogue of a split tile, run by the 128 epilogue threads (named barrier 1).  acc holds this
+// thread's accumulator row (rpad fp32 values).  With S > 1 the row is stored as partial `split`
+// at partial + (split * rows_total + row) * rpad; the last CTA of the tile (counter) then replaces
+// acc with the sum over splits 0..S-1 and returns true; other CTAs return false.  With S == 1 it
+// returns true with acc unchanged.  All 128 threads must call it (rows outside the problem pass
+// row_ok = false and take part in the barriers only).
+__device__ __forceinline__ bool split_reduce(float (&acc)[64], int rpad, int S, int split,
+                                            float* partial, size_t rows_total, int row, bool row_ok,
+                                            int* counter, volatile int* last_flag, int et) {
+  if (S == 1) return true;
+  if (row_ok) {
+    float* dst = partial + (size_t(split) * rows_total + size_t(row)) * rpad;
+#pragma unroll
+    for (int c = 0; c < 64; c += 4)
+      if (c < rpad) __stcg(reinterpret_cast<float4*>(dst + c), make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
+  }
+  __threadfence();
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (et == 0) {
+    const int old = atomicAdd(counter, 1);
+    *last_flag = (old == S - 1) ? 1 : 0;
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (!*last_flag) return false;
+  __threadfence();
+  if (row_ok) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
+    for (int sp = 0; sp < S; ++sp) {
+      const float* src = partial + (size_t(sp) * rows_total + size_t(row)) * rpad;
+      float4 v[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        if (4 * c < rpad) v[c] = __ldcg(reinterpret_cast<const float4*>(src + 4 * c));
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        if (4 * c < rpad) {
+          acc[4 * c] += v[c].x; acc[4 * c + 1] += v[c].y; acc[4 * c + 2] += v[c].z; acc[4 * c + 3] += v[c].w;
+        }
+    }
+  }
+  if (et == 0) *counter = 0;   // ready for the next call on this workspace
+  return true;
+}
+
+// Load this thread's accumulator row (rpad columns) from tensor memory.
+__device__ __forceinline__ void load_acc_row(uint32_t taddr, int rpad, float (&acc)[64]) {
+#pragma unroll
+  for (int c = 0; c < 64; c += 16) {
+    if (c < rpad) {
+      uint32_t v[16];
+      ptx::tmem_ld_32x32b_x16(taddr + c, v);
+      ptx::tmem_ld_wait();
+#pragma unroll
+      for (int g = 0; g < 16; ++g) acc[c + g] = __uint_as_float(v[g]);
+    } else {
+#pragma unroll
+      for (int g = 0; g < 16; ++g) acc[c + g] = 0.0f;
+    }
+  }
+}
+
 struct DownParams {
   CUtensorMap tm_act;  // X [M, K] or dY [M, N] bf16, box {64, 128}, SW128
   CUtensorMap tm_r;    // T: A [r, K] box {64, rpad} SW128; U: B [N, r] box {rpad, 64} SW(2 rpad)
   const float* tensor_scale;
   __nv_bfloat16* z;    // [M, r]
   __nv_bfloat16* zs;   // [M, r]
+  float* partial;      // [S, M, rpad] fp32 (S > 1)
+  int* counters;       // [m tiles]
   int* status;
-  int M, r, rpad, num_k;
+  int M, r, rpad, num_k, S, steps_per_split;
   float s;
 };
 
@@ -57,16 +123,23 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(rs + NS * R_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   const uint32_t b0 = ptx::smem_u32(bars);
   auto full = [&](uint32_t s) { return b0 + 8u * s; };
   auto empty = [&](uint32_t s) { return b0 + 8u * (NS + s); };
   const uint32_t acc_full = b0 + 8u * (2 * NS);
+
+  const int tile = blockIdx.x / p.S, split = blockIdx.x % p.S;
+  const int m0 = tile * BM;
+  const int ks0 = split * p.steps_per_split;
+  const int ks1 = min(ks0 + p.steps_per_split, p.num_k);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) { ptx::mbar_init(full(s), 1); ptx::mbar_init(empty(s), 1); }
     ptx::mbar_init(acc_full, 1);
     *abort_flag = 0;
+    *last_flag = 0;
     ptx::fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -77,14 +150,14 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int m0 = blockIdx.x * BM;
   const uint32_t rowb = uint32_t(p.rpad) * 2u;
   const uint32_t r_bytes = uint32_t(p.rpad) * 128u;
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int ks = 0; ks < p.num_k; ++ks) {
-        const uint32_t s = ks % NS, ph = (ks / NS) & 1;
+      for (int ks = ks0; ks < ks1; ++ks) {
+        const int it = ks - ks0;
+        const uint32_t s = it % NS, ph = (it / NS) & 1;
         if (!ptx::mbar_wait(empty(s), ph ^ 1u, p.status, abort_flag)) break;
         ptx::mbar_arrive_expect_tx(full(s), A_BYTES + r_bytes);
         ptx::tma_load_2d(ptx::smem_u32(as + s * A_BYTES), &p.tm_act, full(s), ks * BK, m0);
@@ -93,11 +166,12 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && ks1 > ks0) {
       const uint32_t idesc = ptx::idesc_bf16(128, uint32_t(p.rpad), 0, R_MN ? 1u : 0u);
       bool ok = true;
-      for (int ks = 0; ks < p.num_k; ++ks) {
-        const uint32_t s = ks % NS, ph = (ks / NS) & 1;
+      for (int ks = ks0; ks < ks1; ++ks) {
+        const int it = ks - ks0;
+        const uint32_t s = it % NS, ph = (it / NS) & 1;
         if (!ptx::mbar_wait(full(s), ph, p.status, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
         const uint32_t a = ptx::smem_u32(as + s * A_BYTES), b = ptx::smem_u32(rs + s * R_BYTES);
@@ -106,7 +180,7 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
           const uint64_t bd = R_MN ? ptx::smem_desc(b + kk * 16 * rowb, 64 * rowb, 8 * rowb,
                                                     swz_mode_for_row_bytes(rowb))
                                    : ptx::smem_desc(b + kk * 32, 16, 1024, ptx::kSw128);
-          ptx::mma_bf16(tmem, ad, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+          ptx::mma_bf16(tmem, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
         }
         ptx::mma_commit(empty(s));
       }
@@ -114,32 +188,36 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
     }
   } else {
     const int q = warp & 3;
+    const int et = threadIdx.x - 64;
     const int row = m0 + q * 32 + lane;
-    if (ptx::mbar_wait(acc_full, 0, p.status, abort_flag)) {
-      ptx::tc_fence_after();
-      const float ts = p.tensor_scale ? __ldg(p.tensor_scale) : 1.0f;
-      const float zscale = p.s / ts;
-#pragma unroll 1
-      for (int c = 0; c < p.rpad; c += 16) {
-        uint32_t v[16];
-        ptx::tmem_ld_32x32b_x16(tmem + (uint32_t(q * 32) << 16) + c, v);
-        ptx::tmem_ld_wait();
-        if (row < p.M) {
+    const bool have = ks1 > ks0;
+    if (have) ptx::mbar_wait(acc_full, 0, p.status, abort_flag);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (*abort_flag == 0) {
+      float acc[64];
+      if (have) {
+        ptx::tc_fence_after();
+        load_acc_row(tmem + (uint32_t(q * 32) << 16), p.rpad, acc);
+      } else {
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            const int col = c + g * 8;
-            if (col < p.r) {
-              uint4 z, zs;
-              const float* f = reinterpret_cast<const float*>(v + g * 8);
-              z.x = ptx::cvt_bf16x2(f[0], f[1]); z.y = ptx::cvt_bf16x2(f[2], f[3]);
-              z.z = ptx::cvt_bf16x2(f[4], f[5]); z.w = ptx::cvt_bf16x2(f[6], f[7]);
-              zs.x = ptx::cvt_bf16x2(f[0] * zscale, f[1] * zscale);
-              zs.y = ptx::cvt_bf16x2(f[2] * zscale, f[3] * zscale);
-              zs.z = ptx::cvt_bf16x2(f[4] * zscale, f[5] * zscale);
-              zs.w = ptx::cvt_bf16x2(f[6] * zscale, f[7] * zscale);
-              *reinterpret_cast<uint4*>(p.z + size_t(row) * p.r + col) = z;
-              *reinterpret_cast<uint4*>(p.zs + size_t(row) * p.r + col) = zs;
-            }
+        for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
+      }
+      if (split_reduce(acc, p.rpad, p.S, split, p.partial, size_t(p.M), row, row < p.M,
+                       p.counters + tile, last_flag, et) && row < p.M) {
+        const float ts = p.tensor_scale ? __ldg(p.tensor_scale) : 1.0f;
+        const float zscale = p.s / ts;
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
+          if (c < p.r) {
+            uint4 z, zs;
+            z.x = ptx::cvt_bf16x2(acc[c], acc[c + 1]); z.y = ptx::cvt_bf16x2(acc[c + 2], acc[c + 3]);
+            z.z = ptx::cvt_bf16x2(acc[c + 4], acc[c + 5]); z.w = ptx::cvt_bf16x2(acc[c + 6], acc[c + 7]);
+            zs.x = ptx::cvt_bf16x2(acc[c] * zscale, acc[c + 1] * zscale);
+            zs.y = ptx::cvt_bf16x2(acc[c + 2] * zscale, acc[c + 3] * zscale);
+            zs.z = ptx::cvt_bf16x2(acc[c + 4] * zscale, acc[c + 5] * zscale);
+            zs.w = ptx::cvt_bf16x2(acc[c + 6] * zscale, acc[c + 7] * zscale);
+            *reinterpret_cast<uint4*>(p.z + size_t(row) * p.r + c) = z;
+            *reinterpret_cast<uint4*>(p.zs + size_t(row) * p.r + c) = zs;
           }
         }
       }
@@ -250,58 +328,34 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
     // every epilogue thread takes the same branch below: a thread whose wait gave up set
     // abort_flag before this barrier
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    const bool ok = *abort_flag == 0;
-    if (ok && have) ptx::tc_fence_after();
-    const int Ptot = p.P0 + p.P1;
-    const int poff = prob ? p.P0 : 0;
-    auto write_out = [&](int j, float v) {
-      const __nv_bfloat16 b = __float2bfloat16_rn(v * p.s);
-      if (prob == 0) p.out0[size_t(prow) * p.r + j] = b;
-      else p.out1[size_t(j) * p.P1 + prow] = b;
-    };
-    if (ok) {
-#pragma unroll 1
-      for (int c = 0; c < p.rpad; c += 16) {
-        uint32_t v[16];
-        if (have) {
-          ptx::tmem_ld_32x32b_x16(tmem + (uint32_t(q * 32) << 16) + c, v);
-          ptx::tmem_ld_wait();
-        } else {
+    if (*abort_flag == 0) {
+      float acc[64];
+      if (have) {
+        ptx::tc_fence_after();
+        load_acc_row(tmem + (uint32_t(q * 32) << 16), p.rpad, acc);
+      } else {
 #pragma unroll
-          for (int g = 0; g < 16; ++g) v[g] = 0u;
-        }
-        if (prow < P) {
-          if (p.S == 1) {
-            for (int g = 0; g < 16 && c + g < p.r; ++g) write_out(c + g, __uint_as_float(v[g]));
-          } else {
-            float* dst = p.partial + (size_t(split) * Ptot + poff + prow) * p.rpad + c;
-#pragma unroll
-            for (int g = 0; g < 16; g += 4)
-              __stcg(reinterpret_cast<float4*>(dst + g),
-                     make_float4(__uint_as_float(v[g]), __uint_as_float(v[g + 1]),
-                                 __uint_as_float(v[g + 2]), __uint_as_float(v[g + 3])));
-          }
-        }
+        for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
       }
-      if (p.S > 1) {
-        __threadfence();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (et == 0) {
-          const int old = atomicAdd(&p.counters[tile], 1);
-          *last_flag = (old == p.S - 1) ? 1 : 0;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (*last_flag) {
-          __threadfence();
-          if (prow < P) {
-            for (int j = 0; j < p.r; ++j) {
-              float acc = 0.0f;
-              for (int sp = 0; sp < p.S; ++sp)
-                acc += __ldcg(p.partial + (size_t(sp) * Ptot + poff + prow) * p.rpad + j);
-              write_out(j, acc);
+      const int poff = prob ? p.P0 : 0;
+      if (split_reduce(acc, p.rpad, p.S, split, p.partial, size_t(p.P0 + p.P1), poff + prow,
+                       prow < P, p.counters + tile, last_flag, et) && prow < P) {
+        if (prob == 0) {
+#pragma unroll
+          for (int c = 0; c < 64; c += 8) {
+            if (c < p.r) {
+              uint4 o;
+              o.x = ptx::cvt_bf16x2(acc[c] * p.s, acc[c + 1] * p.s);
+              o.y = ptx::cvt_bf16x2(acc[c + 2] * p.s, acc[c + 3] * p.s);
+              o.z = ptx::cvt_bf16x2(acc[c + 4] * p.s, acc[c + 5] * p.s);
+              o.w = ptx::cvt_bf16x2(acc[c + 6] * p.s, acc[c + 7] * p.s);
+              *reinterpret_cast<uint4*>(p.out0 + size_t(prow) * p.r + c) = o;
             }
           }
-          if (et == 0) p.counters[tile] = 0;
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c < p.r) p.out1[size_t(c) * p.P1 + prow] = __float2bfloat16_rn(acc[c] * p.s);
         }
       }
     }
