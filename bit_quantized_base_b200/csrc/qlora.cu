@@ -28,8 +28,6 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int rank_pad(int r) { return (r + 15) / 16 * 16; }
 bool rank_ok(int r) { return r == 8 || r == 16 || r == 32 || r == 64; }
 
-int block_size(int fmt) { return fmt == QLORA_FMT_NF4 ? 64 : (fmt == QLORA_FMT_MXFP4 ? 32 : 16); }
-
 int current_device() {
   int d = 0;
   cudaGetDevice(&d);
@@ -106,36 +104,36 @@ qlora_status_t check_weight(const qlora_weight_t* W) {
 bool ptr_ok(const void* p) { return p && aligned16(p); }
 
 // ------------------------------------------------------------------------------- workspace
-// Reduction plan of the dA/dB kernel: tiles of 128 rows of N (dB) and of K (dA), M split into
-// S ranges of whole 64-row steps.
+// E = number of experts (1 for a single layer); M = all rows.
+// Reduction plan of the dA/dB kernel: per expert, tiles of 128 rows of N (dB) and of K (dA); each
+// expert's rows split into S ranges of whole 64-row chunks (the ranges are resolved on the device
+// from the offsets).
 struct WgradPlan {
-  int tiles0, tiles1, S, sps, total_steps;
+  int tiles0, tiles1, S;
 };
 
-WgradPlan wgrad_plan(int64_t N, int64_t K, int64_t M, int sms) {
+WgradPlan wgrad_plan(int64_t N, int64_t K, int64_t M, int E, int sms) {
   WgradPlan p{};
   p.tiles0 = int((N + 127) / 128);
   p.tiles1 = int((K + 127) / 128);
-  p.total_steps = int((M + 63) / 64);
-  const int tiles = p.tiles0 + p.tiles1;
-  int S = (sms + tiles - 1) / tiles;                         // about one wave of long splits
+  const int64_t tiles = int64_t(E) * (p.tiles0 + p.tiles1);
+  int S = int((sms + tiles - 1) / tiles);                    // about one wave of long splits
   S = S < 1 ? 1 : (S > 16 ? 16 : S);
-  if (S > p.total_steps) S = p.total_steps > 0 ? p.total_steps : 1;
-  p.sps = (p.total_steps + S - 1) / S;
-  if (p.sps < 1) p.sps = 1;
-  p.S = p.total_steps > 0 ? (p.total_steps + p.sps - 1) / p.sps : 1;
+  const int64_t chunks = (M + 63) / 64;                      // of one expert holding every row
+  if (S > chunks) S = chunks > 0 ? int(chunks) : 1;
+  p.S = S;
   return p;
 }
 
-// Split plan of the lora_down kernel: 128-row tiles, the contraction (Kc) split into S ranges of
-// whole 64-deep steps, at least 2 steps per split.
+// Split plan of the lora_down kernel: 128-row tiles (at most ceil(M/128) + E - 1 over all
+// experts), the contraction (Kc) split into S ranges of whole 64-deep steps, >= 2 steps each.
 struct DownPlan {
   int tiles, S, sps, num_k;
 };
 
-DownPlan down_plan(int64_t M, int64_t Kc, int sms) {
+DownPlan down_plan(int64_t M, int64_t Kc, int E, int sms) {
   DownPlan p{};
-  p.tiles = int((M + 127) / 128);
+  p.tiles = int((M + 127) / 128) + (E > 1 ? E - 1 : 0);
   p.num_k = int((Kc + 63) / 64);
   int S = p.tiles > 0 ? (sms + p.tiles - 1) / p.tiles : 1;   // about one wave of long splits
   S = S < 1 ? 1 : (S > 16 ? 16 : S);
@@ -146,16 +144,17 @@ DownPlan down_plan(int64_t M, int64_t Kc, int sms) {
   return p;
 }
 
-size_t down_partial_bytes(int64_t M, int64_t Kc, int r, int sms) {
-  const DownPlan dp = down_plan(M, Kc, sms);
+size_t down_partial_bytes(int64_t M, int64_t Kc, int r, int E, int sms) {
+  const DownPlan dp = down_plan(M, Kc, E, sms);
   return dp.S > 1 ? size_t(dp.S) * size_t(M) * size_t(rank_pad(r)) * 4 : 0;
 }
 
 struct WsLayout {
   size_t zs, t, u, partial, partial_bytes, total;
+  int counters_needed;
 };
 
-WsLayout ws_layout(int64_t N, int64_t K, int64_t M, int r, bool bwd, int sms) {
+WsLayout ws_layout(int64_t N, int64_t K, int64_t M, int r, bool bwd, int E, int sms) {
   WsLayout L{};
   size_t off = kHeaderBytes + kCounterBytes;
   const size_t mr = align_up(size_t(M > 0 ? M : 0) * size_t(r) * 2, 256);
@@ -164,13 +163,16 @@ WsLayout ws_layout(int64_t N, int64_t K, int64_t M, int r, bool bwd, int sms) {
   L.u = off; off += bwd ? mr : 0;
   L.partial = off;
   // fp32 split partials, shared by the (sequential) lora_down and lora_wgrad launches
-  size_t pb = down_partial_bytes(M, K, r, sms);
+  size_t pb = down_partial_bytes(M, K, r, E, sms);
+  L.counters_needed = down_plan(M, K, E, sms).tiles;
   if (bwd) {
-    const size_t pu = down_partial_bytes(M, N, r, sms);
+    const size_t pu = down_partial_bytes(M, N, r, E, sms);
     pb = pu > pb ? pu : pb;
-    const WgradPlan wp = wgrad_plan(N, K, M, sms);
-    const size_t pw = wp.S > 1 ? size_t(wp.S) * size_t(N + K) * size_t(rank_pad(r)) * 4 : 0;
+    const WgradPlan wp = wgrad_plan(N, K, M, E, sms);
+    const size_t pw = wp.S > 1 ? size_t(wp.S) * size_t(E) * size_t(N + K) * size_t(rank_pad(r)) * 4 : 0;
     pb = pw > pb ? pw : pb;
+    const int wc = E * (wp.tiles0 + wp.tiles1);
+    if (wc > L.counters_needed) L.counters_needed = wc;
   }
   L.partial_bytes = align_up(pb, 256);
   off += L.partial_bytes;
@@ -218,15 +220,31 @@ struct LaunchScope {
 };
 
 // ---------------------------------------------------------------------------------- launches
-// partial / partial_bytes: fp32 scratch for the split contraction (the split count is reduced
-// until its partials fit); counters: one zeroed int per 128-row tile.
+// 3-D row-major tensor [d2, d1, d0] (d0 contiguous), box {b0, b1, 1}.
+bool tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+             uint32_t b1, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Z = Act . R for every expert's rows: R is A [E, r, Kc] (r_mn false, T = X A^T) or
+// B [E, Kc, r] (r_mn true, U = dY B).  partial / partial_bytes: fp32 scratch for the split
+// contraction (the split count is reduced until its partials fit); counters: zeroed ints, one per
+// row tile.  offsets == nullptr: one expert of M rows.
 qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t Kc, const void* R,
-                                int64_t R_rows, int r, float s, const float* ts, void* z, void* zs,
-                                int* status, float* partial, size_t partial_bytes, int* counters,
-                                cudaStream_t st) {
+                                int r, float s, const float* ts, void* z, void* zs, int* status,
+                                float* partial, size_t partial_bytes, int* counters,
+                                const int32_t* offsets, int E, bool grouped, cudaStream_t st) {
   DownParams p{};
   const int rpad = rank_pad(r);
-  DownPlan dp = down_plan(M, Kc, num_sms());
+  DownPlan dp = down_plan(M, Kc, E, num_sms());
   while (dp.S > 1 && size_t(dp.S) * size_t(M) * size_t(rpad) * 4 > partial_bytes) {
     dp.sps = (dp.num_k + dp.S - 2) / (dp.S - 1);
     dp.S = (dp.num_k + dp.sps - 1) / dp.sps;
@@ -235,51 +253,53 @@ qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t K
   if (!tmap_2d(&p.tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, uint64_t(Kc), uint64_t(M),
                uint64_t(Kc) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
-  if (!r_mn) {  // R = A [r, K]: K-major rows, box {64, rpad}
-    if (!tmap_2d(&p.tm_r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, uint64_t(Kc), uint64_t(r),
-                 uint64_t(Kc) * 2, 64, uint32_t(rpad), CU_TENSOR_MAP_SWIZZLE_128B))
-      return QLORA_ERR_CUDA;
-  } else {      // R = B [N, r]: MN-major, box {rpad, 64}
-    if (!tmap_2d(&p.tm_r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, uint64_t(r), uint64_t(R_rows),
-                 uint64_t(r) * 2, uint32_t(rpad), 64, swizzle_for_bytes(uint32_t(rpad) * 2)))
-      return QLORA_ERR_CUDA;
-  }
+  const bool okm = !r_mn
+      ? tmap_3d(&p.tm_r, R, uint64_t(Kc), uint64_t(r), uint64_t(E), 64, uint32_t(rpad),
+                CU_TENSOR_MAP_SWIZZLE_128B)
+      : tmap_3d(&p.tm_r, R, uint64_t(r), uint64_t(Kc), uint64_t(E), uint32_t(rpad), 64,
+                swizzle_for_bytes(uint32_t(rpad) * 2));
+  if (!okm) return QLORA_ERR_CUDA;
   p.tensor_scale = ts;
   p.z = static_cast<__nv_bfloat16*>(z);
   p.zs = static_cast<__nv_bfloat16*>(zs);
   p.status = status;
   p.partial = partial;
   p.counters = counters;
+  p.offsets = offsets;
   p.M = int(M);
   p.r = r;
   p.rpad = rpad;
   p.num_k = dp.num_k;
   p.S = dp.S;
   p.steps_per_split = dp.sps;
+  p.E = E;
   p.s = s;
   const dim3 grid(unsigned(dp.tiles * dp.S));
-  LaunchScope scope(r_mn ? kKindDownU : kKindDownT, st);
+  const size_t smem = lora::smem_bytes(E);
+  LaunchScope scope(grouped ? (r_mn ? kKindGDownU : kKindGDownT) : (r_mn ? kKindDownU : kKindDownT), st);
   if (r_mn) {
-    if (!set_smem(qlora_lora_down_kernel<true>, lora::kSmemBytes)) return QLORA_ERR_CUDA;
-    qlora_lora_down_kernel<true><<<grid, lora::kThreads, lora::kSmemBytes, st>>>(p);
+    if (!set_smem(qlora_lora_down_kernel<true>, smem)) return QLORA_ERR_CUDA;
+    qlora_lora_down_kernel<true><<<grid, lora::kThreads, smem, st>>>(p);
   } else {
-    if (!set_smem(qlora_lora_down_kernel<false>, lora::kSmemBytes)) return QLORA_ERR_CUDA;
-    qlora_lora_down_kernel<false><<<grid, lora::kThreads, lora::kSmemBytes, st>>>(p);
+    if (!set_smem(qlora_lora_down_kernel<false>, smem)) return QLORA_ERR_CUDA;
+    qlora_lora_down_kernel<false><<<grid, lora::kThreads, smem, st>>>(p);
   }
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 template <int FMT, bool DX>
-qlora_status_t launch_fused_t(const FusedParams& p, int grid, cudaStream_t st) {
-  if (!set_smem(qlora_fused_gemm_kernel<FMT, DX>, fused::kSmemBytes)) return QLORA_ERR_CUDA;
-  LaunchScope scope(DX ? kKindFusedDx : kKindFusedFwd, st);
-  qlora_fused_gemm_kernel<FMT, DX><<<grid, fused::kThreads, fused::kSmemBytes, st>>>(p);
+qlora_status_t launch_fused_t(const FusedParams& p, int grid, bool grouped, cudaStream_t st) {
+  const size_t smem = fused::smem_bytes(p.E);
+  if (!set_smem(qlora_fused_gemm_kernel<FMT, DX>, smem)) return QLORA_ERR_CUDA;
+  LaunchScope scope(grouped ? (DX ? kKindGFusedDx : kKindGFusedFwd) : (DX ? kKindFusedDx : kKindFusedFwd), st);
+  qlora_fused_gemm_kernel<FMT, DX><<<grid, fused::kThreads, smem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// W: one weight (E = 1) or E stacked weights; lora_up: B [E, N, r] (forward) or A [E, r, K] (dX).
 qlora_status_t launch_fused(const qlora_weight_t* W, bool dx, const void* act, const void* zs,
                             const void* lora_up, void* out, int64_t M, int r, int* status,
-                            cudaStream_t st) {
+                            const int32_t* offsets, int E, bool grouped, cudaStream_t st) {
   FusedParams p{};
   const int64_t N = W->N, K = W->K;
   const int64_t Kc = dx ? N : K;
@@ -288,11 +308,11 @@ qlora_status_t launch_fused(const qlora_weight_t* W, bool dx, const void* act, c
     return QLORA_ERR_CUDA;
   if (!dx) {
     if (!tmap_2d(&p.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, uint64_t(K / 2),
-                 uint64_t(N), uint64_t(K / 2), 32, 128, CU_TENSOR_MAP_SWIZZLE_32B))
+                 uint64_t(N) * uint64_t(E), uint64_t(K / 2), 32, 128, CU_TENSOR_MAP_SWIZZLE_32B))
       return QLORA_ERR_CUDA;
   } else {
     if (!tmap_2d(&p.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, uint64_t(K / 2),
-                 uint64_t(N), uint64_t(K / 2), 64, 64, CU_TENSOR_MAP_SWIZZLE_64B))
+                 uint64_t(N) * uint64_t(E), uint64_t(K / 2), 64, 64, CU_TENSOR_MAP_SWIZZLE_64B))
       return QLORA_ERR_CUDA;
   }
   if (!tmap_2d(&p.tm_zs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, zs, uint64_t(r), uint64_t(M),
@@ -302,48 +322,54 @@ qlora_status_t launch_fused(const qlora_weight_t* W, bool dx, const void* act, c
   p.tensor_scale = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
   p.lora_up = static_cast<const __nv_bfloat16*>(lora_up);
   p.out = static_cast<__nv_bfloat16*>(out);
+  p.offsets = offsets;
   p.status = status;
   p.M = int(M);
   p.N = int(N);
   p.K = int(K);
   p.r = r;
-  p.num_m = int((M + fused::BM - 1) / fused::BM);
+  p.E = E;
   p.num_n = int(((dx ? K : N) + fused::BN - 1) / fused::BN);
   p.num_k = int((Kc + fused::BK - 1) / fused::BK);
-  // one CTA pair per pair tile, at most one pair per two SMs (persistent beyond that)
-  const int tiles = p.num_m * p.num_n;
-  const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
-  const int grid = 2 * (pairs > 0 ? pairs : 1);
+  // one CTA pair per pair tile, at most one pair per two SMs (persistent beyond that); the tile
+  // count of a grouped launch is known only on the device: at most ceil(M/256) + E - 1 row tiles
+  const int64_t tiles = ((M + fused::BM - 1) / fused::BM + (E > 1 ? E - 1 : 0)) * p.num_n;
+  const int64_t pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
+  const int grid = int(2 * (pairs > 0 ? pairs : 1));
   switch (W->fmt * 2 + (dx ? 1 : 0)) {
-    case 0: return launch_fused_t<kFmtNF4, false>(p, grid, st);
-    case 1: return launch_fused_t<kFmtNF4, true>(p, grid, st);
-    case 2: return launch_fused_t<kFmtMXFP4, false>(p, grid, st);
-    case 3: return launch_fused_t<kFmtMXFP4, true>(p, grid, st);
-    case 4: return launch_fused_t<kFmtNVFP4, false>(p, grid, st);
-    default: return launch_fused_t<kFmtNVFP4, true>(p, grid, st);
+    case 0: return launch_fused_t<kFmtNF4, false>(p, grid, grouped, st);
+    case 1: return launch_fused_t<kFmtNF4, true>(p, grid, grouped, st);
+    case 2: return launch_fused_t<kFmtMXFP4, false>(p, grid, grouped, st);
+    case 3: return launch_fused_t<kFmtMXFP4, true>(p, grid, grouped, st);
+    case 4: return launch_fused_t<kFmtNVFP4, false>(p, grid, grouped, st);
+    default: return launch_fused_t<kFmtNVFP4, true>(p, grid, grouped, st);
   }
 }
 
+// dB [E, N, r] = s dY_e^T T_e and dA [E, r, K] = s U_e^T X_e over each expert's rows.
 qlora_status_t launch_wgrad(const void* X, const void* dY, const void* T, const void* U, int64_t M,
                             int64_t N, int64_t K, int r, float s, void* dA, void* dB, void* ws,
-                            const WsLayout& L, cudaStream_t st) {
+                            const WsLayout& L, const int32_t* offsets, int E, bool grouped,
+                            cudaStream_t st) {
   WgradParams p{};
   const int rpad = rank_pad(r);
-  const WgradPlan wp = wgrad_plan(N, K, M, num_sms());
+  const WgradPlan wp = wgrad_plan(N, K, M, E, num_sms());
   const CUtensorMapSwizzle rsw = swizzle_for_bytes(uint32_t(rpad) * 2);
-  if (!tmap_2d(&p.tm_l[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, uint64_t(N), uint64_t(M),
+  const uint64_t rows = uint64_t(M > 0 ? M : 1);
+  if (!tmap_2d(&p.tm_l[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, uint64_t(N), rows,
                uint64_t(N) * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !tmap_2d(&p.tm_l[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, uint64_t(K), uint64_t(M),
+      !tmap_2d(&p.tm_l[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, uint64_t(K), rows,
                uint64_t(K) * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !tmap_2d(&p.tm_r[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, uint64_t(r), uint64_t(M),
+      !tmap_2d(&p.tm_r[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, uint64_t(r), rows,
                uint64_t(r) * 2, uint32_t(rpad), 64, rsw) ||
-      !tmap_2d(&p.tm_r[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U, uint64_t(r), uint64_t(M),
+      !tmap_2d(&p.tm_r[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U, uint64_t(r), rows,
                uint64_t(r) * 2, uint32_t(rpad), 64, rsw))
     return QLORA_ERR_CUDA;
   p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.partial);
   p.counters = ws_counters(ws);
   p.out0 = static_cast<__nv_bfloat16*>(dB);
   p.out1 = static_cast<__nv_bfloat16*>(dA);
+  p.offsets = offsets;
   p.status = ws_status(ws);
   p.M = int(M);
   p.P0 = int(N);
@@ -353,14 +379,14 @@ qlora_status_t launch_wgrad(const void* X, const void* dY, const void* T, const 
   p.S = wp.S;
   p.tiles0 = wp.tiles0;
   p.tiles1 = wp.tiles1;
-  p.steps_per_split = wp.sps;
-  p.total_steps = wp.total_steps;
+  p.E = E;
   p.s = s;
-  if (wp.tiles0 + wp.tiles1 > kMaxCounters) return QLORA_ERR_UNSUPPORTED;
-  if (!set_smem(qlora_lora_wgrad_kernel, lora::kSmemBytes)) return QLORA_ERR_CUDA;
-  const unsigned grid = unsigned((wp.tiles0 + wp.tiles1) * wp.S);
-  LaunchScope scope(kKindWgrad, st);
-  qlora_lora_wgrad_kernel<<<grid, lora::kThreads, lora::kSmemBytes, st>>>(p);
+  if (int64_t(E) * (wp.tiles0 + wp.tiles1) > kMaxCounters) return QLORA_ERR_UNSUPPORTED;
+  const size_t smem = lora::smem_bytes(E);
+  if (!set_smem(qlora_lora_wgrad_kernel, smem)) return QLORA_ERR_CUDA;
+  const unsigned grid = unsigned(int64_t(E) * (wp.tiles0 + wp.tiles1) * wp.S);
+  LaunchScope scope(grouped ? kKindGWgrad : kKindWgrad, st);
+  qlora_lora_wgrad_kernel<<<grid, lora::kThreads, smem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
@@ -395,10 +421,13 @@ using namespace qlora;
 extern "C" {
 
 size_t qlora_workspace_size(int op, const qlora_weight_t* W, int64_t M, int r, int E) {
-  (void)E;
   if (check_weight(W) != QLORA_OK || M < 0 || !rank_ok(r)) return 0;
-  if (op != QLORA_OP_FWD && op != QLORA_OP_BWD) return 0;
-  return ws_layout(W->N, W->K, M, r, op == QLORA_OP_BWD, num_sms()).total;
+  const bool grouped = op == QLORA_OP_GROUPED_FWD || op == QLORA_OP_GROUPED_BWD;
+  if (!grouped && op != QLORA_OP_FWD && op != QLORA_OP_BWD) return 0;
+  if (grouped && (E < 1 || E > kMaxExperts)) return 0;
+  const WsLayout L = ws_layout(W->N, W->K, M, r, op == QLORA_OP_BWD || op == QLORA_OP_GROUPED_BWD,
+                               grouped ? E : 1, num_sms());
+  return L.counters_needed > kMaxCounters ? 0 : L.total;
 }
 
 qlora_status_t qlora_workspace_init(void* ws, size_t ws_bytes, qlora_stream_t stream) {
@@ -409,36 +438,108 @@ qlora_status_t qlora_workspace_init(void* ws, size_t ws_bytes, qlora_stream_t st
              : QLORA_ERR_CUDA;
 }
 
-qlora_status_t qlora_linear_fwd(const qlora_weight_t* W, const void* X, const void* A,
-                                const void* B, void* Y, void* T_save, int64_t M, int r,
-                                float scale, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+}  // extern "C"
+
+namespace qlora {
+namespace {
+
+// An [M, ...] activation: required (and 16-byte aligned) when M > 0, may be NULL when M == 0.
+bool act_ok(const void* q, int64_t M) { return M == 0 ? (q == nullptr || aligned16(q)) : ptr_ok(q); }
+
+// Shared argument checks of the four training entry points.
+qlora_status_t check_common(const qlora_weight_t* W, int64_t M, int r) {
   qlora_status_t st = check_weight(W);
   if (st != QLORA_OK) return st;
   if (M < 0 || M > (int64_t(1) << 31) - 512) return QLORA_ERR_INVALID_ARG;
   if (!rank_ok(r)) return (r > 0 && r <= 256) ? QLORA_ERR_UNSUPPORTED : QLORA_ERR_INVALID_ARG;
-  if (!ptr_ok(X) || !ptr_ok(A) || !ptr_ok(B) || !ptr_ok(Y) || (T_save && !aligned16(T_save)))
+  return QLORA_OK;
+}
+
+// Forward over E experts (offsets == nullptr: one layer of M rows).
+qlora_status_t run_fwd(const qlora_weight_t* W, int E, const int32_t* offsets, bool grouped,
+                       const void* X, const void* A, const void* B, void* Y, void* T_save,
+                       int64_t M, int r, float scale, void* ws, size_t ws_bytes, cudaStream_t s) {
+  if (!act_ok(X, M) || !ptr_ok(A) || !ptr_ok(B) || !act_ok(Y, M) || (T_save && !aligned16(T_save)))
     return QLORA_ERR_INVALID_ARG;
-  const WsLayout L = ws_layout(W->N, W->K, M, r, false, num_sms());
+  const WsLayout L = ws_layout(W->N, W->K, M, r, false, E, num_sms());
+  if (L.counters_needed > kMaxCounters) return QLORA_ERR_UNSUPPORTED;
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (M == 0) return QLORA_OK;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* w = static_cast<uint8_t*>(ws);
   void* T = T_save ? T_save : w + L.t;
   void* Zs = w + L.zs;
   const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
-  st = launch_lora_down(false, X, M, W->K, A, r, r, scale, ts, T, Zs, ws_status(ws),
-                        reinterpret_cast<float*>(w + L.partial), L.partial_bytes, ws_counters(ws), s);
+  qlora_status_t st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, T, Zs, ws_status(ws),
+                                       reinterpret_cast<float*>(w + L.partial), L.partial_bytes,
+                                       ws_counters(ws), offsets, E, grouped, s);
   if (st != QLORA_OK) return st;
-  return launch_fused(W, false, X, Zs, B, Y, M, r, ws_status(ws), s);
+  return launch_fused(W, false, X, Zs, B, Y, M, r, ws_status(ws), offsets, E, grouped, s);
+}
+
+// Backward over E experts (offsets == nullptr: one layer of M rows).
+qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, bool grouped,
+                       const void* X, const void* A, const void* B, const void* T, const void* dY,
+                       void* dX, void* dA, void* dB, int64_t M, int r, float scale, void* ws,
+                       size_t ws_bytes, cudaStream_t s) {
+  if (!act_ok(X, M) || !ptr_ok(A) || !ptr_ok(B) || !act_ok(dY, M) || !ptr_ok(dA) || !ptr_ok(dB) ||
+      (T && !aligned16(T)) || (dX && !aligned16(dX)))
+    return QLORA_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(W->N, W->K, M, r, true, E, num_sms());
+  if (L.counters_needed > kMaxCounters) return QLORA_ERR_UNSUPPORTED;
+  if (!ws || !aligned16(ws) || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (M == 0) {
+    if (cudaMemsetAsync(dA, 0, size_t(E) * r * W->K * 2, s) != cudaSuccess ||
+        cudaMemsetAsync(dB, 0, size_t(E) * W->N * r * 2, s) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
+  void* Zs = w + L.zs;
+  void* U = w + L.u;
+  float* part = reinterpret_cast<float*>(w + L.partial);
+  qlora_status_t st;
+  if (!T) {  // recompute T = X A^T (its scaled copy lands in Zs and is overwritten below)
+    st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, w + L.t, Zs, ws_status(ws), part,
+                          L.partial_bytes, ws_counters(ws), offsets, E, grouped, s);
+    if (st != QLORA_OK) return st;
+    T = w + L.t;
+  }
+  st = launch_lora_down(true, dY, M, W->N, B, r, scale, ts, U, Zs, ws_status(ws), part,
+                        L.partial_bytes, ws_counters(ws), offsets, E, grouped, s);
+  if (st != QLORA_OK) return st;
+  if (dX) {
+    st = launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), offsets, E, grouped, s);
+    if (st != QLORA_OK) return st;
+  }
+  return launch_wgrad(X, dY, T, U, M, W->N, W->K, r, scale, dA, dB, ws, L, offsets, E, grouped, s);
+}
+
+qlora_status_t check_groups(int E, const int32_t* d_offsets) {
+  if (E < 1 || E > kMaxExperts) return QLORA_ERR_UNSUPPORTED;
+  if (!d_offsets || (reinterpret_cast<uintptr_t>(d_offsets) & 3u) != 0) return QLORA_ERR_INVALID_ARG;
+  return QLORA_OK;
+}
+
+}  // namespace
+}  // namespace qlora
+
+extern "C" {
+
+qlora_status_t qlora_linear_fwd(const qlora_weight_t* W, const void* X, const void* A,
+                                const void* B, void* Y, void* T_save, int64_t M, int r,
+                                float scale, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  const qlora_status_t st = check_common(W, M, r);
+  if (st != QLORA_OK) return st;
+  return run_fwd(W, 1, nullptr, false, X, A, B, Y, T_save, M, r, scale, ws, ws_bytes,
+                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const void* X, const void* A,
                                         const void* B, void* Y, void* T_save, int64_t M, int r,
                                         float scale, qlora_stream_t stream) {
-  qlora_status_t st = check_weight(W);
+  qlora_status_t st = check_common(W, M, r);
   if (st != QLORA_OK) return st;
-  if (M < 0 || M > (int64_t(1) << 31) - 512) return QLORA_ERR_INVALID_ARG;
-  if (!rank_ok(r)) return (r > 0 && r <= 256) ? QLORA_ERR_UNSUPPORTED : QLORA_ERR_INVALID_ARG;
   if (!ptr_ok(X) || !ptr_ok(A) || !ptr_ok(B) || !ptr_ok(Y) || (T_save && !aligned16(T_save)))
     return QLORA_ERR_INVALID_ARG;
   const size_t mr = align_up(size_t(M) * size_t(r) * 2, 256);
@@ -458,60 +559,31 @@ qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const void* X, 
   float* part = reinterpret_cast<float*>(w + used);
   const size_t part_bytes = kNoAllocScratchBytes - used;
   int* counters = reinterpret_cast<int*>(w + 128);   // 32 tile counters inside the header
-  st = launch_lora_down(false, X, M, W->K, A, r, r, scale, ts, T, Zs, status, part,
-                        (M + 127) / 128 <= 32 ? part_bytes : 0, counters, s);
+  st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, T, Zs, status, part,
+                        (M + 127) / 128 <= 32 ? part_bytes : 0, counters, nullptr, 1, false, s);
   if (st != QLORA_OK) return st;
-  return launch_fused(W, false, X, Zs, B, Y, M, r, status, s);
+  return launch_fused(W, false, X, Zs, B, Y, M, r, status, nullptr, 1, false, s);
 }
 
 qlora_status_t qlora_linear_bwd(const qlora_weight_t* W, const void* X, const void* A,
                                 const void* B, const void* T, const void* dY, void* dX, void* dA,
                                 void* dB, int64_t M, int r, float scale, void* ws, size_t ws_bytes,
                                 qlora_stream_t stream) {
-  qlora_status_t st = check_weight(W);
+  const qlora_status_t st = check_common(W, M, r);
   if (st != QLORA_OK) return st;
-  if (M < 0 || M > (int64_t(1) << 31) - 512) return QLORA_ERR_INVALID_ARG;
-  if (!rank_ok(r)) return (r > 0 && r <= 256) ? QLORA_ERR_UNSUPPORTED : QLORA_ERR_INVALID_ARG;
-  if (!ptr_ok(X) || !ptr_ok(A) || !ptr_ok(B) || !ptr_ok(dY) || !ptr_ok(dA) || !ptr_ok(dB) ||
-      (T && !aligned16(T)) || (dX && !aligned16(dX)))
-    return QLORA_ERR_INVALID_ARG;
-  const WsLayout L = ws_layout(W->N, W->K, M, r, true, num_sms());
-  if (!ws || !aligned16(ws) || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (M == 0) {
-    if (cudaMemsetAsync(dA, 0, size_t(r) * W->K * 2, s) != cudaSuccess ||
-        cudaMemsetAsync(dB, 0, size_t(W->N) * r * 2, s) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    return QLORA_OK;
-  }
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
-  void* Zs = w + L.zs;
-  void* U = w + L.u;
-  float* part = reinterpret_cast<float*>(w + L.partial);
-  if (!T) {  // recompute T = X A^T (its scaled copy lands in Zs and is overwritten below)
-    st = launch_lora_down(false, X, M, W->K, A, r, r, scale, ts, w + L.t, Zs, ws_status(ws), part,
-                          L.partial_bytes, ws_counters(ws), s);
-    if (st != QLORA_OK) return st;
-    T = w + L.t;
-  }
-  st = launch_lora_down(true, dY, M, W->N, B, W->N, r, scale, ts, U, Zs, ws_status(ws), part,
-                        L.partial_bytes, ws_counters(ws), s);
-  if (st != QLORA_OK) return st;
-  if (dX) {
-    st = launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), s);
-    if (st != QLORA_OK) return st;
-  }
-  return launch_wgrad(X, dY, T, U, M, W->N, W->K, r, scale, dA, dB, ws, L, s);
+  return run_bwd(W, 1, nullptr, false, X, A, B, T, dY, dX, dA, dB, M, r, scale, ws, ws_bytes,
+                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 qlora_status_t qlora_grouped_fwd(const qlora_weight_t* W, int E, const int32_t* d_offsets,
                                  int64_t M_total, const void* X, const void* A, const void* B,
                                  void* Y, void* T_save, int r, float scale, void* ws,
                                  size_t ws_bytes, qlora_stream_t stream) {
-  (void)W; (void)E; (void)d_offsets; (void)M_total; (void)X; (void)A; (void)B; (void)Y;
-  (void)T_save; (void)r; (void)scale; (void)ws; (void)ws_bytes; (void)stream;
-  return QLORA_ERR_UNSUPPORTED;
+  qlora_status_t st = check_common(W, M_total, r);
+  if (st != QLORA_OK) return st;
+  if ((st = check_groups(E, d_offsets)) != QLORA_OK) return st;
+  return run_fwd(W, E, d_offsets, true, X, A, B, Y, T_save, M_total, r, scale, ws, ws_bytes,
+                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 qlora_status_t qlora_grouped_bwd(const qlora_weight_t* W, int E, const int32_t* d_offsets,
@@ -519,9 +591,11 @@ qlora_status_t qlora_grouped_bwd(const qlora_weight_t* W, int E, const int32_t* 
                                  const void* T, const void* dY, void* dX, void* dA, void* dB,
                                  int r, float scale, void* ws, size_t ws_bytes,
                                  qlora_stream_t stream) {
-  (void)W; (void)E; (void)d_offsets; (void)M_total; (void)X; (void)A; (void)B; (void)T; (void)dY;
-  (void)dX; (void)dA; (void)dB; (void)r; (void)scale; (void)ws; (void)ws_bytes; (void)stream;
-  return QLORA_ERR_UNSUPPORTED;
+  qlora_status_t st = check_common(W, M_total, r);
+  if (st != QLORA_OK) return st;
+  if ((st = check_groups(E, d_offsets)) != QLORA_OK) return st;
+  return run_bwd(W, E, d_offsets, true, X, A, B, T, dY, dX, dA, dB, M_total, r, scale, ws,
+                 ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 qlora_status_t qlora_get_device_status(void* ws, qlora_stream_t stream) {

@@ -43,13 +43,14 @@
 #include <cuda_bf16.h>
 #include "qlora_ptx.cuh"
 #include "qlora_dequant.cuh"
+#include "qlora_groups.cuh"
 
 namespace qlora {
 namespace fused {
 constexpr int BM = 256, BN = 256;      // pair tile
 constexpr int HM = 128, HN = 128;      // per-CTA halves
 constexpr int BK = 64;
-constexpr int NS = 6, NC = 8;         // operand stages (activation + weight halves), code stages
+constexpr int NS = 6, NC = 6;         // operand stages (activation + weight halves), code stages
 constexpr int X_BYTES = HM * BK * 2;   // 16 KB
 constexpr int W_BYTES = HN * BK * 2;   // 16 KB
 constexpr int C_BYTES = HN * BK / 2;   // 4 KB of packed codes
@@ -58,20 +59,23 @@ constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;
 constexpr int kTmemCols = 512;         // 2 buffers x 256 columns
 constexpr int GM = 8;                  // m-tiles per raster group
 constexpr int kNumBars = 2 * NS + 2 * NC + 4;
-constexpr size_t kSmemBytes = 1024 + size_t(NS) * (X_BYTES + W_BYTES) + size_t(NC) * C_BYTES + 1024;
+constexpr size_t kSmemBase = 1024 + size_t(NS) * (X_BYTES + W_BYTES) + size_t(NC) * C_BYTES + 1024;
+// plus the expert table: 2 x (E + 1) ints
+__host__ __device__ constexpr size_t smem_bytes(int E) { return kSmemBase + size_t(2) * (E + 1) * 4; }
 }  // namespace fused
 
 struct FusedParams {
   CUtensorMap tm_act;    // activations [M, Kc] bf16, box {64, 128}, SW128
-  CUtensorMap tm_codes;  // codes [N, K/2] u8: fwd box {32, 128} SW32; dX box {64, 64} SW64
+  CUtensorMap tm_codes;  // codes [E*N, K/2] u8: fwd box {32, 128} SW32; dX box {64, 64} SW64
   CUtensorMap tm_zs;     // Zs [M, r] bf16, box {64, 128}, SW128 (zero fill beyond r)
-  const void* scales;
-  const float* tensor_scale;         // NVFP4 device scalar, else nullptr
-  const __nv_bfloat16* lora_up;      // fwd: B [N, r]; dX: A [r, K]
+  const void* scales;                // [E, N, K/bs]
+  const float* tensor_scale;         // NVFP4: [E] device floats, else nullptr
+  const __nv_bfloat16* lora_up;      // fwd: B [E, N, r]; dX: A [E, r, K]
   __nv_bfloat16* out;                // fwd: Y [M, N]; dX: dX [M, K]
+  const int32_t* offsets;            // grouped: device [E+1] row offsets; nullptr: one expert
   int* status;
-  int M, N, K, r;
-  int num_m, num_n, num_k;           // pair tiles over rows, over output columns; contraction steps
+  int M, N, K, r, E;                 // M: all rows (packed over experts)
+  int num_n, num_k;                  // pair tiles over output columns; contraction steps
 };
 
 __device__ __forceinline__ void fused_tile_coords(int t, int num_m, int num_n, int& mt, int& nt) {
@@ -84,18 +88,40 @@ __device__ __forceinline__ void fused_tile_coords(int t, int num_m, int num_n, i
   nt = within / gm;
 }
 
-// Block-scale word of the item that starts at weight element (n, kcol).
+// Block-scale word of the item that starts at element (n, kcol) of the weight whose rows begin
+// at row `nrow0` of the (stacked) scale array.
 template <int FMT>
-__device__ __forceinline__ ItemScale load_item_scale(const void* scales, int n, int kcol, int K) {
+__device__ __forceinline__ ItemScale load_item_scale(const void* scales, int n, int kcol, int K,
+                                                     size_t nrow0 = 0) {
   ItemScale s;
+  const size_t row = nrow0 + size_t(n);
   if constexpr (FMT == kFmtNF4) {
-    s.raw = __ldg(reinterpret_cast<const uint32_t*>(scales) + size_t(n) * (K / 64) + kcol / 64);
+    s.raw = __ldg(reinterpret_cast<const uint32_t*>(scales) + row * (K / 64) + kcol / 64);
   } else if constexpr (FMT == kFmtMXFP4) {
-    s.raw = __ldg(reinterpret_cast<const uint16_t*>(scales) + (size_t(n) * (K / 32) + kcol / 32) / 2);
+    s.raw = __ldg(reinterpret_cast<const uint16_t*>(scales) + (row * (K / 32) + kcol / 32) / 2);
   } else {
-    s.raw = __ldg(reinterpret_cast<const uint32_t*>(scales) + (size_t(n) * (K / 16) + kcol / 16) / 4);
+    s.raw = __ldg(reinterpret_cast<const uint32_t*>(scales) + (row * (K / 16) + kcol / 16) / 4);
   }
   return s;
+}
+
+// Pair tile t of a (grouped) launch: expert e, rows [row0, row0 + 256) of which rows below
+// row_end belong to the expert, output-column tile nt.
+struct PairTile {
+  int e, row0, row_end, nt;
+};
+__device__ __forceinline__ PairTile pair_tile_at(const GroupView& g, int t, int num_n) {
+  PairTile pt;
+  pt.e = g.expert_of(t);
+  const int local = t - g.first[pt.e];
+  const int rows = g.off[pt.e + 1] - g.off[pt.e];
+  const int mtiles = (rows + fused::BM - 1) / fused::BM;
+  int mt, nt;
+  fused_tile_coords(local, mtiles, num_n, mt, nt);
+  pt.row0 = g.off[pt.e] + mt * fused::BM;
+  pt.row_end = g.off[pt.e + 1];
+  pt.nt = nt;
+  return pt;
 }
 
 // Shared-memory geometry of one dequant item (thread tg = 0..127 of a dequant group) in a CTA's
@@ -140,6 +166,8 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(cs + NC * C_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_off = reinterpret_cast<int*>(smem + (kSmemBase - 1024));
+  int* s_first = s_off + (p.E + 1);
 
   const uint32_t b0 = ptx::smem_u32(bars);
   auto full_s = [&](uint32_t s) { return b0 + 8u * s; };
@@ -173,13 +201,15 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), kTmemCols);
     ptx::tmem_relinquish_pair();
   }
+  const GroupView grp_view =
+      build_group_view(p.offsets, p.E, p.M, BM, p.num_n, s_off, s_first, p.status);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::cluster_sync();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int num_tiles = p.num_m * p.num_n;
+  const int num_tiles = grp_view.total();
   const int nk = p.num_k;
 
   if (warp == kTmaWarp) {
@@ -187,9 +217,8 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     if (lane == 0) {
       uint32_t i = 0;
       for (int t = pair; t < num_tiles; t += npairs) {
-        int mt, nt;
-        fused_tile_coords(t, p.num_m, p.num_n, mt, nt);
-        const int m0 = mt * BM + int(rank) * HM;      // this CTA's activation rows
+        const PairTile pt = pair_tile_at(grp_view, t, p.num_n);
+        const int m0 = pt.row0 + int(rank) * HM;      // this CTA's activation rows
         bool ok = true;
         for (int ks = 0; ks <= nk; ++ks, ++i) {
           const uint32_t sx = i % NS, px = (i / NS) & 1u;
@@ -208,17 +237,17 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     if (lane == 0) {
       uint32_t j = 0;
       for (int t = pair; t < num_tiles; t += npairs) {
-        int mt, nt;
-        fused_tile_coords(t, p.num_m, p.num_n, mt, nt);
-        const int h0 = nt * BN + int(rank) * HN;      // this CTA's weight half
+        const PairTile pt = pair_tile_at(grp_view, t, p.num_n);
+        const int h0 = pt.nt * BN + int(rank) * HN;   // this CTA's weight half
+        const int wrow0 = pt.e * p.N;                 // the expert's first row of the codes
         bool ok = true;
         for (int ks = 0; ks < nk; ++ks, ++j) {
           const uint32_t sc = j % NC, pc = (j / NC) & 1u;
           if (!ptx::mbar_wait(empty_c(sc), pc ^ 1u, p.status, abort_flag)) { ok = false; break; }
           ptx::mbar_arrive_expect_tx(full_c(sc), C_BYTES);
           const uint32_t cd = ptx::smem_u32(cs + sc * C_BYTES);
-          if (!DX) ptx::tma_load_2d(cd, &p.tm_codes, full_c(sc), ks * (BK / 2), h0);
-          else ptx::tma_load_2d(cd, &p.tm_codes, full_c(sc), h0 / 2, ks * BK);
+          if (!DX) ptx::tma_load_2d(cd, &p.tm_codes, full_c(sc), ks * (BK / 2), wrow0 + h0);
+          else ptx::tma_load_2d(cd, &p.tm_codes, full_c(sc), h0 / 2, wrow0 + ks * BK);
         }
         if (!ok) break;
       }
@@ -270,15 +299,14 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
   } else if (warp < kEpiWarps) {
     // ------------------------------------------------------------------ epilogue
     const int q = warp;  // tensor-memory lanes 32q .. 32q+31
-    const float ts = (FMT == kFmtNVFP4 && p.tensor_scale) ? __ldg(p.tensor_scale) : 1.0f;
     const int ncols = DX ? p.K : p.N;
     const uint32_t acc_empty_leader0 = ptx::mapa(acc_empty(0), 0);
     uint32_t tc = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++tc) {
-      int mt, nt;
-      fused_tile_coords(t, p.num_m, p.num_n, mt, nt);
-      const int row = mt * BM + int(rank) * HM + q * 32 + lane;
-      const int c0 = nt * BN;
+      const PairTile pt = pair_tile_at(grp_view, t, p.num_n);
+      const int row = pt.row0 + int(rank) * HM + q * 32 + lane;
+      const int c0 = pt.nt * BN;
+      const float ts = (FMT == kFmtNVFP4 && p.tensor_scale) ? __ldg(p.tensor_scale + pt.e) : 1.0f;
       const uint32_t buf = tc & 1u;
       if (!ptx::mbar_wait(acc_full(buf), (tc >> 1) & 1u, p.status, abort_flag)) break;
       ptx::tc_fence_after();
@@ -287,7 +315,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
         uint32_t v[32];
         ptx::tmem_ld_32x32b_x32(tmem + (uint32_t(q * 32) << 16) + buf * BN + cb * 32, v);
         ptx::tmem_ld_wait();
-        if (row < p.M) {
+        if (row < pt.row_end) {
           __nv_bfloat16* orow = p.out + size_t(row) * ncols;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
@@ -316,12 +344,14 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     // Cursor over this group's steps (every other step of the CTA's pipeline): tile t (the lt-th
     // of this pair), step ks of the tile (ks == nk is the LoRA step), weight-half origin h0.
     struct Cursor {
-      int t, lt, ks, h0;
+      int t, lt, ks, h0, e;
     };
-    auto tile_h0 = [&](int t) {
-      int mt, nt;
-      fused_tile_coords(t, p.num_m, p.num_n, mt, nt);
-      return nt * BN + int(rank) * HN;
+    auto set_tile = [&](Cursor& c) {
+      if (c.t < num_tiles) {
+        const PairTile pt = pair_tile_at(grp_view, c.t, p.num_n);
+        c.h0 = pt.nt * BN + int(rank) * HN;
+        c.e = pt.e;
+      }
     };
     auto advance2 = [&](Cursor& c) {
       c.ks += 2;
@@ -329,7 +359,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
         c.ks -= nk + 1;
         c.t += npairs;
         ++c.lt;
-        if (c.t < num_tiles) c.h0 = tile_h0(c.t);
+        set_tile(c);
       }
     };
     auto scale_for = [&](const Cursor& c) {
@@ -337,11 +367,13 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
       if (c.t < num_tiles && c.ks < nk) {
         const int n = DX ? c.ks * BK + geo.row : c.h0 + geo.row;
         const int kcol = DX ? c.h0 + geo.chunk * 64 : c.ks * BK;
-        if (n < p.N && kcol < p.K) sc = load_item_scale<FMT>(p.scales, n, kcol, p.K);
+        if (n < p.N && kcol < p.K)
+          sc = load_item_scale<FMT>(p.scales, n, kcol, p.K, size_t(c.e) * p.N);
       }
       return sc;
     };
-    Cursor cur{pair, 0, grp, pair < num_tiles ? tile_h0(pair) : 0};
+    Cursor cur{pair, 0, grp, 0, 0};
+    set_tile(cur);
     Cursor pf = cur;
     advance2(pf);
     ItemScale s_cur = scale_for(cur), s_next = scale_for(pf);
@@ -376,19 +408,20 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
       } else {
         // LoRA step: rows of B (forward, K-major) or of A (dX, MN-major), zero padded.
         uint4 v[8];
+        const __nv_bfloat16* up = p.lora_up + size_t(cur.e) * size_t(p.r) * (DX ? p.K : p.N);
         if (!DX) {
           const int n = cur.h0 + geo.row;
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj)
             v[jj] = (n < p.N && jj * 8 < p.r)
-                        ? __ldg(reinterpret_cast<const uint4*>(p.lora_up + size_t(n) * p.r + jj * 8))
+                        ? __ldg(reinterpret_cast<const uint4*>(up + size_t(n) * p.r + jj * 8))
                         : make_uint4(0, 0, 0, 0);
         } else {
           const int rj = geo.row, kc = cur.h0 + geo.chunk * 64;
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj)
             v[jj] = (rj < p.r && kc < p.K)
-                        ? __ldg(reinterpret_cast<const uint4*>(p.lora_up + size_t(rj) * p.K + kc + jj * 8))
+                        ? __ldg(reinterpret_cast<const uint4*>(up + size_t(rj) * p.K + kc + jj * 8))
                         : make_uint4(0, 0, 0, 0);
         }
         if (!ptx::mbar_wait(empty_s(sw), pw ^ 1u, p.status, abort_flag)) break;

@@ -14,6 +14,12 @@
 //   [M, P] and R [M, r]: an M=128 x N=rpad tcgen05 GEMM per 128-row tile of P whose operands are
 //   both MN-major (M is the contraction), M split over S CTAs per tile.
 //
+// Grouped launches (expert e owns rows [off[e], off[e+1]) of the packed activations, with its own
+// adapters) run the same kernels over a device-side table of (expert, tile) built from the
+// offsets; a single layer is one expert.  lora_down computes rows beyond an expert's end with
+// that expert's adapter and drops them at the store; lora_wgrad zeroes them in shared memory
+// before the MMA, so no row of another expert enters a reduction.
+//
 // Both kernels are memory bound (they stream an activation once) and have few output tiles, so
 // the contraction is split to fill the GPU.  Each split stores its fp32 partial tile; the last
 // split to finish (an atomic counter per tile, reset by that CTA for the next call) adds the S
@@ -21,6 +27,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include "qlora_ptx.cuh"
+#include "qlora_groups.cuh"
 
 namespace qlora {
 namespace lora {
@@ -29,7 +36,8 @@ constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int R_BYTES = 64 * 128;     // up to 64 x 128 B
 constexpr int kThreads = 6 * 32;      // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int kTmemCols = 64;
-constexpr size_t kSmemBytes = 1024 + size_t(NS) * (A_BYTES + R_BYTES) + 512;
+constexpr size_t kSmemBase = 1024 + size_t(NS) * (A_BYTES + R_BYTES) + 512;
+__host__ __device__ constexpr size_t smem_bytes(int E) { return kSmemBase + size_t(2) * (E + 1) * 4; }
 }  // namespace lora
 
 __device__ __forceinline__ uint32_t swz_mode_for_row_bytes(uint32_t rowb) {
@@ -100,14 +108,15 @@ __device__ __forceinline__ void load_acc_row(uint32_t taddr, int rpad, float (&a
 
 struct DownParams {
   CUtensorMap tm_act;  // X [M, K] or dY [M, N] bf16, box {64, 128}, SW128
-  CUtensorMap tm_r;    // T: A [r, K] box {64, rpad} SW128; U: B [N, r] box {rpad, 64} SW(2 rpad)
-  const float* tensor_scale;
+  CUtensorMap tm_r;    // T: A [E, r, K] box {64, rpad, 1} SW128; U: B [E, N, r] box {rpad, 64, 1}
+  const float* tensor_scale;   // NVFP4: [E], else nullptr
   __nv_bfloat16* z;    // [M, r]
   __nv_bfloat16* zs;   // [M, r]
   float* partial;      // [S, M, rpad] fp32 (S > 1)
-  int* counters;       // [m tiles]
+  int* counters;       // [row tiles]
+  const int32_t* offsets;      // grouped: device [E+1]; nullptr: one expert
   int* status;
-  int M, r, rpad, num_k, S, steps_per_split;
+  int M, r, rpad, num_k, S, steps_per_split, E;
   float s;
 };
 
@@ -124,13 +133,22 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  int* s_off = reinterpret_cast<int*>(smem + (kSmemBase - 1024));
+  int* s_first = s_off + (p.E + 1);
   const uint32_t b0 = ptx::smem_u32(bars);
   auto full = [&](uint32_t s) { return b0 + 8u * s; };
   auto empty = [&](uint32_t s) { return b0 + 8u * (NS + s); };
   const uint32_t acc_full = b0 + 8u * (2 * NS);
 
-  const int tile = blockIdx.x / p.S, split = blockIdx.x % p.S;
-  const int m0 = tile * BM;
+  // (expert, 128-row tile, split) of this CTA; CTAs beyond the table's last tile have no work
+  const GroupView gv = build_group_view(p.offsets, p.E, p.M, BM, p.S, s_off, s_first, p.status);
+  if (int(blockIdx.x) >= gv.total()) return;
+  const int e = gv.expert_of(blockIdx.x);
+  const int local = int(blockIdx.x) - gv.first[e];
+  const int mt = local / p.S, split = local % p.S;
+  const int tile = gv.first[e] / p.S + mt;               // row-tile index (counters)
+  const int m0 = gv.off[e] + mt * BM;
+  const int row_end = gv.off[e + 1];
   const int ks0 = split * p.steps_per_split;
   const int ks1 = min(ks0 + p.steps_per_split, p.num_k);
 
@@ -161,8 +179,8 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
         if (!ptx::mbar_wait(empty(s), ph ^ 1u, p.status, abort_flag)) break;
         ptx::mbar_arrive_expect_tx(full(s), A_BYTES + r_bytes);
         ptx::tma_load_2d(ptx::smem_u32(as + s * A_BYTES), &p.tm_act, full(s), ks * BK, m0);
-        if (!R_MN) ptx::tma_load_2d(ptx::smem_u32(rs + s * R_BYTES), &p.tm_r, full(s), ks * BK, 0);
-        else ptx::tma_load_2d(ptx::smem_u32(rs + s * R_BYTES), &p.tm_r, full(s), 0, ks * BK);
+        if (!R_MN) ptx::tma_load_3d(ptx::smem_u32(rs + s * R_BYTES), &p.tm_r, full(s), ks * BK, 0, e);
+        else ptx::tma_load_3d(ptx::smem_u32(rs + s * R_BYTES), &p.tm_r, full(s), 0, ks * BK, e);
       }
     }
   } else if (warp == 1) {
@@ -202,9 +220,10 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
       }
-      if (split_reduce(acc, p.rpad, p.S, split, p.partial, size_t(p.M), row, row < p.M,
-                       p.counters + tile, last_flag, et) && row < p.M) {
-        const float ts = p.tensor_scale ? __ldg(p.tensor_scale) : 1.0f;
+      const bool row_ok = row < row_end;
+      if (split_reduce(acc, p.rpad, p.S, split, p.partial, size_t(p.M), row, row_ok,
+                       p.counters + tile, last_flag, et) && row_ok) {
+        const float ts = p.tensor_scale ? __ldg(p.tensor_scale + e) : 1.0f;
         const float zscale = p.s / ts;
 #pragma unroll
         for (int c = 0; c < 64; c += 8) {
@@ -232,12 +251,13 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
 struct WgradParams {
   CUtensorMap tm_l[2];  // L: dY [M, N] (problem 0, dB) / X [M, K] (problem 1, dA); box {64, 64} SW128
   CUtensorMap tm_r[2];  // R: T [M, r] / U [M, r]; box {rpad, 64} SW(2 rpad)
-  float* partial;       // [S, P0 + P1, rpad] fp32 (S > 1)
-  int* counters;        // [tiles0 + tiles1], zero between calls
-  __nv_bfloat16* out0;  // dB [N, r]: (p, j) at p * r + j
-  __nv_bfloat16* out1;  // dA [r, K]: (p, j) at j * K + p
+  float* partial;       // [S, E * (P0 + P1), rpad] fp32 (S > 1)
+  int* counters;        // [E * (tiles0 + tiles1)], zero between calls
+  __nv_bfloat16* out0;  // dB [E, N, r]: (p, j) at p * r + j
+  __nv_bfloat16* out1;  // dA [E, r, K]: (p, j) at j * K + p
+  const int32_t* offsets;       // grouped: device [E+1]; nullptr: one expert of M rows
   int* status;
-  int M, P0, P1, r, rpad, S, tiles0, tiles1, steps_per_split, total_steps;
+  int M, P0, P1, r, rpad, S, tiles0, tiles1, E;
   float s;
 };
 
@@ -253,17 +273,28 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  int* s_off = reinterpret_cast<int*>(smem + (kSmemBase - 1024));
+  int* s_first = s_off + (p.E + 1);
   const uint32_t b0 = ptx::smem_u32(bars);
   auto full = [&](uint32_t s) { return b0 + 8u * s; };
   auto empty = [&](uint32_t s) { return b0 + 8u * (NS + s); };
   const uint32_t acc_full = b0 + 8u * (2 * NS);
 
+  // tile = (expert, output tile of dB or dA); the expert's rows are split into S ranges of
+  // whole 64-row chunks
+  const GroupView gv = build_group_view(p.offsets, p.E, p.M, 64, 1, s_off, s_first, p.status);
+  const int tiles_pe = p.tiles0 + p.tiles1;
   const int tile = blockIdx.x / p.S, split = blockIdx.x % p.S;
-  const int prob = tile < p.tiles0 ? 0 : 1;
-  const int p0 = (tile - (prob ? p.tiles0 : 0)) * BM;
+  const int e = tile / tiles_pe, et_tile = tile - e * tiles_pe;
+  const int prob = et_tile < p.tiles0 ? 0 : 1;
+  const int p0 = (et_tile - (prob ? p.tiles0 : 0)) * BM;
   const int P = prob ? p.P1 : p.P0;
-  const int ks0 = split * p.steps_per_split;
-  const int ks1 = min(ks0 + p.steps_per_split, p.total_steps);
+  const bool table_ok = gv.total() > 0 || p.M == 0;
+  const int row_begin = gv.off[e], row_end = gv.off[e + 1];
+  const int chunks = table_ok ? (row_end - row_begin + 63) / 64 : 0;
+  const int sps = (chunks + p.S - 1) / p.S;
+  const int ks0 = split * sps;
+  const int ks1 = min(ks0 + sps, chunks);
   const CUtensorMap* tml = &p.tm_l[prob];
   const CUtensorMap* tmr = &p.tm_r[prob];
 
@@ -294,13 +325,16 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
         if (!ptx::mbar_wait(empty(s), ph ^ 1u, p.status, abort_flag)) break;
         ptx::mbar_arrive_expect_tx(full(s), A_BYTES + r_bytes);
         const uint32_t ad = ptx::smem_u32(as + s * A_BYTES);
-        ptx::tma_load_2d(ad, tml, full(s), p0, ks * BK);
-        ptx::tma_load_2d(ad + A_BYTES / 2, tml, full(s), p0 + 64, ks * BK);
-        ptx::tma_load_2d(ptx::smem_u32(rs + s * R_BYTES), tmr, full(s), 0, ks * BK);
+        const int m = row_begin + ks * BK;
+        ptx::tma_load_2d(ad, tml, full(s), p0, m);
+        ptx::tma_load_2d(ad + A_BYTES / 2, tml, full(s), p0 + 64, m);
+        ptx::tma_load_2d(ptx::smem_u32(rs + s * R_BYTES), tmr, full(s), 0, m);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && ks1 > ks0) {
+    // the whole warp runs the loop: it zeroes the rows of a chunk that lie past the expert's
+    // last row (both operands) before lane 0 issues the MMAs
+    if (ks1 > ks0) {
       const uint32_t idesc = ptx::idesc_bf16(128, uint32_t(p.rpad), 1u, 1u);
       const uint32_t rsw = swz_mode_for_row_bytes(rowb);
       bool ok = true;
@@ -308,16 +342,33 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
         const int it = ks - ks0;
         const uint32_t s = it % NS, ph = (it / NS) & 1;
         if (!ptx::mbar_wait(full(s), ph, p.status, abort_flag)) { ok = false; break; }
-        ptx::tc_fence_after();
         const uint32_t a = ptx::smem_u32(as + s * A_BYTES), b = ptx::smem_u32(rs + s * R_BYTES);
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = ptx::smem_desc(a + kk * 2048, 8192, 1024, ptx::kSw128);
-          const uint64_t bd = ptx::smem_desc(b + kk * 16 * rowb, 64 * rowb, 8 * rowb, rsw);
-          ptx::mma_bf16(tmem, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+        const int valid = row_end - (row_begin + ks * BK);
+        if (valid < BK) {
+          // L tile: 2 blocks x 64 rows x 128 B; R tile: 64 rows x rowb bytes
+          for (int idx = lane; idx < (BK - valid) * 16; idx += 32) {
+            const int rr = valid + idx / 16, c = idx % 16;
+            ptx::st_shared_v4(a + (c / 8) * 8192 + rr * 128 + (c % 8) * 16, 0, 0, 0, 0);
+          }
+          for (int idx = lane; idx < (BK - valid) * int(rowb / 16); idx += 32) {
+            const int rr = valid + idx / int(rowb / 16), c = idx % int(rowb / 16);
+            ptx::st_shared_v4(b + rr * rowb + c * 16, 0, 0, 0, 0);
+          }
+          ptx::fence_proxy_async_smem();
         }
-        ptx::mma_commit(empty(s));
+        __syncwarp();
+        if (lane == 0) {
+          ptx::tc_fence_after();
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = ptx::smem_desc(a + kk * 2048, 8192, 1024, ptx::kSw128);
+            const uint64_t bd = ptx::smem_desc(b + kk * 16 * rowb, 64 * rowb, 8 * rowb, rsw);
+            ptx::mma_bf16(tmem, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+          }
+          ptx::mma_commit(empty(s));
+        }
+        __syncwarp();
       }
-      if (ok) ptx::mma_commit(acc_full);
+      if (ok && lane == 0) ptx::mma_commit(acc_full);
     }
   } else {
     const int q = warp & 3;
@@ -337,9 +388,11 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
       }
-      const int poff = prob ? p.P0 : 0;
-      if (split_reduce(acc, p.rpad, p.S, split, p.partial, size_t(p.P0 + p.P1), poff + prow,
-                       prow < P, p.counters + tile, last_flag, et) && prow < P) {
+      const int poff = e * (p.P0 + p.P1) + (prob ? p.P0 : 0);
+      if (split_reduce(acc, p.rpad, p.S, split, p.partial, size_t(p.E) * (p.P0 + p.P1),
+                       poff + prow, prow < P, p.counters + tile, last_flag, et) && prow < P) {
+        __nv_bfloat16* out0 = p.out0 + size_t(e) * p.P0 * p.r;
+        __nv_bfloat16* out1 = p.out1 + size_t(e) * p.r * p.P1;
         if (prob == 0) {
 #pragma unroll
           for (int c = 0; c < 64; c += 8) {
@@ -349,13 +402,13 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
               o.y = ptx::cvt_bf16x2(acc[c + 2] * p.s, acc[c + 3] * p.s);
               o.z = ptx::cvt_bf16x2(acc[c + 4] * p.s, acc[c + 5] * p.s);
               o.w = ptx::cvt_bf16x2(acc[c + 6] * p.s, acc[c + 7] * p.s);
-              *reinterpret_cast<uint4*>(p.out0 + size_t(prow) * p.r + c) = o;
+              *reinterpret_cast<uint4*>(out0 + size_t(prow) * p.r + c) = o;
             }
           }
         } else {
 #pragma unroll
           for (int c = 0; c < 64; ++c)
-            if (c < p.r) p.out1[size_t(c) * p.P1 + prow] = __float2bfloat16_rn(acc[c] * p.s);
+            if (c < p.r) out1[size_t(c) * p.P1 + prow] = __float2bfloat16_rn(acc[c] * p.s);
         }
       }
     }

@@ -310,3 +310,32 @@ def small_layer(fmt: str, M: int, N: int, K: int, r: int, s: float = 2.0, seed: 
     dY = to_bf16_bits(_normal(rng, (M, N), dy_std))
     return dict(fmt=fmt, M=M, N=N, K=K, r=r, s=s, codes=codes, scales=scales, tensor_scale=ts,
                 X=X, A=A, B=B, dY=dY)
+
+
+def small_grouped(fmt: str, counts, N: int, K: int, r: int, s: float = 2.0, seed: int = 0,
+                  b_std=0.01):
+    """A small seeded grouped (MoE) problem: expert e owns counts[e] consecutive rows of the packed
+    activations.  Expert e's weight is N(0, 0.02 * (1 + e % 3)) quantised, so NVFP4 experts get
+    different tensor scales.  Returns a dict with offsets int64 [E+1] and stacked arrays."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    E = len(counts)
+    offsets = np.zeros(E + 1, np.int64)
+    offsets[1:] = np.cumsum(np.asarray(counts, np.int64))
+    M = int(offsets[-1])
+    codes = np.empty((E, N, K // 2), np.uint8)
+    scales = None
+    ts = np.ones(E, np.float32)
+    for e in range(E):
+        c, sc, t = encode(fmt, _normal(rng, (N, K), 0.02 * (1 + e % 3)))
+        if scales is None:
+            scales = np.empty((E,) + sc.shape, sc.dtype)
+        codes[e], scales[e] = c, sc
+        if t is not None:
+            ts[e] = t
+    bound = 1.0 / math.sqrt(K)
+    A = to_bf16_bits(rng.uniform(-bound, bound, size=(E, r, K)).astype(np.float32))
+    B = to_bf16_bits(_normal(rng, (E, N, r), b_std))
+    X = to_bf16_bits(_normal(rng, (M, K), 1.0))
+    dY = to_bf16_bits(_normal(rng, (M, N), 1.0))
+    return dict(fmt=fmt, E=E, offsets=offsets, M=M, N=N, K=K, r=r, s=s, codes=codes,
+                scales=scales, tensor_scale=ts if fmt == "nvfp4" else None, X=X, A=A, B=B, dY=dY)

@@ -29,7 +29,8 @@
  *     gives up, the kernel records QLORA_ERR_DEVICE_TIMEOUT in the workspace and ends, and
  *     qlora_get_device_status() reports it.
  *   - Shape limits: K % 64 == 0, N % 16 == 0, K >= 64, N >= 16, M >= 0 (M == 0 is a no-op that
- *     still overwrites dA and dB with zeros), r in {8, 16, 32, 64}; every pointer 16-byte aligned.
+ *     still overwrites dA and dB with zeros), r in {8, 16, 32, 64}; every pointer 16-byte aligned
+ *     (with M == 0 the [M, ...] activation pointers may be NULL).  Grouped ops: 1 <= E <= 1024.
  *   - Outputs are overwritten, never accumulated (gradient accumulation across micro-batches is the
  *     caller's job).  Results are deterministic: the same inputs give bitwise-identical outputs.
  *   - Calls that share a workspace must be ordered on one stream.
