@@ -19,9 +19,13 @@ Layouts (row-major, K contiguous):
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
+from functools import lru_cache
 
 import numpy as np
+import torch
 
 FORMATS = ("nf4", "mxfp4", "nvfp4")
 FMT_ID = {"nf4": 0, "mxfp4": 1, "nvfp4": 2}
@@ -37,13 +41,23 @@ def rng_for(cfg: int, tensor: str, proj: int = 0) -> np.random.Generator:
 # bf16 bit patterns
 # ---------------------------------------------------------------------------------------------
 def to_bf16_bits(x) -> np.ndarray:
-    """float -> bf16 bit patterns (uint16), round to nearest even; NaN kept as a quiet NaN."""
+    """float -> bf16 bit patterns (uint16), round to nearest even; NaN kept as a quiet NaN.
+
+    Normal numbers, zeros and infinities go through torch's CPU conversion (round to nearest
+    even, multi-threaded); fp32 subnormals and NaNs, which a vectorised conversion may flush or
+    canonicalise, are rounded from their bit patterns here."""
     f = np.ascontiguousarray(x, dtype=np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    nan = np.isnan(f)
-    rounded = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
-    rounded[nan] = ((u[nan] >> 16) | 0x40).astype(np.uint16)
-    return rounded
+    out = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    out = out.reshape(f.shape)
+    a = np.abs(f)
+    odd = ~(a >= np.float32(1.17549435e-38)) & (f != 0)      # subnormal or NaN
+    if odd.any():
+        u = f.view(np.uint32)[odd].astype(np.uint64)
+        nan = np.isnan(f[odd])
+        r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+        r[nan] = ((u[nan] >> 16) | 0x40).astype(np.uint16)
+        out[odd] = r
+    return out
 
 
 def bf16_bits_to_f32(h) -> np.ndarray:
@@ -59,6 +73,7 @@ def pack_nibbles(c: np.ndarray) -> np.ndarray:
 # ---------------------------------------------------------------------------------------------
 # Encoders (test-data quantisers; the layer never runs these)
 # ---------------------------------------------------------------------------------------------
+@lru_cache(maxsize=1)
 def _nf4_grid() -> np.ndarray:
     # The generator's own approximate NF4 grid (any grid gives valid codes).
     from scipy.special import ndtri
@@ -108,11 +123,38 @@ def _e4m3_code(v: np.ndarray) -> np.ndarray:
 
 
 def encode(fmt: str, W: np.ndarray):
-    """Quantise a float weight [N,K] -> (codes [N,K/2], scales, tensor_scale)."""
+    """Quantise a float weight [N,K] -> (codes [N,K/2], scales, tensor_scale).
+
+    Rows are independent given the (NVFP4) tensor scale, so row chunks are encoded on a thread
+    pool; the result does not depend on the chunking."""
     W = np.asarray(W, np.float32)
     N, K = W.shape
     bs = BLOCK[fmt]
     assert K % bs == 0
+    ts = None
+    if fmt == "nvfp4":
+        tmax = float(np.abs(W).max())
+        ts = np.float32(tmax / (6 * 448)) if tmax > 0 else np.float32(1.0)
+    codes = np.empty((N, K // 2), np.uint8)
+    scales = np.empty((N, K // bs), np.float32 if fmt == "nf4" else np.uint8)
+    step = max(1, min(N, (1 << 21) // K))
+
+    def run(n0):
+        n1 = min(N, n0 + step)
+        codes[n0:n1], scales[n0:n1] = _encode_rows(fmt, W[n0:n1], ts)
+
+    starts = range(0, N, step)
+    if len(starts) > 1:
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(run, starts))
+    else:
+        run(0)
+    return codes, scales, ts
+
+
+def _encode_rows(fmt: str, W: np.ndarray, ts):
+    N, K = W.shape
+    bs = BLOCK[fmt]
     Wb = W.reshape(N, K // bs, bs)
     amax = np.abs(Wb).max(axis=2)
     if fmt == "nf4":
@@ -123,23 +165,21 @@ def encode(fmt: str, W: np.ndarray):
         x = (Wb / safe).astype(np.float64)
         c = np.searchsorted(mids, x, side="left").astype(np.uint8)
         c[np.broadcast_to(absmax[:, :, None] == 0, c.shape)] = 7
-        return pack_nibbles(c.reshape(N, K)), absmax, None
+        return pack_nibbles(c.reshape(N, K)), absmax
     if fmt == "mxfp4":
         with np.errstate(divide="ignore"):
             e = np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 2 + 127
         e = np.where(amax > 0, np.clip(e, 0, 254), 0).astype(np.uint8)
         scale = np.exp2(e.astype(np.float64) - 127)[:, :, None]
         c = _e2m1_code(Wb / scale)
-        return pack_nibbles(c.reshape(N, K)), e, None
+        return pack_nibbles(c.reshape(N, K)), e
     # nvfp4
-    tmax = float(np.abs(W).max())
-    ts = np.float32(tmax / (6 * 448)) if tmax > 0 else np.float32(1.0)
     sb = _e4m3_code(amax / (6 * float(ts)))
     sval = _E4M3[sb.astype(np.int64)] * float(ts)
     safe = np.where(sval > 0, sval, 1.0)[:, :, None]
     c = _e2m1_code(Wb / safe)
     c[np.broadcast_to(sval[:, :, None] == 0, c.shape)] = 0
-    return pack_nibbles(c.reshape(N, K)), sb, np.float32(ts)
+    return pack_nibbles(c.reshape(N, K)), sb
 
 
 def random_stored_weight(fmt: str, N: int, K: int, rng: np.random.Generator,
