@@ -13,6 +13,7 @@
 #include "qlora_debug.cuh"
 #include "qlora_fused.cuh"
 #include "qlora_lora.cuh"
+#include "qlora_stream.cuh"
 
 namespace qlora {
 namespace {
@@ -84,8 +85,12 @@ CUtensorMapSwizzle swizzle_for_bytes(uint32_t b) {
 
 template <typename K>
 bool set_smem(K kernel, size_t bytes) {
+  // every kernel of the library asks for the largest shared-memory carveout, so that consecutive
+  // launches never make the SMs switch their L1 / shared-memory split
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(bytes)) == cudaSuccess;
+                              static_cast<int>(bytes)) == cudaSuccess &&
+         cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              cudaSharedmemCarveoutMaxShared) == cudaSuccess;
 }
 
 qlora_status_t check_weight(const qlora_weight_t* W) {
@@ -149,6 +154,41 @@ size_t down_partial_bytes(int64_t M, int64_t Kc, int r, int E, int sms) {
   return dp.S > 1 ? size_t(dp.S) * size_t(M) * size_t(rank_pad(r)) * 4 : 0;
 }
 
+// Short batches (M <= 256 rows, one weight) use the weight-streaming kernels: the flat space of
+// (256-column output tile, 64-deep step) iterations, plus one LoRA step per tile, cut into equal
+// contiguous ranges, one per CTA.
+struct StreamPlan {
+  int tiles, nk, iters, grid, segments;
+  long long lcm;
+  size_t partial_bytes;
+};
+
+bool use_stream(int64_t M, int E) { return E == 1 && M > 0 && M <= stream::kMaxRows; }
+
+StreamPlan stream_plan(int64_t N, int64_t K, int64_t M, bool dx, int sms) {
+  StreamPlan p{};
+  p.tiles = int(((dx ? K : N) + stream::BN - 1) / stream::BN);
+  p.nk = int(((dx ? N : K) + stream::BK - 1) / stream::BK);
+  const int64_t total = int64_t(p.tiles) * (p.nk + 1);
+  int64_t L = (total + sms - 1) / sms;
+  if (L < 2) L = 2;
+  p.iters = int(L);
+  p.grid = int((total + L - 1) / L);
+  const int64_t nk1 = p.nk + 1;
+  int64_t a = L, b = nk1;
+  while (b) { const int64_t t = a % b; a = b; b = t; }
+  p.lcm = L / a * nk1;
+  p.segments = int(p.grid + p.tiles - (total + p.lcm - 1) / p.lcm);
+  p.partial_bytes = size_t(p.segments) * size_t(M) * stream::BN * 4;
+  return p;
+}
+
+// The streaming path is taken when the batch is short and the workspace's partial region (all
+// of the workspace from its start) holds its fp32 partials; otherwise the tiled kernels run.
+bool stream_fits(const qlora_weight_t* W, int64_t M, int E, bool dx, size_t region) {
+  return use_stream(M, E) && stream_plan(W->N, W->K, M, dx, num_sms()).partial_bytes <= region;
+}
+
 struct WsLayout {
   size_t zs, t, u, partial, partial_bytes, total;
   int counters_needed;
@@ -174,6 +214,14 @@ WsLayout ws_layout(int64_t N, int64_t K, int64_t M, int r, bool bwd, int E, int 
     const int wc = E * (wp.tiles0 + wp.tiles1);
     if (wc > L.counters_needed) L.counters_needed = wc;
   }
+  if (use_stream(M, E)) {
+    const size_t sf = stream_plan(N, K, M, false, sms).partial_bytes;
+    pb = sf > pb ? sf : pb;
+    if (bwd) {
+      const size_t sd = stream_plan(N, K, M, true, sms).partial_bytes;
+      pb = sd > pb ? sd : pb;
+    }
+  }
   L.partial_bytes = align_up(pb, 256);
   off += L.partial_bytes;
   L.total = off;
@@ -186,12 +234,13 @@ int* ws_counters(void* ws) { return reinterpret_cast<int*>(static_cast<uint8_t*>
 // ---------------------------------------------------------------------------------- profiling
 enum Kind : int {
   kKindFusedFwd = 0, kKindFusedDx, kKindDownT, kKindDownU, kKindWgrad,
-  kKindGFusedFwd, kKindGFusedDx, kKindGDownT, kKindGDownU, kKindGWgrad, kNumKinds
+  kKindGFusedFwd, kKindGFusedDx, kKindGDownT, kKindGDownU, kKindGWgrad,
+  kKindStreamFwd, kKindStreamDx, kKindStreamReduce, kNumKinds
 };
 const char* const kKindNames[kNumKinds] = {
     "fused_fwd", "fused_dx", "lora_down_T", "lora_down_U", "lora_wgrad",
     "grouped_fused_fwd", "grouped_fused_dx", "grouped_lora_down_T", "grouped_lora_down_U",
-    "grouped_lora_wgrad"};
+    "grouped_lora_wgrad", "stream_fwd", "stream_dx", "stream_reduce"};
 constexpr int kMaxProfiled = 65536;
 
 std::atomic<int64_t> g_launches{0};
@@ -346,6 +395,87 @@ qlora_status_t launch_fused(const qlora_weight_t* W, bool dx, const void* act, c
   }
 }
 
+template <int FMT, bool DX, int MT>
+qlora_status_t launch_stream_t(const StreamParams& p, int grid, cudaStream_t st) {
+  const size_t smem = stream::smem_bytes(MT);
+  if (!set_smem(qlora_stream_gemm_kernel<FMT, DX, MT>, smem)) return QLORA_ERR_CUDA;
+  LaunchScope scope(DX ? kKindStreamDx : kKindStreamFwd, st);
+  qlora_stream_gemm_kernel<FMT, DX, MT><<<grid, stream::kThreads, smem, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// Short-batch path of the fused GEMM (same operands and result as launch_fused with one expert):
+// the streaming kernel writes fp32 partials into `partial`, the reduce kernel writes `out`.
+qlora_status_t launch_stream(const qlora_weight_t* W, bool dx, const void* act, const void* zs,
+                             const void* lora_up, void* out, int64_t M, int r, int* status,
+                             float* partial, size_t partial_bytes, cudaStream_t st) {
+  const int64_t N = W->N, K = W->K;
+  const int64_t Kc = dx ? N : K;
+  const StreamPlan sp = stream_plan(N, K, M, dx, num_sms());
+  if (sp.partial_bytes > partial_bytes) return QLORA_ERR_WORKSPACE;
+  StreamParams p{};
+  if (!tmap_2d(&p.tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, uint64_t(Kc), uint64_t(M),
+               uint64_t(Kc) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return QLORA_ERR_CUDA;
+  const bool okc = !dx
+      ? tmap_2d(&p.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, uint64_t(K / 2), uint64_t(N),
+                uint64_t(K / 2), 32, 128, CU_TENSOR_MAP_SWIZZLE_32B)
+      : tmap_2d(&p.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, uint64_t(K / 2), uint64_t(N),
+                uint64_t(K / 2), 64, 64, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (!okc) return QLORA_ERR_CUDA;
+  if (!tmap_2d(&p.tm_zs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, zs, uint64_t(r), uint64_t(M),
+               uint64_t(r) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return QLORA_ERR_CUDA;
+  p.scales = W->scales;
+  p.lora_up = static_cast<const __nv_bfloat16*>(lora_up);
+  p.partial = partial;
+  p.status = status;
+  p.M = int(M);
+  p.N = int(N);
+  p.K = int(K);
+  p.r = r;
+  p.num_k = sp.nk;
+  p.num_tiles = sp.tiles;
+  p.iters = sp.iters;
+  p.lcm = sp.lcm;
+  const int mt = M <= 128 ? 1 : 2;
+  qlora_status_t rc;
+  switch ((W->fmt * 2 + (dx ? 1 : 0)) * 2 + (mt - 1)) {
+    case 0: rc = launch_stream_t<kFmtNF4, false, 1>(p, sp.grid, st); break;
+    case 1: rc = launch_stream_t<kFmtNF4, false, 2>(p, sp.grid, st); break;
+    case 2: rc = launch_stream_t<kFmtNF4, true, 1>(p, sp.grid, st); break;
+    case 3: rc = launch_stream_t<kFmtNF4, true, 2>(p, sp.grid, st); break;
+    case 4: rc = launch_stream_t<kFmtMXFP4, false, 1>(p, sp.grid, st); break;
+    case 5: rc = launch_stream_t<kFmtMXFP4, false, 2>(p, sp.grid, st); break;
+    case 6: rc = launch_stream_t<kFmtMXFP4, true, 1>(p, sp.grid, st); break;
+    case 7: rc = launch_stream_t<kFmtMXFP4, true, 2>(p, sp.grid, st); break;
+    case 8: rc = launch_stream_t<kFmtNVFP4, false, 1>(p, sp.grid, st); break;
+    case 9: rc = launch_stream_t<kFmtNVFP4, false, 2>(p, sp.grid, st); break;
+    case 10: rc = launch_stream_t<kFmtNVFP4, true, 1>(p, sp.grid, st); break;
+    default: rc = launch_stream_t<kFmtNVFP4, true, 2>(p, sp.grid, st); break;
+  }
+  if (rc != QLORA_OK) return rc;
+  StreamReduceParams rp{};
+  rp.partial = partial;
+  rp.tensor_scale = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
+  rp.out = static_cast<__nv_bfloat16*>(out);
+  rp.M = int(M);
+  rp.ncols = int(dx ? K : N);
+  rp.num_tiles = sp.tiles;
+  rp.nk1 = sp.nk + 1;
+  rp.iters = sp.iters;
+  {
+    const long long total = (long long)sp.tiles * (sp.nk + 1);
+    rp.lcm = int(sp.lcm < total + 1 ? sp.lcm : total + 1);
+  }
+  rp.segments = sp.segments;
+  const int64_t threads = M * int64_t(sp.tiles) * (stream::BN / 4);
+  if (!set_smem(qlora_stream_reduce_kernel, 0)) return QLORA_ERR_CUDA;
+  LaunchScope scope(kKindStreamReduce, st);
+  qlora_stream_reduce_kernel<<<unsigned((threads + 255) / 256), 256, 0, st>>>(rp);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 // dB [E, N, r] = s dY_e^T T_e and dA [E, r, K] = s U_e^T X_e over each expert's rows.
 qlora_status_t launch_wgrad(const void* X, const void* dY, const void* T, const void* U, int64_t M,
                             int64_t N, int64_t K, int r, float s, void* dA, void* dB, void* ws,
@@ -473,6 +603,9 @@ qlora_status_t run_fwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
                                        reinterpret_cast<float*>(w + L.partial), L.partial_bytes,
                                        ws_counters(ws), offsets, E, grouped, s);
   if (st != QLORA_OK) return st;
+  if (stream_fits(W, M, E, false, ws_bytes - L.partial))
+    return launch_stream(W, false, X, Zs, B, Y, M, r, ws_status(ws),
+                         reinterpret_cast<float*>(w + L.partial), ws_bytes - L.partial, s);
   return launch_fused(W, false, X, Zs, B, Y, M, r, ws_status(ws), offsets, E, grouped, s);
 }
 
@@ -509,7 +642,10 @@ qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
                         L.partial_bytes, ws_counters(ws), offsets, E, grouped, s);
   if (st != QLORA_OK) return st;
   if (dX) {
-    st = launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), offsets, E, grouped, s);
+    st = stream_fits(W, M, E, true, ws_bytes - L.partial)
+             ? launch_stream(W, true, dY, Zs, A, dX, M, r, ws_status(ws), part, ws_bytes - L.partial, s)
+                          : launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), offsets, E,
+                                         grouped, s);
     if (st != QLORA_OK) return st;
   }
   return launch_wgrad(X, dY, T, U, M, W->N, W->K, r, scale, dA, dB, ws, L, offsets, E, grouped, s);

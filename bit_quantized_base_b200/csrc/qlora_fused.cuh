@@ -105,6 +105,26 @@ __device__ __forceinline__ ItemScale load_item_scale(const void* scales, int n, 
   return s;
 }
 
+// The 4-byte word of the scale array that holds the block-scale material of the item starting at
+// element (n, kcol), and the right shift that brings it to the low bits (for an asynchronous
+// 4-byte copy into shared memory): NF4 the fp32 absmax; MXFP4 the two E8M0 bytes (2-byte
+// aligned, so the word is the aligned one around them); NVFP4 the four E4M3 bytes.
+template <int FMT>
+__device__ __forceinline__ const void* item_scale_word(const void* scales, int n, int kcol, int K,
+                                                       size_t nrow0, uint32_t& shift) {
+  const size_t row = nrow0 + size_t(n);
+  shift = 0;
+  if constexpr (FMT == kFmtNF4) {
+    return reinterpret_cast<const uint32_t*>(scales) + row * (K / 64) + kcol / 64;
+  } else if constexpr (FMT == kFmtMXFP4) {
+    const size_t off = row * (K / 32) + kcol / 32;
+    shift = uint32_t(off & 2u) * 8u;
+    return reinterpret_cast<const uint8_t*>(scales) + (off & ~size_t(3));
+  } else {
+    return reinterpret_cast<const uint8_t*>(scales) + row * (K / 16) + kcol / 16;
+  }
+}
+
 // Pair tile t of a (grouped) launch: expert e, rows [row0, row0 + 256) of which rows below
 // row_end belong to the expert, output-column tile nt.
 struct PairTile {

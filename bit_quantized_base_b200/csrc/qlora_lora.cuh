@@ -45,14 +45,15 @@ __device__ __forceinline__ uint32_t swz_mode_for_row_bytes(uint32_t rowb) {
 }
 
 // Epilogue of a split tile, run by the 128 epilogue threads (named barrier 1).  acc holds this
-// thread's accumulator row (rpad fp32 values).  With S > 1 the row is stored as partial `split`
-// at partial + (split * rows_total + row) * rpad; the last CTA of the tile (counter) then replaces
-// acc with the sum over splits 0..S-1 and returns true; other CTAs return false.  With S == 1 it
-// returns true with acc unchanged.  All 128 threads must call it (rows outside the problem pass
-// row_ok = false and take part in the barriers only).
-__device__ __forceinline__ bool split_reduce(float (&acc)[64], int rpad, int S, int split,
-                                            float* partial, size_t rows_total, int row, bool row_ok,
-                                            int* counter, volatile int* last_flag, int et) {
+// thread's accumulator row (rpad fp32 values); with S > 1 it is stored as partial `split` at
+// partial + (split * rows_total + row) * rpad and the tile's counter is incremented.  Returns true
+// in the last CTA of the tile to arrive (which then calls split_sum; the counter is reset for the
+// next call), and true with S == 1 (nothing stored: the caller writes acc directly).  All 128
+// threads must call it (rows outside the problem pass row_ok = false and take part in the
+// barriers only).
+__device__ __forceinline__ bool split_arrive(const float (&acc)[64], int rpad, int S, int split,
+                                             float* partial, size_t rows_total, int row, bool row_ok,
+                                             int* counter, volatile int* last_flag, int et) {
   if (S == 1) return true;
   if (row_ok) {
     float* dst = partial + (size_t(split) * rows_total + size_t(row)) * rpad;
@@ -67,26 +68,46 @@ __device__ __forceinline__ bool split_reduce(float (&acc)[64], int rpad, int S, 
     *last_flag = (old == S - 1) ? 1 : 0;
   }
   asm volatile("bar.sync 1, 128;" ::: "memory");
-  if (!*last_flag) return false;
-  __threadfence();
-  if (row_ok) {
-#pragma unroll
-    for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
-    for (int sp = 0; sp < S; ++sp) {
-      const float* src = partial + (size_t(sp) * rows_total + size_t(row)) * rpad;
-      float4 v[16];
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        if (4 * c < rpad) v[c] = __ldcg(reinterpret_cast<const float4*>(src + 4 * c));
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        if (4 * c < rpad) {
-          acc[4 * c] += v[c].x; acc[4 * c + 1] += v[c].y; acc[4 * c + 2] += v[c].z; acc[4 * c + 3] += v[c].w;
-        }
-    }
+  const bool last = *last_flag != 0;
+  if (last) {
+    __threadfence();
+    if (et == 0) *counter = 0;   // ready for the next call on this workspace
   }
-  if (et == 0) *counter = 0;   // ready for the next call on this workspace
-  return true;
+  return last;
+}
+
+// In the last CTA of a split tile: the 128 epilogue threads share out the (row, 8-column chunk)
+// items of rows [row0, row0 + nrows); each adds the S partials of its item in split order
+// 0..S-1 (loads issued four splits at a time) and hands the sum to write(row, c0, v[8]).
+template <class F>
+__device__ __forceinline__ void split_sum(int rpad, int S, const float* partial, size_t rows_total,
+                                          int row0, int nrows, int et, F&& write) {
+  const int chunks = rpad / 8;
+  const int items = nrows * chunks;
+  const size_t sstride = rows_total * size_t(rpad);
+  for (int it = et; it < items; it += 128) {
+    const int rr = it / chunks, c0 = (it - rr * chunks) * 8;
+    const float* src = partial + size_t(row0 + rr) * rpad + c0;
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int sp = 0; sp < S; sp += 4) {
+      float4 a[4], b[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (sp + u < S) {
+          a[u] = __ldcg(reinterpret_cast<const float4*>(src + size_t(sp + u) * sstride));
+          b[u] = __ldcg(reinterpret_cast<const float4*>(src + size_t(sp + u) * sstride + 4));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (sp + u < S) {
+          v[0] += a[u].x; v[1] += a[u].y; v[2] += a[u].z; v[3] += a[u].w;
+          v[4] += b[u].x; v[5] += b[u].y; v[6] += b[u].z; v[7] += b[u].w;
+        }
+      }
+    }
+    write(row0 + rr, c0, v);
+  }
 }
 
 // Load this thread's accumulator row (rpad columns) from tensor memory.
@@ -221,24 +242,34 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
         for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
       }
       const bool row_ok = row < row_end;
-      if (split_reduce(acc, p.rpad, p.S, split, p.partial, size_t(p.M), row, row_ok,
-                       p.counters + tile, last_flag, et) && row_ok) {
-        const float ts = p.tensor_scale ? __ldg(p.tensor_scale + e) : 1.0f;
-        const float zscale = p.s / ts;
+      const float ts = p.tensor_scale ? __ldg(p.tensor_scale + e) : 1.0f;
+      const float zscale = p.s / ts;
+      // Z and Zs = bf16(Z * s / ts) for columns c .. c+7 of row rw
+      auto write8 = [&](int rw, int c, const float (&v)[8]) {
+        if (c >= p.r) return;
+        uint4 z, zs;
+        z.x = ptx::cvt_bf16x2(v[0], v[1]); z.y = ptx::cvt_bf16x2(v[2], v[3]);
+        z.z = ptx::cvt_bf16x2(v[4], v[5]); z.w = ptx::cvt_bf16x2(v[6], v[7]);
+        zs.x = ptx::cvt_bf16x2(v[0] * zscale, v[1] * zscale);
+        zs.y = ptx::cvt_bf16x2(v[2] * zscale, v[3] * zscale);
+        zs.z = ptx::cvt_bf16x2(v[4] * zscale, v[5] * zscale);
+        zs.w = ptx::cvt_bf16x2(v[6] * zscale, v[7] * zscale);
+        *reinterpret_cast<uint4*>(p.z + size_t(rw) * p.r + c) = z;
+        *reinterpret_cast<uint4*>(p.zs + size_t(rw) * p.r + c) = zs;
+      };
+      if (p.S == 1) {
+        if (row_ok) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 8) {
-          if (c < p.r) {
-            uint4 z, zs;
-            z.x = ptx::cvt_bf16x2(acc[c], acc[c + 1]); z.y = ptx::cvt_bf16x2(acc[c + 2], acc[c + 3]);
-            z.z = ptx::cvt_bf16x2(acc[c + 4], acc[c + 5]); z.w = ptx::cvt_bf16x2(acc[c + 6], acc[c + 7]);
-            zs.x = ptx::cvt_bf16x2(acc[c] * zscale, acc[c + 1] * zscale);
-            zs.y = ptx::cvt_bf16x2(acc[c + 2] * zscale, acc[c + 3] * zscale);
-            zs.z = ptx::cvt_bf16x2(acc[c + 4] * zscale, acc[c + 5] * zscale);
-            zs.w = ptx::cvt_bf16x2(acc[c + 6] * zscale, acc[c + 7] * zscale);
-            *reinterpret_cast<uint4*>(p.z + size_t(row) * p.r + c) = z;
-            *reinterpret_cast<uint4*>(p.zs + size_t(row) * p.r + c) = zs;
+          for (int c = 0; c < 64; c += 8) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = acc[c + u];
+            write8(row, c, v);
           }
         }
+      } else if (split_arrive(acc, p.rpad, p.S, split, p.partial, size_t(p.M), row, row_ok,
+                              p.counters + tile, last_flag, et)) {
+        split_sum(p.rpad, p.S, p.partial, size_t(p.M), m0, min(BM, row_end - m0), et, write8);
       }
     }
   }
@@ -389,27 +420,38 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
         for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
       }
       const int poff = e * (p.P0 + p.P1) + (prob ? p.P0 : 0);
-      if (split_reduce(acc, p.rpad, p.S, split, p.partial, size_t(p.E) * (p.P0 + p.P1),
-                       poff + prow, prow < P, p.counters + tile, last_flag, et) && prow < P) {
-        __nv_bfloat16* out0 = p.out0 + size_t(e) * p.P0 * p.r;
-        __nv_bfloat16* out1 = p.out1 + size_t(e) * p.r * p.P1;
+      __nv_bfloat16* out0 = p.out0 + size_t(e) * p.P0 * p.r;
+      __nv_bfloat16* out1 = p.out1 + size_t(e) * p.r * p.P1;
+      // s * the reduction for columns c .. c+7 of output row pr (dB row-major, dA transposed)
+      auto write8 = [&](int pr, int c, const float (&v)[8]) {
+        if (c >= p.r) return;
         if (prob == 0) {
-#pragma unroll
-          for (int c = 0; c < 64; c += 8) {
-            if (c < p.r) {
-              uint4 o;
-              o.x = ptx::cvt_bf16x2(acc[c] * p.s, acc[c + 1] * p.s);
-              o.y = ptx::cvt_bf16x2(acc[c + 2] * p.s, acc[c + 3] * p.s);
-              o.z = ptx::cvt_bf16x2(acc[c + 4] * p.s, acc[c + 5] * p.s);
-              o.w = ptx::cvt_bf16x2(acc[c + 6] * p.s, acc[c + 7] * p.s);
-              *reinterpret_cast<uint4*>(out0 + size_t(prow) * p.r + c) = o;
-            }
-          }
+          uint4 o;
+          o.x = ptx::cvt_bf16x2(v[0] * p.s, v[1] * p.s);
+          o.y = ptx::cvt_bf16x2(v[2] * p.s, v[3] * p.s);
+          o.z = ptx::cvt_bf16x2(v[4] * p.s, v[5] * p.s);
+          o.w = ptx::cvt_bf16x2(v[6] * p.s, v[7] * p.s);
+          *reinterpret_cast<uint4*>(out0 + size_t(pr) * p.r + c) = o;
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c < p.r) out1[size_t(c) * p.P1 + prow] = __float2bfloat16_rn(acc[c] * p.s);
+          for (int u = 0; u < 8; ++u) out1[size_t(c + u) * p.P1 + pr] = __float2bfloat16_rn(v[u] * p.s);
         }
+      };
+      if (p.S == 1) {
+        if (prow < P) {
+#pragma unroll
+          for (int c = 0; c < 64; c += 8) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = acc[c + u];
+            write8(prow, c, v);
+          }
+        }
+      } else if (split_arrive(acc, p.rpad, p.S, split, p.partial, size_t(p.E) * (p.P0 + p.P1),
+                              poff + prow, prow < P, p.counters + tile, last_flag, et)) {
+        split_sum(p.rpad, p.S, p.partial, size_t(p.E) * (p.P0 + p.P1), poff + p0,
+                  min(BM, P - p0), et,
+                  [&](int prw, int c, const float (&v)[8]) { write8(prw - poff, c, v); });
       }
     }
   }

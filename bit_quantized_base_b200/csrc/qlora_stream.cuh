@@ -1,0 +1,433 @@
+// qlora_stream.cuh -- the dequant-GEMM for short batches (M <= 256 rows): weight streaming.
+//
+//   forward : Y  = ( X  deq(W)^T + (s/ts) T B^T ) * ts     contraction over K, tiles over N
+//   backward: dX = ( dY deq(W)   + (s/ts) U A   ) * ts     contraction over N, tiles over K
+//
+// With few rows the layer is a stream over the 4-bit weight: every weight element is decoded once
+// and meets only M activation rows, so the work is the decode, not the tensor-core math.  The
+// pair-tiled kernel (qlora_fused.cuh) would give such a batch one tile row, ceil(N/256) tiles, and
+// leave most SMs idle; here the whole (output tile, contraction step) iteration space is instead
+// cut into equal contiguous ranges, one per CTA (one CTA per SM), so every SM decodes the same
+// number of weight elements.  A range may start or end inside an output tile; each piece of a tile
+// (a segment) is accumulated in tensor memory and stored as an fp32 partial, and a second small
+// kernel adds the partials of each tile in range order (a fixed order: results are deterministic),
+// applies the NVFP4 tensor scale and writes bf16.
+//
+// A tile is 256 output columns (two 128-column weight halves, each decoded exactly as one CTA's
+// half in the pair kernel) by all M rows: one tcgen05.mma (cta_group::1) of M=128, N=256 per
+// 16-deep step and 128-row block of activations (one block for M <= 128, two for M <= 256, sharing
+// the decoded weight).  The LoRA term is one extra step per tile (operands Zs and rows of B or A),
+// as in the pair kernel.
+//
+// Warp roles (480 threads, one CTA per SM):
+//   warps 0-3   epilogue: tensor memory -> fp32 partial (global, L2-resident)
+//   warp  4     TMA producer of the activation blocks (and Zs for the LoRA step)
+//   warp  5     TMA producer of the packed-code tiles, on its own deeper ring
+//   warp  6     tensor-memory allocation and the single MMA-issuing thread
+//   warps 7-14  dequant: two groups of 4 warps taking alternate steps; thread tg of a group
+//               decodes 64-element item tg of both 128-column weight halves of its step (a row of
+//               the forward tile, or a row x column chunk of the dX tile); block scales are copied
+//               asynchronously into a shared ring four own steps ahead of their use
+#pragma once
+#include <cuda_bf16.h>
+#include "qlora_ptx.cuh"
+#include "qlora_dequant.cuh"
+#include "qlora_fused.cuh"
+
+namespace qlora {
+namespace stream {
+constexpr int BN = 256, HN = 128, BK = 64;
+constexpr int X_BYTES = 128 * BK * 2;     // one 128-row activation block: 16 KB
+constexpr int W_BYTES = BN * BK * 2;      // 32 KB (two 16 KB halves)
+constexpr int HW_BYTES = HN * BK * 2;     // 16 KB
+constexpr int C_BYTES = BN * BK / 2;      // 8 KB of packed codes (two 4 KB halves)
+constexpr int HC_BYTES = HN * BK / 2;
+constexpr int NC = 6;                     // code stages
+constexpr int kEpiWarps = 4, kTmaWarp = 4, kCodeWarp = 5, kMmaWarp = 6, kDqWarp0 = 7, kDqWarps = 8;
+constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;
+constexpr int kTmemCols = 512;
+constexpr int kMaxRows = 256;
+constexpr int SCALE_RING_BYTES = 4 * 2 * 256 * 4;   // kPf slots x 2 halves x 256 threads
+// operand stages: MT activation blocks + one weight tile
+__host__ __device__ constexpr int num_stages(int MT) { return MT == 1 ? 3 : 2; }
+__host__ __device__ constexpr size_t stage_bytes(int MT) { return size_t(MT) * X_BYTES + W_BYTES; }
+__host__ __device__ constexpr size_t smem_bytes(int MT) {
+  return 1024 + size_t(num_stages(MT)) * stage_bytes(MT) + size_t(NC) * C_BYTES + SCALE_RING_BYTES + 1024;
+}
+}  // namespace stream
+
+struct StreamParams {
+  CUtensorMap tm_act;    // activations [M, Kc] bf16, box {64, 128}, SW128
+  CUtensorMap tm_codes;  // codes [N, K/2] u8, per weight half: fwd box {32, 128} SW32; dX box {64, 64} SW64
+  CUtensorMap tm_zs;     // Zs [M, r] bf16, box {64, 128}, SW128
+  const void* scales;                // [N, K/bs]
+  const __nv_bfloat16* lora_up;      // fwd: B [N, r]; dX: A [r, K]
+  float* partial;                    // [segments][M][256] fp32
+  int* status;
+  int M, N, K, r;
+  int num_k;                         // contraction steps of 64 (the LoRA step comes after them)
+  int num_tiles;                     // 256-column output tiles
+  int iters;                         // L: (tile, step) iterations per CTA
+  long long lcm;                     // lcm(L, num_k + 1)
+};
+
+// Segments are the pieces of the iteration space between consecutive CTA-range starts (multiples
+// of L) and tile starts (multiples of nk1); a segment's index is the number of such starts below
+// its own start `st` (multiples of both counted once).
+__device__ __forceinline__ int stream_segment(long long st, int L, int nk1, long long lcm) {
+  return int((st + L - 1) / L + (st + nk1 - 1) / nk1 - (st + lcm - 1) / lcm);
+}
+
+// Segment bookkeeping shared by the producer, MMA and epilogue roles: iteration g of the flat
+// (tile, step) space is tile g / (num_k + 1), step g % (num_k + 1).
+struct StreamRange {
+  int g0, g1, nk1;
+  __device__ __forceinline__ int tile(int g) const { return g / nk1; }
+  __device__ __forceinline__ int step(int g) const { return g - (g / nk1) * nk1; }
+  __device__ __forceinline__ bool seg_end(int g) const { return g + 1 == g1 || step(g) == nk1 - 1; }
+};
+
+template <int FMT, bool DX, int MT>
+__global__ void __launch_bounds__(stream::kThreads, 1)
+qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
+  using namespace stream;
+  constexpr int NS = num_stages(MT);
+  constexpr uint32_t STAGE = uint32_t(stage_bytes(MT));
+  constexpr int NB = MT == 1 ? 2 : 1;          // accumulator buffers
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stages = smem;                      // per stage: MT activation blocks, then the weight tile
+  uint8_t* cs = stages + NS * STAGE;
+  uint8_t* scr = cs + NC * C_BYTES;            // scale ring: kPf slots x 2 halves x 256 threads x 4 B
+  uint64_t* bars = reinterpret_cast<uint64_t*>(scr + SCALE_RING_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 2 * NC + 2 * NB);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t b0 = ptx::smem_u32(bars);
+  auto full_s = [&](uint32_t s) { return b0 + 8u * s; };
+  auto empty_s = [&](uint32_t s) { return b0 + 8u * (NS + s); };
+  auto full_c = [&](uint32_t s) { return b0 + 8u * (2 * NS + s); };
+  auto empty_c = [&](uint32_t s) { return b0 + 8u * (2 * NS + NC + s); };
+  auto acc_full = [&](uint32_t b) { return b0 + 8u * (2 * NS + 2 * NC + b); };
+  auto acc_empty = [&](uint32_t b) { return b0 + 8u * (2 * NS + 2 * NC + NB + b); };
+  auto xs = [&](uint32_t s) { return ptx::smem_u32(stages) + s * STAGE; };
+  auto wsm = [&](uint32_t s) { return ptx::smem_u32(stages) + s * STAGE + MT * X_BYTES; };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = p.num_k;
+  const int total = p.num_tiles * (nk + 1);
+  StreamRange rg;
+  rg.nk1 = nk + 1;
+  rg.g0 = int(blockIdx.x) * p.iters;
+  rg.g1 = min(rg.g0 + p.iters, total);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      ptx::mbar_init(full_s(s), 1 + kDqWarps / 2);   // producer's expect-tx arrive + one dequant group
+      ptx::mbar_init(empty_s(s), 1);
+    }
+    for (int s = 0; s < NC; ++s) { ptx::mbar_init(full_c(s), 1); ptx::mbar_init(empty_c(s), kDqWarps / 2); }
+    for (int b = 0; b < NB; ++b) { ptx::mbar_init(acc_full(b), 1); ptx::mbar_init(acc_empty(b), kEpiWarps); }
+    *abort_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  if (warp == kTmaWarp && lane == 0) {
+    ptx::prefetch_tmap(&p.tm_act);
+    ptx::prefetch_tmap(&p.tm_zs);
+  }
+  if (warp == kCodeWarp && lane == 0) ptx::prefetch_tmap(&p.tm_codes);
+  if (warp == kMmaWarp) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------------ activation producer
+    if (lane == 0) {
+      for (int g = rg.g0; g < rg.g1; ++g) {
+        const uint32_t i = uint32_t(g - rg.g0), s = i % NS;
+        if (!ptx::mbar_wait(empty_s(s), ((i / NS) & 1u) ^ 1u, p.status, abort_flag)) break;
+        ptx::mbar_arrive_expect_tx(full_s(s), MT * X_BYTES);
+        const int ks = rg.step(g);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          if (ks < nk) ptx::tma_load_2d(xs(s) + mt * X_BYTES, &p.tm_act, full_s(s), ks * BK, mt * 128);
+          else ptx::tma_load_2d(xs(s) + mt * X_BYTES, &p.tm_zs, full_s(s), 0, mt * 128);
+        }
+      }
+    }
+  } else if (warp == kCodeWarp) {
+    // ------------------------------------------------------------------ code producer
+    if (lane == 0) {
+      uint32_t j = 0;
+      for (int g = rg.g0; g < rg.g1; ++g) {
+        const int ks = rg.step(g);
+        if (ks == nk) continue;
+        const uint32_t sc = j % NC;
+        if (!ptx::mbar_wait(empty_c(sc), ((j / NC) & 1u) ^ 1u, p.status, abort_flag)) break;
+        ptx::mbar_arrive_expect_tx(full_c(sc), C_BYTES);
+        const uint32_t cd = ptx::smem_u32(cs + sc * C_BYTES);
+        const int c0 = rg.tile(g) * BN;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (!DX) ptx::tma_load_2d(cd + h * HC_BYTES, &p.tm_codes, full_c(sc), ks * (BK / 2), c0 + h * HN);
+          else ptx::tma_load_2d(cd + h * HC_BYTES, &p.tm_codes, full_c(sc), (c0 + h * HN) / 2, ks * BK);
+        }
+        ++j;
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = ptx::idesc_bf16(128, BN, 0, DX ? 1u : 0u);
+      const int lora_kk = (p.r + 15) / 16;
+      uint32_t seg = 0;
+      bool first = true;
+      for (int g = rg.g0; g < rg.g1; ++g) {
+        const uint32_t i = uint32_t(g - rg.g0), s = i % NS;
+        const uint32_t b = seg % NB;
+        if (first) {
+          if (!ptx::mbar_wait(acc_empty(b), ((seg / NB) & 1u) ^ 1u, p.status, abort_flag)) break;
+          ptx::tc_fence_after();
+        }
+        if (!ptx::mbar_wait(full_s(s), (i / NS) & 1u, p.status, abort_flag)) break;
+        ptx::tc_fence_after();
+        const int ks = rg.step(g);
+        const int nkk = ks < nk ? BK / 16 : lora_kk;
+        const uint32_t xa = xs(s), wb = wsm(s);
+        for (int kk = 0; kk < nkk; ++kk) {
+          const uint64_t bd = DX ? ptx::smem_desc(wb + kk * 2048, 8192, 1024, ptx::kSw128)
+                                 : ptx::smem_desc(wb + kk * 32, 16, 1024, ptx::kSw128);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            const uint64_t ad = ptx::smem_desc(xa + mt * X_BYTES + kk * 32, 16, 1024, ptx::kSw128);
+            const uint32_t d = tmem + uint32_t(MT == 1 ? b * BN : mt * BN);
+            ptx::mma_bf16(d, ad, bd, idesc, (!first || kk > 0) ? 1u : 0u);
+          }
+        }
+        ptx::mma_commit(empty_s(s));
+        first = false;
+        if (rg.seg_end(g)) {
+          ptx::mma_commit(acc_full(b));
+          ++seg;
+          first = true;
+        }
+      }
+    }
+  } else if (warp < kEpiWarps) {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp;   // tensor-memory lanes 32q .. 32q+31
+    uint32_t seg = 0;
+    for (int g = rg.g0; g < rg.g1; ++g) {
+      if (!rg.seg_end(g)) continue;
+      const uint32_t b = seg % NB;
+      if (!ptx::mbar_wait(acc_full(b), (seg / NB) & 1u, p.status, abort_flag)) break;
+      ptx::tc_fence_after();
+      const long long st = max((long long)rg.g0, (long long)rg.tile(g) * rg.nk1);
+      float* base = p.partial + size_t(stream_segment(st, p.iters, rg.nk1, p.lcm)) * size_t(p.M) * BN;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const int row = mt * 128 + q * 32 + lane;
+#pragma unroll 1
+        for (int cb = 0; cb < BN / 32; ++cb) {
+          uint32_t v[32];
+          ptx::tmem_ld_32x32b_x32(tmem + (uint32_t(q * 32) << 16) + uint32_t(MT == 1 ? b * BN : mt * BN) + cb * 32, v);
+          ptx::tmem_ld_wait();
+          if (row < p.M) {
+            float4* dst = reinterpret_cast<float4*>(base + size_t(row) * BN + cb * 32);
+#pragma unroll
+            for (int g4 = 0; g4 < 8; ++g4)
+              __stcg(dst + g4, make_float4(__uint_as_float(v[4 * g4]), __uint_as_float(v[4 * g4 + 1]),
+                                           __uint_as_float(v[4 * g4 + 2]), __uint_as_float(v[4 * g4 + 3])));
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(acc_empty(b));
+      ++seg;
+    }
+  } else {
+    // ------------------------------------------------------------------ dequant
+    // Two groups of 4 warps take alternate steps, so one group's barrier waits and bookkeeping
+    // overlap the other's decode; thread tg of a group decodes item tg of both weight halves.
+    const int dt = threadIdx.x - kDqWarp0 * 32;   // 0..255
+    const int grp = dt >> 7;
+    const ItemGeom<DX> geo(dt & 127);
+    // Block scales travel global -> shared by per-thread 4-byte asynchronous copies issued kPf own
+    // steps ahead of their use (one copy group per own step, empty for steps without a scale), so
+    // the decode never waits on a global load.  Positions advance incrementally (no divisions on
+    // the decode path).
+    constexpr int kPf = 4;
+    const uint32_t sring = ptx::smem_u32(scr) + uint32_t(dt) * 4u;   // (slot, half) at + (2 slot + half) * 1024
+    struct Cursor {
+      int g, t, ks;
+      uint32_t i, j;   // step index within the range; code-step index within the range
+    };
+    auto advance1 = [&](Cursor& c) {
+      if (c.ks < nk) ++c.j;
+      ++c.g;
+      ++c.i;
+      if (++c.ks == rg.nk1) { c.ks = 0; ++c.t; }
+    };
+    auto advance2 = [&](Cursor& c) { advance1(c); advance1(c); };
+    // weight row n and first column kcol of this thread's item in weight half hh at cursor c
+    auto item_at = [&](const Cursor& c, int hh, int& n, int& kcol) {
+      const int h0 = c.t * BN + hh * HN;
+      n = DX ? c.ks * BK + geo.row : h0 + geo.row;
+      kcol = DX ? h0 + geo.chunk * 64 : c.ks * BK;
+    };
+    auto scale_fetch = [&](const Cursor& c, uint32_t slot, uint32_t dep) {
+      if (c.g < rg.g1 && c.ks < nk) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          int n, kcol;
+          item_at(c, hh, n, kcol);
+          uint32_t sh;
+          if (n < p.N && kcol < p.K)
+            ptx::cp_async_4(sring + (2u * slot + hh) * 1024u + dep,
+                            item_scale_word<FMT>(p.scales, n, kcol, p.K, 0, sh));
+        }
+      }
+      ptx::cp_async_commit();
+    };
+    Cursor cur{rg.g0, rg.g0 / rg.nk1, rg.g0 - (rg.g0 / rg.nk1) * rg.nk1, 0u, 0u};
+    if (grp) advance1(cur);
+    Cursor pf = cur;
+#pragma unroll
+    for (int d = 0; d < kPf; ++d) {
+      scale_fetch(pf, uint32_t(d), 0u);
+      advance2(pf);
+    }
+    uint32_t slot = 0;
+    for (; cur.g < rg.g1; advance2(cur), advance2(pf)) {
+      ptx::cp_async_wait<kPf - 1>();
+      const uint32_t s = cur.i % NS, pw = (cur.i / NS) & 1u;
+      uint32_t sdep = 0;   // zero, but only once the slot has been read: orders the refill after it
+      bool ok = true;
+      if (cur.ks < nk) {
+        const uint32_t scs = cur.j % NC;
+        if (!ptx::mbar_wait(full_c(scs), (cur.j / NC) & 1u, p.status, abort_flag)) break;
+        uint32_t used = 0;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          int n, kcol;
+          item_at(cur, hh, n, kcol);
+          uint32_t sh = 0;
+          if (FMT == kFmtMXFP4) item_scale_word<FMT>(p.scales, n, kcol, p.K, 0, sh);
+          ItemScale sc;
+          sc.raw = ptx::ld_shared_u32(sring + (2u * slot + hh) * 1024u) >> sh;
+          sdep |= sc.raw;
+          const uint32_t cb = ptx::smem_u32(cs + scs * C_BYTES) + hh * HC_BYTES;
+          const uint4 c_lo = ptx::ld_shared_v4(cb + geo.code_off(0));
+          const uint4 c_hi = ptx::ld_shared_v4(cb + geo.code_off(1));
+          const uint32_t cw[8] = {c_lo.x, c_lo.y, c_lo.z, c_lo.w, c_hi.x, c_hi.y, c_hi.z, c_hi.w};
+          if (hh == 0 && !ptx::mbar_wait(empty_s(s), pw ^ 1u, p.status, abort_flag)) { ok = false; break; }
+          const uint32_t rb = geo.op_row_base(wsm(s) + hh * HW_BYTES);
+          if (n < p.N && kcol < p.K) dequant_item_store<FMT>(cw, sc, rb, geo.swz());
+          else zero_item_store(rb);
+          used ^= (c_lo.x ^ c_lo.y ^ c_lo.z ^ c_lo.w) ^ (c_hi.x ^ c_hi.y ^ c_hi.z ^ c_hi.w);
+        }
+        if (!ok) break;
+        // release the code stage only once the loaded words have been consumed
+        uint32_t dep;
+        asm volatile("and.b32 %0, %1, 0;" : "=r"(dep) : "r"(used));
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(empty_c(scs) + dep);
+      } else {
+        // LoRA step: rows of B (forward, K-major) or of A (dX, MN-major), zero padded
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          const int h0 = cur.t * BN + hh * HN;
+          uint4 v[8];
+          if (!DX) {
+            const int n = h0 + geo.row;
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+              v[jj] = (n < p.N && jj * 8 < p.r)
+                          ? __ldg(reinterpret_cast<const uint4*>(p.lora_up + size_t(n) * p.r + jj * 8))
+                          : make_uint4(0, 0, 0, 0);
+          } else {
+            const int rj = geo.row, kc = h0 + geo.chunk * 64;
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+              v[jj] = (rj < p.r && kc < p.K)
+                          ? __ldg(reinterpret_cast<const uint4*>(p.lora_up + size_t(rj) * p.K + kc + jj * 8))
+                          : make_uint4(0, 0, 0, 0);
+          }
+          if (hh == 0 && !ptx::mbar_wait(empty_s(s), pw ^ 1u, p.status, abort_flag)) { ok = false; break; }
+          const uint32_t rb = geo.op_row_base(wsm(s) + hh * HW_BYTES);
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj)
+            ptx::st_shared_v4(rb + ((uint32_t(jj) ^ geo.swz()) << 4), v[jj].x, v[jj].y, v[jj].z, v[jj].w);
+        }
+        if (!ok) break;
+      }
+      asm volatile("and.b32 %0, %1, 0;" : "=r"(sdep) : "r"(sdep));
+      scale_fetch(pf, slot, sdep);
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(full_s(s));
+      slot = slot + 1 == kPf ? 0 : slot + 1;
+    }
+    ptx::cp_async_wait<0>();
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+// out[m, c] = bf16( ts * sum over the segments of tile c / 256, in range order ), for m < M and
+// c < ncols.  One thread per 4 consecutive columns of one row.  The segments of tile t are the
+// consecutive indices from the rank of its first iteration t * nk1 to the rank of (t+1) * nk1.
+struct StreamReduceParams {
+  const float* partial;
+  const float* tensor_scale;   // NVFP4: device float, else nullptr
+  __nv_bfloat16* out;          // [M, ncols]
+  int M, ncols, num_tiles, nk1, iters, lcm, segments;   // lcm clamped to at most total + 1
+};
+
+__device__ __forceinline__ int stream_rank32(int st, int L, int nk1, int lcm) {
+  return (st + L - 1) / L + (st + nk1 - 1) / nk1 - (st + lcm - 1) / lcm;
+}
+
+__global__ void __launch_bounds__(256)
+qlora_stream_reduce_kernel(const __grid_constant__ StreamReduceParams p) {
+  constexpr int BN = stream::BN, Q4 = BN / 4;
+  const int idx = int(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int per_row = p.num_tiles * Q4;
+  if (idx >= per_row * p.M) return;
+  const int m = idx / per_row;
+  const int rem = idx - m * per_row;
+  const int t = rem / Q4, col = (rem - t * Q4) * 4;
+  if (t * BN + col >= p.ncols) return;
+  const int seg0 = stream_rank32(t * p.nk1, p.iters, p.nk1, p.lcm);
+  const int seg1 = t + 1 == p.num_tiles ? p.segments
+                                        : stream_rank32((t + 1) * p.nk1, p.iters, p.nk1, p.lcm);
+  const float* src = p.partial + (size_t(seg0) * p.M + m) * BN + col;
+  const size_t sstride = size_t(p.M) * BN;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int sg = seg0; sg < seg1; sg += 4) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (sg + u < seg1) v[u] = __ldcg(reinterpret_cast<const float4*>(src + size_t(sg - seg0 + u) * sstride));
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (sg + u < seg1) { acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w; }
+  }
+  const float ts = p.tensor_scale ? __ldg(p.tensor_scale) : 1.0f;
+  uint2 o;
+  o.x = ptx::cvt_bf16x2(acc.x * ts, acc.y * ts);
+  o.y = ptx::cvt_bf16x2(acc.z * ts, acc.w * ts);
+  *reinterpret_cast<uint2*>(p.out + size_t(m) * p.ncols + t * BN + col) = o;
+}
+
+}  // namespace qlora

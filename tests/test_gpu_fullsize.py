@@ -52,6 +52,27 @@ def test_full_size_layer_sampled(cfg_id, proj):
     assert_close(to_f64(dB), ref["dB"], "dB")
 
 
+SHORT = [(2, 16), (2, 256), (3, 64)]
+
+
+@pytest.mark.parametrize("cfg_id,M", SHORT, ids=[f"{synth.CONFIGS[c].fmt}-M{m}" for c, m in SHORT])
+def test_full_size_weight_short_batch(cfg_id, M):
+    # the full-size weights of the NF4 up-proj and the MXFP4 gate-proj under the short batches of
+    # the weight-stream sweep: every output row is checked
+    from oracle import oracle
+    p = synth.layer_inputs(cfg_id, 0, M=M)
+    g = GpuLayer(p)
+    Y, T = g.fwd()
+    dX, dA, dB = g.bwd(T)
+    torch.cuda.synchronize()
+    assert g.status() == 0
+    ref = oracle.layer(p["fmt"], p["M"], p["N"], p["K"], p["r"], p["s"], p["codes"], p["scales"],
+                       p["tensor_scale"], p["X"], p["A"], p["B"], p["dY"],
+                       want=("Y", "dX", "T", "dA", "dB"))
+    for name, got in (("Y", Y), ("dX", dX), ("T", T), ("dA", dA), ("dB", dB)):
+        assert_close(to_f64(got), ref[name], name)
+
+
 @pytest.mark.parametrize("proj", [0, 1, 2], ids=["gate", "up", "down"])
 def test_full_size_grouped_sampled(proj):
     from oracle import oracle

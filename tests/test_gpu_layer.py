@@ -114,6 +114,12 @@ CASES = [
     ("mxfp4", 255, 144, 640, 16),
     ("nvfp4", 256, 256, 256, 16),
     ("nvfp4", 513, 528, 448, 64),
+    # short batches (weight-streaming kernels): many output tiles, ranges that split tiles
+    ("nf4", 16, 1024, 2048, 16),
+    ("mxfp4", 64, 2048, 1024, 64),
+    ("nvfp4", 200, 768, 4096, 8),
+    ("nf4", 128, 4096, 512, 32),
+    ("mxfp4", 2, 16, 64, 8),
 ]
 
 
