@@ -397,7 +397,7 @@ qlora_status_t launch_fused(const qlora_weight_t* W, bool dx, const void* act, c
 
 template <int FMT, bool DX, int MT>
 qlora_status_t launch_stream_t(const StreamParams& p, int grid, cudaStream_t st) {
-  const size_t smem = stream::smem_bytes(MT);
+  const size_t smem = stream::smem_bytes(p.xrows);
   if (!set_smem(qlora_stream_gemm_kernel<FMT, DX, MT>, smem)) return QLORA_ERR_CUDA;
   LaunchScope scope(DX ? kKindStreamDx : kKindStreamFwd, st);
   qlora_stream_gemm_kernel<FMT, DX, MT><<<grid, stream::kThreads, smem, st>>>(p);
@@ -414,8 +414,10 @@ qlora_status_t launch_stream(const qlora_weight_t* W, bool dx, const void* act, 
   const StreamPlan sp = stream_plan(N, K, M, dx, num_sms());
   if (sp.partial_bytes > partial_bytes) return QLORA_ERR_WORKSPACE;
   StreamParams p{};
+  p.xrows = int((M + 15) / 16 * 16);
+  const int mt = p.xrows <= 128 ? 1 : 2;
   if (!tmap_2d(&p.tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, uint64_t(Kc), uint64_t(M),
-               uint64_t(Kc) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+               uint64_t(Kc) * 2, 64, uint32_t(p.xrows), CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
   const bool okc = !dx
       ? tmap_2d(&p.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, uint64_t(K / 2), uint64_t(N),
@@ -424,7 +426,7 @@ qlora_status_t launch_stream(const qlora_weight_t* W, bool dx, const void* act, 
                 uint64_t(K / 2), 64, 64, CU_TENSOR_MAP_SWIZZLE_64B);
   if (!okc) return QLORA_ERR_CUDA;
   if (!tmap_2d(&p.tm_zs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, zs, uint64_t(r), uint64_t(M),
-               uint64_t(r) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+               uint64_t(r) * 2, 64, uint32_t(p.xrows), CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
   p.scales = W->scales;
   p.lora_up = static_cast<const __nv_bfloat16*>(lora_up);
@@ -438,7 +440,6 @@ qlora_status_t launch_stream(const qlora_weight_t* W, bool dx, const void* act, 
   p.num_tiles = sp.tiles;
   p.iters = sp.iters;
   p.lcm = sp.lcm;
-  const int mt = M <= 128 ? 1 : 2;
   qlora_status_t rc;
   switch ((W->fmt * 2 + (dx ? 1 : 0)) * 2 + (mt - 1)) {
     case 0: rc = launch_stream_t<kFmtNF4, false, 1>(p, sp.grid, st); break;

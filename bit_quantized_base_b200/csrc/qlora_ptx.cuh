@@ -65,6 +65,28 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* de
   }
 }
 
+// As mbar_wait, for roles that wait long and whose wake-up latency does not matter (epilogues,
+// producers running ahead): the thread sleeps between polls, so it does not take issue slots
+// from the warps that do the work.
+__device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity, int* dev_status,
+                                               volatile int* abort_flag,
+                                               unsigned long long limit = QLORA_WAIT_LIMIT_CYCLES) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(128);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 15u) == 0u) {
+      if (abort_flag && *abort_flag) return false;
+      if (static_cast<unsigned long long>(clock64() - t0) > limit) {
+        if (dev_status) atomicCAS(dev_status, 0, 5 /* QLORA_ERR_DEVICE_TIMEOUT */);
+        if (abort_flag) *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------- CTA pairs
 // A cluster of two CTAs shares one tcgen05.mma.cta_group::2: rank 0 (the leader) issues it, each
 // CTA supplies half of the operands from its own shared memory and receives its half of D in its

@@ -14,10 +14,13 @@
 // applies the NVFP4 tensor scale and writes bf16.
 //
 // A tile is 256 output columns (two 128-column weight halves, each decoded exactly as one CTA's
-// half in the pair kernel) by all M rows: one tcgen05.mma (cta_group::1) of M=128, N=256 per
-// 16-deep step and 128-row block of activations (one block for M <= 128, two for M <= 256, sharing
-// the decoded weight).  The LoRA term is one extra step per tile (operands Zs and rows of B or A),
-// as in the pair kernel.
+// half in the pair kernel) by all M rows.  The MMA runs with the operands swapped: a decoded
+// weight half is the A operand (M = 128 output columns), the activation rows are the B operand
+// (N = M rounded up to 16), so the tensor core computes only the batch's own rows, and the
+// accumulator holds the tile transposed (tensor-memory lane = output column, column = batch row).
+// The LoRA term is one extra step per tile (operands rows of B or A, and Zs), as in the pair
+// kernel.  Every step has one operand stage (activation rows + weight tile) with one full and one
+// empty barrier.
 //
 // Warp roles (480 threads, one CTA per SM):
 //   warps 0-3   epilogue: tensor memory -> fp32 partial (global, L2-resident)
@@ -37,29 +40,31 @@
 namespace qlora {
 namespace stream {
 constexpr int BN = 256, HN = 128, BK = 64;
-constexpr int X_BYTES = 128 * BK * 2;     // one 128-row activation block: 16 KB
 constexpr int W_BYTES = BN * BK * 2;      // 32 KB (two 16 KB halves)
 constexpr int HW_BYTES = HN * BK * 2;     // 16 KB
 constexpr int C_BYTES = BN * BK / 2;      // 8 KB of packed codes (two 4 KB halves)
 constexpr int HC_BYTES = HN * BK / 2;
-constexpr int NC = 6;                     // code stages
 constexpr int kEpiWarps = 4, kTmaWarp = 4, kCodeWarp = 5, kMmaWarp = 6, kDqWarp0 = 7, kDqWarps = 8;
 constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;
 constexpr int kTmemCols = 512;
 constexpr int kMaxRows = 256;
 constexpr int SCALE_RING_BYTES = 4 * 2 * 256 * 4;   // kPf slots x 2 halves x 256 threads
-// operand stages: MT activation blocks + one weight tile
-__host__ __device__ constexpr int num_stages(int MT) { return MT == 1 ? 3 : 2; }
-__host__ __device__ constexpr size_t stage_bytes(int MT) { return size_t(MT) * X_BYTES + W_BYTES; }
-__host__ __device__ constexpr size_t smem_bytes(int MT) {
-  return 1024 + size_t(num_stages(MT)) * stage_bytes(MT) + size_t(NC) * C_BYTES + SCALE_RING_BYTES + 1024;
+// Operand stages: xrows activation rows (M rounded up to 16) plus one weight tile; the stage count
+// depends on xrows, so every role tracks its stage index and phase incrementally.  MT = 1 for
+// xrows <= 128 (double-buffered accumulators: 2 x 2 halves x xrows tensor-memory columns), 2 above.
+__host__ __device__ constexpr int num_stages(int xrows) { return xrows <= 64 ? 4 : (xrows <= 128 ? 3 : 2); }
+constexpr int kMaxStages = 4;
+constexpr int NC = 6;                     // code stages
+__host__ __device__ constexpr size_t smem_bytes(int xrows) {
+  return 1024 + size_t(num_stages(xrows)) * (size_t(xrows) * 128 + W_BYTES) + size_t(NC) * C_BYTES +
+         SCALE_RING_BYTES + 1024;
 }
 }  // namespace stream
 
 struct StreamParams {
-  CUtensorMap tm_act;    // activations [M, Kc] bf16, box {64, 128}, SW128
+  CUtensorMap tm_act;    // activations [M, Kc] bf16, box {64, xrows}, SW128
   CUtensorMap tm_codes;  // codes [N, K/2] u8, per weight half: fwd box {32, 128} SW32; dX box {64, 64} SW64
-  CUtensorMap tm_zs;     // Zs [M, r] bf16, box {64, 128}, SW128
+  CUtensorMap tm_zs;     // Zs [M, r] bf16, box {64, xrows}, SW128
   const void* scales;                // [N, K/bs]
   const __nv_bfloat16* lora_up;      // fwd: B [N, r]; dX: A [r, K]
   float* partial;                    // [segments][M][256] fp32
@@ -69,6 +74,7 @@ struct StreamParams {
   int num_tiles;                     // 256-column output tiles
   int iters;                         // L: (tile, step) iterations per CTA
   long long lcm;                     // lcm(L, num_k + 1)
+  int xrows;                         // M rounded up to 16: activation rows per stage, MMA N
 };
 
 // Segments are the pieces of the iteration space between consecutive CTA-range starts (multiples
@@ -91,28 +97,29 @@ template <int FMT, bool DX, int MT>
 __global__ void __launch_bounds__(stream::kThreads, 1)
 qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
   using namespace stream;
-  constexpr int NS = num_stages(MT);
-  constexpr uint32_t STAGE = uint32_t(stage_bytes(MT));
   constexpr int NB = MT == 1 ? 2 : 1;          // accumulator buffers
+  const int NS = num_stages(p.xrows);
+  const uint32_t XSTAGE = uint32_t(p.xrows) * 128u;   // bytes of one activation stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* stages = smem;                      // per stage: MT activation blocks, then the weight tile
-  uint8_t* cs = stages + NS * STAGE;
+  uint8_t* xst = smem;                         // NS activation stages, then NS weight tiles
+  uint8_t* wst = xst + NS * XSTAGE;
+  uint8_t* cs = wst + NS * W_BYTES;
   uint8_t* scr = cs + NC * C_BYTES;            // scale ring: kPf slots x 2 halves x 256 threads x 4 B
   uint64_t* bars = reinterpret_cast<uint64_t*>(scr + SCALE_RING_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 2 * NC + 2 * NB);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kMaxStages + 2 * NC + 2 * NB);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t b0 = ptx::smem_u32(bars);
   auto full_s = [&](uint32_t s) { return b0 + 8u * s; };
-  auto empty_s = [&](uint32_t s) { return b0 + 8u * (NS + s); };
-  auto full_c = [&](uint32_t s) { return b0 + 8u * (2 * NS + s); };
-  auto empty_c = [&](uint32_t s) { return b0 + 8u * (2 * NS + NC + s); };
-  auto acc_full = [&](uint32_t b) { return b0 + 8u * (2 * NS + 2 * NC + b); };
-  auto acc_empty = [&](uint32_t b) { return b0 + 8u * (2 * NS + 2 * NC + NB + b); };
-  auto xs = [&](uint32_t s) { return ptx::smem_u32(stages) + s * STAGE; };
-  auto wsm = [&](uint32_t s) { return ptx::smem_u32(stages) + s * STAGE + MT * X_BYTES; };
+  auto empty_s = [&](uint32_t s) { return b0 + 8u * (kMaxStages + s); };
+  auto full_c = [&](uint32_t s) { return b0 + 8u * (2 * kMaxStages + s); };
+  auto empty_c = [&](uint32_t s) { return b0 + 8u * (2 * kMaxStages + NC + s); };
+  auto acc_full = [&](uint32_t b) { return b0 + 8u * (2 * kMaxStages + 2 * NC + b); };
+  auto acc_empty = [&](uint32_t b) { return b0 + 8u * (2 * kMaxStages + 2 * NC + NB + b); };
+  auto xs = [&](uint32_t s) { return ptx::smem_u32(xst) + s * XSTAGE; };
+  auto wsm = [&](uint32_t s) { return ptx::smem_u32(wst) + s * uint32_t(W_BYTES); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = p.num_k;
@@ -149,108 +156,108 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------------ activation producer
     if (lane == 0) {
+      uint32_t s = 0, ph = 0;
+      int ks = rg.step(rg.g0);
       for (int g = rg.g0; g < rg.g1; ++g) {
-        const uint32_t i = uint32_t(g - rg.g0), s = i % NS;
-        if (!ptx::mbar_wait(empty_s(s), ((i / NS) & 1u) ^ 1u, p.status, abort_flag)) break;
-        ptx::mbar_arrive_expect_tx(full_s(s), MT * X_BYTES);
-        const int ks = rg.step(g);
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          if (ks < nk) ptx::tma_load_2d(xs(s) + mt * X_BYTES, &p.tm_act, full_s(s), ks * BK, mt * 128);
-          else ptx::tma_load_2d(xs(s) + mt * X_BYTES, &p.tm_zs, full_s(s), 0, mt * 128);
-        }
+        if (!ptx::mbar_wait_idle(empty_s(s), ph ^ 1u, p.status, abort_flag)) break;
+        ptx::mbar_arrive_expect_tx(full_s(s), XSTAGE);
+        if (ks < nk) ptx::tma_load_2d(xs(s), &p.tm_act, full_s(s), ks * BK, 0);
+        else ptx::tma_load_2d(xs(s), &p.tm_zs, full_s(s), 0, 0);
+        if (++s == uint32_t(NS)) { s = 0; ph ^= 1u; }
+        if (++ks == rg.nk1) ks = 0;
       }
     }
   } else if (warp == kCodeWarp) {
     // ------------------------------------------------------------------ code producer
     if (lane == 0) {
-      uint32_t j = 0;
+      uint32_t sc = 0, ph = 0;
+      int ks = rg.step(rg.g0), c0 = rg.tile(rg.g0) * BN;
       for (int g = rg.g0; g < rg.g1; ++g) {
-        const int ks = rg.step(g);
-        if (ks == nk) continue;
-        const uint32_t sc = j % NC;
-        if (!ptx::mbar_wait(empty_c(sc), ((j / NC) & 1u) ^ 1u, p.status, abort_flag)) break;
-        ptx::mbar_arrive_expect_tx(full_c(sc), C_BYTES);
-        const uint32_t cd = ptx::smem_u32(cs + sc * C_BYTES);
-        const int c0 = rg.tile(g) * BN;
+        if (ks < nk) {
+          if (!ptx::mbar_wait_idle(empty_c(sc), ph ^ 1u, p.status, abort_flag)) break;
+          ptx::mbar_arrive_expect_tx(full_c(sc), C_BYTES);
+          const uint32_t cd = ptx::smem_u32(cs + sc * C_BYTES);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (!DX) ptx::tma_load_2d(cd + h * HC_BYTES, &p.tm_codes, full_c(sc), ks * (BK / 2), c0 + h * HN);
-          else ptx::tma_load_2d(cd + h * HC_BYTES, &p.tm_codes, full_c(sc), (c0 + h * HN) / 2, ks * BK);
+          for (int h = 0; h < 2; ++h) {
+            if (!DX) ptx::tma_load_2d(cd + h * HC_BYTES, &p.tm_codes, full_c(sc), ks * (BK / 2), c0 + h * HN);
+            else ptx::tma_load_2d(cd + h * HC_BYTES, &p.tm_codes, full_c(sc), (c0 + h * HN) / 2, ks * BK);
+          }
+          if (++sc == uint32_t(NC)) { sc = 0; ph ^= 1u; }
         }
-        ++j;
+        if (++ks == rg.nk1) { ks = 0; c0 += BN; }
       }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = ptx::idesc_bf16(128, BN, 0, DX ? 1u : 0u);
+      const uint32_t idesc = ptx::idesc_bf16(128, uint32_t(p.xrows), DX ? 1u : 0u, 0u);
       const int lora_kk = (p.r + 15) / 16;
-      uint32_t seg = 0;
+      uint32_t b = 0, bph = 0, s = 0, ph = 0;
+      int ks = rg.step(rg.g0);
       bool first = true;
       for (int g = rg.g0; g < rg.g1; ++g) {
-        const uint32_t i = uint32_t(g - rg.g0), s = i % NS;
-        const uint32_t b = seg % NB;
         if (first) {
-          if (!ptx::mbar_wait(acc_empty(b), ((seg / NB) & 1u) ^ 1u, p.status, abort_flag)) break;
+          if (!ptx::mbar_wait(acc_empty(b), bph ^ 1u, p.status, abort_flag)) break;
           ptx::tc_fence_after();
         }
-        if (!ptx::mbar_wait(full_s(s), (i / NS) & 1u, p.status, abort_flag)) break;
+        if (!ptx::mbar_wait(full_s(s), ph, p.status, abort_flag)) break;
         ptx::tc_fence_after();
-        const int ks = rg.step(g);
         const int nkk = ks < nk ? BK / 16 : lora_kk;
         const uint32_t xa = xs(s), wb = wsm(s);
+        const uint32_t d0 = tmem + b * 2u * uint32_t(p.xrows);
         for (int kk = 0; kk < nkk; ++kk) {
-          const uint64_t bd = DX ? ptx::smem_desc(wb + kk * 2048, 8192, 1024, ptx::kSw128)
-                                 : ptx::smem_desc(wb + kk * 32, 16, 1024, ptx::kSw128);
+          const uint64_t bd = ptx::smem_desc(xa + kk * 32, 16, 1024, ptx::kSw128);
 #pragma unroll
-          for (int mt = 0; mt < MT; ++mt) {
-            const uint64_t ad = ptx::smem_desc(xa + mt * X_BYTES + kk * 32, 16, 1024, ptx::kSw128);
-            const uint32_t d = tmem + uint32_t(MT == 1 ? b * BN : mt * BN);
-            ptx::mma_bf16(d, ad, bd, idesc, (!first || kk > 0) ? 1u : 0u);
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t wh = wb + hh * HW_BYTES;
+            const uint64_t ad = DX ? ptx::smem_desc(wh + kk * 2048, 8192, 1024, ptx::kSw128)
+                                   : ptx::smem_desc(wh + kk * 32, 16, 1024, ptx::kSw128);
+            ptx::mma_bf16(d0 + hh * uint32_t(p.xrows), ad, bd, idesc, (!first || kk > 0) ? 1u : 0u);
           }
         }
         ptx::mma_commit(empty_s(s));
         first = false;
-        if (rg.seg_end(g)) {
+        if (++s == uint32_t(NS)) { s = 0; ph ^= 1u; }
+        const bool end = g + 1 == rg.g1 || ks == nk;
+        if (++ks == rg.nk1) ks = 0;
+        if (end) {
           ptx::mma_commit(acc_full(b));
-          ++seg;
+          if (++b == uint32_t(NB)) { b = 0; bph ^= 1u; }
           first = true;
         }
       }
     }
   } else if (warp < kEpiWarps) {
     // ------------------------------------------------------------------ epilogue
-    const int q = warp;   // tensor-memory lanes 32q .. 32q+31
-    uint32_t seg = 0;
+    // Tensor-memory lane 32q + lane holds output column hh * 128 + 32q + lane of the tile; its
+    // accumulator columns are the batch rows.  Each store instruction writes 32 consecutive floats
+    // of one partial row.
+    const int q = warp;
+    uint32_t b = 0, bph = 0;
     for (int g = rg.g0; g < rg.g1; ++g) {
       if (!rg.seg_end(g)) continue;
-      const uint32_t b = seg % NB;
-      if (!ptx::mbar_wait(acc_full(b), (seg / NB) & 1u, p.status, abort_flag)) break;
+      if (!ptx::mbar_wait_idle(acc_full(b), bph, p.status, abort_flag)) break;
       ptx::tc_fence_after();
       const long long st = max((long long)rg.g0, (long long)rg.tile(g) * rg.nk1);
       float* base = p.partial + size_t(stream_segment(st, p.iters, rg.nk1, p.lcm)) * size_t(p.M) * BN;
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        const int row = mt * 128 + q * 32 + lane;
 #pragma unroll 1
-        for (int cb = 0; cb < BN / 32; ++cb) {
-          uint32_t v[32];
-          ptx::tmem_ld_32x32b_x32(tmem + (uint32_t(q * 32) << 16) + uint32_t(MT == 1 ? b * BN : mt * BN) + cb * 32, v);
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t tcol = tmem + (uint32_t(q * 32) << 16) + b * 2u * uint32_t(p.xrows) + hh * uint32_t(p.xrows);
+        float* col = base + hh * HN + q * 32 + lane;
+#pragma unroll 1
+        for (int m0 = 0; m0 < p.xrows; m0 += 16) {
+          uint32_t v[16];
+          ptx::tmem_ld_32x32b_x16(tcol + m0, v);
           ptx::tmem_ld_wait();
-          if (row < p.M) {
-            float4* dst = reinterpret_cast<float4*>(base + size_t(row) * BN + cb * 32);
 #pragma unroll
-            for (int g4 = 0; g4 < 8; ++g4)
-              __stcg(dst + g4, make_float4(__uint_as_float(v[4 * g4]), __uint_as_float(v[4 * g4 + 1]),
-                                           __uint_as_float(v[4 * g4 + 2]), __uint_as_float(v[4 * g4 + 3])));
-          }
+          for (int u = 0; u < 16; ++u)
+            if (m0 + u < p.M) __stcg(col + size_t(m0 + u) * BN, __uint_as_float(v[u]));
         }
       }
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(acc_empty(b));
-      ++seg;
+      if (++b == uint32_t(NB)) { b = 0; bph ^= 1u; }
     }
   } else {
     // ------------------------------------------------------------------ dequant
@@ -305,9 +312,10 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
       advance2(pf);
     }
     uint32_t slot = 0;
+    uint32_t s = cur.i, pw = 0;   // operand stage of the step and its phase (own steps are 2 apart)
+    if (s >= uint32_t(NS)) { s -= NS; pw ^= 1u; }
     for (; cur.g < rg.g1; advance2(cur), advance2(pf)) {
       ptx::cp_async_wait<kPf - 1>();
-      const uint32_t s = cur.i % NS, pw = (cur.i / NS) & 1u;
       uint32_t sdep = 0;   // zero, but only once the slot has been read: orders the refill after it
       bool ok = true;
       if (cur.ks < nk) {
@@ -374,6 +382,8 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(full_s(s));
       slot = slot + 1 == kPf ? 0 : slot + 1;
+      s += 2;
+      if (s >= uint32_t(NS)) { s -= NS; pw ^= 1u; }
     }
     ptx::cp_async_wait<0>();
   }
