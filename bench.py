@@ -185,6 +185,122 @@ def max_over_ranks(ws, x):
     return float(t.item())
 
 
+def short_batch_sweep(Q, torch, p, Ws, X, dY, A, B, peaks):
+    """fwd+bwd at M in {16, 32, 64, 128, 256} on one weight (rotating device copies whose total
+    exceeds 3x L2): weight bytes read per step (two passes) / time, TFLOP/s, and the fraction of
+    the binding roofline max(flops / bf16 peak, bytes / HBM peak)."""
+    fmt, N, K, r, s = p["fmt"], p["N"], p["K"], p["r"], p["s"]
+    wbytes = weight_bytes(fmt, N, K)
+    nw = int(math.ceil(3 * 126e6 / wbytes)) + 1
+    base = list(Ws) if Ws else []
+    Wsw = base + [Q.weight_from_numpy(fmt, p["codes"], p["scales"], p["tensor_scale"])
+                  for _ in range(max(0, nw - len(base)))]
+    if X is None:
+        X, dY = Q.bf16_from_bits(p["X"]), Q.bf16_from_bits(p["dY"])
+        A, B = Q.bf16_from_bits(p["A"]), Q.bf16_from_bits(p["B"])
+    Y = torch.empty((256, N), dtype=torch.bfloat16, device="cuda")
+    T = torch.empty((256, r), dtype=torch.bfloat16, device="cuda")
+    dX = torch.empty((256, K), dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty((r, K), dtype=torch.bfloat16, device="cuda")
+    dB = torch.empty((N, r), dtype=torch.bfloat16, device="cuda")
+    out = {}
+    for Ms in (16, 32, 64, 128, 256):
+        Xm, dYm, Ym, Tm, dXm = X[:Ms], dY[:Ms], Y[:Ms], T[:Ms], dX[:Ms]
+        wsm = Q.alloc_workspace(Q.OP_BWD, Wsw[0], Ms, r)
+        Q.qlora_workspace_init(wsm)
+
+        def sstep(i):
+            w = Wsw[i % len(Wsw)]
+            Q.qlora_linear_fwd(w, Xm, A, B, Ym, Tm, Ms, r, s, wsm)
+            Q.qlora_linear_bwd(w, Xm, A, B, Tm, dYm, dXm, dA, dB, Ms, r, s, wsm)
+
+        for i in range(5):
+            sstep(i)
+        torch.cuda.synchronize()
+        n_it = 60
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for i in range(n_it):
+            sstep(i)
+        a1.record()
+        a1.synchronize()
+        if Q.qlora_get_device_status(wsm) != 0:
+            raise RuntimeError("device status in the short-batch sweep")
+        t = a0.elapsed_time(a1) / n_it * 1e-3
+        fl = flops(Ms, N, K, r)
+        byt = 2 * wbytes + 2 * (2 * Ms * K + 2 * Ms * N)
+        t_roof = max(fl / (peaks["bf16_tflops"] * 1e12), byt / (peaks["hbm_gbs"] * 1e9))
+        out[str(Ms)] = {"us_per_step": round(t * 1e6, 1),
+                        "weight_gbs": round(2 * wbytes / t / 1e9, 1),
+                        "tflops": round(fl / t / 1e12, 1),
+                        "roofline_frac": round(t_roof / t, 4),
+                        "bound": "tensor" if fl / (peaks["bf16_tflops"] * 1e12) > byt / (peaks["hbm_gbs"] * 1e9) else "hbm"}
+    del Wsw
+    torch.cuda.empty_cache()
+    return out
+
+
+def grouped_moe(Q, torch, synth, peaks):
+    """One fwd+bwd of each MoE expert projection (64 experts, MXFP4, Zipf top-8 routing of 16384
+    tokens): TFLOP/s.  Timing inputs: seeded random stored codes with a realistic E8M0 scale range
+    and seeded normal activations generated on the device (values do not change the timing)."""
+    cfg = synth.CONFIGS[5]
+    offs = synth.moe_routing(cfg)
+    E, r, s = cfg.experts, cfg.r, cfg.scale
+    M = int(offs[-1])
+    off = torch.from_numpy(offs.astype("int32")).cuda()
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5000)
+    res = {"experts": E, "rows": M, "counts_min": int((offs[1:] - offs[:-1]).min()),
+           "counts_max": int((offs[1:] - offs[:-1]).max()), "data": "random stored codes"}
+    tot_fl, tot_t = 0.0, 0.0
+    for pr in cfg.projs:
+        N, K = pr.N, pr.K
+        codes = torch.randint(0, 256, (E, N, K // 2), dtype=torch.uint8, device="cuda", generator=g)
+        scales = torch.randint(118, 124, (E, N, K // 32), dtype=torch.uint8, device="cuda", generator=g)
+        W = Q.Weight("mxfp4", N, K, codes, scales, None)
+        X = torch.randn(M, K, device="cuda", generator=g).bfloat16()
+        dY = torch.randn(M, N, device="cuda", generator=g).bfloat16()
+        A = (torch.rand(E, r, K, device="cuda", generator=g) * 0.02 - 0.01).bfloat16()
+        B = (torch.randn(E, N, r, device="cuda", generator=g) * 0.01).bfloat16()
+        Y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+        T = torch.empty(M, r, device="cuda", dtype=torch.bfloat16)
+        dX = torch.empty(M, K, device="cuda", dtype=torch.bfloat16)
+        dA = torch.empty(E, r, K, device="cuda", dtype=torch.bfloat16)
+        dB = torch.empty(E, N, r, device="cuda", dtype=torch.bfloat16)
+        ws = Q.alloc_workspace(Q.OP_GROUPED_BWD, W, M, r, E)
+        Q.qlora_workspace_init(ws)
+
+        def step():
+            Q.qlora_grouped_fwd(W, E, off, M, X, A, B, Y, T, r, s, ws)
+            Q.qlora_grouped_bwd(W, E, off, M, X, A, B, T, dY, dX, dA, dB, r, s, ws)
+
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        n_it = 10
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for _ in range(n_it):
+            step()
+        a1.record()
+        a1.synchronize()
+        if Q.qlora_get_device_status(ws) != 0:
+            raise RuntimeError("device status in the grouped run")
+        t = a0.elapsed_time(a1) / n_it * 1e-3
+        fl = flops(M, N, K, r)
+        tot_fl += fl
+        tot_t += t
+        res[pr.name] = {"ms_per_step": round(t * 1e3, 3), "tflops": round(fl / t / 1e12, 1)}
+        del codes, scales, W, X, dY, A, B, Y, T, dX, dA, dB, ws
+        torch.cuda.empty_cache()
+    res["tflops_all"] = round(tot_fl / tot_t / 1e12, 1)
+    res["frac_of_bf16_peak"] = round(tot_fl / tot_t / 1e12 / peaks["bf16_tflops"], 4)
+    return res
+
+
 def run_own(args):
     import numpy as np
     import torch
@@ -251,8 +367,8 @@ def run_own(args):
     if Q.qlora_get_device_status(ws) != 0:
         raise RuntimeError("device status after the timed region: %d" % Q.qlora_get_device_status(ws))
 
-    # ---- dominant kernel and its roofline
     peaks, peak_src = load_peaks()
+    # ---- dominant kernel and its roofline
     kflops = {"fused_fwd": 2.0 * M * N * K + 2.0 * M * N * r,
               "fused_dx": 2.0 * M * N * K + 2.0 * M * K * r,
               "lora_down_T": 2.0 * M * K * r, "lora_down_U": 2.0 * M * N * r,
@@ -308,40 +424,19 @@ def run_own(args):
            "d2h_bytes_per_step": int((hdA.numel() + hdB.numel()) * 2),
            "ms_per_step": round(e2e_ms / e2e_steps, 4)}
 
-    # ---- small-M weight-stream sweep on the same weight
+    # ---- short-batch weight-stream sweeps: the NF4 up-proj weight and the MXFP4 gate-proj weight
     sweep = None
     if not args.no_sweep:
-        sweep = {}
-        wbytes = weight_bytes(fmt, N, K)
-        nw = int(math.ceil(3 * 126e6 / wbytes)) + 1
-        Wsw = Ws + [Q.weight_from_numpy(fmt, p["codes"], p["scales"], p["tensor_scale"])
-                    for _ in range(max(0, nw - ncopy))]
-        for Ms in (16, 32, 64, 128, 256):
-            Xm, dYm = Xs[0][:Ms], dYs[0][:Ms]
-            Ym, Tm, dXm = Y[:Ms], T[:Ms], dX[:Ms]
-            wsm = Q.alloc_workspace(Q.OP_BWD, Wsw[0], Ms, r)
-            Q.qlora_workspace_init(wsm)
+        sweep = {"nf4_up_14336x4096": short_batch_sweep(Q, torch, p, Ws, Xs[0], dYs[0], A, B, peaks)}
+        p3 = synth.layer_inputs(3, M=256)
+        sweep["mxfp4_gate_28672x8192"] = short_batch_sweep(Q, torch, p3, None, None, None, None, None,
+                                                           peaks)
+        del p3
 
-            def sstep(i):
-                w = Wsw[i % len(Wsw)]
-                Q.qlora_linear_fwd(w, Xm, A, B, Ym, Tm, Ms, r, s, wsm)
-                Q.qlora_linear_bwd(w, Xm, A, B, Tm, dYm, dXm, dA, dB, Ms, r, s, wsm)
-
-            for i in range(5):
-                sstep(i)
-            torch.cuda.synchronize()
-            n_it = 60
-            a0 = torch.cuda.Event(enable_timing=True)
-            a1 = torch.cuda.Event(enable_timing=True)
-            a0.record()
-            for i in range(n_it):
-                sstep(i)
-            a1.record()
-            a1.synchronize()
-            t = a0.elapsed_time(a1) / n_it * 1e-3
-            sweep[str(Ms)] = {"us_per_step": round(t * 1e6, 1),
-                              "weight_gbs": round(2 * wbytes / t / 1e9, 1),
-                              "tflops": round(flops(Ms, N, K, r) / t / 1e12, 1)}
+    # ---- grouped (MoE) experts: 64 experts, 16384 tokens x top-8, one fwd+bwd per projection
+    grouped = None
+    if not args.no_sweep:
+        grouped = grouped_moe(Q, torch, synth, peaks)
 
     # ---- CPU baseline: the oracle on a bounded sample of the same workload
     cpu = None
@@ -364,6 +459,7 @@ def run_own(args):
         "kernel_breakdown": breakdown,
         "e2e": e2e,
         "weight_stream_small_m": sweep,
+        "grouped_moe": grouped,
         "cpu_baseline": cpu,
     }
     if rank == 0:
