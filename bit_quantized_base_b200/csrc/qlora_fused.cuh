@@ -8,15 +8,20 @@
 // lora_down kernel), its B operand the rows of B (forward) or A (backward), so it accumulates into
 // the same fp32 tensor-memory accumulator as the base product and the epilogue only scales by ts.
 //
-// The kernel runs on CTA pairs (clusters of 2) sharing one tcgen05.mma.cta_group::2 of M=256,
-// N=256 per 16-deep step.  A pair tile is 256 rows x 256 output columns; CTA rank r holds rows
-// [128r, 128r+128) of the activation operand and output columns [128r, 128r+128) of the
-// dequantised weight operand, and receives rows [128r, 128r+128) x all 256 columns of the fp32
-// accumulator in its own tensor memory (double buffered: 2 x 256 columns).  Each weight element is
-// decoded once per 256 rows, and each activation tile is fetched once per 256 output columns.
+// The kernel runs on CTA pairs (clusters of 2) issuing tcgen05.mma.cta_group::2 of M=256, N=256.
+// A pair tile is 512 rows x 256 output columns: two MMA blocks of 256 rows share each 16-deep
+// step's dequantised weight operand.  CTA rank r holds rows [256b + 128r, 256b + 128r + 128) of
+// activation block b and output columns [128r, 128r+128) of the weight operand, and receives rows
+// [256b + 128r, +128) x all 256 columns of block b's fp32 accumulator in its own tensor memory
+// (2 blocks x 256 columns, all 512 columns, single buffered).  Each weight element is decoded once
+// per 512 rows (8 decoded weights per clock per SM keep the MMA at full rate), and each step issues
+// 8 pair MMAs per barrier round, which keeps the fixed per-step cost of the issuing thread small
+// against the 1024 cycles of tensor work.  The epilogue of one tile delays the next tile's first
+// MMA (the accumulator is not double buffered); the dequant warps keep decoding into free stages
+// meanwhile.
 //
 // Warp roles per CTA (480 threads, one CTA per SM, persistent over pair tiles):
-//   warps 0-3   epilogue: tensor memory -> registers -> * ts -> bf16 -> global
+//   warps 0-3   epilogue: tensor memory (both blocks) -> registers -> * ts -> bf16 -> global
 //   warp  4     TMA producer of this CTA's activation half (completion counted on the leader's
 //               barrier)
 //   warp  6     TMA producer of this CTA's packed-code tiles, running ahead of the activation
@@ -47,19 +52,20 @@
 
 namespace qlora {
 namespace fused {
-constexpr int BM = 256, BN = 256;      // pair tile
-constexpr int HM = 128, HN = 128;      // per-CTA halves
+constexpr int BM = 512, BN = 256;      // pair tile
+constexpr int HM = 128, HN = 128;      // per-CTA rows of one MMA block; per-CTA weight half
+constexpr int MB = 2;                  // MMA blocks of 256 rows per pair tile
 constexpr int BK = 64;
-constexpr int NS = 6, NC = 6;         // operand stages (activation + weight halves), code stages
-constexpr int X_BYTES = HM * BK * 2;   // 16 KB
+constexpr int NS = 4, NC = 6;         // operand stages (activation blocks + weight half), code stages
+constexpr int X_BYTES = HM * BK * 2;   // 16 KB per block
 constexpr int W_BYTES = HN * BK * 2;   // 16 KB
 constexpr int C_BYTES = HN * BK / 2;   // 4 KB of packed codes
 constexpr int kEpiWarps = 4, kTmaWarp = 4, kMmaWarp = 5, kCodeWarp = 6, kDqWarp0 = 7, kDqWarps = 8;
 constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;
-constexpr int kTmemCols = 512;         // 2 buffers x 256 columns
+constexpr int kTmemCols = 512;         // 2 blocks x 256 columns
 constexpr int GM = 8;                  // m-tiles per raster group
-constexpr int kNumBars = 2 * NS + 2 * NC + 4;
-constexpr size_t kSmemBase = 1024 + size_t(NS) * (X_BYTES + W_BYTES) + size_t(NC) * C_BYTES + 1024;
+constexpr int kNumBars = 2 * NS + 2 * NC + 2;
+constexpr size_t kSmemBase = 1024 + size_t(NS) * (MB * X_BYTES + W_BYTES) + size_t(NC) * C_BYTES + 1024;
 // plus the expert table: 2 x (E + 1) ints
 __host__ __device__ constexpr size_t smem_bytes(int E) { return kSmemBase + size_t(2) * (E + 1) * 4; }
 }  // namespace fused
@@ -180,8 +186,8 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* xs = smem;                      // NS activation halves
-  uint8_t* wsm = xs + NS * X_BYTES;        // NS weight halves
+  uint8_t* xs = smem;                      // NS stages of this CTA's MB activation blocks
+  uint8_t* wsm = xs + NS * MB * X_BYTES;   // NS weight halves
   uint8_t* cs = wsm + NS * W_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(cs + NC * C_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
@@ -194,8 +200,8 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
   auto empty_s = [&](uint32_t s) { return b0 + 8u * (NS + s); };
   auto full_c = [&](uint32_t s) { return b0 + 8u * (2 * NS + s); };
   auto empty_c = [&](uint32_t s) { return b0 + 8u * (2 * NS + NC + s); };
-  auto acc_full = [&](uint32_t b) { return b0 + 8u * (2 * NS + 2 * NC + b); };
-  auto acc_empty = [&](uint32_t b) { return b0 + 8u * (2 * NS + 2 * NC + 2 + b); };
+  const uint32_t acc_full = b0 + 8u * (2 * NS + 2 * NC);
+  const uint32_t acc_empty = b0 + 8u * (2 * NS + 2 * NC + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();
@@ -208,7 +214,8 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
       ptx::mbar_init(empty_s(s), 1);
     }
     for (int s = 0; s < NC; ++s) { ptx::mbar_init(full_c(s), 1); ptx::mbar_init(empty_c(s), kDqWarps / 2); }
-    for (int b = 0; b < 2; ++b) { ptx::mbar_init(acc_full(b), 1); ptx::mbar_init(acc_empty(b), 2 * kEpiWarps); }
+    ptx::mbar_init(acc_full, 1);
+    ptx::mbar_init(acc_empty, 2 * kEpiWarps);
     *abort_flag = 0;
     ptx::fence_mbarrier_init();
   }
@@ -238,16 +245,19 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
       uint32_t i = 0;
       for (int t = pair; t < num_tiles; t += npairs) {
         const PairTile pt = pair_tile_at(grp_view, t, p.num_n);
-        const int m0 = pt.row0 + int(rank) * HM;      // this CTA's activation rows
+        const int m0 = pt.row0 + int(rank) * HM;      // this CTA's rows of block 0 (+256: block 1)
         bool ok = true;
         for (int ks = 0; ks <= nk; ++ks, ++i) {
           const uint32_t sx = i % NS, px = (i / NS) & 1u;
           if (!ptx::mbar_wait(empty_s(sx), px ^ 1u, p.status, abort_flag)) { ok = false; break; }
-          if (rank == 0) ptx::mbar_arrive_expect_tx(full_s(sx), 2 * X_BYTES);
-          const uint32_t xd = ptx::smem_u32(xs + sx * X_BYTES);
+          if (rank == 0) ptx::mbar_arrive_expect_tx(full_s(sx), 2 * MB * X_BYTES);
           const uint32_t fx = ptx::mapa(full_s(sx), 0);
-          if (ks < nk) ptx::tma_load_2d_pair(xd, &p.tm_act, fx, ks * BK, m0);
-          else ptx::tma_load_2d_pair(xd, &p.tm_zs, fx, 0, m0);
+#pragma unroll
+          for (int blk = 0; blk < MB; ++blk) {
+            const uint32_t xd = ptx::smem_u32(xs + (sx * MB + blk) * X_BYTES);
+            if (ks < nk) ptx::tma_load_2d_pair(xd, &p.tm_act, fx, ks * BK, m0 + blk * 2 * HM);
+            else ptx::tma_load_2d_pair(xd, &p.tm_zs, fx, 0, m0 + blk * 2 * HM);
+          }
         }
         if (!ok) break;
       }
@@ -279,28 +289,29 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
       const int lora_kk = (p.r + 15) / 16;
       uint32_t i = 0, tc = 0;
       for (int t = pair; t < num_tiles; t += npairs, ++tc) {
-        const uint32_t buf = tc & 1u;
-        if (!ptx::mbar_wait_cluster(acc_empty(buf), ((tc >> 1) & 1u) ^ 1u, p.status, abort_flag)) break;
+        if (!ptx::mbar_wait_cluster(acc_empty, (tc & 1u) ^ 1u, p.status, abort_flag)) break;
         ptx::tc_fence_after();
-        const uint32_t d = tmem + buf * BN;
         bool ok = true;
         for (int ks = 0; ks <= nk; ++ks, ++i) {
           const uint32_t st = i % NS;
           if (!ptx::mbar_wait_cluster(full_s(st), (i / NS) & 1u, p.status, abort_flag)) { ok = false; break; }
           ptx::tc_fence_after();
-          const uint32_t xa = ptx::smem_u32(xs + st * X_BYTES);
+          const uint32_t xa = ptx::smem_u32(xs + st * MB * X_BYTES);
           const uint32_t wb = ptx::smem_u32(wsm + st * W_BYTES);
           const int nkk = ks < nk ? BK / 16 : lora_kk;
           for (int kk = 0; kk < nkk; ++kk) {
-            const uint64_t ad = ptx::smem_desc(xa + kk * 32, 16, 1024, ptx::kSw128);
             const uint64_t bd = DX ? ptx::smem_desc(wb + kk * 2048, 8192, 1024, ptx::kSw128)
                                    : ptx::smem_desc(wb + kk * 32, 16, 1024, ptx::kSw128);
-            ptx::mma_bf16_pair(d, ad, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int blk = 0; blk < MB; ++blk) {
+              const uint64_t ad = ptx::smem_desc(xa + blk * X_BYTES + kk * 32, 16, 1024, ptx::kSw128);
+              ptx::mma_bf16_pair(tmem + blk * BN, ad, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           ptx::mma_commit_pair(empty_s(st), 3);
         }
         if (!ok) break;
-        ptx::mma_commit_pair(acc_full(buf), 3);
+        ptx::mma_commit_pair(acc_full, 3);
       }
     } else if (lane == 0) {
       // relay (other CTA): this CTA's weight half of step i is complete -> tell the leader
@@ -320,40 +331,43 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     // ------------------------------------------------------------------ epilogue
     const int q = warp;  // tensor-memory lanes 32q .. 32q+31
     const int ncols = DX ? p.K : p.N;
-    const uint32_t acc_empty_leader0 = ptx::mapa(acc_empty(0), 0);
+    const uint32_t acc_empty_leader = ptx::mapa(acc_empty, 0);
     uint32_t tc = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++tc) {
       const PairTile pt = pair_tile_at(grp_view, t, p.num_n);
-      const int row = pt.row0 + int(rank) * HM + q * 32 + lane;
       const int c0 = pt.nt * BN;
       const float ts = (FMT == kFmtNVFP4 && p.tensor_scale) ? __ldg(p.tensor_scale + pt.e) : 1.0f;
-      const uint32_t buf = tc & 1u;
-      if (!ptx::mbar_wait(acc_full(buf), (tc >> 1) & 1u, p.status, abort_flag)) break;
+      if (!ptx::mbar_wait(acc_full, tc & 1u, p.status, abort_flag)) break;
       ptx::tc_fence_after();
 #pragma unroll 1
-      for (int cb = 0; cb < BN / 32; ++cb) {
-        uint32_t v[32];
-        ptx::tmem_ld_32x32b_x32(tmem + (uint32_t(q * 32) << 16) + buf * BN + cb * 32, v);
-        ptx::tmem_ld_wait();
-        if (row < pt.row_end) {
-          __nv_bfloat16* orow = p.out + size_t(row) * ncols;
+      for (int blk = 0; blk < MB; ++blk) {
+        const int row = pt.row0 + blk * 2 * HM + int(rank) * HM + q * 32 + lane;
+        if (pt.row0 + blk * 2 * HM + int(rank) * HM + q * 32 >= pt.row_end) continue;   // warp-uniform
+#pragma unroll 1
+        for (int cb = 0; cb < BN / 32; ++cb) {
+          uint32_t v[32];
+          ptx::tmem_ld_32x32b_x32(tmem + (uint32_t(q * 32) << 16) + blk * BN + cb * 32, v);
+          ptx::tmem_ld_wait();
+          if (row < pt.row_end) {
+            __nv_bfloat16* orow = p.out + size_t(row) * ncols;
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int col = c0 + cb * 32 + g * 8;
-            if (col < ncols) {
-              uint4 o;
-              o.x = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 0]) * ts, __uint_as_float(v[g * 8 + 1]) * ts);
-              o.y = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 2]) * ts, __uint_as_float(v[g * 8 + 3]) * ts);
-              o.z = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 4]) * ts, __uint_as_float(v[g * 8 + 5]) * ts);
-              o.w = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 6]) * ts, __uint_as_float(v[g * 8 + 7]) * ts);
-              *reinterpret_cast<uint4*>(orow + col) = o;
+            for (int g = 0; g < 4; ++g) {
+              const int col = c0 + cb * 32 + g * 8;
+              if (col < ncols) {
+                uint4 o;
+                o.x = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 0]) * ts, __uint_as_float(v[g * 8 + 1]) * ts);
+                o.y = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 2]) * ts, __uint_as_float(v[g * 8 + 3]) * ts);
+                o.z = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 4]) * ts, __uint_as_float(v[g * 8 + 5]) * ts);
+                o.w = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 6]) * ts, __uint_as_float(v[g * 8 + 7]) * ts);
+                *reinterpret_cast<uint4*>(orow + col) = o;
+              }
             }
           }
         }
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive_remote(acc_empty_leader0 + 8u * buf);
+      if (lane == 0) ptx::mbar_arrive_remote(acc_empty_leader);
     }
   } else {
     // ------------------------------------------------------------------ dequant
