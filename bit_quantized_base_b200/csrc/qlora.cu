@@ -521,6 +521,37 @@ qlora_status_t launch_wgrad(const void* X, const void* dY, const void* T, const 
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------------------ side stream
+// One non-blocking stream per device for work that may overlap the caller's stream inside a call,
+// with a ring of fork/join event pairs (re-recording an event is safe once its earlier waits have
+// been enqueued).  Created on first use and kept for the life of the process.
+struct SideStream {
+  static constexpr int kEvents = 32;
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork[kEvents] = {};
+  cudaEvent_t join[kEvents] = {};
+  std::atomic<int> next{0};
+};
+SideStream g_side[kMaxDevices];
+bool g_side_ok[kMaxDevices] = {false};
+std::mutex g_side_mu;
+
+SideStream* side_stream() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_side_mu);
+  if (!g_side_ok[d]) {
+    SideStream& ss = g_side[d];
+    if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    for (int i = 0; i < SideStream::kEvents; ++i)
+      if (cudaEventCreateWithFlags(&ss.fork[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&ss.join[i], cudaEventDisableTiming) != cudaSuccess)
+        return nullptr;
+    g_side_ok[d] = true;
+  }
+  return &g_side[d];
+}
+
 // ------------------------------------------------------------------- fixed scratch (no alloc)
 // Scratch of qlora_linear_fwd_noalloc: a file-scope device array, present on every GPU that loads
 // the library.  Host code must not pass the symbol itself to a kernel (on the host it names a
@@ -642,11 +673,30 @@ qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   st = launch_lora_down(true, dY, M, W->N, B, r, scale, ts, U, Zs, ws_status(ws), part,
                         L.partial_bytes, ws_counters(ws), offsets, E, grouped, s);
   if (st != QLORA_OK) return st;
+  const bool short_dx = dX && stream_fits(W, M, E, true, ws_bytes - L.partial);
+  if (dX && !short_dx) {
+    // The adapter gradients need only T, U, X and dY, so they run on a side stream beside the
+    // tiled dX kernel, filling the SMs its last wave of tiles leaves idle (the two kernels share
+    // no workspace region).  Joined back into `s` before returning.
+    SideStream* side = side_stream();
+    if (side) {
+      const int slot = side->next.fetch_add(1, std::memory_order_relaxed) % SideStream::kEvents;
+      if (cudaEventRecord(side->fork[slot], s) != cudaSuccess ||
+          cudaStreamWaitEvent(side->stream, side->fork[slot], 0) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+      st = launch_wgrad(X, dY, T, U, M, W->N, W->K, r, scale, dA, dB, ws, L, offsets, E, grouped,
+                        side->stream);
+      if (st != QLORA_OK) return st;
+      if (cudaEventRecord(side->join[slot], side->stream) != cudaSuccess) return QLORA_ERR_CUDA;
+      st = launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), offsets, E, grouped, s);
+      if (cudaStreamWaitEvent(s, side->join[slot], 0) != cudaSuccess) return QLORA_ERR_CUDA;
+      return st;
+    }
+  }
   if (dX) {
-    st = stream_fits(W, M, E, true, ws_bytes - L.partial)
-             ? launch_stream(W, true, dY, Zs, A, dX, M, r, ws_status(ws), part, ws_bytes - L.partial, s)
-                          : launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), offsets, E,
-                                         grouped, s);
+    st = short_dx ? launch_stream(W, true, dY, Zs, A, dX, M, r, ws_status(ws), part,
+                                  ws_bytes - L.partial, s)
+                  : launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), offsets, E, grouped, s);
     if (st != QLORA_OK) return st;
   }
   return launch_wgrad(X, dY, T, U, M, W->N, W->K, r, scale, dA, dB, ws, L, offsets, E, grouped, s);
