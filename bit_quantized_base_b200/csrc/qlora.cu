@@ -93,6 +93,24 @@ bool set_smem(K kernel, size_t bytes) {
                               cudaSharedmemCarveoutMaxShared) == cudaSuccess;
 }
 
+// Launch with programmatic stream serialization: the kernel may begin while the previous kernel of
+// the stream runs; it waits for it (griddepcontrol.wait) after its own prologue.
+template <typename P>
+cudaError_t launch_pdl(void (*kernel)(P), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       const P& params) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, params);
+}
+
 qlora_status_t check_weight(const qlora_weight_t* W) {
   if (!W) return QLORA_ERR_INVALID_ARG;
   if (W->fmt < QLORA_FMT_NF4 || W->fmt > QLORA_FMT_NVFP4) return QLORA_ERR_INVALID_ARG;
@@ -122,7 +140,7 @@ WgradPlan wgrad_plan(int64_t N, int64_t K, int64_t M, int E, int sms) {
   p.tiles0 = int((N + 127) / 128);
   p.tiles1 = int((K + 127) / 128);
   const int64_t tiles = int64_t(E) * (p.tiles0 + p.tiles1);
-  int S = int((sms + tiles - 1) / tiles);                    // about one wave of long splits
+  int S = int(sms / tiles);                                  // at most one wave of long splits
   S = S < 1 ? 1 : (S > 16 ? 16 : S);
   const int64_t chunks = (M + 63) / 64;                      // of one expert holding every row
   if (S > chunks) S = chunks > 0 ? int(chunks) : 1;
@@ -140,7 +158,7 @@ DownPlan down_plan(int64_t M, int64_t Kc, int E, int sms) {
   DownPlan p{};
   p.tiles = int((M + 127) / 128) + (E > 1 ? E - 1 : 0);
   p.num_k = int((Kc + 63) / 64);
-  int S = p.tiles > 0 ? (sms + p.tiles - 1) / p.tiles : 1;   // about one wave of long splits
+  int S = p.tiles > 0 ? sms / p.tiles : 1;                   // at most one wave of long splits
   S = S < 1 ? 1 : (S > 16 ? 16 : S);
   const int max_s = p.num_k / 2 > 0 ? p.num_k / 2 : 1;
   if (S > max_s) S = max_s;
@@ -328,10 +346,12 @@ qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t K
   LaunchScope scope(grouped ? (r_mn ? kKindGDownU : kKindGDownT) : (r_mn ? kKindDownU : kKindDownT), st);
   if (r_mn) {
     if (!set_smem(qlora_lora_down_kernel<true>, smem)) return QLORA_ERR_CUDA;
-    qlora_lora_down_kernel<true><<<grid, lora::kThreads, smem, st>>>(p);
+    if (launch_pdl(qlora_lora_down_kernel<true>, grid, dim3(lora::kThreads), smem, st, p) != cudaSuccess)
+      return QLORA_ERR_CUDA;
   } else {
     if (!set_smem(qlora_lora_down_kernel<false>, smem)) return QLORA_ERR_CUDA;
-    qlora_lora_down_kernel<false><<<grid, lora::kThreads, smem, st>>>(p);
+    if (launch_pdl(qlora_lora_down_kernel<false>, grid, dim3(lora::kThreads), smem, st, p) != cudaSuccess)
+      return QLORA_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
@@ -341,7 +361,9 @@ qlora_status_t launch_fused_t(const FusedParams& p, int grid, bool grouped, cuda
   const size_t smem = fused::smem_bytes(p.E);
   if (!set_smem(qlora_fused_gemm_kernel<FMT, DX>, smem)) return QLORA_ERR_CUDA;
   LaunchScope scope(grouped ? (DX ? kKindGFusedDx : kKindGFusedFwd) : (DX ? kKindFusedDx : kKindFusedFwd), st);
-  qlora_fused_gemm_kernel<FMT, DX><<<grid, fused::kThreads, smem, st>>>(p);
+  if (launch_pdl(qlora_fused_gemm_kernel<FMT, DX>, dim3(grid), dim3(fused::kThreads), smem, st, p) !=
+      cudaSuccess)
+    return QLORA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
@@ -400,7 +422,9 @@ qlora_status_t launch_stream_t(const StreamParams& p, int grid, cudaStream_t st)
   const size_t smem = stream::smem_bytes(p.xrows);
   if (!set_smem(qlora_stream_gemm_kernel<FMT, DX, MT>, smem)) return QLORA_ERR_CUDA;
   LaunchScope scope(DX ? kKindStreamDx : kKindStreamFwd, st);
-  qlora_stream_gemm_kernel<FMT, DX, MT><<<grid, stream::kThreads, smem, st>>>(p);
+  if (launch_pdl(qlora_stream_gemm_kernel<FMT, DX, MT>, dim3(grid), dim3(stream::kThreads), smem, st,
+                 p) != cudaSuccess)
+    return QLORA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
@@ -473,7 +497,9 @@ qlora_status_t launch_stream(const qlora_weight_t* W, bool dx, const void* act, 
   const int64_t threads = M * int64_t(sp.tiles) * (stream::BN / 4);
   if (!set_smem(qlora_stream_reduce_kernel, 0)) return QLORA_ERR_CUDA;
   LaunchScope scope(kKindStreamReduce, st);
-  qlora_stream_reduce_kernel<<<unsigned((threads + 255) / 256), 256, 0, st>>>(rp);
+  if (launch_pdl(qlora_stream_reduce_kernel, dim3(unsigned((threads + 255) / 256)), dim3(256), 0, st,
+                 rp) != cudaSuccess)
+    return QLORA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
@@ -517,7 +543,8 @@ qlora_status_t launch_wgrad(const void* X, const void* dY, const void* T, const 
   if (!set_smem(qlora_lora_wgrad_kernel, smem)) return QLORA_ERR_CUDA;
   const unsigned grid = unsigned(int64_t(E) * (wp.tiles0 + wp.tiles1) * wp.S);
   LaunchScope scope(grouped ? kKindGWgrad : kKindWgrad, st);
-  qlora_lora_wgrad_kernel<<<grid, lora::kThreads, smem, st>>>(p);
+  if (launch_pdl(qlora_lora_wgrad_kernel, dim3(grid), dim3(lora::kThreads), smem, st, p) != cudaSuccess)
+    return QLORA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 

@@ -235,6 +235,8 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
   ptx::cluster_sync();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
 
   const int num_tiles = grp_view.total();
   const int nk = p.num_k;

@@ -31,7 +31,7 @@
 
 namespace qlora {
 namespace lora {
-constexpr int BM = 128, BK = 64, NS = 6;
+constexpr int BM = 128, BK = 64, NS = 8;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int R_BYTES = 64 * 128;     // up to 64 x 128 B
 constexpr int kThreads = 6 * 32;      // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
@@ -189,6 +189,8 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   const uint32_t rowb = uint32_t(p.rpad) * 2u;
   const uint32_t r_bytes = uint32_t(p.rpad) * 128u;
 
@@ -345,6 +347,8 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   const uint32_t rowb = uint32_t(p.rpad) * 2u;
   const uint32_t r_bytes = 64u * rowb;
 

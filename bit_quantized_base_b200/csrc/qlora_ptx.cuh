@@ -87,6 +87,16 @@ __device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity, in
   }
 }
 
+// Programmatic dependent launch.  Every kernel of the library is launched so that it may start
+// while the previous kernel of the stream is still running: it does its prologue (barriers, tensor
+// memory, descriptor prefetch), then waits for the previous grid to complete and flush
+// (griddep_wait) before touching global memory, then lets the next kernel of the stream launch
+// (griddep_launch_dependents; its CTAs only take SMs this grid has left, and wait in turn).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------- CTA pairs
 // A cluster of two CTAs shares one tcgen05.mma.cta_group::2: rank 0 (the leader) issues it, each
 // CTA supplies half of the operands from its own shared memory and receives its half of D in its

@@ -152,6 +152,8 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------------ activation producer
@@ -411,6 +413,8 @@ __device__ __forceinline__ int stream_rank32(int st, int L, int nk1, int lcm) {
 __global__ void __launch_bounds__(256)
 qlora_stream_reduce_kernel(const __grid_constant__ StreamReduceParams p) {
   constexpr int BN = stream::BN, Q4 = BN / 4;
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   const int idx = int(blockIdx.x) * blockDim.x + threadIdx.x;
   const int per_row = p.num_tiles * Q4;
   if (idx >= per_row * p.M) return;
