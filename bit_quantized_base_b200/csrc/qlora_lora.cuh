@@ -77,36 +77,52 @@ __device__ __forceinline__ bool split_arrive(const float (&acc)[64], int rpad, i
 }
 
 // In the last CTA of a split tile: the 128 epilogue threads share out the (row, 8-column chunk)
-// items of rows [row0, row0 + nrows); each adds the S partials of its item in split order
-// 0..S-1 (loads issued four splits at a time) and hands the sum to write(row, c0, v[8]).
+// items of rows [row0, row0 + nrows), two items per round; each adds the S partials of its items
+// in split order 0..S-1, with the loads of up to eight splits of both items in flight at once, and
+// hands each sum to write(row, c0, v[8]).
 template <class F>
 __device__ __forceinline__ void split_sum(int rpad, int S, const float* partial, size_t rows_total,
                                           int row0, int nrows, int et, F&& write) {
   const int chunks = rpad / 8;
   const int items = nrows * chunks;
   const size_t sstride = rows_total * size_t(rpad);
-  for (int it = et; it < items; it += 128) {
-    const int rr = it / chunks, c0 = (it - rr * chunks) * 8;
-    const float* src = partial + size_t(row0 + rr) * rpad + c0;
-    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int sp = 0; sp < S; sp += 4) {
-      float4 a[4], b[4];
+  for (int it0 = et; it0 < items; it0 += 256) {
+    const float* src[2];
+    bool have[2];
+    int rr[2], c0[2];
+    float v[2][8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (sp + u < S) {
-          a[u] = __ldcg(reinterpret_cast<const float4*>(src + size_t(sp + u) * sstride));
-          b[u] = __ldcg(reinterpret_cast<const float4*>(src + size_t(sp + u) * sstride + 4));
-        }
-      }
+    for (int u = 0; u < 2; ++u) {
+      const int it = it0 + u * 128;
+      have[u] = it < items;
+      rr[u] = have[u] ? it / chunks : 0;
+      c0[u] = have[u] ? (it - rr[u] * chunks) * 8 : 0;
+      src[u] = partial + size_t(row0 + rr[u]) * rpad + c0[u];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (sp + u < S) {
-          v[0] += a[u].x; v[1] += a[u].y; v[2] += a[u].z; v[3] += a[u].w;
-          v[4] += b[u].x; v[5] += b[u].y; v[6] += b[u].z; v[7] += b[u].w;
-        }
-      }
+      for (int c = 0; c < 8; ++c) v[u][c] = 0.f;
     }
-    write(row0 + rr, c0, v);
+    for (int sp = 0; sp < S; sp += 8) {
+      float4 a[2][8], b[2][8];
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (have[u] && sp + q < S) {
+            a[u][q] = __ldcg(reinterpret_cast<const float4*>(src[u] + size_t(sp + q) * sstride));
+            b[u][q] = __ldcg(reinterpret_cast<const float4*>(src[u] + size_t(sp + q) * sstride + 4));
+          }
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (have[u] && sp + q < S) {
+            v[u][0] += a[u][q].x; v[u][1] += a[u][q].y; v[u][2] += a[u][q].z; v[u][3] += a[u][q].w;
+            v[u][4] += b[u][q].x; v[u][5] += b[u][q].y; v[u][6] += b[u][q].z; v[u][7] += b[u][q].w;
+          }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+      if (have[u]) write(row0 + rr[u], c0[u], v[u]);
   }
 }
 
