@@ -404,8 +404,17 @@ qlora_status_t launch_fused(const qlora_weight_t* W, bool dx, const void* act, c
   p.num_k = int((Kc + fused::BK - 1) / fused::BK);
   // one CTA pair per pair tile, at most one pair per two SMs (persistent beyond that); the tile
   // count of a grouped launch is known only on the device: at most ceil(M/256) + E - 1 row tiles
-  const int64_t tiles = ((M + fused::BM - 1) / fused::BM + (E > 1 ? E - 1 : 0)) * p.num_n;
-  const int64_t pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
+  int64_t tiles = ((M + fused::BM - 1) / fused::BM + (E > 1 ? E - 1 : 0)) * p.num_n;
+  int64_t pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
+  // One layer whose last wave of tiles would leave most pairs idle: split that wave's 512-row
+  // tiles in two 256-row tiles each, scheduled last, so the wave takes about half as long.
+  p.tail_split = 0;
+  if (!grouped && E == 1 && pairs > 0) {
+    const int64_t rem = tiles % pairs;
+    if (rem > 0 && 2 * rem <= pairs && tiles > pairs) p.tail_split = int(rem);
+  }
+  tiles += p.tail_split;
+  pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
   const int grid = int(2 * (pairs > 0 ? pairs : 1));
   switch (W->fmt * 2 + (dx ? 1 : 0)) {
     case 0: return launch_fused_t<kFmtNF4, false>(p, grid, grouped, st);

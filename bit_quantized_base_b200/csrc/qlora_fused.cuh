@@ -82,6 +82,7 @@ struct FusedParams {
   int* status;
   int M, N, K, r, E;                 // M: all rows (packed over experts)
   int num_n, num_k;                  // pair tiles over output columns; contraction steps
+  int tail_split;                    // the last tail_split 512-row tiles run as 2 x 256-row tiles
 };
 
 __device__ __forceinline__ void fused_tile_coords(int t, int num_m, int num_n, int& mt, int& nt) {
@@ -134,10 +135,19 @@ __device__ __forceinline__ const void* item_scale_word(const void* scales, int n
 // Pair tile t of a (grouped) launch: expert e, rows [row0, row0 + 256) of which rows below
 // row_end belong to the expert, output-column tile nt.
 struct PairTile {
-  int e, row0, row_end, nt;
+  int e, row0, row_end, nt, nb;   // nb: MMA blocks of 256 rows in the tile (2, or 1 for a split tile)
 };
-__device__ __forceinline__ PairTile pair_tile_at(const GroupView& g, int t, int num_n) {
+// Tiles [0, total - tail) are the 512-row tiles of the table; when the last wave of tiles would
+// leave most pairs idle, the host asks for the last `tail` of them to be split in two 256-row
+// tiles each, scheduled after all others (indices total - tail .. total + tail - 1).
+__device__ __forceinline__ PairTile pair_tile_at(const GroupView& g, int t, int num_n, int tail) {
   PairTile pt;
+  int half = -1;
+  const int nbig = g.total() - tail;
+  if (t >= nbig) {
+    half = (t - nbig) & 1;
+    t = nbig + ((t - nbig) >> 1);
+  }
   pt.e = g.expert_of(t);
   const int local = t - g.first[pt.e];
   const int rows = g.off[pt.e + 1] - g.off[pt.e];
@@ -147,6 +157,12 @@ __device__ __forceinline__ PairTile pair_tile_at(const GroupView& g, int t, int 
   pt.row0 = g.off[pt.e] + mt * fused::BM;
   pt.row_end = g.off[pt.e + 1];
   pt.nt = nt;
+  pt.nb = fused::MB;
+  if (half >= 0) {
+    pt.row0 += half * 2 * fused::HM;
+    pt.row_end = min(pt.row_end, pt.row0 + 2 * fused::HM);
+    pt.nb = 1;
+  }
   return pt;
 }
 
@@ -238,7 +254,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
 
-  const int num_tiles = grp_view.total();
+  const int num_tiles = grp_view.total() + p.tail_split;
   const int nk = p.num_k;
 
   if (warp == kTmaWarp) {
@@ -246,16 +262,15 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     if (lane == 0) {
       uint32_t i = 0;
       for (int t = pair; t < num_tiles; t += npairs) {
-        const PairTile pt = pair_tile_at(grp_view, t, p.num_n);
+        const PairTile pt = pair_tile_at(grp_view, t, p.num_n, p.tail_split);
         const int m0 = pt.row0 + int(rank) * HM;      // this CTA's rows of block 0 (+256: block 1)
         bool ok = true;
         for (int ks = 0; ks <= nk; ++ks, ++i) {
           const uint32_t sx = i % NS, px = (i / NS) & 1u;
           if (!ptx::mbar_wait(empty_s(sx), px ^ 1u, p.status, abort_flag)) { ok = false; break; }
-          if (rank == 0) ptx::mbar_arrive_expect_tx(full_s(sx), 2 * MB * X_BYTES);
+          if (rank == 0) ptx::mbar_arrive_expect_tx(full_s(sx), 2 * pt.nb * X_BYTES);
           const uint32_t fx = ptx::mapa(full_s(sx), 0);
-#pragma unroll
-          for (int blk = 0; blk < MB; ++blk) {
+          for (int blk = 0; blk < pt.nb; ++blk) {
             const uint32_t xd = ptx::smem_u32(xs + (sx * MB + blk) * X_BYTES);
             if (ks < nk) ptx::tma_load_2d_pair(xd, &p.tm_act, fx, ks * BK, m0 + blk * 2 * HM);
             else ptx::tma_load_2d_pair(xd, &p.tm_zs, fx, 0, m0 + blk * 2 * HM);
@@ -269,7 +284,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     if (lane == 0) {
       uint32_t j = 0;
       for (int t = pair; t < num_tiles; t += npairs) {
-        const PairTile pt = pair_tile_at(grp_view, t, p.num_n);
+        const PairTile pt = pair_tile_at(grp_view, t, p.num_n, p.tail_split);
         const int h0 = pt.nt * BN + int(rank) * HN;   // this CTA's weight half
         const int wrow0 = pt.e * p.N;                 // the expert's first row of the codes
         bool ok = true;
@@ -291,6 +306,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
       const int lora_kk = (p.r + 15) / 16;
       uint32_t i = 0, tc = 0;
       for (int t = pair; t < num_tiles; t += npairs, ++tc) {
+        const int nb = pair_tile_at(grp_view, t, p.num_n, p.tail_split).nb;
         if (!ptx::mbar_wait_cluster(acc_empty, (tc & 1u) ^ 1u, p.status, abort_flag)) break;
         ptx::tc_fence_after();
         bool ok = true;
@@ -304,11 +320,11 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
           for (int kk = 0; kk < nkk; ++kk) {
             const uint64_t bd = DX ? ptx::smem_desc(wb + kk * 2048, 8192, 1024, ptx::kSw128)
                                    : ptx::smem_desc(wb + kk * 32, 16, 1024, ptx::kSw128);
-#pragma unroll
-            for (int blk = 0; blk < MB; ++blk) {
-              const uint64_t ad = ptx::smem_desc(xa + blk * X_BYTES + kk * 32, 16, 1024, ptx::kSw128);
-              ptx::mma_bf16_pair(tmem + blk * BN, ad, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
-            }
+            const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
+            ptx::mma_bf16_pair(tmem, ptx::smem_desc(xa + kk * 32, 16, 1024, ptx::kSw128), bd, idesc, acc);
+            if (nb == 2)
+              ptx::mma_bf16_pair(tmem + BN, ptx::smem_desc(xa + X_BYTES + kk * 32, 16, 1024, ptx::kSw128),
+                                 bd, idesc, acc);
           }
           ptx::mma_commit_pair(empty_s(st), 3);
         }
@@ -336,13 +352,13 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     const uint32_t acc_empty_leader = ptx::mapa(acc_empty, 0);
     uint32_t tc = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++tc) {
-      const PairTile pt = pair_tile_at(grp_view, t, p.num_n);
+      const PairTile pt = pair_tile_at(grp_view, t, p.num_n, p.tail_split);
       const int c0 = pt.nt * BN;
       const float ts = (FMT == kFmtNVFP4 && p.tensor_scale) ? __ldg(p.tensor_scale + pt.e) : 1.0f;
       if (!ptx::mbar_wait(acc_full, tc & 1u, p.status, abort_flag)) break;
       ptx::tc_fence_after();
 #pragma unroll 1
-      for (int blk = 0; blk < MB; ++blk) {
+      for (int blk = 0; blk < pt.nb; ++blk) {
         const int row = pt.row0 + blk * 2 * HM + int(rank) * HM + q * 32 + lane;
         if (pt.row0 + blk * 2 * HM + int(rank) * HM + q * 32 >= pt.row_end) continue;   // warp-uniform
 #pragma unroll 1
@@ -384,7 +400,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     };
     auto set_tile = [&](Cursor& c) {
       if (c.t < num_tiles) {
-        const PairTile pt = pair_tile_at(grp_view, c.t, p.num_n);
+        const PairTile pt = pair_tile_at(grp_view, c.t, p.num_n, p.tail_split);
         c.h0 = pt.nt * BN + int(rank) * HN;
         c.e = pt.e;
       }
