@@ -302,8 +302,18 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer (leader)
     if (lane == 0 && rank == 0) {
+      // Lean issue loop: the issuing thread shares its SM sub-partition with busy dequant warps, so
+      // every instruction between two steps' MMAs costs several cycles of tensor-pipe time.
+      // Descriptors are the stage-0 descriptors plus constant offsets (the 14-bit address field
+      // never carries), the four 16-deep sub-steps are unrolled, and the stage ring is a power of 2.
+      static_assert((NS & (NS - 1)) == 0, "stage count must be a power of two");
       const uint32_t idesc = ptx::idesc_bf16(256, BN, 0, DX ? 1u : 0u);
       const int lora_kk = (p.r + 15) / 16;
+      const uint64_t a0 = ptx::smem_desc(ptx::smem_u32(xs), 16, 1024, ptx::kSw128);
+      const uint64_t b0d = DX ? ptx::smem_desc(ptx::smem_u32(wsm), 8192, 1024, ptx::kSw128)
+                              : ptx::smem_desc(ptx::smem_u32(wsm), 16, 1024, ptx::kSw128);
+      constexpr uint64_t kAStage = (MB * X_BYTES) >> 4, kBStage = W_BYTES >> 4;
+      constexpr uint64_t kABlk = X_BYTES >> 4, kAkk = 32 >> 4, kBkk = DX ? (2048 >> 4) : (32 >> 4);
       uint32_t i = 0, tc = 0;
       for (int t = pair; t < num_tiles; t += npairs, ++tc) {
         const int nb = pair_tile_at(grp_view, t, p.num_n, p.tail_split).nb;
@@ -311,20 +321,28 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
         ptx::tc_fence_after();
         bool ok = true;
         for (int ks = 0; ks <= nk; ++ks, ++i) {
-          const uint32_t st = i % NS;
+          const uint32_t st = i & (NS - 1);
           if (!ptx::mbar_wait_cluster(full_s(st), (i / NS) & 1u, p.status, abort_flag)) { ok = false; break; }
           ptx::tc_fence_after();
-          const uint32_t xa = ptx::smem_u32(xs + st * MB * X_BYTES);
-          const uint32_t wb = ptx::smem_u32(wsm + st * W_BYTES);
-          const int nkk = ks < nk ? BK / 16 : lora_kk;
-          for (int kk = 0; kk < nkk; ++kk) {
-            const uint64_t bd = DX ? ptx::smem_desc(wb + kk * 2048, 8192, 1024, ptx::kSw128)
-                                   : ptx::smem_desc(wb + kk * 32, 16, 1024, ptx::kSw128);
-            const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
-            ptx::mma_bf16_pair(tmem, ptx::smem_desc(xa + kk * 32, 16, 1024, ptx::kSw128), bd, idesc, acc);
-            if (nb == 2)
-              ptx::mma_bf16_pair(tmem + BN, ptx::smem_desc(xa + X_BYTES + kk * 32, 16, 1024, ptx::kSw128),
-                                 bd, idesc, acc);
+          const uint64_t a = a0 + st * kAStage, b = b0d + st * kBStage;
+          if (ks < nk) {
+            const uint32_t acc0 = ks > 0 ? 1u : 0u;
+            if (nb == 2) {
+#pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk) {
+                ptx::mma_bf16_pair(tmem, a + kk * kAkk, b + kk * kBkk, idesc, kk ? 1u : acc0);
+                ptx::mma_bf16_pair(tmem + BN, a + kABlk + kk * kAkk, b + kk * kBkk, idesc, kk ? 1u : acc0);
+              }
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk)
+                ptx::mma_bf16_pair(tmem, a + kk * kAkk, b + kk * kBkk, idesc, kk ? 1u : acc0);
+            }
+          } else {
+            for (int kk = 0; kk < lora_kk; ++kk) {
+              ptx::mma_bf16_pair(tmem, a + kk * kAkk, b + kk * kBkk, idesc, 1u);
+              if (nb == 2) ptx::mma_bf16_pair(tmem + BN, a + kABlk + kk * kAkk, b + kk * kBkk, idesc, 1u);
+            }
           }
           ptx::mma_commit_pair(empty_s(st), 3);
         }
