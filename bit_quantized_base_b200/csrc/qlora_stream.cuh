@@ -192,8 +192,17 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      // Lean issue loop (the thread shares its SM sub-partition with busy dequant warps):
+      // descriptors are stage-0 descriptors plus constant offsets, the 16-deep sub-steps unrolled.
       const uint32_t idesc = ptx::idesc_bf16(128, uint32_t(p.xrows), DX ? 1u : 0u, 0u);
       const int lora_kk = (p.r + 15) / 16;
+      const uint64_t bx0 = ptx::smem_desc(xs(0), 16, 1024, ptx::kSw128);
+      const uint64_t aw0 = DX ? ptx::smem_desc(wsm(0), 8192, 1024, ptx::kSw128)
+                              : ptx::smem_desc(wsm(0), 16, 1024, ptx::kSw128);
+      const uint64_t kXStage = XSTAGE >> 4;
+      constexpr uint64_t kWStage = W_BYTES >> 4, kWHalf = HW_BYTES >> 4;
+      constexpr uint64_t kXkk = 32 >> 4, kWkk = DX ? (2048 >> 4) : (32 >> 4);
+      const uint32_t xr = uint32_t(p.xrows);
       uint32_t b = 0, bph = 0, s = 0, ph = 0;
       int ks = rg.step(rg.g0);
       bool first = true;
@@ -204,17 +213,19 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
         }
         if (!ptx::mbar_wait(full_s(s), ph, p.status, abort_flag)) break;
         ptx::tc_fence_after();
-        const int nkk = ks < nk ? BK / 16 : lora_kk;
-        const uint32_t xa = xs(s), wb = wsm(s);
-        const uint32_t d0 = tmem + b * 2u * uint32_t(p.xrows);
-        for (int kk = 0; kk < nkk; ++kk) {
-          const uint64_t bd = ptx::smem_desc(xa + kk * 32, 16, 1024, ptx::kSw128);
+        const uint64_t bx = bx0 + s * kXStage, aw = aw0 + s * kWStage;
+        const uint32_t d0 = tmem + b * 2u * xr;
+        const uint32_t acc0 = first ? 0u : 1u;
+        if (ks < nk) {
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const uint32_t wh = wb + hh * HW_BYTES;
-            const uint64_t ad = DX ? ptx::smem_desc(wh + kk * 2048, 8192, 1024, ptx::kSw128)
-                                   : ptx::smem_desc(wh + kk * 32, 16, 1024, ptx::kSw128);
-            ptx::mma_bf16(d0 + hh * uint32_t(p.xrows), ad, bd, idesc, (!first || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            ptx::mma_bf16(d0, aw + kk * kWkk, bx + kk * kXkk, idesc, kk ? 1u : acc0);
+            ptx::mma_bf16(d0 + xr, aw + kWHalf + kk * kWkk, bx + kk * kXkk, idesc, kk ? 1u : acc0);
+          }
+        } else {
+          for (int kk = 0; kk < lora_kk; ++kk) {
+            ptx::mma_bf16(d0, aw + kk * kWkk, bx + kk * kXkk, idesc, kk ? 1u : acc0);
+            ptx::mma_bf16(d0 + xr, aw + kWHalf + kk * kWkk, bx + kk * kXkk, idesc, kk ? 1u : acc0);
           }
         }
         ptx::mma_commit(empty_s(s));
