@@ -21,7 +21,8 @@
 // meanwhile.
 //
 // Warp roles per CTA (480 threads, one CTA per SM, persistent over pair tiles):
-//   warps 0-3   epilogue: tensor memory (both blocks) -> registers -> * ts -> bf16 -> global
+//   warps 0-3   epilogue: tensor memory (both blocks) -> registers -> * ts -> bf16 -> a per-warp
+//               staging tile in shared memory -> coalesced 64-byte row segments to global
 //   warp  4     TMA producer of this CTA's activation half (completion counted on the leader's
 //               barrier)
 //   warp  6     TMA producer of this CTA's packed-code tiles, running ahead of the activation
@@ -56,7 +57,7 @@ constexpr int BM = 512, BN = 256;      // pair tile
 constexpr int HM = 128, HN = 128;      // per-CTA rows of one MMA block; per-CTA weight half
 constexpr int MB = 2;                  // MMA blocks of 256 rows per pair tile
 constexpr int BK = 64;
-constexpr int NS = 4, NC = 6;         // operand stages (activation blocks + weight half), code stages
+constexpr int NS = 4, NC = 4;         // operand stages (activation blocks + weight half), code stages
 constexpr int X_BYTES = HM * BK * 2;   // 16 KB per block
 constexpr int W_BYTES = HN * BK * 2;   // 16 KB
 constexpr int C_BYTES = HN * BK / 2;   // 4 KB of packed codes
@@ -65,7 +66,10 @@ constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;
 constexpr int kTmemCols = 512;         // 2 blocks x 256 columns
 constexpr int GM = 8;                  // m-tiles per raster group
 constexpr int kNumBars = 2 * NS + 2 * NC + 2;
-constexpr size_t kSmemBase = 1024 + size_t(NS) * (MB * X_BYTES + W_BYTES) + size_t(NC) * C_BYTES + 1024;
+// epilogue staging: per epilogue warp one tile of 32 rows x 32 output columns (bf16)
+constexpr int STG_BYTES = 32 * 32 * 2;
+constexpr size_t kStgOff = size_t(NS) * (MB * X_BYTES + W_BYTES) + size_t(NC) * C_BYTES + 1024;
+constexpr size_t kSmemBase = 1024 + kStgOff + size_t(kEpiWarps) * STG_BYTES;
 // plus the expert table: 2 x (E + 1) ints
 __host__ __device__ constexpr size_t smem_bytes(int E) { return kSmemBase + size_t(2) * (E + 1) * 4; }
 }  // namespace fused
@@ -365,9 +369,17 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     }
   } else if (warp < kEpiWarps) {
     // ------------------------------------------------------------------ epilogue
+    // Each warp drains its 32 accumulator lanes (rows) 32 columns at a time: scaled, rounded to
+    // bf16 and written as one row per lane into a 32 x 32 staging tile (16-byte chunks XOR-swizzled
+    // by row, so neither the row writes nor the column reads conflict), then read back 8 rows x
+    // 64 bytes per warp instruction, so each global store covers 8 row segments of 64 contiguous
+    // bytes instead of 32 scattered 16-byte pieces.
     const int q = warp;  // tensor-memory lanes 32q .. 32q+31
     const int ncols = DX ? p.K : p.N;
     const uint32_t acc_empty_leader = ptx::mapa(acc_empty, 0);
+    const uint32_t stg = ptx::smem_u32(smem + kStgOff) + uint32_t(q) * STG_BYTES;
+    const uint32_t wsw = (uint32_t(lane) >> 1) & 3u;             // write swizzle of row `lane`
+    const int rr0 = lane >> 2, rc = lane & 3;                     // read: row rr0 + 8 it, chunk rc
     uint32_t tc = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++tc) {
       const PairTile pt = pair_tile_at(grp_view, t, p.num_n, p.tail_split);
@@ -377,27 +389,39 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
       ptx::tc_fence_after();
 #pragma unroll 1
       for (int blk = 0; blk < pt.nb; ++blk) {
-        const int row = pt.row0 + blk * 2 * HM + int(rank) * HM + q * 32 + lane;
-        if (pt.row0 + blk * 2 * HM + int(rank) * HM + q * 32 >= pt.row_end) continue;   // warp-uniform
+        const int rbase = pt.row0 + blk * 2 * HM + int(rank) * HM + q * 32;
+        if (rbase >= pt.row_end) continue;   // warp-uniform
+        const uint32_t tb = tmem + (uint32_t(q * 32) << 16) + uint32_t(blk * BN);
 #pragma unroll 1
         for (int cb = 0; cb < BN / 32; ++cb) {
           uint32_t v[32];
-          ptx::tmem_ld_32x32b_x32(tmem + (uint32_t(q * 32) << 16) + blk * BN + cb * 32, v);
-          ptx::tmem_ld_wait();
-          if (row < pt.row_end) {
-            __nv_bfloat16* orow = p.out + size_t(row) * ncols;
+          ptx::tmem_ld_32x32b_x32(tb + uint32_t(cb) * 32u, v);
+          ptx::tmem_ld_wait(v);
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const int col = c0 + cb * 32 + g * 8;
-              if (col < ncols) {
-                uint4 o;
-                o.x = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 0]) * ts, __uint_as_float(v[g * 8 + 1]) * ts);
-                o.y = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 2]) * ts, __uint_as_float(v[g * 8 + 3]) * ts);
-                o.z = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 4]) * ts, __uint_as_float(v[g * 8 + 5]) * ts);
-                o.w = ptx::cvt_bf16x2(__uint_as_float(v[g * 8 + 6]) * ts, __uint_as_float(v[g * 8 + 7]) * ts);
-                *reinterpret_cast<uint4*>(orow + col) = o;
-              }
+          for (int g = 0; g < 4; ++g) {
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float lo = __uint_as_float(v[g * 8 + 2 * j]), hi = __uint_as_float(v[g * 8 + 2 * j + 1]);
+              if constexpr (FMT == kFmtNVFP4) { lo *= ts; hi *= ts; }
+              w[j] = ptx::cvt_bf16x2(lo, hi);
             }
+            ptx::st_shared_v4(stg + uint32_t(lane) * 64u + ((uint32_t(g) ^ wsw) << 4), w[0], w[1], w[2], w[3]);
+          }
+          __syncwarp();
+          uint4 o[4];
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const uint32_t rr = uint32_t(it * 8 + rr0);
+            o[it] = ptx::ld_shared_v4(stg + rr * 64u + ((uint32_t(rc) ^ ((rr >> 1) & 3u)) << 4));
+          }
+          __syncwarp();
+          const int col = c0 + cb * 32 + rc * 8;
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int row = rbase + it * 8 + rr0;
+            if (row < pt.row_end && col < ncols)
+              *reinterpret_cast<uint4*>(p.out + size_t(row) * ncols + col) = o[it];
           }
         }
       }

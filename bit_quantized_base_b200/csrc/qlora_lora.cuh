@@ -133,7 +133,7 @@ __device__ __forceinline__ void load_acc_row(uint32_t taddr, int rpad, float (&a
     if (c < rpad) {
       uint32_t v[16];
       ptx::tmem_ld_32x32b_x16(taddr + c, v);
-      ptx::tmem_ld_wait();
+      ptx::tmem_ld_wait(v);
 #pragma unroll
       for (int g = 0; g < 16; ++g) acc[c + g] = __uint_as_float(v[g]);
     } else {

@@ -261,7 +261,7 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
         for (int m0 = 0; m0 < p.xrows; m0 += 16) {
           uint32_t v[16];
           ptx::tmem_ld_32x32b_x16(tcol + m0, v);
-          ptx::tmem_ld_wait();
+          ptx::tmem_ld_wait(v);
 #pragma unroll
           for (int u = 0; u < 16; ++u)
             if (m0 + u < p.M) __stcg(col + size_t(m0 + u) * BN, __uint_as_float(v[u]));
