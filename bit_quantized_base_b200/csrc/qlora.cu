@@ -20,8 +20,7 @@ namespace {
 
 // ------------------------------------------------------------------------------------ helpers
 constexpr size_t kHeaderBytes = 256;        // [0]: device status word
-constexpr int kMaxCounters = 16384;         // reduction tile counters
-constexpr size_t kCounterBytes = size_t(kMaxCounters) * 4;
+constexpr int kMaxClusterSplits = 8;        // split-K CTAs of one LoRA tile (one portable cluster)
 constexpr int kMaxDevices = 64;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -111,6 +110,28 @@ cudaError_t launch_pdl(void (*kernel)(P), dim3 grid, dim3 block, size_t smem, cu
   return cudaLaunchKernelEx(&cfg, kernel, params);
 }
 
+// As launch_pdl, with the grid cut into thread-block clusters of `cluster` CTAs along x (1: no
+// clusters).
+template <typename P>
+cudaError_t launch_pdl_cluster(void (*kernel)(P), dim3 grid, dim3 block, size_t smem,
+                               cudaStream_t st, const P& params, unsigned cluster) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cluster > 1 ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kernel, params);
+}
+
 qlora_status_t check_weight(const qlora_weight_t* W) {
   if (!W) return QLORA_ERR_INVALID_ARG;
   if (W->fmt < QLORA_FMT_NF4 || W->fmt > QLORA_FMT_NVFP4) return QLORA_ERR_INVALID_ARG;
@@ -141,7 +162,7 @@ WgradPlan wgrad_plan(int64_t N, int64_t K, int64_t M, int E, int sms) {
   p.tiles1 = int((K + 127) / 128);
   const int64_t tiles = int64_t(E) * (p.tiles0 + p.tiles1);
   int S = int(sms / tiles);                                  // at most one wave of long splits
-  S = S < 1 ? 1 : (S > 16 ? 16 : S);
+  S = S < 1 ? 1 : (S > kMaxClusterSplits ? kMaxClusterSplits : S);
   const int64_t chunks = (M + 63) / 64;                      // of one expert holding every row
   if (S > chunks) S = chunks > 0 ? int(chunks) : 1;
   p.S = S;
@@ -159,17 +180,12 @@ DownPlan down_plan(int64_t M, int64_t Kc, int E, int sms) {
   p.tiles = int((M + 127) / 128) + (E > 1 ? E - 1 : 0);
   p.num_k = int((Kc + 63) / 64);
   int S = p.tiles > 0 ? sms / p.tiles : 1;                   // at most one wave of long splits
-  S = S < 1 ? 1 : (S > 16 ? 16 : S);
+  S = S < 1 ? 1 : (S > kMaxClusterSplits ? kMaxClusterSplits : S);
   const int max_s = p.num_k / 2 > 0 ? p.num_k / 2 : 1;
   if (S > max_s) S = max_s;
   p.sps = (p.num_k + S - 1) / S;
   p.S = (p.num_k + p.sps - 1) / p.sps;
   return p;
-}
-
-size_t down_partial_bytes(int64_t M, int64_t Kc, int r, int E, int sms) {
-  const DownPlan dp = down_plan(M, Kc, E, sms);
-  return dp.S > 1 ? size_t(dp.S) * size_t(M) * size_t(rank_pad(r)) * 4 : 0;
 }
 
 // Short batches (M <= 256 rows, one weight) use the weight-streaming kernels: the flat space of
@@ -209,29 +225,18 @@ bool stream_fits(const qlora_weight_t* W, int64_t M, int E, bool dx, size_t regi
 
 struct WsLayout {
   size_t zs, t, u, partial, partial_bytes, total;
-  int counters_needed;
 };
 
 WsLayout ws_layout(int64_t N, int64_t K, int64_t M, int r, bool bwd, int E, int sms) {
   WsLayout L{};
-  size_t off = kHeaderBytes + kCounterBytes;
+  size_t off = kHeaderBytes;
   const size_t mr = align_up(size_t(M > 0 ? M : 0) * size_t(r) * 2, 256);
   L.zs = off; off += mr;
   L.t = off; off += mr;
   L.u = off; off += bwd ? mr : 0;
   L.partial = off;
-  // fp32 split partials, shared by the (sequential) lora_down and lora_wgrad launches
-  size_t pb = down_partial_bytes(M, K, r, E, sms);
-  L.counters_needed = down_plan(M, K, E, sms).tiles;
-  if (bwd) {
-    const size_t pu = down_partial_bytes(M, N, r, E, sms);
-    pb = pu > pb ? pu : pb;
-    const WgradPlan wp = wgrad_plan(N, K, M, E, sms);
-    const size_t pw = wp.S > 1 ? size_t(wp.S) * size_t(E) * size_t(N + K) * size_t(rank_pad(r)) * 4 : 0;
-    pb = pw > pb ? pw : pb;
-    const int wc = E * (wp.tiles0 + wp.tiles1);
-    if (wc > L.counters_needed) L.counters_needed = wc;
-  }
+  // fp32 partials of the short-batch weight-streaming kernels
+  size_t pb = 0;
   if (use_stream(M, E)) {
     const size_t sf = stream_plan(N, K, M, false, sms).partial_bytes;
     pb = sf > pb ? sf : pb;
@@ -247,7 +252,6 @@ WsLayout ws_layout(int64_t N, int64_t K, int64_t M, int r, bool bwd, int E, int 
 }
 
 int* ws_status(void* ws) { return reinterpret_cast<int*>(ws); }
-int* ws_counters(void* ws) { return reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + kHeaderBytes); }
 
 // ---------------------------------------------------------------------------------- profiling
 enum Kind : int {
@@ -302,21 +306,13 @@ bool tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_
 }
 
 // Z = Act . R for every expert's rows: R is A [E, r, Kc] (r_mn false, T = X A^T) or
-// B [E, Kc, r] (r_mn true, U = dY B).  partial / partial_bytes: fp32 scratch for the split
-// contraction (the split count is reduced until its partials fit); counters: zeroed ints, one per
-// row tile.  offsets == nullptr: one expert of M rows.
+// B [E, Kc, r] (r_mn true, U = dY B).  offsets == nullptr: one expert of M rows.
 qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t Kc, const void* R,
                                 int r, float s, const float* ts, void* z, void* zs, int* status,
-                                float* partial, size_t partial_bytes, int* counters,
                                 const int32_t* offsets, int E, bool grouped, cudaStream_t st) {
   DownParams p{};
   const int rpad = rank_pad(r);
-  DownPlan dp = down_plan(M, Kc, E, num_sms());
-  while (dp.S > 1 && size_t(dp.S) * size_t(M) * size_t(rpad) * 4 > partial_bytes) {
-    dp.sps = (dp.num_k + dp.S - 2) / (dp.S - 1);
-    dp.S = (dp.num_k + dp.sps - 1) / dp.sps;
-  }
-  if (dp.tiles > kMaxCounters) return QLORA_ERR_UNSUPPORTED;
+  const DownPlan dp = down_plan(M, Kc, E, num_sms());
   if (!tmap_2d(&p.tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, uint64_t(Kc), uint64_t(M),
                uint64_t(Kc) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
@@ -330,8 +326,6 @@ qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t K
   p.z = static_cast<__nv_bfloat16*>(z);
   p.zs = static_cast<__nv_bfloat16*>(zs);
   p.status = status;
-  p.partial = partial;
-  p.counters = counters;
   p.offsets = offsets;
   p.M = int(M);
   p.r = r;
@@ -346,11 +340,13 @@ qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t K
   LaunchScope scope(grouped ? (r_mn ? kKindGDownU : kKindGDownT) : (r_mn ? kKindDownU : kKindDownT), st);
   if (r_mn) {
     if (!set_smem(qlora_lora_down_kernel<true>, smem)) return QLORA_ERR_CUDA;
-    if (launch_pdl(qlora_lora_down_kernel<true>, grid, dim3(lora::kThreads), smem, st, p) != cudaSuccess)
+    if (launch_pdl_cluster(qlora_lora_down_kernel<true>, grid, dim3(lora::kThreads), smem, st, p,
+                           unsigned(dp.S)) != cudaSuccess)
       return QLORA_ERR_CUDA;
   } else {
     if (!set_smem(qlora_lora_down_kernel<false>, smem)) return QLORA_ERR_CUDA;
-    if (launch_pdl(qlora_lora_down_kernel<false>, grid, dim3(lora::kThreads), smem, st, p) != cudaSuccess)
+    if (launch_pdl_cluster(qlora_lora_down_kernel<false>, grid, dim3(lora::kThreads), smem, st, p,
+                           unsigned(dp.S)) != cudaSuccess)
       return QLORA_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
@@ -531,8 +527,6 @@ qlora_status_t launch_wgrad(const void* X, const void* dY, const void* T, const 
       !tmap_2d(&p.tm_r[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U, uint64_t(r), rows,
                uint64_t(r) * 2, uint32_t(rpad), 64, rsw))
     return QLORA_ERR_CUDA;
-  p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.partial);
-  p.counters = ws_counters(ws);
   p.out0 = static_cast<__nv_bfloat16*>(dB);
   p.out1 = static_cast<__nv_bfloat16*>(dA);
   p.offsets = offsets;
@@ -547,12 +541,12 @@ qlora_status_t launch_wgrad(const void* X, const void* dY, const void* T, const 
   p.tiles1 = wp.tiles1;
   p.E = E;
   p.s = s;
-  if (int64_t(E) * (wp.tiles0 + wp.tiles1) > kMaxCounters) return QLORA_ERR_UNSUPPORTED;
   const size_t smem = lora::smem_bytes(E);
   if (!set_smem(qlora_lora_wgrad_kernel, smem)) return QLORA_ERR_CUDA;
   const unsigned grid = unsigned(int64_t(E) * (wp.tiles0 + wp.tiles1) * wp.S);
   LaunchScope scope(grouped ? kKindGWgrad : kKindWgrad, st);
-  if (launch_pdl(qlora_lora_wgrad_kernel, dim3(grid), dim3(lora::kThreads), smem, st, p) != cudaSuccess)
+  if (launch_pdl_cluster(qlora_lora_wgrad_kernel, dim3(grid), dim3(lora::kThreads), smem, st, p,
+                         unsigned(wp.S)) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
@@ -625,12 +619,12 @@ size_t qlora_workspace_size(int op, const qlora_weight_t* W, int64_t M, int r, i
   if (grouped && (E < 1 || E > kMaxExperts)) return 0;
   const WsLayout L = ws_layout(W->N, W->K, M, r, op == QLORA_OP_BWD || op == QLORA_OP_GROUPED_BWD,
                                grouped ? E : 1, num_sms());
-  return L.counters_needed > kMaxCounters ? 0 : L.total;
+  return L.total;
 }
 
 qlora_status_t qlora_workspace_init(void* ws, size_t ws_bytes, qlora_stream_t stream) {
-  if (!ws || !aligned16(ws) || ws_bytes < kHeaderBytes + kCounterBytes) return QLORA_ERR_WORKSPACE;
-  return cudaMemsetAsync(ws, 0, kHeaderBytes + kCounterBytes, reinterpret_cast<cudaStream_t>(stream)) ==
+  if (!ws || !aligned16(ws) || ws_bytes < kHeaderBytes) return QLORA_ERR_WORKSPACE;
+  return cudaMemsetAsync(ws, 0, kHeaderBytes, reinterpret_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
              ? QLORA_OK
              : QLORA_ERR_CUDA;
@@ -660,7 +654,6 @@ qlora_status_t run_fwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   if (!act_ok(X, M) || !ptr_ok(A) || !ptr_ok(B) || !act_ok(Y, M) || (T_save && !aligned16(T_save)))
     return QLORA_ERR_INVALID_ARG;
   const WsLayout L = ws_layout(W->N, W->K, M, r, false, E, num_sms());
-  if (L.counters_needed > kMaxCounters) return QLORA_ERR_UNSUPPORTED;
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (M == 0) return QLORA_OK;
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -668,8 +661,7 @@ qlora_status_t run_fwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   void* Zs = w + L.zs;
   const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
   qlora_status_t st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, T, Zs, ws_status(ws),
-                                       reinterpret_cast<float*>(w + L.partial), L.partial_bytes,
-                                       ws_counters(ws), offsets, E, grouped, s);
+                                       offsets, E, grouped, s);
   if (st != QLORA_OK) return st;
   if (stream_fits(W, M, E, false, ws_bytes - L.partial))
     return launch_stream(W, false, X, Zs, B, Y, M, r, ws_status(ws),
@@ -686,7 +678,6 @@ qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
       (T && !aligned16(T)) || (dX && !aligned16(dX)))
     return QLORA_ERR_INVALID_ARG;
   const WsLayout L = ws_layout(W->N, W->K, M, r, true, E, num_sms());
-  if (L.counters_needed > kMaxCounters) return QLORA_ERR_UNSUPPORTED;
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (M == 0) {
     if (cudaMemsetAsync(dA, 0, size_t(E) * r * W->K * 2, s) != cudaSuccess ||
@@ -701,13 +692,13 @@ qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   float* part = reinterpret_cast<float*>(w + L.partial);
   qlora_status_t st;
   if (!T) {  // recompute T = X A^T (its scaled copy lands in Zs and is overwritten below)
-    st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, w + L.t, Zs, ws_status(ws), part,
-                          L.partial_bytes, ws_counters(ws), offsets, E, grouped, s);
+    st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, w + L.t, Zs, ws_status(ws), offsets,
+                          E, grouped, s);
     if (st != QLORA_OK) return st;
     T = w + L.t;
   }
-  st = launch_lora_down(true, dY, M, W->N, B, r, scale, ts, U, Zs, ws_status(ws), part,
-                        L.partial_bytes, ws_counters(ws), offsets, E, grouped, s);
+  st = launch_lora_down(true, dY, M, W->N, B, r, scale, ts, U, Zs, ws_status(ws), offsets, E,
+                        grouped, s);
   if (st != QLORA_OK) return st;
   const bool short_dx = dX && stream_fits(W, M, E, true, ws_bytes - L.partial);
   if (dX && !short_dx) {
@@ -777,13 +768,7 @@ qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const void* X, 
   void* Zs = w + kHeaderBytes;
   void* T = T_save ? T_save : w + kHeaderBytes + mr;
   const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
-  // the rest of the array holds the lora_down split partials (fewer splits if it is short)
-  const size_t used = kHeaderBytes + 256 + mr + (T_save ? 0 : mr);
-  float* part = reinterpret_cast<float*>(w + used);
-  const size_t part_bytes = kNoAllocScratchBytes - used;
-  int* counters = reinterpret_cast<int*>(w + 128);   // 32 tile counters inside the header
-  st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, T, Zs, status, part,
-                        (M + 127) / 128 <= 32 ? part_bytes : 0, counters, nullptr, 1, false, s);
+  st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, T, Zs, status, nullptr, 1, false, s);
   if (st != QLORA_OK) return st;
   return launch_fused(W, false, X, Zs, B, Y, M, r, status, nullptr, 1, false, s);
 }

@@ -21,9 +21,9 @@
 // before the MMA, so no row of another expert enters a reduction.
 //
 // Both kernels are memory bound (they stream an activation once) and have few output tiles, so
-// the contraction is split to fill the GPU.  Each split stores its fp32 partial tile; the last
-// split to finish (an atomic counter per tile, reset by that CTA for the next call) adds the S
-// partials in split order 0..S-1, so the result is bitwise deterministic.
+// the contraction is split over S CTAs per tile to fill the GPU.  The S CTAs of a tile run as one
+// thread-block cluster and add their fp32 partial tiles through distributed shared memory, in
+// split order 0..S-1, so the result is bitwise deterministic.
 #pragma once
 #include <cuda_bf16.h>
 #include "qlora_ptx.cuh"
@@ -44,85 +44,64 @@ __device__ __forceinline__ uint32_t swz_mode_for_row_bytes(uint32_t rowb) {
   return rowb == 128 ? ptx::kSw128 : (rowb == 64 ? ptx::kSw64 : ptx::kSw32);
 }
 
-// Epilogue of a split tile, run by the 128 epilogue threads (named barrier 1).  acc holds this
-// thread's accumulator row (rpad fp32 values); with S > 1 it is stored as partial `split` at
-// partial + (split * rows_total + row) * rpad and the tile's counter is incremented.  Returns true
-// in the last CTA of the tile to arrive (which then calls split_sum; the counter is reset for the
-// next call), and true with S == 1 (nothing stored: the caller writes acc directly).  All 128
-// threads must call it (rows outside the problem pass row_ok = false and take part in the
-// barriers only).
-__device__ __forceinline__ bool split_arrive(const float (&acc)[64], int rpad, int S, int split,
-                                             float* partial, size_t rows_total, int row, bool row_ok,
-                                             int* counter, volatile int* last_flag, int et) {
-  if (S == 1) return true;
-  if (row_ok) {
-    float* dst = partial + (size_t(split) * rows_total + size_t(row)) * rpad;
-#pragma unroll
-    for (int c = 0; c < 64; c += 4)
-      if (c < rpad) __stcg(reinterpret_cast<float4*>(dst + c), make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
-  }
-  __threadfence();
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-  if (et == 0) {
-    const int old = atomicAdd(counter, 1);
-    *last_flag = (old == S - 1) ? 1 : 0;
-  }
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-  const bool last = *last_flag != 0;
-  if (last) {
-    __threadfence();
-    if (et == 0) *counter = 0;   // ready for the next call on this workspace
-  }
-  return last;
+// Split-K reduction through distributed shared memory.  The S CTAs that share one 128-row output
+// tile form a thread-block cluster (cluster rank = split).  Each stores its fp32 partial tile
+// (128 rows x rpad, row-major, 16-byte chunks XOR-swizzled by row so that the row-per-lane stores
+// of a warp do not conflict) in its own shared memory; after a cluster barrier, CTA `split` sums
+// rows [split * ceil(128 / S), ...) of all S partials, read in split order 0..S-1 -- so the result
+// is bitwise deterministic -- and a second cluster barrier keeps every partial in place until all
+// reads are done.
+__device__ __forceinline__ uint32_t part_off(int row, int chunk, uint32_t rowb) {
+  const uint32_t sw = rowb >= 128u ? (uint32_t(row) & 7u) : ((uint32_t(row) >> 1) & 3u);
+  return uint32_t(row) * rowb + ((uint32_t(chunk) ^ sw) << 4);
 }
 
-// In the last CTA of a split tile: the 128 epilogue threads share out the (row, 8-column chunk)
-// items of rows [row0, row0 + nrows), two items per round; each adds the S partials of its items
-// in split order 0..S-1, with the loads of up to eight splits of both items in flight at once, and
-// hands each sum to write(row, c0, v[8]).
+// This thread's accumulator row (rpad fp32 values) as row `lrow` of the partial tile at `part`.
+__device__ __forceinline__ void store_partial_row(uint32_t part, int lrow, const float (&acc)[64],
+                                                  int rpad) {
+  const uint32_t rowb = uint32_t(rpad) * 4u;
+#pragma unroll
+  for (int c = 0; c < 16; ++c)
+    if (c * 4 < rpad)
+      ptx::st_shared_v4(part + part_off(lrow, c, rowb), __float_as_uint(acc[4 * c]),
+                        __float_as_uint(acc[4 * c + 1]), __float_as_uint(acc[4 * c + 2]),
+                        __float_as_uint(acc[4 * c + 3]));
+}
+
+// Run by the 128 epilogue threads (et = 0..127) between the two cluster barriers: rows [0, nrows)
+// of the tile exist; write(row, c0, v[8]) receives the sum of columns c0 .. c0+7 of a row.
 template <class F>
-__device__ __forceinline__ void split_sum(int rpad, int S, const float* partial, size_t rows_total,
-                                          int row0, int nrows, int et, F&& write) {
-  const int chunks = rpad / 8;
-  const int items = nrows * chunks;
-  const size_t sstride = rows_total * size_t(rpad);
-  for (int it0 = et; it0 < items; it0 += 256) {
-    const float* src[2];
-    bool have[2];
-    int rr[2], c0[2];
-    float v[2][8];
+__device__ __forceinline__ void cluster_sum(uint32_t part, int rpad, int S, int split, int nrows,
+                                            int et, F&& write) {
+  const int rows_per = (lora::BM + S - 1) / S;
+  const int r0 = split * rows_per;
+  const int r1 = min(nrows, r0 + rows_per);
+  const int g8 = rpad / 8;
+  const int items = r1 > r0 ? (r1 - r0) * g8 : 0;
+  const uint32_t rowb = uint32_t(rpad) * 4u;
+  for (int it = et; it < items; it += 128) {
+    const int lr = r0 + it / g8, c8 = it % g8;
+    const uint32_t o0 = part_off(lr, 2 * c8, rowb), o1 = part_off(lr, 2 * c8 + 1, rowb);
+    float v[8];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int it = it0 + u * 128;
-      have[u] = it < items;
-      rr[u] = have[u] ? it / chunks : 0;
-      c0[u] = have[u] ? (it - rr[u] * chunks) * 8 : 0;
-      src[u] = partial + size_t(row0 + rr[u]) * rpad + c0[u];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) v[u][c] = 0.f;
-    }
+    for (int c = 0; c < 8; ++c) v[c] = 0.f;
     for (int sp = 0; sp < S; sp += 8) {
-      float4 a[2][8], b[2][8];
+      float4 a[8], b[8];
 #pragma unroll
-      for (int u = 0; u < 2; ++u)
+      for (int q = 0; q < 8; ++q)
+        if (sp + q < S) {
+          const uint32_t rb = ptx::mapa(part, uint32_t(sp + q));
+          a[q] = ptx::ld_dsmem_f4(rb + o0);
+          b[q] = ptx::ld_dsmem_f4(rb + o1);
+        }
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (have[u] && sp + q < S) {
-            a[u][q] = __ldcg(reinterpret_cast<const float4*>(src[u] + size_t(sp + q) * sstride));
-            b[u][q] = __ldcg(reinterpret_cast<const float4*>(src[u] + size_t(sp + q) * sstride + 4));
-          }
-#pragma unroll
-      for (int u = 0; u < 2; ++u)
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (have[u] && sp + q < S) {
-            v[u][0] += a[u][q].x; v[u][1] += a[u][q].y; v[u][2] += a[u][q].z; v[u][3] += a[u][q].w;
-            v[u][4] += b[u][q].x; v[u][5] += b[u][q].y; v[u][6] += b[u][q].z; v[u][7] += b[u][q].w;
-          }
+      for (int q = 0; q < 8; ++q)
+        if (sp + q < S) {
+          v[0] += a[q].x; v[1] += a[q].y; v[2] += a[q].z; v[3] += a[q].w;
+          v[4] += b[q].x; v[5] += b[q].y; v[6] += b[q].z; v[7] += b[q].w;
+        }
     }
-#pragma unroll
-    for (int u = 0; u < 2; ++u)
-      if (have[u]) write(row0 + rr[u], c0[u], v[u]);
+    write(lr, c8 * 8, v);
   }
 }
 
@@ -149,8 +128,6 @@ struct DownParams {
   const float* tensor_scale;   // NVFP4: [E], else nullptr
   __nv_bfloat16* z;    // [M, r]
   __nv_bfloat16* zs;   // [M, r]
-  float* partial;      // [S, M, rpad] fp32 (S > 1)
-  int* counters;       // [row tiles]
   const int32_t* offsets;      // grouped: device [E+1]; nullptr: one expert
   int* status;
   int M, r, rpad, num_k, S, steps_per_split, E;
@@ -169,7 +146,6 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(rs + NS * R_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   int* s_off = reinterpret_cast<int*>(smem + (kSmemBase - 1024));
   int* s_first = s_off + (p.E + 1);
   const uint32_t b0 = ptx::smem_u32(bars);
@@ -177,13 +153,14 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
   auto empty = [&](uint32_t s) { return b0 + 8u * (NS + s); };
   const uint32_t acc_full = b0 + 8u * (2 * NS);
 
-  // (expert, 128-row tile, split) of this CTA; CTAs beyond the table's last tile have no work
+  // (expert, 128-row tile, split) of this CTA; CTAs beyond the table's last tile have no work.
+  // The table's tile count and the grid are multiples of S, so the S CTAs of a cluster either
+  // all leave here or all stay.
   const GroupView gv = build_group_view(p.offsets, p.E, p.M, BM, p.S, s_off, s_first, p.status);
   if (int(blockIdx.x) >= gv.total()) return;
   const int e = gv.expert_of(blockIdx.x);
   const int local = int(blockIdx.x) - gv.first[e];
   const int mt = local / p.S, split = local % p.S;
-  const int tile = gv.first[e] / p.S + mt;               // row-tile index (counters)
   const int m0 = gv.off[e] + mt * BM;
   const int row_end = gv.off[e + 1];
   const int ks0 = split * p.steps_per_split;
@@ -194,7 +171,6 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
     for (int s = 0; s < NS; ++s) { ptx::mbar_init(full(s), 1); ptx::mbar_init(empty(s), 1); }
     ptx::mbar_init(acc_full, 1);
     *abort_flag = 0;
-    *last_flag = 0;
     ptx::fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -209,6 +185,21 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
   ptx::griddep_launch_dependents();
   const uint32_t rowb = uint32_t(p.rpad) * 2u;
   const uint32_t r_bytes = uint32_t(p.rpad) * 128u;
+  const float ts = p.tensor_scale ? __ldg(p.tensor_scale + e) : 1.0f;
+  const float zscale = p.s / ts;
+  // Z and Zs = bf16(Z * s / ts) for columns c .. c+7 of row rw
+  auto write8 = [&](int rw, int c, const float (&v)[8]) {
+    if (c >= p.r) return;
+    uint4 z, zs;
+    z.x = ptx::cvt_bf16x2(v[0], v[1]); z.y = ptx::cvt_bf16x2(v[2], v[3]);
+    z.z = ptx::cvt_bf16x2(v[4], v[5]); z.w = ptx::cvt_bf16x2(v[6], v[7]);
+    zs.x = ptx::cvt_bf16x2(v[0] * zscale, v[1] * zscale);
+    zs.y = ptx::cvt_bf16x2(v[2] * zscale, v[3] * zscale);
+    zs.z = ptx::cvt_bf16x2(v[4] * zscale, v[5] * zscale);
+    zs.w = ptx::cvt_bf16x2(v[6] * zscale, v[7] * zscale);
+    *reinterpret_cast<uint4*>(p.z + size_t(rw) * p.r + c) = z;
+    *reinterpret_cast<uint4*>(p.zs + size_t(rw) * p.r + c) = zs;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -245,7 +236,6 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
     }
   } else {
     const int q = warp & 3;
-    const int et = threadIdx.x - 64;
     const int row = m0 + q * 32 + lane;
     const bool have = ks1 > ks0;
     if (have) ptx::mbar_wait(acc_full, 0, p.status, abort_flag);
@@ -259,24 +249,8 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
       }
-      const bool row_ok = row < row_end;
-      const float ts = p.tensor_scale ? __ldg(p.tensor_scale + e) : 1.0f;
-      const float zscale = p.s / ts;
-      // Z and Zs = bf16(Z * s / ts) for columns c .. c+7 of row rw
-      auto write8 = [&](int rw, int c, const float (&v)[8]) {
-        if (c >= p.r) return;
-        uint4 z, zs;
-        z.x = ptx::cvt_bf16x2(v[0], v[1]); z.y = ptx::cvt_bf16x2(v[2], v[3]);
-        z.z = ptx::cvt_bf16x2(v[4], v[5]); z.w = ptx::cvt_bf16x2(v[6], v[7]);
-        zs.x = ptx::cvt_bf16x2(v[0] * zscale, v[1] * zscale);
-        zs.y = ptx::cvt_bf16x2(v[2] * zscale, v[3] * zscale);
-        zs.z = ptx::cvt_bf16x2(v[4] * zscale, v[5] * zscale);
-        zs.w = ptx::cvt_bf16x2(v[6] * zscale, v[7] * zscale);
-        *reinterpret_cast<uint4*>(p.z + size_t(rw) * p.r + c) = z;
-        *reinterpret_cast<uint4*>(p.zs + size_t(rw) * p.r + c) = zs;
-      };
       if (p.S == 1) {
-        if (row_ok) {
+        if (row < row_end) {
 #pragma unroll
           for (int c = 0; c < 64; c += 8) {
             float v[8];
@@ -285,11 +259,18 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
             write8(row, c, v);
           }
         }
-      } else if (split_arrive(acc, p.rpad, p.S, split, p.partial, size_t(p.M), row, row_ok,
-                              p.counters + tile, last_flag, et)) {
-        split_sum(p.rpad, p.S, p.partial, size_t(p.M), m0, min(BM, row_end - m0), et, write8);
+      } else {
+        // the operand stages are free: every MMA has completed and every load was consumed
+        store_partial_row(ptx::smem_u32(as), q * 32 + lane, acc, p.rpad);
       }
     }
+  }
+  if (p.S > 1) {
+    ptx::cluster_sync();
+    if (warp >= 2 && *abort_flag == 0)
+      cluster_sum(ptx::smem_u32(as), p.rpad, p.S, split, min(BM, row_end - m0), threadIdx.x - 64,
+                  [&](int lr, int c, const float (&v)[8]) { write8(m0 + lr, c, v); });
+    ptx::cluster_sync();
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -300,8 +281,6 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
 struct WgradParams {
   CUtensorMap tm_l[2];  // L: dY [M, N] (problem 0, dB) / X [M, K] (problem 1, dA); box {64, 64} SW128
   CUtensorMap tm_r[2];  // R: T [M, r] / U [M, r]; box {rpad, 64} SW(2 rpad)
-  float* partial;       // [S, E * (P0 + P1), rpad] fp32 (S > 1)
-  int* counters;        // [E * (tiles0 + tiles1)], zero between calls
   __nv_bfloat16* out0;  // dB [E, N, r]: (p, j) at p * r + j
   __nv_bfloat16* out1;  // dA [E, r, K]: (p, j) at j * K + p
   const int32_t* offsets;       // grouped: device [E+1]; nullptr: one expert of M rows
@@ -321,7 +300,6 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(rs + NS * R_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   int* s_off = reinterpret_cast<int*>(smem + (kSmemBase - 1024));
   int* s_first = s_off + (p.E + 1);
   const uint32_t b0 = ptx::smem_u32(bars);
@@ -352,7 +330,6 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
     for (int s = 0; s < NS; ++s) { ptx::mbar_init(full(s), 1); ptx::mbar_init(empty(s), 1); }
     ptx::mbar_init(acc_full, 1);
     *abort_flag = 0;
-    *last_flag = 0;
     ptx::fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -367,6 +344,23 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
   ptx::griddep_launch_dependents();
   const uint32_t rowb = uint32_t(p.rpad) * 2u;
   const uint32_t r_bytes = 64u * rowb;
+  __nv_bfloat16* out0 = p.out0 + size_t(e) * p.P0 * p.r;
+  __nv_bfloat16* out1 = p.out1 + size_t(e) * p.r * p.P1;
+  // s * the reduction for columns c .. c+7 of output row pr (dB row-major, dA transposed)
+  auto write8 = [&](int pr, int c, const float (&v)[8]) {
+    if (c >= p.r) return;
+    if (prob == 0) {
+      uint4 o;
+      o.x = ptx::cvt_bf16x2(v[0] * p.s, v[1] * p.s);
+      o.y = ptx::cvt_bf16x2(v[2] * p.s, v[3] * p.s);
+      o.z = ptx::cvt_bf16x2(v[4] * p.s, v[5] * p.s);
+      o.w = ptx::cvt_bf16x2(v[6] * p.s, v[7] * p.s);
+      *reinterpret_cast<uint4*>(out0 + size_t(pr) * p.r + c) = o;
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) out1[size_t(c + u) * p.P1 + pr] = __float2bfloat16_rn(v[u] * p.s);
+    }
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -423,7 +417,6 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
     }
   } else {
     const int q = warp & 3;
-    const int et = threadIdx.x - 64;   // 0..127
     const int prow = p0 + q * 32 + lane;
     const bool have = ks1 > ks0;
     if (have) ptx::mbar_wait(acc_full, 0, p.status, abort_flag);
@@ -439,24 +432,6 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
       }
-      const int poff = e * (p.P0 + p.P1) + (prob ? p.P0 : 0);
-      __nv_bfloat16* out0 = p.out0 + size_t(e) * p.P0 * p.r;
-      __nv_bfloat16* out1 = p.out1 + size_t(e) * p.r * p.P1;
-      // s * the reduction for columns c .. c+7 of output row pr (dB row-major, dA transposed)
-      auto write8 = [&](int pr, int c, const float (&v)[8]) {
-        if (c >= p.r) return;
-        if (prob == 0) {
-          uint4 o;
-          o.x = ptx::cvt_bf16x2(v[0] * p.s, v[1] * p.s);
-          o.y = ptx::cvt_bf16x2(v[2] * p.s, v[3] * p.s);
-          o.z = ptx::cvt_bf16x2(v[4] * p.s, v[5] * p.s);
-          o.w = ptx::cvt_bf16x2(v[6] * p.s, v[7] * p.s);
-          *reinterpret_cast<uint4*>(out0 + size_t(pr) * p.r + c) = o;
-        } else {
-#pragma unroll
-          for (int u = 0; u < 8; ++u) out1[size_t(c + u) * p.P1 + pr] = __float2bfloat16_rn(v[u] * p.s);
-        }
-      };
       if (p.S == 1) {
         if (prow < P) {
 #pragma unroll
@@ -467,13 +442,18 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
             write8(prow, c, v);
           }
         }
-      } else if (split_arrive(acc, p.rpad, p.S, split, p.partial, size_t(p.E) * (p.P0 + p.P1),
-                              poff + prow, prow < P, p.counters + tile, last_flag, et)) {
-        split_sum(p.rpad, p.S, p.partial, size_t(p.E) * (p.P0 + p.P1), poff + p0,
-                  min(BM, P - p0), et,
-                  [&](int prw, int c, const float (&v)[8]) { write8(prw - poff, c, v); });
+      } else {
+        // the operand stages are free: every MMA has completed and every load was consumed
+        store_partial_row(ptx::smem_u32(as), q * 32 + lane, acc, p.rpad);
       }
     }
+  }
+  if (p.S > 1) {
+    ptx::cluster_sync();
+    if (warp >= 2 && *abort_flag == 0)
+      cluster_sum(ptx::smem_u32(as), p.rpad, p.S, split, min(BM, P - p0), threadIdx.x - 64,
+                  [&](int lr, int c, const float (&v)[8]) { write8(p0 + lr, c, v); });
+    ptx::cluster_sync();
   }
   ptx::tc_fence_before();
   __syncthreads();

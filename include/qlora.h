@@ -108,7 +108,7 @@ typedef enum {
  * arguments.  A workspace sized for an op and shapes also serves smaller M. */
 QLORA_API size_t qlora_workspace_size(int op, const qlora_weight_t* W, int64_t M, int r, int E);
 
-/* Zero the workspace's status word and reduction counters.  Call once after allocating a
+/* Zero the workspace's status word.  Call once after allocating a
  * workspace (or zero it yourself), and again after a QLORA_ERR_DEVICE_TIMEOUT.  Async on stream. */
 QLORA_API qlora_status_t qlora_workspace_init(void* ws, size_t ws_bytes, qlora_stream_t stream);
 
@@ -155,10 +155,9 @@ QLORA_API qlora_status_t qlora_grouped_bwd(const qlora_weight_t* W, int E, const
  * synchronise the device and fragment its memory), or plain C callers with no allocator of their
  * own.  The paper has no counterpart of this entry point; it only changes who provides scratch.
  *   Scratch is a fixed 4 MiB array inside the library (every GPU that loads the library holds it
- *   until the process exits): 256 bytes of status and counters, the [M,r] bf16 operand Zs and,
- *   when T_save is NULL, an [M,r] bf16 T; what is left holds fp32 partial sums when the T = X A^T
- *   contraction is split over several CTAs (fewer splits when it is short, results within the
- *   same tolerance).  Sizes that do not fit -- M*r > 2,097,024 with T_save, or
+ *   until the process exits): 256 bytes of status, the [M,r] bf16 operand Zs and, when T_save is
+ *   NULL, an [M,r] bf16 T; results are bitwise those of qlora_linear_fwd.  Sizes that do not fit
+ *   -- M*r > 2,097,024 with T_save, or
  *   M*r > 1,048,512 without -- are rejected with QLORA_ERR_WORKSPACE before anything is enqueued.
  *   The call allocates nothing (no cudaMalloc/cudaFree, no allocating library routine); it clears
  *   the status word on `stream` each call.
