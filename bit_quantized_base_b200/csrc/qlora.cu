@@ -19,8 +19,11 @@ namespace qlora {
 namespace {
 
 // ------------------------------------------------------------------------------------ helpers
-constexpr size_t kHeaderBytes = 256;        // [0]: device status word
+constexpr size_t kHeaderBytes = 256;        // [0]: device status word, [1]: pair-kernel ticket
 constexpr int kMaxClusterSplits = 8;        // split-K CTAs of one LoRA tile (one portable cluster)
+// CTAs of a lora_down launch that feeds the pair kernel: the pair kernel starts beside it on the
+// other SMs and waits for its output only at the end of its first tile
+constexpr int kDownCtasBesidePair = 32;
 constexpr int kMaxDevices = 64;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -175,11 +178,11 @@ struct DownPlan {
   int tiles, S, sps, num_k;
 };
 
-DownPlan down_plan(int64_t M, int64_t Kc, int E, int sms) {
+DownPlan down_plan(int64_t M, int64_t Kc, int E, int ctas) {
   DownPlan p{};
   p.tiles = int((M + 127) / 128) + (E > 1 ? E - 1 : 0);
   p.num_k = int((Kc + 63) / 64);
-  int S = p.tiles > 0 ? sms / p.tiles : 1;                   // at most one wave of long splits
+  int S = p.tiles > 0 ? ctas / p.tiles : 1;                  // at most `ctas` CTAs of long splits
   S = S < 1 ? 1 : (S > kMaxClusterSplits ? kMaxClusterSplits : S);
   const int max_s = p.num_k / 2 > 0 ? p.num_k / 2 : 1;
   if (S > max_s) S = max_s;
@@ -306,13 +309,15 @@ bool tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_
 }
 
 // Z = Act . R for every expert's rows: R is A [E, r, Kc] (r_mn false, T = X A^T) or
-// B [E, Kc, r] (r_mn true, U = dY B).  offsets == nullptr: one expert of M rows.
+// B [E, Kc, r] (r_mn true, U = dY B).  offsets == nullptr: one expert of M rows.  beside_pair:
+// the next launch of the stream is the pair kernel, which overlaps this one (fewer CTAs).
 qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t Kc, const void* R,
                                 int r, float s, const float* ts, void* z, void* zs, int* status,
-                                const int32_t* offsets, int E, bool grouped, cudaStream_t st) {
+                                const int32_t* offsets, int E, bool grouped, bool beside_pair,
+                                cudaStream_t st) {
   DownParams p{};
   const int rpad = rank_pad(r);
-  const DownPlan dp = down_plan(M, Kc, E, num_sms());
+  const DownPlan dp = down_plan(M, Kc, E, beside_pair ? kDownCtasBesidePair : num_sms());
   if (!tmap_2d(&p.tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, uint64_t(Kc), uint64_t(M),
                uint64_t(Kc) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
@@ -391,6 +396,7 @@ qlora_status_t launch_fused(const qlora_weight_t* W, bool dx, const void* act, c
   p.out = static_cast<__nv_bfloat16*>(out);
   p.offsets = offsets;
   p.status = status;
+  p.ticket = reinterpret_cast<unsigned*>(status + 1);
   p.M = int(M);
   p.N = int(N);
   p.K = int(K);
@@ -660,10 +666,11 @@ qlora_status_t run_fwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   void* T = T_save ? T_save : w + L.t;
   void* Zs = w + L.zs;
   const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
+  const bool short_fwd = stream_fits(W, M, E, false, ws_bytes - L.partial);
   qlora_status_t st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, T, Zs, ws_status(ws),
-                                       offsets, E, grouped, s);
+                                       offsets, E, grouped, !short_fwd, s);
   if (st != QLORA_OK) return st;
-  if (stream_fits(W, M, E, false, ws_bytes - L.partial))
+  if (short_fwd)
     return launch_stream(W, false, X, Zs, B, Y, M, r, ws_status(ws),
                          reinterpret_cast<float*>(w + L.partial), ws_bytes - L.partial, s);
   return launch_fused(W, false, X, Zs, B, Y, M, r, ws_status(ws), offsets, E, grouped, s);
@@ -693,14 +700,14 @@ qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   qlora_status_t st;
   if (!T) {  // recompute T = X A^T (its scaled copy lands in Zs and is overwritten below)
     st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, w + L.t, Zs, ws_status(ws), offsets,
-                          E, grouped, s);
+                          E, grouped, false, s);
     if (st != QLORA_OK) return st;
     T = w + L.t;
   }
-  st = launch_lora_down(true, dY, M, W->N, B, r, scale, ts, U, Zs, ws_status(ws), offsets, E,
-                        grouped, s);
-  if (st != QLORA_OK) return st;
   const bool short_dx = dX && stream_fits(W, M, E, true, ws_bytes - L.partial);
+  st = launch_lora_down(true, dY, M, W->N, B, r, scale, ts, U, Zs, ws_status(ws), offsets, E,
+                        grouped, dX && !short_dx, s);
+  if (st != QLORA_OK) return st;
   if (dX && !short_dx) {
     // The adapter gradients need only T, U, X and dY, so they run on a side stream beside the
     // tiled dX kernel, filling the SMs its last wave of tiles leaves idle (the two kernels share
@@ -768,7 +775,8 @@ qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const void* X, 
   void* Zs = w + kHeaderBytes;
   void* T = T_save ? T_save : w + kHeaderBytes + mr;
   const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
-  st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, T, Zs, status, nullptr, 1, false, s);
+  st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, T, Zs, status, nullptr, 1, false, true,
+                        s);
   if (st != QLORA_OK) return st;
   return launch_fused(W, false, X, Zs, B, Y, M, r, status, nullptr, 1, false, s);
 }

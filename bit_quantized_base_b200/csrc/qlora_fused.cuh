@@ -84,6 +84,7 @@ struct FusedParams {
   __nv_bfloat16* out;                // fwd: Y [M, N]; dX: dX [M, K]
   const int32_t* offsets;            // grouped: device [E+1] row offsets; nullptr: one expert
   int* status;
+  unsigned* ticket;                  // pair-rank ticket, 0 between launches (wraps back to 0)
   int M, N, K, r, E;                 // M: all rows (packed over experts)
   int num_n, num_k;                  // pair tiles over output columns; contraction steps
   int tail_split;                    // the last tail_split 512-row tiles run as 2 x 256-row tiles
@@ -212,6 +213,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(cs + NC * C_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* pair_slot = tmem_slot + 2;
   int* s_off = reinterpret_cast<int*>(smem + (kSmemBase - 1024));
   int* s_first = s_off + (p.E + 1);
 
@@ -225,7 +227,18 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();
-  const int pair = int(blockIdx.x >> 1), npairs = int(gridDim.x >> 1);
+  const int npairs = int(gridDim.x >> 1);
+  if (threadIdx.x == 0 && rank == 0) {
+    // Pair ranks in order of arrival: pairs that start late (their SMs still held by the previous
+    // kernel) get the last ranks, whose static share of tiles is the smaller one.  atomicInc
+    // wraps at npairs, so the npairs tickets of a launch are a permutation of 0..npairs-1 and
+    // leave the ticket where it started.
+    const uint32_t r = atomicInc(p.ticket, unsigned(npairs - 1));
+    if (r >= uint32_t(npairs) && p.status)   // the workspace header was never zeroed
+      atomicCAS(p.status, 0, 1 /* QLORA_ERR_INVALID_ARG */);
+    *pair_slot = r;
+    ptx::st_cluster_u32(ptx::mapa(ptx::smem_u32(pair_slot), 1), r);
+  }
   if (threadIdx.x == 0) {
     // stage full: leader = producer's expect-tx arrive + 4 dequant warps + 1 relayed arrive;
     // other CTA = its 4 dequant warps (waited on by its relay).  acc_empty is used in the leader.
@@ -255,7 +268,10 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
   ptx::cluster_sync();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  ptx::griddep_wait();
+  const int pair = int(*pair_slot) % npairs;
+  // The previous kernel of the stream (the lora_down launch that writes Zs) may still be running:
+  // only the Zs loads of the LoRA steps wait for it (griddep_wait in the activation producer).
+  // Everything else this kernel reads was complete before that kernel let this one launch.
   ptx::griddep_launch_dependents();
 
   const int num_tiles = grp_view.total() + p.tail_split;
@@ -265,6 +281,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     // ------------------------------------------------------------------ activation producer
     if (lane == 0) {
       uint32_t i = 0;
+      bool waited = false;
       for (int t = pair; t < num_tiles; t += npairs) {
         const PairTile pt = pair_tile_at(grp_view, t, p.num_n, p.tail_split);
         const int m0 = pt.row0 + int(rank) * HM;      // this CTA's rows of block 0 (+256: block 1)
@@ -272,6 +289,10 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
         for (int ks = 0; ks <= nk; ++ks, ++i) {
           const uint32_t sx = i % NS, px = (i / NS) & 1u;
           if (!ptx::mbar_wait(empty_s(sx), px ^ 1u, p.status, abort_flag)) { ok = false; break; }
+          if (ks == nk && !waited) {
+            ptx::griddep_wait();
+            waited = true;
+          }
           if (rank == 0) ptx::mbar_arrive_expect_tx(full_s(sx), 2 * pt.nb * X_BYTES);
           const uint32_t fx = ptx::mapa(full_s(sx), 0);
           for (int blk = 0; blk < pt.nb; ++blk) {

@@ -361,6 +361,10 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
 }
+// 32-bit store to the shared memory of any CTA of the cluster (shared::cluster address).
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
 // 16-byte load from the shared memory of any CTA of the cluster (shared::cluster address, as
 // returned by mapa).
 __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t cluster_addr) {
