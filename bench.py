@@ -337,9 +337,9 @@ def run_own(args):
     if Q.qlora_get_device_status(ws) != 0:
         raise RuntimeError("device status after warm-up: %d" % Q.qlora_get_device_status(ws))
 
-    # ---- timed region (device time, CUDA events on the launching stream)
-    Q.qlora_profile_enable(True)
-    Q.qlora_profile_reset()
+    # ---- timed region (device time, CUDA events on the launching stream).  No per-kernel events
+    # inside it: an event recorded between two launches would stop the next kernel from starting
+    # beside the previous one (programmatic dependent launch).
     clk = ClockSampler(local)
     clk.start()
     barrier(ws_n)
@@ -357,9 +357,17 @@ def run_own(args):
     launches = Q.qlora_launch_count() - launches0
     clocks = clk.stop()
     ms_local = ev0.elapsed_time(ev1)
+    ms_total = max_over_ranks(ws_n, ms_local)
+
+    # ---- per-kernel durations: a separate pass with an event pair around every launch
+    prof_steps = max(3, min(args.steps, 50))
+    Q.qlora_profile_enable(True)
+    Q.qlora_profile_reset()
+    for i in range(prof_steps):
+        step(args.warmup + args.steps + i)
+    torch.cuda.synchronize()
     prof = Q.qlora_profile_read()
     Q.qlora_profile_enable(False)
-    ms_total = max_over_ranks(ws_n, ms_local)
     ms_step = ms_total / args.steps
     fl = flops(M, N, K, r)
     value = ws_n * fl * args.steps / (ms_total * 1e-3) / 1e12
@@ -457,6 +465,8 @@ def run_own(args):
         "clocks": clocks,
         "roofline": roofline,
         "kernel_breakdown": breakdown,
+        "kernel_breakdown_method": f"separate pass of {prof_steps} steps after the timed region, "
+                                   "CUDA events around every launch (launches serialised)",
         "e2e": e2e,
         "weight_stream_small_m": sweep,
         "grouped_moe": grouped,
