@@ -24,6 +24,9 @@ constexpr int kMaxClusterSplits = 8;        // split-K CTAs of one LoRA tile (on
 // CTAs of a lora_down launch that feeds the pair kernel: the pair kernel starts beside it on the
 // other SMs and waits for its output only at the end of its first tile
 constexpr int kDownCtasBesidePair = 32;
+// The same for the short-batch streaming kernel, which up to 64 rows also leaves that many SMs to
+// lora_down (its ranges are equal, so a late CTA would delay the whole launch)
+constexpr int kDownCtasBesideStream = 16;
 constexpr int kMaxDevices = 64;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -204,6 +207,9 @@ bool use_stream(int64_t M, int E) { return E == 1 && M > 0 && M <= stream::kMaxR
 
 StreamPlan stream_plan(int64_t N, int64_t K, int64_t M, bool dx, int sms) {
   StreamPlan p{};
+  // Up to 64 rows the launch is short next to lora_down: leave it its SMs.  Above, the decode
+  // work per SM is larger than lora_down's duration is worth.
+  if (M <= 64 && sms > 4 * kDownCtasBesideStream) sms -= kDownCtasBesideStream;
   p.tiles = int(((dx ? K : N) + stream::BN - 1) / stream::BN);
   p.nk = int(((dx ? N : K) + stream::BK - 1) / stream::BK);
   const int64_t total = int64_t(p.tiles) * (p.nk + 1);
@@ -310,14 +316,15 @@ bool tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_
 
 // Z = Act . R for every expert's rows: R is A [E, r, Kc] (r_mn false, T = X A^T) or
 // B [E, Kc, r] (r_mn true, U = dY B).  offsets == nullptr: one expert of M rows.  beside_pair:
-// the next launch of the stream is the pair kernel, which overlaps this one (fewer CTAs).
+// max_ctas > 0: the next launch of the stream (pair or streaming kernel) runs beside this one,
+// which then uses at most that many CTAs.
 qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t Kc, const void* R,
                                 int r, float s, const float* ts, void* z, void* zs, int* status,
-                                const int32_t* offsets, int E, bool grouped, bool beside_pair,
+                                const int32_t* offsets, int E, bool grouped, int max_ctas,
                                 cudaStream_t st) {
   DownParams p{};
   const int rpad = rank_pad(r);
-  const DownPlan dp = down_plan(M, Kc, E, beside_pair ? kDownCtasBesidePair : num_sms());
+  const DownPlan dp = down_plan(M, Kc, E, max_ctas > 0 ? max_ctas : num_sms());
   if (!tmap_2d(&p.tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, uint64_t(Kc), uint64_t(M),
                uint64_t(Kc) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
@@ -668,7 +675,8 @@ qlora_status_t run_fwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
   const bool short_fwd = stream_fits(W, M, E, false, ws_bytes - L.partial);
   qlora_status_t st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, T, Zs, ws_status(ws),
-                                       offsets, E, grouped, !short_fwd, s);
+                                       offsets, E, grouped,
+                                       short_fwd ? kDownCtasBesideStream : kDownCtasBesidePair, s);
   if (st != QLORA_OK) return st;
   if (short_fwd)
     return launch_stream(W, false, X, Zs, B, Y, M, r, ws_status(ws),
@@ -700,13 +708,13 @@ qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   qlora_status_t st;
   if (!T) {  // recompute T = X A^T (its scaled copy lands in Zs and is overwritten below)
     st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, w + L.t, Zs, ws_status(ws), offsets,
-                          E, grouped, false, s);
+                          E, grouped, 0, s);
     if (st != QLORA_OK) return st;
     T = w + L.t;
   }
   const bool short_dx = dX && stream_fits(W, M, E, true, ws_bytes - L.partial);
   st = launch_lora_down(true, dY, M, W->N, B, r, scale, ts, U, Zs, ws_status(ws), offsets, E,
-                        grouped, dX && !short_dx, s);
+                        grouped, !dX ? 0 : (short_dx ? kDownCtasBesideStream : kDownCtasBesidePair), s);
   if (st != QLORA_OK) return st;
   if (dX && !short_dx) {
     // The adapter gradients need only T, U, X and dY, so they run on a side stream beside the
@@ -775,8 +783,8 @@ qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const void* X, 
   void* Zs = w + kHeaderBytes;
   void* T = T_save ? T_save : w + kHeaderBytes + mr;
   const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
-  st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, T, Zs, status, nullptr, 1, false, true,
-                        s);
+  st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, T, Zs, status, nullptr, 1, false,
+                        kDownCtasBesidePair, s);
   if (st != QLORA_OK) return st;
   return launch_fused(W, false, X, Zs, B, Y, M, r, status, nullptr, 1, false, s);
 }

@@ -14,10 +14,12 @@
 // applies the NVFP4 tensor scale and writes bf16.
 //
 // A tile is 256 output columns (two 128-column weight halves, each decoded exactly as one CTA's
-// half in the pair kernel) by all M rows.  The MMA runs with the operands swapped: a decoded
-// weight half is the A operand (M = 128 output columns), the activation rows are the B operand
-// (N = M rounded up to 16), so the tensor core computes only the batch's own rows, and the
-// accumulator holds the tile transposed (tensor-memory lane = output column, column = batch row).
+// half in the pair kernel) by all M rows.  Up to 128 rows (MT = 1) the activation rows are the A
+// operand (M = 128; lanes past the batch are never read) and the whole decoded 256-row weight tile
+// the B operand (N = 256): one MMA per 16-deep sub-step, an N at which the tensor core runs at
+// its proportional rate.  Above 128 rows (MT = 2) the operands are swapped: each weight half is an
+// A operand and the batch rows the B operand (N = M rounded up to 16), and the accumulator holds
+// the tile transposed (tensor-memory lane = output column, column = batch row).
 // The LoRA term is one extra step per tile (operands rows of B or A, and Zs), as in the pair
 // kernel.  Every step has one operand stage (activation rows + weight tile) with one full and one
 // empty barrier.
@@ -51,7 +53,8 @@ constexpr int kMaxRows = 256;
 constexpr int SCALE_RING_BYTES = 4 * 2 * 256 * 4;   // kPf slots x 2 halves x 256 threads
 // Operand stages: xrows activation rows (M rounded up to 16) plus one weight tile; the stage count
 // depends on xrows, so every role tracks its stage index and phase incrementally.  MT = 1 for
-// xrows <= 128 (double-buffered accumulators: 2 x 2 halves x xrows tensor-memory columns), 2 above.
+// xrows <= 128 (double-buffered accumulators: 2 x 256 tensor-memory columns), 2 above (one
+// accumulator: 2 halves x xrows columns).
 __host__ __device__ constexpr int num_stages(int xrows) { return xrows <= 64 ? 4 : (xrows <= 128 ? 3 : 2); }
 constexpr int kMaxStages = 4;
 constexpr int NC = 6;                     // code stages
@@ -152,7 +155,9 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  ptx::griddep_wait();
+  // The previous kernel of the stream (the lora_down launch that writes Zs, on SMs this launch
+  // leaves free) may still be running: only the Zs loads of the LoRA steps wait for it.
+  // Everything else this kernel reads was complete before that kernel let this one launch.
   ptx::griddep_launch_dependents();
 
   if (warp == kTmaWarp) {
@@ -160,7 +165,12 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
     if (lane == 0) {
       uint32_t s = 0, ph = 0;
       int ks = rg.step(rg.g0);
+      bool waited = false;
       for (int g = rg.g0; g < rg.g1; ++g) {
+        if (ks == nk && !waited) {
+          ptx::griddep_wait();
+          waited = true;
+        }
         if (!ptx::mbar_wait_idle(empty_s(s), ph ^ 1u, p.status, abort_flag)) break;
         ptx::mbar_arrive_expect_tx(full_s(s), XSTAGE);
         if (ks < nk) ptx::tma_load_2d(xs(s), &p.tm_act, full_s(s), ks * BK, 0);
@@ -194,14 +204,21 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
     if (lane == 0) {
       // Lean issue loop (the thread shares its SM sub-partition with busy dequant warps):
       // descriptors are stage-0 descriptors plus constant offsets, the 16-deep sub-steps unrolled.
-      const uint32_t idesc = ptx::idesc_bf16(128, uint32_t(p.xrows), DX ? 1u : 0u, 0u);
       const int lora_kk = (p.r + 15) / 16;
-      const uint64_t bx0 = ptx::smem_desc(xs(0), 16, 1024, ptx::kSw128);
-      const uint64_t aw0 = DX ? ptx::smem_desc(wsm(0), 8192, 1024, ptx::kSw128)
-                              : ptx::smem_desc(wsm(0), 16, 1024, ptx::kSw128);
+      const uint64_t x0 = ptx::smem_desc(xs(0), 16, 1024, ptx::kSw128);
+      const uint64_t w0 = DX ? ptx::smem_desc(wsm(0), 8192, 1024, ptx::kSw128)
+                             : ptx::smem_desc(wsm(0), 16, 1024, ptx::kSw128);
       const uint64_t kXStage = XSTAGE >> 4;
       constexpr uint64_t kWStage = W_BYTES >> 4, kWHalf = HW_BYTES >> 4;
       constexpr uint64_t kXkk = 32 >> 4, kWkk = DX ? (2048 >> 4) : (32 >> 4);
+      // MT == 1: the activation rows are the A operand (M = 128: rows past xrows read whatever
+      // follows in shared memory and land in accumulator lanes nobody reads) and the whole
+      // 256-row weight tile the B operand (N = 256), one MMA per 16-deep sub-step; accumulator
+      // buffer b = tensor-memory columns [256 b, 256 b + 256), lane = batch row.
+      // MT == 2: each 128-row weight half is the A operand and the batch rows the B operand
+      // (N = xrows), two MMAs per sub-step; the accumulator holds the tile transposed.
+      const uint32_t idesc = MT == 1 ? ptx::idesc_bf16(128, 256, 0u, DX ? 1u : 0u)
+                                     : ptx::idesc_bf16(128, uint32_t(p.xrows), DX ? 1u : 0u, 0u);
       const uint32_t xr = uint32_t(p.xrows);
       uint32_t b = 0, bph = 0, s = 0, ph = 0;
       int ks = rg.step(rg.g0);
@@ -213,19 +230,32 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
         }
         if (!ptx::mbar_wait(full_s(s), ph, p.status, abort_flag)) break;
         ptx::tc_fence_after();
-        const uint64_t bx = bx0 + s * kXStage, aw = aw0 + s * kWStage;
-        const uint32_t d0 = tmem + b * 2u * xr;
+        const uint64_t xd = x0 + s * kXStage, wd = w0 + s * kWStage;
         const uint32_t acc0 = first ? 0u : 1u;
-        if (ks < nk) {
+        const int nkk = ks < nk ? BK / 16 : lora_kk;
+        if constexpr (MT == 1) {
+          const uint32_t d0 = tmem + b * uint32_t(BN);
+          if (nkk == BK / 16) {
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            ptx::mma_bf16(d0, aw + kk * kWkk, bx + kk * kXkk, idesc, kk ? 1u : acc0);
-            ptx::mma_bf16(d0 + xr, aw + kWHalf + kk * kWkk, bx + kk * kXkk, idesc, kk ? 1u : acc0);
+            for (int kk = 0; kk < BK / 16; ++kk)
+              ptx::mma_bf16(d0, xd + kk * kXkk, wd + kk * kWkk, idesc, kk ? 1u : acc0);
+          } else {
+            for (int kk = 0; kk < nkk; ++kk)
+              ptx::mma_bf16(d0, xd + kk * kXkk, wd + kk * kWkk, idesc, kk ? 1u : acc0);
           }
         } else {
-          for (int kk = 0; kk < lora_kk; ++kk) {
-            ptx::mma_bf16(d0, aw + kk * kWkk, bx + kk * kXkk, idesc, kk ? 1u : acc0);
-            ptx::mma_bf16(d0 + xr, aw + kWHalf + kk * kWkk, bx + kk * kXkk, idesc, kk ? 1u : acc0);
+          const uint32_t d0 = tmem + b * 2u * xr;
+          if (nkk == BK / 16) {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              ptx::mma_bf16(d0, wd + kk * kWkk, xd + kk * kXkk, idesc, kk ? 1u : acc0);
+              ptx::mma_bf16(d0 + xr, wd + kWHalf + kk * kWkk, xd + kk * kXkk, idesc, kk ? 1u : acc0);
+            }
+          } else {
+            for (int kk = 0; kk < nkk; ++kk) {
+              ptx::mma_bf16(d0, wd + kk * kWkk, xd + kk * kXkk, idesc, kk ? 1u : acc0);
+              ptx::mma_bf16(d0 + xr, wd + kWHalf + kk * kWkk, xd + kk * kXkk, idesc, kk ? 1u : acc0);
+            }
           }
         }
         ptx::mma_commit(empty_s(s));
@@ -242,9 +272,6 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
     }
   } else if (warp < kEpiWarps) {
     // ------------------------------------------------------------------ epilogue
-    // Tensor-memory lane 32q + lane holds output column hh * 128 + 32q + lane of the tile; its
-    // accumulator columns are the batch rows.  Each store instruction writes 32 consecutive floats
-    // of one partial row.
     const int q = warp;
     uint32_t b = 0, bph = 0;
     for (int g = rg.g0; g < rg.g1; ++g) {
@@ -253,18 +280,44 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
       ptx::tc_fence_after();
       const long long st = max((long long)rg.g0, (long long)rg.tile(g) * rg.nk1);
       float* base = p.partial + size_t(stream_segment(st, p.iters, rg.nk1, p.lcm)) * size_t(p.M) * BN;
+      if constexpr (MT == 1) {
+        // Tensor-memory lane 32q + lane holds batch row 32q + lane; its 256 columns are the tile's
+        // output columns.  Warps whose rows are all past the batch have nothing to store.
+        const int m = q * 32 + lane;
+        if (q * 32 < p.M) {
+          const uint32_t trow = tmem + (uint32_t(q * 32) << 16) + b * uint32_t(BN);
+          float* row = base + size_t(m) * BN;
 #pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        const uint32_t tcol = tmem + (uint32_t(q * 32) << 16) + b * 2u * uint32_t(p.xrows) + hh * uint32_t(p.xrows);
-        float* col = base + hh * HN + q * 32 + lane;
-#pragma unroll 1
-        for (int m0 = 0; m0 < p.xrows; m0 += 16) {
-          uint32_t v[16];
-          ptx::tmem_ld_32x32b_x16(tcol + m0, v);
-          ptx::tmem_ld_wait(v);
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            uint32_t v[32];
+            ptx::tmem_ld_32x32b_x32(trow + uint32_t(c0), v);
+            ptx::tmem_ld_wait(v);
+            if (m < p.M) {
 #pragma unroll
-          for (int u = 0; u < 16; ++u)
-            if (m0 + u < p.M) __stcg(col + size_t(m0 + u) * BN, __uint_as_float(v[u]));
+              for (int u = 0; u < 32; u += 4)
+                __stcg(reinterpret_cast<float4*>(row + c0 + u),
+                       make_float4(__uint_as_float(v[u]), __uint_as_float(v[u + 1]),
+                                   __uint_as_float(v[u + 2]), __uint_as_float(v[u + 3])));
+            }
+          }
+        }
+      } else {
+        // Tensor-memory lane 32q + lane holds output column hh * 128 + 32q + lane of the tile; its
+        // accumulator columns are the batch rows.  Each store instruction writes 32 consecutive
+        // floats of one partial row.
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t tcol = tmem + (uint32_t(q * 32) << 16) + b * 2u * uint32_t(p.xrows) + hh * uint32_t(p.xrows);
+          float* col = base + hh * HN + q * 32 + lane;
+#pragma unroll 1
+          for (int m0 = 0; m0 < p.xrows; m0 += 16) {
+            uint32_t v[16];
+            ptx::tmem_ld_32x32b_x16(tcol + m0, v);
+            ptx::tmem_ld_wait(v);
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+              if (m0 + u < p.M) __stcg(col + size_t(m0 + u) * BN, __uint_as_float(v[u]));
+          }
         }
       }
       ptx::tc_fence_before();
