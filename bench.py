@@ -405,32 +405,55 @@ def run_own(args):
     hdA = torch.empty((r, K), dtype=torch.bfloat16).pin_memory()
     hdB = torch.empty((N, r), dtype=torch.bfloat16).pin_memory()
     e2e_steps = max(3, min(args.steps, 30))
+    # Step i's inputs are copied from pinned host memory on a copy stream into device set i % ncopy
+    # while the compute stream runs step i - 1 (the copy of set c waits for the step that last
+    # read it); the compute stream waits for its inputs, then reads dA and dB back.
+    comp = torch.cuda.current_stream()
+    copy_st = torch.cuda.Stream()
+    copied = [torch.cuda.Event() for _ in range(ncopy)]
+    consumed = [torch.cuda.Event() for _ in range(ncopy)]
+
+    def e2e_copy(i):
+        c = i % ncopy
+        with torch.cuda.stream(copy_st):
+            copy_st.wait_event(consumed[c])
+            Xs[c].copy_(hX, non_blocking=True)
+            dYs[c].copy_(hdY, non_blocking=True)
+            copied[c].record(copy_st)
 
     def e2e_step(i):
         c = i % ncopy
-        Xs[c].copy_(hX, non_blocking=True)
-        dYs[c].copy_(hdY, non_blocking=True)
+        comp.wait_event(copied[c])
         Q.qlora_linear_fwd(Ws[c], Xs[c], A, B, Y, T, M, r, s, ws)
         Q.qlora_linear_bwd(Ws[c], Xs[c], A, B, T, dYs[c], dX, dA, dB, M, r, s, ws)
+        consumed[c].record(comp)
         hdA.copy_(dA, non_blocking=True)
         hdB.copy_(dB, non_blocking=True)
 
-    for i in range(2):
+    for ev in consumed:
+        ev.record(comp)
+    for i in range(2):   # warm-up
+        e2e_copy(i)
         e2e_step(i)
     barrier(ws_n)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
-    for i in range(e2e_steps):
-        e2e_step(i)
+    e2e_copy(2)   # every timed step's copy is issued inside the timed region
+    for j in range(e2e_steps):
+        if j + 1 < e2e_steps:
+            e2e_copy(j + 3)
+        e2e_step(j + 2)
     e1.record()
     e1.synchronize()
     e2e_ms = max_over_ranks(ws_n, e0.elapsed_time(e1))
     e2e = {"value": round(ws_n * fl * e2e_steps / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
            "h2d_bytes_per_step": int((hX.numel() + hdY.numel()) * 2),
            "d2h_bytes_per_step": int((hdA.numel() + hdB.numel()) * 2),
-           "ms_per_step": round(e2e_ms / e2e_steps, 4)}
+           "ms_per_step": round(e2e_ms / e2e_steps, 4),
+           "note": "host->device copies of each step's X and dY on a copy stream overlap the "
+                   "previous step's compute; all of them inside the timed region"}
 
     # ---- short-batch weight-stream sweeps: the NF4 up-proj weight and the MXFP4 gate-proj weight
     sweep = None
