@@ -152,6 +152,72 @@ class ClockSampler:
         return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
 
 
+class NvmlSampler:
+    """SM clock, power draw and clock-event reasons of this process's GPU, read through NVML every
+    5 ms on a host thread while the timed region runs (reads only; no setting is changed).  Falls
+    back to the nvidia-smi sampler when NVML is unavailable."""
+
+    BITS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+            ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+            ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+            ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.fallback = None
+        self.samples = []
+        self.reasons = set()
+        self.thread = None
+        self.stop_flag = False
+
+    def start(self):
+        try:
+            import threading
+            import pynvml as N
+            import torch
+            N.nvmlInit()
+            pr = torch.cuda.get_device_properties(self.dev)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            self.N, self.h = N, N.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.fallback = ClockSampler(self.dev)
+            self.fallback.start()
+
+    def _run(self):
+        N = self.N
+        while not self.stop_flag:
+            try:
+                mhz = N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM)
+                mw = N.nvmlDeviceGetPowerUsage(self.h)
+                rs = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                break
+            self.samples.append((mhz, mw / 1000.0))
+            for name, attr in self.BITS:
+                if rs & getattr(N, attr):
+                    self.reasons.add(name)
+            time.sleep(0.005)
+
+    def stop(self):
+        if self.fallback is not None:
+            return self.fallback.stop()
+        self.stop_flag = True
+        self.thread.join(timeout=5)
+        try:
+            self.N.nvmlShutdown()
+        except Exception:
+            pass
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "power_w_max": round(max(w for _, w in self.samples), 1),
+                "source": "NVML every 5 ms during the timed region"}
+
+
 # ------------------------------------------------------------------------------- own arm
 def dist_setup(args):
     import torch
@@ -340,7 +406,7 @@ def run_own(args):
     # ---- timed region (device time, CUDA events on the launching stream).  No per-kernel events
     # inside it: an event recorded between two launches would stop the next kernel from starting
     # beside the previous one (programmatic dependent launch).
-    clk = ClockSampler(local)
+    clk = NvmlSampler(local)
     clk.start()
     barrier(ws_n)
     torch.cuda.synchronize()
