@@ -168,6 +168,29 @@ def test_deterministic_reruns():
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+def test_pair_ticket_from_any_start():
+    # The pair kernel draws pair ranks from a ticket in the workspace header (32-bit word 1) that
+    # wraps at the pair count: npairs draws from any start below it are a permutation of the
+    # ranks, so results do not depend on where the ticket stands, and every launch leaves it
+    # where it found it.
+    p = synth.small_layer("mxfp4", 1300, 2048, 1024, 16, seed=21)   # pair path
+    g = GpuLayer(p)
+    Y0, T0 = g.fwd()
+    r0 = g.bwd(T0)
+    torch.cuda.synchronize()
+    ticket = g.ws[4:8].view(torch.int32)
+    assert int(ticket.item()) == 0
+    ticket.fill_(3)
+    Y1, T1 = g.fwd()
+    r1 = g.bwd(T1)
+    torch.cuda.synchronize()
+    assert g.status() == 0
+    assert int(ticket.item()) == 3
+    assert torch.equal(Y0.view(torch.int16), Y1.view(torch.int16))
+    for a, b in zip(r0, r1):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
 def test_step0_init_on_gpu():
     # B = 0 -> dA == 0 exactly and Y equals the base product ("Initialization matters")
     p = synth.small_layer("nf4", 64, 128, 256, 16, seed=2)
