@@ -254,9 +254,16 @@ def max_over_ranks(ws, x):
 def short_batch_sweep(Q, torch, p, Ws, X, dY, A, B, peaks):
     """fwd+bwd at M in {16, 32, 64, 128, 256} on one weight (rotating device copies whose total
     exceeds 3x L2): weight bytes read per step (two passes) / time, TFLOP/s, and the fraction of
-    the binding roofline max(flops / bf16 peak, bytes / HBM peak)."""
+    the binding roofline max(flops / bf16 peak, bytes / HBM peak, decoded weights / decode peak).
+    The decode peak is the library's own dequant stage measured on every SM of this GPU
+    (qlora_debug_decode_rate: decoded weights per SM clock) x SMs x the maximum SM clock; it binds
+    the short batches, where each decoded weight meets only M activation rows."""
     fmt, N, K, r, s = p["fmt"], p["N"], p["K"], p["r"], p["s"]
     wbytes = weight_bytes(fmt, N, K)
+    per_clk = Q.qlora_debug_decode_rate(fmt)
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    clk_hz = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    decode_peak = per_clk * sms * clk_hz                      # weights / s
     nw = int(math.ceil(3 * 126e6 / wbytes)) + 1
     base = list(Ws) if Ws else []
     Wsw = base + [Q.weight_from_numpy(fmt, p["codes"], p["scales"], p["tensor_scale"])
@@ -296,12 +303,18 @@ def short_batch_sweep(Q, torch, p, Ws, X, dY, A, B, peaks):
         t = a0.elapsed_time(a1) / n_it * 1e-3
         fl = flops(Ms, N, K, r)
         byt = 2 * wbytes + 2 * (2 * Ms * K + 2 * Ms * N)
-        t_roof = max(fl / (peaks["bf16_tflops"] * 1e12), byt / (peaks["hbm_gbs"] * 1e9))
+        bounds = {"tensor": fl / (peaks["bf16_tflops"] * 1e12),
+                  "hbm": byt / (peaks["hbm_gbs"] * 1e9),
+                  "alu": 2.0 * N * K / decode_peak}
+        bound = max(bounds, key=bounds.get)
         out[str(Ms)] = {"us_per_step": round(t * 1e6, 1),
                         "weight_gbs": round(2 * wbytes / t / 1e9, 1),
                         "tflops": round(fl / t / 1e12, 1),
-                        "roofline_frac": round(t_roof / t, 4),
-                        "bound": "tensor" if fl / (peaks["bf16_tflops"] * 1e12) > byt / (peaks["hbm_gbs"] * 1e9) else "hbm"}
+                        "roofline_frac": round(bounds[bound] / t, 4),
+                        "bound": bound}
+    out["decode_peak"] = {"weights_per_clk_per_sm": round(per_clk, 2), "sms": sms,
+                          "sm_mhz": clk_hz / 1e6, "weights_per_s": round(decode_peak / 1e12, 3),
+                          "unit": "T weights/s", "source": "qlora_debug_decode_rate (measured)"}
     del Wsw
     torch.cuda.empty_cache()
     return out

@@ -863,6 +863,35 @@ qlora_status_t qlora_debug_dequant(const qlora_weight_t* W, int transposed, void
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+qlora_status_t qlora_debug_decode_rate(int fmt, int iters, double* weights_per_clock_per_sm) {
+  if (!weights_per_clock_per_sm || iters < 1 || iters > (1 << 20) || fmt < QLORA_FMT_NF4 ||
+      fmt > QLORA_FMT_NVFP4)
+    return QLORA_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  unsigned long long* cyc = nullptr;
+  uint32_t* sink = nullptr;
+  if (cudaMalloc(&cyc, sizeof(unsigned long long) * sms) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaMalloc(&sink, 4) != cudaSuccess) {
+    cudaFree(cyc);
+    return QLORA_ERR_CUDA;
+  }
+  if (fmt == QLORA_FMT_NF4) qlora_debug_decode_rate_kernel<kFmtNF4><<<sms, 256>>>(iters, cyc, sink);
+  else if (fmt == QLORA_FMT_MXFP4) qlora_debug_decode_rate_kernel<kFmtMXFP4><<<sms, 256>>>(iters, cyc, sink);
+  else qlora_debug_decode_rate_kernel<kFmtNVFP4><<<sms, 256>>>(iters, cyc, sink);
+  std::vector<unsigned long long> h(sms);
+  const bool ok = cudaGetLastError() == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess &&
+                  cudaMemcpy(h.data(), cyc, sizeof(unsigned long long) * sms,
+                             cudaMemcpyDeviceToHost) == cudaSuccess;
+  cudaFree(cyc);
+  cudaFree(sink);
+  if (!ok) return QLORA_ERR_CUDA;
+  double c = 0;
+  for (int i = 0; i < sms; ++i) c += double(h[i]);
+  c /= sms;
+  *weights_per_clock_per_sm = c > 0 ? double(iters) * 256.0 * 64.0 / c : 0.0;
+  return QLORA_OK;
+}
+
 qlora_status_t qlora_debug_wait_timeout(void* ws, size_t ws_bytes, int limit_us,
                                         qlora_stream_t stream) {
   if (!ws || !aligned16(ws) || ws_bytes < kHeaderBytes) return QLORA_ERR_WORKSPACE;

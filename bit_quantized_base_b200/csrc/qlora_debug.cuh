@@ -67,6 +67,38 @@ qlora_debug_dequant_kernel(const __grid_constant__ DebugDequantParams p) {
   }
 }
 
+// Decode throughput of the layer's own dequant stage on one SM, the bound of the short-batch
+// (weight-streaming) path: 256 threads (the two dequant groups' worth) each decode `iters`
+// 64-element items with dequant_item_store into a swizzled operand tile, fresh codes every item
+// (updated with a multiply-add, so the integer pipe does only decode work).  cycles[b] = the CTA's
+// clock cycles for the loop.
+template <int FMT>
+__global__ void __launch_bounds__(256, 1)
+qlora_debug_decode_rate_kernel(int iters, unsigned long long* cycles, uint32_t* sink) {
+  __shared__ __align__(1024) uint8_t tile[2][fused::W_BYTES];
+  const int tg = threadIdx.x & 127;
+  const ItemGeom<false> geo(tg);
+  const uint32_t rb = geo.op_row_base(ptx::smem_u32(tile[threadIdx.x >> 7]));
+  uint32_t cw[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) cw[j] = (threadIdx.x * 8u + j + blockIdx.x * 7919u) * 0x9E3779B1u;
+  ItemScale sc;
+  sc.raw = FMT == kFmtNF4 ? __float_as_uint(0.01f + 0.001f * float(tg & 7))
+                          : (FMT == kFmtMXFP4 ? 0x7C7Du : 0x38393A3Bu);
+  __syncthreads();
+  const unsigned long long t0 = clock64();
+  for (int it = 0; it < iters; ++it) {
+    dequant_item_store<FMT>(cw, sc, rb, geo.swz());
+#pragma unroll
+    for (int j = 0; j < 8; ++j) cw[j] = cw[j] * 0x9E3779B1u + 0x7F4A7C15u;
+  }
+  __syncthreads();
+  const unsigned long long t1 = clock64();
+  const uint32_t v = ptx::ld_shared_v4(rb).x;
+  if (v == 0x12345678u) sink[0] = v;   // keeps the stores live
+  if (threadIdx.x == 0) cycles[blockIdx.x] = t1 - t0;
+}
+
 __global__ void qlora_debug_wait_kernel(int* status, unsigned long long limit_cycles) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;

@@ -27,7 +27,8 @@ EXPORTS = ("qlora_workspace_size", "qlora_workspace_init", "qlora_linear_fwd", "
            "qlora_grouped_fwd", "qlora_grouped_bwd", "qlora_get_device_status",
            "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_status_string",
            "qlora_build_info", "qlora_launch_count", "qlora_profile_enable",
-           "qlora_profile_reset", "qlora_profile_read", "qlora_linear_fwd_noalloc")
+           "qlora_profile_reset", "qlora_profile_read", "qlora_linear_fwd_noalloc",
+           "qlora_debug_decode_rate")
 
 
 class QLoraError(RuntimeError):
@@ -65,6 +66,7 @@ def _load():
     L.qlora_get_device_status.argtypes = [P, P]
     L.qlora_debug_dequant.argtypes = [W, c.c_int, P, P]
     L.qlora_debug_wait_timeout.argtypes = [P, c.c_size_t, c.c_int, P]
+    L.qlora_debug_decode_rate.argtypes = [c.c_int, c.c_int, c.POINTER(c.c_double)]
     L.qlora_status_string.argtypes = [c.c_int]
     L.qlora_status_string.restype = c.c_char_p
     L.qlora_build_info.restype = c.c_char_p
@@ -76,7 +78,8 @@ def _load():
                                      c.POINTER(c.c_int), c.POINTER(c.c_double)]
     for name in ("qlora_workspace_init", "qlora_linear_fwd", "qlora_linear_bwd",
                  "qlora_grouped_fwd", "qlora_grouped_bwd", "qlora_get_device_status",
-                 "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_profile_enable",
+                 "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_debug_decode_rate",
+                 "qlora_profile_enable",
                  "qlora_profile_reset", "qlora_profile_read"):
         getattr(L, name).restype = c.c_int
     return L
@@ -185,6 +188,14 @@ def qlora_debug_dequant(W: Weight, transposed, out, stream=None):
 def qlora_debug_wait_timeout(ws, limit_us, stream=None):
     _check(lib.qlora_debug_wait_timeout(_p(ws), ws.numel(), int(limit_us), _stream(stream)),
            "qlora_debug_wait_timeout")
+
+
+def qlora_debug_decode_rate(fmt, iters=2000):
+    """Decoded weights per SM clock of the layer's dequant stage, measured on every SM."""
+    v = ctypes.c_double(0.0)
+    _check(lib.qlora_debug_decode_rate(FMT[fmt] if isinstance(fmt, str) else int(fmt), int(iters),
+                                       ctypes.byref(v)), "qlora_debug_decode_rate")
+    return v.value
 
 
 def qlora_build_info():

@@ -193,6 +193,16 @@ QLORA_API qlora_status_t qlora_debug_dequant(const qlora_weight_t* W, int transp
 QLORA_API qlora_status_t qlora_debug_wait_timeout(void* ws, size_t ws_bytes, int limit_us,
                                         qlora_stream_t stream);
 
+/* Benchmark support: measure the decode throughput of the layer's own dequant stage (the code
+ * every GEMM kernel decodes the 4-bit weight with) on every SM -- 256 threads per SM, each
+ * decoding `iters` 64-element items into a shared-memory operand tile -- and return the mean
+ * decoded weights per SM clock cycle in *weights_per_clock_per_sm.  fmt: QLORA_FMT_*; 1 <= iters
+ * <= 2^20.  Synchronises the device and allocates two small device buffers; not for the compute
+ * path.  The result is the ceiling of the short-batch path, where every weight is decoded for a
+ * few activation rows. */
+QLORA_API qlora_status_t qlora_debug_decode_rate(int fmt, int iters,
+                                                 double* weights_per_clock_per_sm);
+
 /* Profiling support for benchmarks.  qlora_launch_count() is the number of kernels this library
  * has launched in the process (always counted).  While profiling is enabled, every launch is also
  * bracketed by two CUDA events recorded on its stream (up to 65536 launches; events are created by

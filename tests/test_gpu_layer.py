@@ -191,6 +191,14 @@ def test_pair_ticket_from_any_start():
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+def test_decode_rate_measurement(fmt):
+    # the benchmark's decode ceiling: a positive rate of the order of the ALU's width
+    from bit_quantized_base_b200 import qlora as Q
+    v = Q.qlora_debug_decode_rate(fmt, 200)
+    assert 2.0 < v < 200.0, v
+
+
 def test_step0_init_on_gpu():
     # B = 0 -> dA == 0 exactly and Y equals the base product ("Initialization matters")
     p = synth.small_layer("nf4", 64, 128, 256, 16, seed=2)
