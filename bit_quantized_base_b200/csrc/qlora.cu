@@ -716,10 +716,11 @@ qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   st = launch_lora_down(true, dY, M, W->N, B, r, scale, ts, U, Zs, ws_status(ws), offsets, E,
                         grouped, !dX ? 0 : (short_dx ? kDownCtasBesideStream : kDownCtasBesidePair), s);
   if (st != QLORA_OK) return st;
-  if (dX && !short_dx) {
-    // The adapter gradients need only T, U, X and dY, so they run on a side stream beside the
-    // tiled dX kernel, filling the SMs its last wave of tiles leaves idle (the two kernels share
-    // no workspace region).  Joined back into `s` before returning.
+  if (dX) {
+    // The adapter gradients need only T, U, X and dY, so they run on a side stream beside the dX
+    // kernel, on the SMs it leaves idle (the tiled kernel's last wave of tiles; the SMs the
+    // streaming kernel leaves to lora_down); the kernels share no workspace region.  Joined back
+    // into `s` before returning.
     SideStream* side = side_stream();
     if (side) {
       const int slot = side->next.fetch_add(1, std::memory_order_relaxed) % SideStream::kEvents;
@@ -730,7 +731,9 @@ qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
                         side->stream);
       if (st != QLORA_OK) return st;
       if (cudaEventRecord(side->join[slot], side->stream) != cudaSuccess) return QLORA_ERR_CUDA;
-      st = launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), offsets, E, grouped, s);
+      st = short_dx ? launch_stream(W, true, dY, Zs, A, dX, M, r, ws_status(ws), part,
+                                    ws_bytes - L.partial, s)
+                    : launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), offsets, E, grouped, s);
       if (cudaStreamWaitEvent(s, side->join[slot], 0) != cudaSuccess) return QLORA_ERR_CUDA;
       return st;
     }
