@@ -706,9 +706,11 @@ qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   void* U = w + L.u;
   float* part = reinterpret_cast<float*>(w + L.partial);
   qlora_status_t st;
-  if (!T) {  // recompute T = X A^T (its scaled copy lands in Zs and is overwritten below)
+  if (!T) {  // recompute T = X A^T (its scaled copy lands in Zs and is overwritten below) with
+             // the forward's split plan, so it equals the forward's T bit for bit
+    const bool short_fwd = stream_fits(W, M, E, false, ws_bytes - L.partial);
     st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, w + L.t, Zs, ws_status(ws), offsets,
-                          E, grouped, 0, s);
+                          E, grouped, short_fwd ? kDownCtasBesideStream : kDownCtasBesidePair, s);
     if (st != QLORA_OK) return st;
     T = w + L.t;
   }

@@ -150,14 +150,16 @@ QLORA_API qlora_status_t qlora_grouped_bwd(const qlora_weight_t* W, int E, const
                                  int r, float scale, void* ws, size_t ws_bytes,
                                  qlora_stream_t stream);
 
-/* Forward without a workspace: the same computation and kernels as qlora_linear_fwd, for callers
+/* Forward without a workspace: the same computation as qlora_linear_fwd, for callers
  * that cannot allocate device memory where they run the layer -- for example runtimes that
  * allocate everything at start-up and forbid allocation on the step path (an allocation can
  * synchronise the device and fragment its memory), or plain C callers with no allocator of their
  * own.  The paper has no counterpart of this entry point; it only changes who provides scratch.
  *   Scratch is a fixed 4 MiB array inside the library (every GPU that loads the library holds it
  *   until the process exits): 256 bytes of status, the [M,r] bf16 operand Zs and, when T_save is
- *   NULL, an [M,r] bf16 T; results are bitwise those of qlora_linear_fwd.  Sizes that do not fit
+ *   NULL, an [M,r] bf16 T.  It always runs the tiled kernels, so for M > 256 its results are
+ *   bitwise those of qlora_linear_fwd; shorter batches, which qlora_linear_fwd runs through the
+ *   weight-streaming kernel, differ from them in rounding only.  Sizes that do not fit
  *   -- M*r > 2,097,024 with T_save, or
  *   M*r > 1,048,512 without -- are rejected with QLORA_ERR_WORKSPACE before anything is enqueued.
  *   The call allocates nothing (no cudaMalloc/cudaFree, no allocating library routine); it clears

@@ -155,6 +155,20 @@ def test_backward_recomputes_T_and_skips_dx():
     assert_close(to_f64(dB), ref["dB"], "dB")
 
 
+@pytest.mark.parametrize("M", [200, 1000])   # streaming and pair paths
+def test_backward_recompute_matches_saved_T(M):
+    # T recomputed in the backward pass uses the forward's plan: same T, bit for bit, so the
+    # gradients equal those computed from the saved T
+    p = synth.small_layer("nf4", M, 768, 1024, 32, seed=4)
+    g = GpuLayer(p)
+    Y, T = g.fwd()
+    saved = g.bwd(T)
+    recomputed = g.bwd(None)
+    torch.cuda.synchronize()
+    for a, b in zip(saved, recomputed):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
 def test_deterministic_reruns():
     p = synth.small_layer("nf4", 1000, 512, 1024, 32, seed=9)
     g = GpuLayer(p)
