@@ -182,6 +182,41 @@ def _encode_rows(fmt: str, W: np.ndarray, ts):
     return pack_nibbles(c.reshape(N, K)), sb
 
 
+DQ_GROUP = 256   # NF4 with double quantisation: first-level codes per fp32 second-level scale
+
+
+def encode_nf4dq(W: np.ndarray):
+    """Quantise a float weight [N,K] to NF4 with a double-quantised absmax -> (codes [N,K/2],
+    first-level E4M3 codes [N,K/64] uint8, second-level fp32 scales [ceil(N*K/64 / 256)]).
+
+    Test-data encoder (its choices are not part of the decode definition): the 64-block absmax
+    is fp32 max|w|; every 256 consecutive absmax values (row-major) share s2 = max / 448; the
+    first-level code is the nearest E4M3 of absmax / s2; the 4-bit codes are the nearest NF4
+    levels of w / (decoded absmax)."""
+    W = np.asarray(W, np.float32)
+    N, K = W.shape
+    assert K % 64 == 0
+    nb = K // 64
+    Wb = W.reshape(N, nb, 64)
+    amax = np.abs(Wb).max(axis=2).astype(np.float32).reshape(-1)
+    G = (amax.size + DQ_GROUP - 1) // DQ_GROUP
+    pad = np.zeros(G * DQ_GROUP, np.float32)
+    pad[:amax.size] = amax
+    gmax = pad.reshape(G, DQ_GROUP).max(axis=1)
+    s2 = np.where(gmax > 0, gmax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    s2_el = np.repeat(s2, DQ_GROUP)[:amax.size]
+    c1 = _e4m3_code(amax / s2_el)
+    absmax_d = (_E4M3[c1.astype(np.int64)].astype(np.float32) * s2_el).astype(np.float32)
+    absmax_d = absmax_d.reshape(N, nb)
+    grid = _nf4_grid()
+    mids = 0.5 * (grid[1:] + grid[:-1])
+    safe = np.where(absmax_d > 0, absmax_d, np.float32(1.0))[:, :, None]
+    x = (Wb / safe).astype(np.float64)
+    c = np.searchsorted(mids, x, side="left").astype(np.uint8)
+    c[np.broadcast_to(absmax_d[:, :, None] == 0, c.shape)] = 7
+    return pack_nibbles(c.reshape(N, K)), c1.reshape(N, nb), s2
+
+
 def random_stored_weight(fmt: str, N: int, K: int, rng: np.random.Generator,
                          scale_codes=None):
     """Uniformly random codes and scales (every code and every scale pattern reachable).
@@ -335,9 +370,14 @@ def layer_inputs(cfg_id: int, proj: int = 0, M: int | None = None):
 
 def small_layer(fmt: str, M: int, N: int, K: int, r: int, s: float = 2.0, seed: int = 0,
                 random_codes: bool = False, x_std=1.0, dy_std=1.0, b_std=0.01):
-    """A small seeded problem for parity tests (W ~ N(0, 0.02) quantised, or random codes)."""
+    """A small seeded problem for parity tests (W ~ N(0, 0.02) quantised, or random codes).
+    fmt "nf4dq" (NF4 with double-quantised absmax) adds scales2, the second-level scales."""
     rng = np.random.Generator(np.random.PCG64(seed))
-    if random_codes:
+    scales2 = None
+    if fmt == "nf4dq":
+        codes, scales, scales2 = encode_nf4dq(_normal(rng, (N, K), 0.02))
+        ts = 1.0
+    elif random_codes:
         codes, scales, ts = random_stored_weight(fmt, N, K, rng)
         ts = 1.0 if ts is None else float(ts)
     else:
@@ -349,7 +389,7 @@ def small_layer(fmt: str, M: int, N: int, K: int, r: int, s: float = 2.0, seed: 
     X = to_bf16_bits(_normal(rng, (M, K), x_std))
     dY = to_bf16_bits(_normal(rng, (M, N), dy_std))
     return dict(fmt=fmt, M=M, N=N, K=K, r=r, s=s, codes=codes, scales=scales, tensor_scale=ts,
-                X=X, A=A, B=B, dY=dY)
+                scales2=scales2, X=X, A=A, B=B, dY=dY)
 
 
 def small_grouped(fmt: str, counts, N: int, K: int, r: int, s: float = 2.0, seed: int = 0,

@@ -13,8 +13,14 @@ import numpy as np
 
 from . import build_oracle
 
-FORMATS = {"nf4": 0, "mxfp4": 1, "nvfp4": 2}
-BLOCK = {0: 64, 1: 32, 2: 16}
+FORMATS = {"nf4": 0, "mxfp4": 1, "nvfp4": 2, "nf4dq": 3}
+BLOCK = {0: 64, 1: 32, 2: 16, 3: 64}
+DQ_GROUP = 256   # NF4-DQ: first-level constants per fp32 second-level scale
+
+
+def dq_groups(N, K):
+    """Second-level scales of one [N, K] NF4-DQ weight."""
+    return (N * (K // 64) + DQ_GROUP - 1) // DQ_GROUP
 
 _lib = None
 
@@ -39,10 +45,10 @@ def lib():
         L.oracle_weight_bytes.argtypes = [c.c_int, c.c_int64, c.c_int64]
         L.oracle_weight_bytes.restype = c.c_int64
         L.oracle_dequant.argtypes = [c.c_int, c.c_int64, c.c_int64, c.c_void_p, c.c_void_p,
-                                     c.c_float, c.c_int, c.c_void_p]
+                                     c.c_void_p, c.c_float, c.c_int, c.c_void_p]
         L.oracle_dequant.restype = c.c_int
         L.oracle_layer.argtypes = [c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_int, c.c_double,
-                                   c.c_void_p, c.c_void_p, c.c_float,
+                                   c.c_void_p, c.c_void_p, c.c_void_p, c.c_float,
                                    c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
                                    c.c_void_p, c.c_int64,
                                    c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
@@ -101,20 +107,26 @@ def weight_bytes(fmt, N, K):
     return lib().oracle_weight_bytes(_fmt(fmt), int(N), int(K))
 
 
-def dequant(fmt, N, K, codes, scales, tensor_scale=1.0, with_tensor_scale=True):
-    """Decoded weight [N,K] as bf16 bit patterns (uint16)."""
+def _scales2(scales2):
+    return None if scales2 is None else np.ascontiguousarray(scales2, np.float32)
+
+
+def dequant(fmt, N, K, codes, scales, tensor_scale=1.0, with_tensor_scale=True, scales2=None):
+    """Decoded weight [N,K] as bf16 bit patterns (uint16).  scales2: NF4-DQ second-level fp32
+    scales [dq_groups(N, K)]."""
     codes = np.ascontiguousarray(codes, np.uint8)
     scales = np.ascontiguousarray(scales)
+    s2 = _scales2(scales2)
     out = np.zeros((N, K), np.uint16)
-    rc = lib().oracle_dequant(_fmt(fmt), N, K, _ptr(codes), _ptr(scales), float(tensor_scale),
-                              1 if with_tensor_scale else 0, _ptr(out))
+    rc = lib().oracle_dequant(_fmt(fmt), N, K, _ptr(codes), _ptr(scales), _ptr(s2),
+                              float(tensor_scale), 1 if with_tensor_scale else 0, _ptr(out))
     if rc != 0:
         raise ValueError("oracle_dequant rejected its arguments")
     return out
 
 
 def layer(fmt, M, N, K, r, s, codes, scales, tensor_scale, X, A, B, dY=None, rows=None,
-          want=("Y", "dX", "T", "U", "dA", "dB")):
+          want=("Y", "dX", "T", "U", "dA", "dB"), scales2=None):
     """fp64 layer forward + backward.  X/A/B/dY are uint16 bf16 bit patterns.
 
     rows: optional int64 array of the rows of Y and dX to produce (None: all rows).
@@ -135,7 +147,8 @@ def layer(fmt, M, N, K, r, s, codes, scales, tensor_scale, X, A, B, dY=None, row
     out["U"] = np.zeros((M, r)) if ("U" in want and dY is not None) else None
     out["dA"] = np.zeros((r, K)) if ("dA" in want and dY is not None) else None
     out["dB"] = np.zeros((N, r)) if ("dB" in want and dY is not None) else None
-    rc = lib().oracle_layer(_fmt(fmt), M, N, K, r, float(s), _ptr(codes), _ptr(scales),
+    s2 = _scales2(scales2)
+    rc = lib().oracle_layer(_fmt(fmt), M, N, K, r, float(s), _ptr(codes), _ptr(scales), _ptr(s2),
                             float(tensor_scale), _ptr(X), _ptr(A), _ptr(B), _ptr(dY),
                             _ptr(rows_arr), nrows,
                             _ptr(out["Y"]), _ptr(out["dX"]), _ptr(out["T"]), _ptr(out["U"]),
@@ -146,12 +159,13 @@ def layer(fmt, M, N, K, r, s, codes, scales, tensor_scale, X, A, B, dY=None, row
 
 
 def grouped_layer(fmt, offsets, N, K, r, s, codes, scales, tensor_scales, X, A, B, dY=None,
-                  rows_per_expert=None, want=("Y", "dX", "T", "U", "dA", "dB")):
+                  rows_per_expert=None, want=("Y", "dX", "T", "U", "dA", "dB"), scales2=None):
     """The grouped (MoE) layer: the single layer above applied to each expert e on its rows
     [offsets[e], offsets[e+1]) of the packed X / dY with that expert's own weight and adapters.
 
     codes [E, N, K/2], scales [E, N, K/bs], tensor_scales [E] (NVFP4) or None, A [E, r, K],
-    B [E, N, r].  rows_per_expert: optional list of local row indices per expert.
+    B [E, N, r], scales2 [E, dq_groups(N, K)] (NF4-DQ) or None.  rows_per_expert: optional list
+    of local row indices per expert.
     Returns a list of per-expert dicts (row indices in each are local to the expert).
     """
     E = len(offsets) - 1
@@ -161,7 +175,8 @@ def grouped_layer(fmt, offsets, N, K, r, s, codes, scales, tensor_scales, X, A, 
         ts = 1.0 if tensor_scales is None else float(tensor_scales[e])
         rows = None if rows_per_expert is None else rows_per_expert[e]
         res.append(layer(fmt, m1 - m0, N, K, r, s, codes[e], scales[e], ts, X[m0:m1], A[e], B[e],
-                         None if dY is None else dY[m0:m1], rows=rows, want=want))
+                         None if dY is None else dY[m0:m1], rows=rows, want=want,
+                         scales2=None if scales2 is None else scales2[e]))
     return res
 
 

@@ -15,6 +15,11 @@
 //               16 along K plus one fp32 tensor scale
 //               ("Fine-Tuning 4-Bit Models: Adapting a Base That Only Ships Quantized", "Case 2:
 //               An NVFP4 deployment checkpoint is what you were handed").
+//       NF4 with double quantisation: as NF4 with absmax = fp32( e4m3(c1) * s2[g] ): the 64-block
+//               absmax is stored as an 8-bit E4M3 code c1, and every 256 consecutive first-level
+//               codes of the weight (row-major [N, K/64] order) share one fp32 second-level
+//               scale s2 ("Training LLMs on a Budget", §3 "The three QLoRA tricks", item 2:
+//               "8-bit FP8 with a second-level absmax over blocks of 256 first-level constants").
 //     Every multiply is IEEE binary32 round-to-nearest-even, subnormals kept (no FTZ).
 //   * The layer, in fp64 on the exact bf16/fp32 input values, with s = alpha/r (or alpha/sqrt r)
 //     multiplying every LoRA term ("Training LLMs on a Budget", §2 "The math": y = Wx + (a/r)BAx,
@@ -174,8 +179,15 @@ double norm_ppf(double p) {
   return (q < 0.0) ? -x : x;
 }
 
+// Formats: 0 NF4, 1 MXFP4, 2 NVFP4, 3 NF4 with double-quantised absmax.
+constexpr int kFmtNf4Dq = 3;
+constexpr int64_t kDqGroup = 256;   // first-level constants per second-level scale
+
 // Block size along K of the scale of each format.
-int block_size(int fmt) { return fmt == 0 ? 64 : (fmt == 1 ? 32 : 16); }
+int block_size(int fmt) { return (fmt == 0 || fmt == kFmtNf4Dq) ? 64 : (fmt == 1 ? 32 : 16); }
+
+// Second-level scales of one [N, K] NF4-DQ weight: ceil(N * K/64 / 256).
+int64_t dq_groups(int64_t N, int64_t K) { return (N * (K / 64) + kDqGroup - 1) / kDqGroup; }
 
 uint32_t code_at(const uint8_t* codes, int64_t K, int64_t n, int64_t k) {
   const uint8_t byte = codes[n * (K / 2) + k / 2];
@@ -184,13 +196,20 @@ uint32_t code_at(const uint8_t* codes, int64_t K, int64_t n, int64_t k) {
 
 // One weight element per the definition at the top of this file.  with_tensor_scale = 0 stops
 // the NVFP4 chain before the tensor scale (the micro-block decode alone).
-uint16_t dequant_element(int fmt, const uint8_t* codes, const void* scales, float tensor_scale,
-                         int with_tensor_scale, int64_t K, int64_t n, int64_t k) {
+uint16_t dequant_element(int fmt, const uint8_t* codes, const void* scales, const float* scales2,
+                         float tensor_scale, int with_tensor_scale, int64_t K, int64_t n,
+                         int64_t k) {
   const uint32_t c = code_at(codes, K, n, k);
   const int64_t nb = K / block_size(fmt);
   const int64_t blk = k / block_size(fmt);
   if (fmt == 0) {
     const float absmax = static_cast<const float*>(scales)[n * nb + blk];
+    const float p = nf4_level(c) * absmax;
+    return f32_to_bf16_rne(p);
+  }
+  if (fmt == kFmtNf4Dq) {
+    const int64_t f = n * nb + blk;   // first-level constant, row-major
+    const float absmax = e4m3_value(static_cast<const uint8_t*>(scales)[f]) * scales2[f / kDqGroup];
     const float p = nf4_level(c) * absmax;
     return f32_to_bf16_rne(p);
   }
@@ -206,7 +225,7 @@ uint16_t dequant_element(int fmt, const uint8_t* codes, const void* scales, floa
 }
 
 bool valid_shape(int fmt, int64_t N, int64_t K) {
-  if (fmt < 0 || fmt > 2 || N < 0 || K < 0) return false;
+  if (fmt < 0 || fmt > kFmtNf4Dq || N < 0 || K < 0) return false;
   return K % block_size(fmt) == 0;
 }
 
@@ -247,24 +266,30 @@ float oracle_decode_e4m3(uint32_t code) { return e4m3_value(code); }
 uint16_t oracle_f32_to_bf16(float x) { return f32_to_bf16_rne(x); }
 float oracle_bf16_to_f32(uint16_t h) { return bf16_to_f32(h); }
 
-// Bytes of one stored weight: codes + block scales (+ 4 for the NVFP4 tensor scale).
+// Bytes of one stored weight: codes + block scales (+ 4 for the NVFP4 tensor scale; + 4 per 256
+// first-level constants for NF4 with double quantisation).
 int64_t oracle_weight_bytes(int fmt, int64_t N, int64_t K) {
   if (!valid_shape(fmt, N, K)) return -1;
   const int64_t codes = N * K / 2;
   const int64_t nb = N * (K / block_size(fmt));
   if (fmt == 0) return codes + 4 * nb;
+  if (fmt == kFmtNf4Dq) return codes + nb + 4 * dq_groups(N, K);
   if (fmt == 1) return codes + nb;
   return codes + nb + 4;
 }
 
-// Decode a whole weight [N,K] to bf16 bit patterns.  Returns 0, or -1 on a bad argument.
+// Decode a whole weight [N,K] to bf16 bit patterns.  scales2: NF4-DQ second-level scales
+// [ceil(N * K/64 / 256)], else unused.  Returns 0, or -1 on a bad argument.
 int oracle_dequant(int fmt, int64_t N, int64_t K, const uint8_t* codes, const void* scales,
-                   float tensor_scale, int with_tensor_scale, uint16_t* out) {
+                   const float* scales2, float tensor_scale, int with_tensor_scale,
+                   uint16_t* out) {
   if (!valid_shape(fmt, N, K) || (N * K > 0 && (!codes || !scales || !out))) return -1;
+  if (fmt == kFmtNf4Dq && N * K > 0 && !scales2) return -1;
 #pragma omp parallel for schedule(static)
   for (int64_t n = 0; n < N; ++n)
     for (int64_t k = 0; k < K; ++k)
-      out[n * K + k] = dequant_element(fmt, codes, scales, tensor_scale, with_tensor_scale, K, n, k);
+      out[n * K + k] = dequant_element(fmt, codes, scales, scales2, tensor_scale,
+                                       with_tensor_scale, K, n, k);
   return 0;
 }
 
@@ -275,7 +300,7 @@ int oracle_dequant(int fmt, int64_t N, int64_t K, const uint8_t* codes, const vo
 //   U [M,r], dA [r,K], dB [N,r].  T, U, dA and dB always cover all M rows.
 // Returns 0, or -1 on a bad argument.
 int oracle_layer(int fmt, int64_t M, int64_t N, int64_t K, int r, double s,
-                 const uint8_t* codes, const void* scales, float tensor_scale,
+                 const uint8_t* codes, const void* scales, const float* scales2, float tensor_scale,
                  const uint16_t* X, const uint16_t* A, const uint16_t* B, const uint16_t* dY,
                  const int64_t* rows, int64_t nrows,
                  double* Y_rows, double* dX_rows, double* T_out, double* U_out,
@@ -289,7 +314,8 @@ int oracle_layer(int fmt, int64_t M, int64_t N, int64_t K, int r, double s,
   std::vector<float> Wd(static_cast<size_t>(N * K));
   {
     std::vector<uint16_t> wb(static_cast<size_t>(N * K));
-    if (N * K > 0 && oracle_dequant(fmt, N, K, codes, scales, tensor_scale, 1, wb.data()) != 0)
+    if (N * K > 0 &&
+        oracle_dequant(fmt, N, K, codes, scales, scales2, tensor_scale, 1, wb.data()) != 0)
       return -1;
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < N * K; ++i) Wd[static_cast<size_t>(i)] = bf16_to_f32(wb[static_cast<size_t>(i)]);

@@ -204,11 +204,78 @@ def test_weight_bytes_pins_memory_table():
             nbytes = O.weight_bytes("nf4", N, K)
             assert nbytes * 8 == N * K * 4.5
             assert round(P * 4.5 / 8 / 1e9, 1) == float(gb)
-        else:
+        elif name == "fp16":
             assert round(P * int(bits) / 8 / 1e9, 1) == float(gb)
+        elif name == "nf4dq":
+            # 8-bit first level per 64 weights + one fp32 per 256 first-level constants
+            N, K = 4096, 16384
+            bpw = O.weight_bytes("nf4dq", N, K) * 8 / (N * K)
+            assert abs(bpw - (4 + 8 / 64 + 32 / (64 * 256))) < 1e-12
+            assert round(bpw, 3) == float(bits)
+            assert round(P * bpw / 8 / 1e9, 1) == float(gb)
+            assert abs((4.5 - bpw) - 0.373) < 5e-4            # "net savings: about 0.373 bits"
     assert O.weight_bytes("mxfp4", 64, 1024) * 8 == 64 * 1024 * 4.25
     assert O.weight_bytes("nvfp4", 64, 1024) * 8 == 64 * 1024 * 4.5 + 32
     assert O.weight_bytes("nf4", 64, 100) == -1                 # K must be a whole number of blocks
+
+
+# ---------------------------------------------------------------- NF4 with double quantisation
+def _e4m3_values32(c1):
+    return np.array([O.decode_e4m3(int(v)) for v in np.asarray(c1).reshape(-1)],
+                    np.float32).reshape(np.asarray(c1).shape)
+
+
+def test_dequant_nf4dq_reduces_to_nf4_with_unit_second_level():
+    # s2 = 1: the absmax is the first-level E4M3 value itself, so the decode must equal the
+    # (separately pinned) NF4 decode with that fp32 absmax, bit for bit, for every E4M3 code
+    rng = np.random.default_rng(3)
+    N, K = 24, 64 * 64
+    codes = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    c1 = rng.integers(0, 256, size=(N, K // 64), dtype=np.uint8)
+    c1.reshape(-1)[:256] = np.arange(256, dtype=np.uint8)        # every first-level code
+    s2 = np.ones(O.dq_groups(N, K), np.float32)
+    got = O.dequant("nf4dq", N, K, codes, c1, scales2=s2)
+    ref = O.dequant("nf4", N, K, codes, _e4m3_values32(c1))
+    assert np.array_equal(got, ref)
+
+
+def test_dequant_nf4dq_second_level_groups():
+    # distinct power-of-two s2 per group (exact products), 300 blocks per row: groups of 256
+    # consecutive first-level constants straddle rows.  Each block must take the s2 of its own
+    # group, i.e. equal NF4 with absmax = e4m3(c1) * s2[f // 256], f the row-major block index.
+    rng = np.random.default_rng(4)
+    N, K = 7, 64 * 300
+    codes = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    c1 = rng.integers(0x20, 0x60, size=(N, K // 64), dtype=np.uint8)
+    G = O.dq_groups(N, K)
+    assert G == math.ceil(N * 300 / 256)
+    s2 = np.ldexp(np.ones(G, np.float32), np.arange(G) - 4).astype(np.float32)
+    got = O.dequant("nf4dq", N, K, codes, c1, scales2=s2)
+    f = np.arange(N * 300).reshape(N, 300)
+    absmax = (_e4m3_values32(c1) * s2[f // 256]).astype(np.float32)
+    ref = O.dequant("nf4", N, K, codes, absmax)
+    assert np.array_equal(got, ref)
+    # and a different group assignment (a shift by one block) would not match
+    wrong = (_e4m3_values32(c1) * s2[(f + 1) // 256]).astype(np.float32)
+    assert not np.array_equal(got, O.dequant("nf4", N, K, codes, wrong))
+
+
+def test_nf4dq_encoder_absmax_within_e4m3_bound():
+    # the test-data encoder's stored absmax (decoded by the oracle: e4m3(c1) * s2) is within the
+    # E4M3 rounding bound (relative 2^-4) of the true block absmax wherever absmax / s2 is in
+    # E4M3's normal range
+    from bit_quantized_base_b200 import synth
+    rng = np.random.default_rng(5)
+    N, K = 40, 64 * 50
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    codes, c1, s2 = synth.encode_nf4dq(W)
+    true = np.abs(W.reshape(N, 50, 64)).max(axis=2).reshape(-1)
+    f = np.arange(true.size)
+    dec = _e4m3_values32(c1).reshape(-1).astype(np.float64) * s2[f // 256]
+    normal = true / s2[f // 256] >= 2.0 ** -6
+    assert normal.mean() > 0.9
+    rel = np.abs(dec[normal] - true[normal]) / true[normal]
+    assert rel.max() <= 2.0 ** -4 + 1e-7
 
 
 def test_dequant_rejects_bad_shape():
