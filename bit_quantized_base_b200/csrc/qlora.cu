@@ -140,13 +140,16 @@ cudaError_t launch_pdl_cluster(void (*kernel)(P), dim3 grid, dim3 block, size_t 
 
 qlora_status_t check_weight(const qlora_weight_t* W) {
   if (!W) return QLORA_ERR_INVALID_ARG;
-  if (W->fmt < QLORA_FMT_NF4 || W->fmt > QLORA_FMT_NVFP4) return QLORA_ERR_INVALID_ARG;
+  if (W->fmt < QLORA_FMT_NF4 || W->fmt > QLORA_FMT_NF4_DQ) return QLORA_ERR_INVALID_ARG;
   if (W->N < 16 || W->N % 16 != 0 || W->K < 64 || W->K % 64 != 0) return QLORA_ERR_INVALID_ARG;
   if (W->N > (int64_t(1) << 30) || W->K > (int64_t(1) << 30)) return QLORA_ERR_INVALID_ARG;
   if (!W->codes || !W->scales || !aligned16(W->codes) || !aligned16(W->scales))
     return QLORA_ERR_INVALID_ARG;
   if (W->fmt == QLORA_FMT_NVFP4 &&
       (!W->tensor_scale || (reinterpret_cast<uintptr_t>(W->tensor_scale) & 3u)))
+    return QLORA_ERR_INVALID_ARG;
+  if (W->fmt == QLORA_FMT_NF4_DQ &&
+      (!W->scales2 || (reinterpret_cast<uintptr_t>(W->scales2) & 3u)))
     return QLORA_ERR_INVALID_ARG;
   return QLORA_OK;
 }
@@ -229,7 +232,9 @@ StreamPlan stream_plan(int64_t N, int64_t K, int64_t M, bool dx, int sms) {
 // The streaming path is taken when the batch is short and the workspace's partial region (all
 // of the workspace from its start) holds its fp32 partials; otherwise the tiled kernels run.
 bool stream_fits(const qlora_weight_t* W, int64_t M, int E, bool dx, size_t region) {
-  return use_stream(M, E) && stream_plan(W->N, W->K, M, dx, num_sms()).partial_bytes <= region;
+  // NF4 with a double-quantised absmax runs the tiled kernels at every batch size
+  return W->fmt != QLORA_FMT_NF4_DQ && use_stream(M, E) &&
+         stream_plan(W->N, W->K, M, dx, num_sms()).partial_bytes <= region;
 }
 
 struct WsLayout {
@@ -398,6 +403,7 @@ qlora_status_t launch_fused(const qlora_weight_t* W, bool dx, const void* act, c
                uint64_t(r) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
   p.scales = W->scales;
+  p.scales2 = W->fmt == QLORA_FMT_NF4_DQ ? W->scales2 : nullptr;
   p.tensor_scale = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
   p.lora_up = static_cast<const __nv_bfloat16*>(lora_up);
   p.out = static_cast<__nv_bfloat16*>(out);
@@ -431,7 +437,9 @@ qlora_status_t launch_fused(const qlora_weight_t* W, bool dx, const void* act, c
     case 2: return launch_fused_t<kFmtMXFP4, false>(p, grid, grouped, st);
     case 3: return launch_fused_t<kFmtMXFP4, true>(p, grid, grouped, st);
     case 4: return launch_fused_t<kFmtNVFP4, false>(p, grid, grouped, st);
-    default: return launch_fused_t<kFmtNVFP4, true>(p, grid, grouped, st);
+    case 5: return launch_fused_t<kFmtNVFP4, true>(p, grid, grouped, st);
+    case 6: return launch_fused_t<kFmtNF4DQ, false>(p, grid, grouped, st);
+    default: return launch_fused_t<kFmtNF4DQ, true>(p, grid, grouped, st);
   }
 }
 
@@ -850,6 +858,7 @@ qlora_status_t qlora_debug_dequant(const qlora_weight_t* W, int transposed, void
                dx ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B))
     return QLORA_ERR_CUDA;
   p.scales = W->scales;
+  p.scales2 = W->fmt == QLORA_FMT_NF4_DQ ? W->scales2 : nullptr;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.status = nullptr;
   p.N = int(N);
@@ -863,15 +872,18 @@ qlora_status_t qlora_debug_dequant(const qlora_weight_t* W, int transposed, void
     case 2: qlora_debug_dequant_kernel<kFmtMXFP4, false><<<grid, 128, 0, s>>>(p); break;
     case 3: qlora_debug_dequant_kernel<kFmtMXFP4, true><<<grid, 128, 0, s>>>(p); break;
     case 4: qlora_debug_dequant_kernel<kFmtNVFP4, false><<<grid, 128, 0, s>>>(p); break;
-    default: qlora_debug_dequant_kernel<kFmtNVFP4, true><<<grid, 128, 0, s>>>(p); break;
+    case 5: qlora_debug_dequant_kernel<kFmtNVFP4, true><<<grid, 128, 0, s>>>(p); break;
+    case 6: qlora_debug_dequant_kernel<kFmtNF4DQ, false><<<grid, 128, 0, s>>>(p); break;
+    default: qlora_debug_dequant_kernel<kFmtNF4DQ, true><<<grid, 128, 0, s>>>(p); break;
   }
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 qlora_status_t qlora_debug_decode_rate(int fmt, int iters, double* weights_per_clock_per_sm) {
   if (!weights_per_clock_per_sm || iters < 1 || iters > (1 << 20) || fmt < QLORA_FMT_NF4 ||
-      fmt > QLORA_FMT_NVFP4)
+      fmt > QLORA_FMT_NF4_DQ)
     return QLORA_ERR_INVALID_ARG;
+  if (fmt == QLORA_FMT_NF4_DQ) fmt = QLORA_FMT_NF4;   // the same item decode once the absmax is formed
   const int sms = num_sms();
   unsigned long long* cyc = nullptr;
   uint32_t* sink = nullptr;

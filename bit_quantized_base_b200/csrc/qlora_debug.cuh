@@ -9,6 +9,7 @@ namespace qlora {
 struct DebugDequantParams {
   CUtensorMap tm_codes;  // same tensor map shape as the fused kernel's
   const void* scales;
+  const float* scales2;  // NF4DQ second-level scales, else unused
   __nv_bfloat16* out;    // [N, K]
   int* status;
   int N, K;
@@ -44,7 +45,10 @@ qlora_debug_dequant_kernel(const __grid_constant__ DebugDequantParams p) {
   const int kcol = DX ? c0 + geo.chunk * 64 : ks * fused::BK;
   const bool valid = n < p.N && kcol < p.K;
   ItemScale sc{0u};
-  if (valid) sc = load_item_scale<FMT>(p.scales, n, kcol, p.K);
+  if (valid) {
+    if constexpr (FMT == kFmtNF4DQ) sc = load_item_scale_dq(p.scales, p.scales2, 0, p.N, n, kcol, p.K);
+    else sc = load_item_scale<FMT>(p.scales, n, kcol, p.K);
+  }
   if (!ptx::mbar_wait(b, 0, p.status, &abort_flag)) return;
   const uint32_t cb = ptx::smem_u32(ctile);
   const uint4 lo = ptx::ld_shared_v4(cb + geo.code_off(0));

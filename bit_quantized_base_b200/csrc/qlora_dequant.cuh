@@ -110,31 +110,41 @@ __device__ __forceinline__ uint32_t e8m0_bf16(uint32_t e) {
   return e << 7;
 }
 
-// E4M3 ("FN": bias 7, no inf, S.1111.111 NaN) -> binary32 (exact), then its bf16 bit pattern
-// (exact: at most 4 significant bits).
-__device__ __forceinline__ uint32_t e4m3_bf16(uint32_t b) {
+// E4M3 ("FN": bias 7, no inf, S.1111.111 NaN) -> binary32 (exact).
+__device__ __forceinline__ float e4m3_f32(uint32_t b) {
   b &= 0xFFu;
   const uint32_t s = b >> 7, e = (b >> 3) & 15u, m = b & 7u;
-  if (e == 15u && m == 7u) return 0x7FC0u;
+  if (e == 15u && m == 7u) return __uint_as_float(0x7FC00000u);
   float mag;
   if (e == 0u) mag = __fmul_rn(static_cast<float>(m), 0.001953125f);   // m/8 * 2^-6
   else mag = __uint_as_float(((e + 120u) << 23) | (m << 20));
-  return (__float_as_uint(mag) >> 16) | (s << 15);
+  return __uint_as_float(__float_as_uint(mag) | (s << 31));
 }
+// ... and its bf16 bit pattern (exact: at most 4 significant bits).
+__device__ __forceinline__ uint32_t e4m3_bf16(uint32_t b) { return __float_as_uint(e4m3_f32(b)) >> 16; }
 
-enum : int { kFmtNF4 = 0, kFmtMXFP4 = 1, kFmtNVFP4 = 2 };
+// kFmtNF4DQ: NF4 whose 64-block absmax is an E4M3 code times an fp32 second-level scale (one per
+// 256 consecutive codes); once the absmax is formed the decode is NF4's.
+enum : int { kFmtNF4 = 0, kFmtMXFP4 = 1, kFmtNVFP4 = 2, kFmtNF4DQ = 3 };
 
 // Per-item scale material, loaded from global memory one step ahead of use.
 struct ItemScale {
-  uint32_t raw;   // NF4: fp32 bits of the absmax; MXFP4: 2 E8M0 bytes; NVFP4: 4 E4M3 bytes
+  uint32_t raw;   // NF4 / NF4DQ: fp32 bits of the absmax; MXFP4: 2 E8M0 bytes; NVFP4: 4 E4M3 bytes
 };
+
+// The absmax of an NF4DQ block: fp32( e4m3(c1) * s2 ), binary32 round-to-nearest-even.
+__device__ __forceinline__ ItemScale nf4dq_item_scale(uint32_t c1, float s2) {
+  ItemScale s;
+  s.raw = __float_as_uint(__fmul_rn(e4m3_f32(c1), s2));
+  return s;
+}
 
 // Decode one item (64 elements: code words cw[0..7], 8 elements each) and store it as eight
 // 16-byte chunks: chunk j goes to shared address row_base + ((j ^ swz) << 4).
 template <int FMT>
 __device__ __forceinline__ void dequant_item_store(const uint32_t (&cw)[8], ItemScale sc,
                                                    uint32_t row_base, uint32_t swz) {
-  if constexpr (FMT == kFmtNF4) {
+  if constexpr (FMT == kFmtNF4 || FMT == kFmtNF4DQ) {
     const Lut16 t = nf4_lut(__uint_as_float(sc.raw));
 #pragma unroll
     for (int j = 0; j < 8; ++j) {

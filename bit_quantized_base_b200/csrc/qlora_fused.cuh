@@ -79,6 +79,7 @@ struct FusedParams {
   CUtensorMap tm_codes;  // codes [E*N, K/2] u8: fwd box {32, 128} SW32; dX box {64, 64} SW64
   CUtensorMap tm_zs;     // Zs [M, r] bf16, box {64, 128}, SW128 (zero fill beyond r)
   const void* scales;                // [E, N, K/bs]
+  const float* scales2;              // NF4DQ: second-level scales [E, ceil(N * K/64 / 256)]
   const float* tensor_scale;         // NVFP4: [E] device floats, else nullptr
   const __nv_bfloat16* lora_up;      // fwd: B [E, N, r]; dX: A [E, r, K]
   __nv_bfloat16* out;                // fwd: Y [M, N]; dX: dX [M, K]
@@ -115,6 +116,18 @@ __device__ __forceinline__ ItemScale load_item_scale(const void* scales, int n, 
     s.raw = __ldg(reinterpret_cast<const uint32_t*>(scales) + (row * (K / 16) + kcol / 16) / 4);
   }
   return s;
+}
+
+// NF4DQ: the absmax of the block of element (n, kcol) of expert e's weight, from its first-level
+// E4M3 code and the second-level scale of its group of 256 consecutive first-level codes in the
+// expert's row-major [N, K/64] array.
+__device__ __forceinline__ ItemScale load_item_scale_dq(const void* scales, const float* scales2,
+                                                        int e, int N, int n, int kcol, int K) {
+  const size_t nb = size_t(K) / 64;
+  const size_t f = size_t(n) * nb + size_t(kcol) / 64;
+  const size_t groups = (size_t(N) * nb + 255) / 256;
+  const uint32_t c1 = __ldg(static_cast<const uint8_t*>(scales) + size_t(e) * size_t(N) * nb + f);
+  return nf4dq_item_scale(c1, __ldg(scales2 + size_t(e) * groups + f / 256));
 }
 
 // The 4-byte word of the scale array that holds the block-scale material of the item starting at
@@ -482,8 +495,10 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
       if (c.t < num_tiles && c.ks < nk) {
         const int n = DX ? c.ks * BK + geo.row : c.h0 + geo.row;
         const int kcol = DX ? c.h0 + geo.chunk * 64 : c.ks * BK;
-        if (n < p.N && kcol < p.K)
-          sc = load_item_scale<FMT>(p.scales, n, kcol, p.K, size_t(c.e) * p.N);
+        if (n < p.N && kcol < p.K) {
+          if constexpr (FMT == kFmtNF4DQ) sc = load_item_scale_dq(p.scales, p.scales2, c.e, p.N, n, kcol, p.K);
+          else sc = load_item_scale<FMT>(p.scales, n, kcol, p.K, size_t(c.e) * p.N);
+        }
       }
       return sc;
     };

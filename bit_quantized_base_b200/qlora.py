@@ -15,7 +15,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqlora.so")
 
-FMT = {"nf4": 0, "mxfp4": 1, "nvfp4": 2}
+FMT = {"nf4": 0, "mxfp4": 1, "nvfp4": 2, "nf4dq": 3}
 BLOCK = {"nf4": 64, "mxfp4": 32, "nvfp4": 16}
 OP_FWD, OP_BWD, OP_GROUPED_FWD, OP_GROUPED_BWD = 0, 1, 2, 3
 
@@ -42,7 +42,7 @@ class qlora_weight_t(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("N", ctypes.c_int64), ("K", ctypes.c_int64),
                 ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
-                ("tensor_scale", ctypes.c_void_p)]
+                ("tensor_scale", ctypes.c_void_p), ("scales2", ctypes.c_void_p)]
 
 
 def _load():
@@ -112,14 +112,15 @@ def _stream(stream):
 
 
 class Weight:
-    """A frozen 4-bit weight resident on the GPU (codes [.., N, K/2] uint8, scales, and for NVFP4
-    the tensor scale as a float32 device tensor)."""
+    """A frozen 4-bit weight resident on the GPU (codes [.., N, K/2] uint8, scales, for NVFP4 the
+    tensor scale and for NF4-DQ the second-level scales, as float32 device tensors)."""
 
-    def __init__(self, fmt, N, K, codes, scales, tensor_scale=None):
+    def __init__(self, fmt, N, K, codes, scales, tensor_scale=None, scales2=None):
         self.fmt, self.N, self.K = fmt, int(N), int(K)
         self.codes, self.scales, self.tensor_scale = codes, scales, tensor_scale
+        self.scales2 = scales2
         self.c = qlora_weight_t(FMT[fmt], 0, self.N, self.K, _p(codes), _p(scales),
-                                _p(tensor_scale))
+                                _p(tensor_scale), _p(scales2))
 
     @property
     def ref(self):
@@ -129,6 +130,8 @@ class Weight:
         n = self.codes.numel() * self.codes.element_size() + self.scales.numel() * self.scales.element_size()
         if self.tensor_scale is not None:
             n += self.tensor_scale.numel() * 4
+        if self.scales2 is not None:
+            n += self.scales2.numel() * 4
         return n
 
 
@@ -239,14 +242,16 @@ def bf16_from_bits(a, device="cuda"):
     return torch.from_numpy(a.view("int16")).view(torch.bfloat16).to(device)
 
 
-def weight_from_numpy(fmt, codes, scales, tensor_scale=None, device="cuda"):
+def weight_from_numpy(fmt, codes, scales, tensor_scale=None, device="cuda", scales2=None):
     """Upload a stored weight (numpy arrays as made by synth) to the GPU."""
+    import numpy as np
     N = codes.shape[-2]
     K = codes.shape[-1] * 2
     c = torch.from_numpy(codes).to(device)
     s = torch.from_numpy(scales).to(device)
-    ts = None
+    ts = s2 = None
     if fmt == "nvfp4":
-        import numpy as np
         ts = torch.from_numpy(np.atleast_1d(np.asarray(tensor_scale, np.float32))).to(device)
-    return Weight(fmt, N, K, c, s, ts)
+    if fmt == "nf4dq":
+        s2 = torch.from_numpy(np.ascontiguousarray(scales2, np.float32)).to(device)
+    return Weight(fmt, N, K, c, s, ts, s2)

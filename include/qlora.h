@@ -63,7 +63,11 @@ typedef enum {
   QLORA_FMT_MXFP4 = 1,
   /* NVFP4: E2M1 elements times one E4M3 scale per 16 along K, times one fp32 tensor scale
    * (same page and section: "a per-block FP8 scale over 16-element micro-blocks"). */
-  QLORA_FMT_NVFP4 = 2
+  QLORA_FMT_NVFP4 = 2,
+  /* NF4 with double quantisation: as NF4, the absmax of each 64-block stored as an 8-bit E4M3
+   * code times an fp32 second-level scale shared by 256 consecutive first-level codes
+   * ("Training LLMs on a Budget", §3 "The three QLoRA tricks", item 2).  4.127 bits/weight. */
+  QLORA_FMT_NF4_DQ = 3
 } qlora_format_t;
 
 typedef enum {
@@ -77,12 +81,17 @@ typedef enum {
 
 /* One frozen 4-bit weight W [N,K] (row n = output feature, K contiguous).
  *   codes  [N, K/2] uint8: element 2j of a row in the low nibble of byte j, 2j+1 in the high.
- *   scales NF4: float [N, K/64]; MXFP4: uint8 E8M0 [N, K/32]; NVFP4: uint8 E4M3 [N, K/16].
+ *   scales NF4: float [N, K/64]; MXFP4: uint8 E8M0 [N, K/32]; NVFP4: uint8 E4M3 [N, K/16];
+ *          NF4_DQ: uint8 E4M3 first-level codes [N, K/64].
  *          Block b of row n covers k in [b*bs, (b+1)*bs).
  *   tensor_scale NVFP4: device float* holding the decode multiplier (grouped: [E] values);
- *          NULL for NF4 and MXFP4.  It must be finite and non-zero.
- * Decode of element (n,k) with code c: NF4 bf16(fp32(level[c] * absmax)); MXFP4
- * bf16(e2m1(c) * 2^(e-127)); NVFP4 bf16(fp32(fp32(e2m1(c) * e4m3(s)) * tensor_scale)), every
+ *          NULL for the other formats.  It must be finite and non-zero.
+ *   scales2 NF4_DQ: device float [G] second-level scales, G = ceil(N * (K/64) / 256); scale g
+ *          serves first-level codes [256 g, 256 g + 256) of the row-major [N, K/64] array
+ *          (grouped: [E, G], per expert).  NULL for the other formats.
+ * Decode of element (n,k) with code c: NF4 bf16(fp32(level[c] * absmax)); NF4_DQ the same with
+ * absmax = fp32(e4m3(c1) * scales2[g]); MXFP4 bf16(e2m1(c) * 2^(e-127)); NVFP4
+ * bf16(fp32(fp32(e2m1(c) * e4m3(s)) * tensor_scale)), every
  * multiply binary32 round-to-nearest-even without flush-to-zero.  The kernels apply the NVFP4
  * tensor scale to the fp32 accumulator rather than to each element (it is uniform over W); the
  * per-element micro-block decode is exact.
@@ -94,6 +103,7 @@ typedef struct {
   const uint8_t* codes;
   const void* scales;
   const float* tensor_scale;
+  const float* scales2;
 } qlora_weight_t;
 
 typedef enum {

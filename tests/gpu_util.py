@@ -42,7 +42,8 @@ class GpuLayer:
         from bit_quantized_base_b200 import qlora as Q
         self.Q = Q
         self.p = p
-        self.W = Q.weight_from_numpy(p["fmt"], p["codes"], p["scales"], p["tensor_scale"], device)
+        self.W = Q.weight_from_numpy(p["fmt"], p["codes"], p["scales"], p["tensor_scale"], device,
+                                     scales2=p.get("scales2"))
         self.X = Q.bf16_from_bits(p["X"], device)
         self.A = Q.bf16_from_bits(p["A"], device)
         self.B = Q.bf16_from_bits(p["B"], device)

@@ -65,6 +65,70 @@ def test_debug_dequant_bit_exact(fmt, transposed):
     assert not mism.any(), f"{mism.sum()} decoded elements differ, first at {np.argwhere(mism)[0]}"
 
 
+def _nf4dq_edge_weight(N, K, seed):
+    """Random codes, every first-level E4M3 code (NaN and subnormals included) and second-level
+    scales that make the absmax product overflow, underflow, vanish or go subnormal."""
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    c1 = rng.integers(0, 256, size=(N, K // 64), dtype=np.uint8)
+    c1.reshape(-1)[:256] = np.arange(256, dtype=np.uint8)
+    pool = np.array([1.0, 2.0 ** -20, 3.3e38, 0.0, 1.5, 7.1e-3, 1e-40, 4.2e35], np.float32)
+    s2 = pool[rng.integers(0, len(pool), size=O.dq_groups(N, K))]
+    return codes, c1, s2
+
+
+@pytest.mark.parametrize("transposed", [0, 1])
+def test_debug_dequant_nf4dq_bit_exact(transposed):
+    from bit_quantized_base_b200 import qlora as Q
+    N, K = 272, 448
+    codes, c1, s2 = _nf4dq_edge_weight(N, K, seed=27 + transposed)
+    W = Q.weight_from_numpy("nf4dq", codes, c1, None, scales2=s2)
+    out = torch.zeros((N, K), dtype=torch.bfloat16, device="cuda")
+    Q.qlora_debug_dequant(W, transposed, out)
+    torch.cuda.synchronize()
+    got = bits(out)
+    ref = O.dequant("nf4dq", N, K, codes, c1, scales2=s2)
+    gnan = (got & 0x7FFF) > 0x7F80
+    rnan = (ref & 0x7FFF) > 0x7F80
+    assert np.array_equal(gnan, rnan), "NaN positions differ"
+    mism = (got != ref) & ~rnan
+    assert not mism.any(), f"{mism.sum()} decoded elements differ, first at {np.argwhere(mism)[0]}"
+
+
+@pytest.mark.parametrize("dx", [False, True])
+def test_fused_nf4dq_identity_is_bit_exact(dx):
+    # X = I (forward) or dY = I (dX) with a zero LoRA term: every output is one decoded weight
+    N, K = 208, 384
+    rng = np.random.default_rng(8 + dx)
+    codes = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    c1 = rng.integers(0x18, 0x70, size=(N, K // 64), dtype=np.uint8)
+    s2 = rng.uniform(1e-4, 1e-2, size=O.dq_groups(N, K)).astype(np.float32)
+    r = 8
+    if not dx:
+        M = K
+        p = dict(fmt="nf4dq", M=M, N=N, K=K, r=r, s=2.0, codes=codes, scales=c1, tensor_scale=1.0,
+                 scales2=s2, X=synth.to_bf16_bits(np.eye(K, dtype=np.float32)),
+                 A=synth.to_bf16_bits(rng.standard_normal((r, K)).astype(np.float32)),
+                 B=np.zeros((N, r), np.uint16), dY=np.zeros((M, N), np.uint16))
+    else:
+        M = N
+        p = dict(fmt="nf4dq", M=M, N=N, K=K, r=r, s=2.0, codes=codes, scales=c1, tensor_scale=1.0,
+                 scales2=s2, X=np.zeros((M, K), np.uint16), A=np.zeros((r, K), np.uint16),
+                 B=synth.to_bf16_bits(rng.standard_normal((N, r)).astype(np.float32)),
+                 dY=synth.to_bf16_bits(np.eye(N, dtype=np.float32)))
+    g = GpuLayer(p)
+    if not dx:
+        out, _ = g.fwd()
+    else:
+        out, _, _ = g.bwd()
+    torch.cuda.synchronize()
+    assert g.status() == 0
+    ref = _fold_signed_zero(O.dequant("nf4dq", N, K, codes, c1, scales2=s2))
+    if not dx:
+        ref = ref.T
+    assert np.array_equal(bits(out), ref), f"{(bits(out) != ref).sum()} elements differ"
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 def test_fused_forward_identity_is_bit_exact(fmt):
     from bit_quantized_base_b200 import qlora as Q
@@ -123,6 +187,11 @@ CASES = [
     # 76 pair tiles on 74 pairs: the last wave's tiles run split in two 256-row tiles (fwd, dX)
     ("nf4", 1000, 9728, 128, 8),
     ("mxfp4", 1024, 128, 9728, 16),
+    # NF4 with double-quantised absmax (tiled kernels at every batch size); K/64 = 5 or 19
+    # blocks per row, so second-level groups of 256 straddle rows
+    ("nf4dq", 5, 272, 320, 8),
+    ("nf4dq", 300, 400, 1216, 64),
+    ("nf4dq", 700, 1040, 576, 16),
 ]
 
 
@@ -135,7 +204,7 @@ def test_layer_parity(fmt, M, N, K, r):
     torch.cuda.synchronize()
     assert g.status() == 0
     ref = O.layer(fmt, M, N, K, r, p["s"], p["codes"], p["scales"], p["tensor_scale"], p["X"],
-                  p["A"], p["B"], p["dY"])
+                  p["A"], p["B"], p["dY"], scales2=p.get("scales2"))
     assert_close(to_f64(T), ref["T"], "T")
     assert_close(to_f64(Y), ref["Y"], "Y")
     assert_close(to_f64(dX), ref["dX"], "dX")
