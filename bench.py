@@ -320,6 +320,50 @@ def short_batch_sweep(Q, torch, p, Ws, X, dY, A, B, peaks):
     return out
 
 
+def nf4dq_step(Q, torch, p, Xs, dYs, A, B, ncopy, steps=60):
+    """fwd+bwd of the same layer with its weight stored as NF4 with a double-quantised absmax
+    (8-bit E4M3 first level, fp32 second level per 256): TFLOP/s.  Timing inputs: the workload's
+    NF4 codes with seeded random first-level codes and second-level scales (values do not change
+    the timing), rotating device copies as in the main loop."""
+    import numpy as np
+    N, K, M, r, s = p["N"], p["K"], p["M"], p["r"], p["s"]
+    rng = np.random.default_rng(77)
+    Ws = []
+    for _ in range(ncopy):
+        c1 = rng.integers(0x18, 0x70, size=(N, K // 64), dtype=np.uint8)
+        s2 = rng.uniform(1e-4, 1e-3, size=(N * (K // 64) + 255) // 256).astype(np.float32)
+        Ws.append(Q.weight_from_numpy("nf4dq", p["codes"], c1, None, scales2=s2))
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    T = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty((r, K), dtype=torch.bfloat16, device="cuda")
+    dB = torch.empty((N, r), dtype=torch.bfloat16, device="cuda")
+    ws = Q.alloc_workspace(Q.OP_BWD, Ws[0], M, r)
+    Q.qlora_workspace_init(ws)
+
+    def step(i):
+        c = i % ncopy
+        Q.qlora_linear_fwd(Ws[c], Xs[c], A, B, Y, T, M, r, s, ws)
+        Q.qlora_linear_bwd(Ws[c], Xs[c], A, B, T, dYs[c], dX, dA, dB, M, r, s, ws)
+
+    for i in range(5):
+        step(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(i)
+    e1.record()
+    e1.synchronize()
+    if Q.qlora_get_device_status(ws) != 0:
+        raise RuntimeError("device status in the NF4-DQ leg")
+    t = e0.elapsed_time(e1) / steps * 1e-3
+    bits = (Ws[0].nbytes()) * 8 / (N * K)
+    return {"ms_per_step": round(t * 1e3, 4), "tflops": round(flops(M, N, K, r) / t / 1e12, 1),
+            "bits_per_weight": round(bits, 4), "data": "workload NF4 codes, random stored scales"}
+
+
 def grouped_moe(Q, torch, synth, peaks):
     """One fwd+bwd of each MoE expert projection (64 experts, MXFP4, Zipf top-8 routing of 16384
     tokens): TFLOP/s.  Timing inputs: seeded random stored codes with a realistic E8M0 scale range
@@ -543,6 +587,11 @@ def run_own(args):
                                                            peaks)
         del p3
 
+    # ---- the same layer with NF4 double quantisation of the absmax
+    dq = None
+    if not args.no_sweep:
+        dq = nf4dq_step(Q, torch, p, Xs, dYs, A, B, ncopy)
+
     # ---- grouped (MoE) experts: 64 experts, 16384 tokens x top-8, one fwd+bwd per projection
     grouped = None
     if not args.no_sweep:
@@ -571,6 +620,7 @@ def run_own(args):
                                    "CUDA events around every launch (launches serialised)",
         "e2e": e2e,
         "weight_stream_small_m": sweep,
+        "nf4_double_quant": dq,
         "grouped_moe": grouped,
         "cpu_baseline": cpu,
     }

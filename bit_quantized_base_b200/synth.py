@@ -404,9 +404,17 @@ def small_grouped(fmt: str, counts, N: int, K: int, r: int, s: float = 2.0, seed
     M = int(offsets[-1])
     codes = np.empty((E, N, K // 2), np.uint8)
     scales = None
+    scales2 = None
     ts = np.ones(E, np.float32)
     for e in range(E):
-        c, sc, t = encode(fmt, _normal(rng, (N, K), 0.02 * (1 + e % 3)))
+        if fmt == "nf4dq":
+            c, sc, s2 = encode_nf4dq(_normal(rng, (N, K), 0.02 * (1 + e % 3)))
+            if scales2 is None:
+                scales2 = np.empty((E,) + s2.shape, np.float32)
+            scales2[e] = s2
+            t = None
+        else:
+            c, sc, t = encode(fmt, _normal(rng, (N, K), 0.02 * (1 + e % 3)))
         if scales is None:
             scales = np.empty((E,) + sc.shape, sc.dtype)
         codes[e], scales[e] = c, sc
@@ -418,4 +426,5 @@ def small_grouped(fmt: str, counts, N: int, K: int, r: int, s: float = 2.0, seed
     X = to_bf16_bits(_normal(rng, (M, K), 1.0))
     dY = to_bf16_bits(_normal(rng, (M, N), 1.0))
     return dict(fmt=fmt, E=E, offsets=offsets, M=M, N=N, K=K, r=r, s=s, codes=codes,
-                scales=scales, tensor_scale=ts if fmt == "nvfp4" else None, X=X, A=A, B=B, dY=dY)
+                scales=scales, tensor_scale=ts if fmt == "nvfp4" else None, scales2=scales2,
+                X=X, A=A, B=B, dY=dY)

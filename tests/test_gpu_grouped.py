@@ -16,7 +16,8 @@ class GpuGrouped:
     def __init__(self, p):
         from bit_quantized_base_b200 import qlora as Q
         self.Q, self.p = Q, p
-        self.W = Q.weight_from_numpy(p["fmt"], p["codes"], p["scales"], p["tensor_scale"])
+        self.W = Q.weight_from_numpy(p["fmt"], p["codes"], p["scales"], p["tensor_scale"],
+                                     scales2=p.get("scales2"))
         self.X = Q.bf16_from_bits(p["X"])
         self.A = Q.bf16_from_bits(p["A"])
         self.B = Q.bf16_from_bits(p["B"])
@@ -50,7 +51,8 @@ class GpuGrouped:
 def oracle_grouped(p):
     from oracle import oracle
     res = oracle.grouped_layer(p["fmt"], p["offsets"], p["N"], p["K"], p["r"], p["s"], p["codes"],
-                               p["scales"], p["tensor_scale"], p["X"], p["A"], p["B"], p["dY"])
+                               p["scales"], p["tensor_scale"], p["X"], p["A"], p["B"], p["dY"],
+                               scales2=p.get("scales2"))
     cat = lambda k, w: (np.concatenate([d[k] for d in res], 0) if p["M"] else np.zeros((0, w)))
     return dict(Y=cat("Y", p["N"]), T=cat("T", p["r"]), dX=cat("dX", p["K"]),
                 dA=np.stack([d["dA"] for d in res]), dB=np.stack([d["dB"] for d in res]))
@@ -61,6 +63,8 @@ GROUPED = [
     ("nf4", [200, 0, 513], 384, 192, 16),
     ("nvfp4", [64, 130, 0, 77], 256, 448, 64),
     ("mxfp4", [3, 5, 0, 2, 1, 7, 0, 0, 9, 4, 6, 8, 1, 1, 2, 40], 128, 256, 32),
+    # per-expert second-level scales: 336 x 5 = 1680 first-level codes per expert (7 groups)
+    ("nf4dq", [150, 0, 600, 33], 336, 320, 16),
 ]
 
 
