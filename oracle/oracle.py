@@ -55,6 +55,9 @@ def lib():
                                    c.c_void_p, c.c_void_p]
         L.oracle_layer.restype = c.c_int
         L.oracle_num_threads.restype = c.c_int
+        L.oracle_encode.argtypes = [c.c_int, c.c_int64, c.c_int64, c.c_void_p, c.c_void_p,
+                                    c.c_void_p, c.c_void_p, c.c_void_p]
+        L.oracle_encode.restype = c.c_int
         _lib = L
     return _lib
 
@@ -178,6 +181,23 @@ def grouped_layer(fmt, offsets, N, K, r, s, codes, scales, tensor_scales, X, A, 
                          None if dY is None else dY[m0:m1], rows=rows, want=want,
                          scales2=None if scales2 is None else scales2[e]))
     return res
+
+
+def encode(fmt, v):
+    """Encode a float weight v [N,K] (float32) per the build's encoder rules.  Returns (codes
+    [N,K/2] uint8, scales, tensor_scale (NVFP4, else None), scales2 (NF4-DQ, else None))."""
+    f = _fmt(fmt)
+    v = np.ascontiguousarray(v, np.float32)
+    N, K = v.shape
+    bs = BLOCK[f]
+    codes = np.zeros((N, K // 2), np.uint8)
+    scales = np.zeros((N, K // bs), np.float32 if f == 0 else np.uint8)
+    ts = np.zeros(1, np.float32)
+    s2 = np.zeros(dq_groups(N, K), np.float32) if f == 3 else None
+    rc = lib().oracle_encode(f, N, K, _ptr(v), _ptr(codes), _ptr(scales), _ptr(ts), _ptr(s2))
+    if rc != 0:
+        raise ValueError("oracle_encode rejected its arguments")
+    return codes, scales, (float(ts[0]) if f == 2 else None), s2
 
 
 def num_threads():

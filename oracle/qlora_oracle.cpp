@@ -229,9 +229,150 @@ bool valid_shape(int fmt, int64_t N, int64_t K) {
   return K % block_size(fmt) == 0;
 }
 
+// ---------------------------------------------------------------------------------------------
+// Encoders (float weight -> stored codes and scales).  The pages give no rounding rules, so the
+// encode is this build's reading, stated once here and in the header (include/qlora.h):
+//   NF4    : absmax = max |v| over the 64-block (binary32, exact); absmax == 0 -> every code 7
+//            (level 0); else code = the number of level midpoints m_i = (L_i + L_{i+1}) / 2 that
+//            are < x = v / absmax, x and m_i in binary64 (ties go to the lower code).
+//   NF4-DQ : the 64-block absmax a as above; per group of 256 consecutive blocks (row-major)
+//            s2 = fp32(gmax / 448) (gmax = the group's largest a; s2 = 1 if gmax == 0);
+//            c1 = E4M3 nearest to a / s2 (binary64 quotient; ties to the even code; saturating
+//            at 448); the element codes as NF4 against the decoded absmax fp32(e4m3(c1) * s2).
+//   MXFP4  : amax = max |v| over the 32-block; e = clamp(floor(log2 amax) - 2 + 127, 0, 254)
+//            (amax == 0 -> e = 0); code = E2M1 nearest to v / 2^(e-127) (binary64), ties to the
+//            even code (mantissa bit 0), magnitude saturating at 6, sign bit only on a non-zero
+//            magnitude.
+//   NVFP4  : tensor amax T; s_t = fp32(T / 2688) (1 if T == 0); per 16-block s_b = E4M3 nearest
+//            to amax_b / (6 s_t) (binary64, ties to even, saturating at 448); code = E2M1 nearest
+//            to v / (e4m3(s_b) * s_t) (binary64 divisor; a zero divisor gives code 0).
+// Inputs must be finite.
+// ---------------------------------------------------------------------------------------------
+
+// Nearest E2M1 code of x (binary64), ties to even, saturating, sign only on non-zero magnitude.
+uint32_t e2m1_encode(double x) {
+  static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  const double a = std::fabs(x) < 6.0 ? std::fabs(x) : 6.0;
+  uint32_t c = 0;
+  for (uint32_t i = 0; i < 7; ++i) {
+    const double mid = 0.5 * (mag[i] + mag[i + 1]);
+    if (a > mid || (a == mid && (i & 1u))) c = i + 1;   // past the midpoint, or a tie toward even
+  }
+  return (c != 0u && std::signbit(x)) ? (c | 8u) : c;
+}
+
+// Nearest positive E4M3 code of q >= 0 (binary64), ties to the even code, saturating at 448.
+uint32_t e4m3_encode_pos(double q) {
+  uint32_t best = 0;
+  for (uint32_t c = 1; c <= 0x7Eu; ++c) {
+    const double lo = e4m3_value(c - 1), hi = e4m3_value(c);
+    const double mid = 0.5 * (lo + hi);
+    if (q > mid || (q == mid && (c & 1u) == 0u)) best = c;
+  }
+  return best;
+}
+
+// NF4 code of v against absmax a (> 0).
+uint32_t nf4_encode(float v, float a) {
+  const double x = static_cast<double>(v) / static_cast<double>(a);
+  uint32_t c = 0;
+  for (uint32_t i = 0; i < 15; ++i) {
+    const double mid = 0.5 * (static_cast<double>(nf4_level(i)) + static_cast<double>(nf4_level(i + 1)));
+    if (mid < x) c = i + 1;
+  }
+  return c;
+}
+
+void put_code(uint8_t* codes, int64_t K, int64_t n, int64_t k, uint32_t c) {
+  uint8_t& b = codes[n * (K / 2) + k / 2];
+  b = (k & 1) ? static_cast<uint8_t>((b & 0x0Fu) | (c << 4)) : static_cast<uint8_t>((b & 0xF0u) | c);
+}
+
 }  // namespace
 
 extern "C" {
+
+// Encode a float weight v [N,K] (binary32, row-major) per the rules above.  Outputs: codes
+// [N,K/2]; scales (NF4 float [N,K/64], NF4-DQ uint8 E4M3 [N,K/64], MXFP4 uint8 [N,K/32], NVFP4
+// uint8 [N,K/16]); *tensor_scale (NVFP4, else untouched); scales2 (NF4-DQ [ceil(N*K/64/256)]).
+// Returns 0, or -1 on a bad argument.
+int oracle_encode(int fmt, int64_t N, int64_t K, const float* v, uint8_t* codes, void* scales,
+                  float* tensor_scale, float* scales2) {
+  if (!valid_shape(fmt, N, K) || (N * K > 0 && (!v || !codes || !scales))) return -1;
+  if (fmt == 2 && !tensor_scale) return -1;
+  if (fmt == kFmtNf4Dq && N * K > 0 && !scales2) return -1;
+  const int bs = block_size(fmt);
+  const int64_t nb = K / bs;
+  std::vector<float> amax(static_cast<size_t>(N * nb), 0.0f);
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t b = 0; b < nb; ++b) {
+      float a = 0.0f;
+      for (int i = 0; i < bs; ++i) a = std::fmax(a, std::fabs(v[n * K + b * bs + i]));
+      amax[static_cast<size_t>(n * nb + b)] = a;
+    }
+  if (fmt == 0 || fmt == kFmtNf4Dq) {
+    std::vector<float> dec(amax);   // the absmax the element codes are taken against
+    if (fmt == kFmtNf4Dq) {
+      const int64_t G = dq_groups(N, K);
+      for (int64_t g = 0; g < G; ++g) {
+        const int64_t f0 = g * kDqGroup, f1 = (f0 + kDqGroup < N * nb) ? f0 + kDqGroup : N * nb;
+        float gmax = 0.0f;
+        for (int64_t f = f0; f < f1; ++f) gmax = std::fmax(gmax, amax[static_cast<size_t>(f)]);
+        const float s2 = gmax > 0.0f ? gmax / 448.0f : 1.0f;
+        scales2[g] = s2;
+        for (int64_t f = f0; f < f1; ++f) {
+          const uint32_t c1 = e4m3_encode_pos(static_cast<double>(amax[static_cast<size_t>(f)]) /
+                                              static_cast<double>(s2));
+          static_cast<uint8_t*>(scales)[f] = static_cast<uint8_t>(c1);
+          dec[static_cast<size_t>(f)] = e4m3_value(c1) * s2;
+        }
+      }
+    } else {
+      for (int64_t f = 0; f < N * nb; ++f) static_cast<float*>(scales)[f] = amax[static_cast<size_t>(f)];
+    }
+    for (int64_t n = 0; n < N; ++n)
+      for (int64_t k = 0; k < K; ++k) {
+        const float a = dec[static_cast<size_t>(n * nb + k / 64)];
+        put_code(codes, K, n, k, a > 0.0f ? nf4_encode(v[n * K + k], a) : 7u);
+      }
+    return 0;
+  }
+  if (fmt == 1) {
+    for (int64_t f = 0; f < N * nb; ++f) {
+      const float a = amax[static_cast<size_t>(f)];
+      uint32_t e = 0;
+      if (a > 0.0f) {
+        int p = 0;
+        std::frexp(a, &p);                       // a = m 2^p, m in [0.5, 1): floor(log2 a) = p - 1
+        const int ee = (p - 1) - 2 + 127;
+        e = static_cast<uint32_t>(ee < 0 ? 0 : (ee > 254 ? 254 : ee));
+      }
+      static_cast<uint8_t*>(scales)[f] = static_cast<uint8_t>(e);
+    }
+    for (int64_t n = 0; n < N; ++n)
+      for (int64_t k = 0; k < K; ++k) {
+        const uint32_t e = static_cast<const uint8_t*>(scales)[n * nb + k / 32];
+        const double sc = std::ldexp(1.0, static_cast<int>(e) - 127);
+        put_code(codes, K, n, k, e2m1_encode(static_cast<double>(v[n * K + k]) / sc));
+      }
+    return 0;
+  }
+  // NVFP4
+  float T = 0.0f;
+  for (int64_t i = 0; i < N * K; ++i) T = std::fmax(T, std::fabs(v[i]));
+  const float st = T > 0.0f ? static_cast<float>(static_cast<double>(T) / 2688.0) : 1.0f;
+  *tensor_scale = st;
+  for (int64_t f = 0; f < N * nb; ++f)
+    static_cast<uint8_t*>(scales)[f] = static_cast<uint8_t>(
+        e4m3_encode_pos(static_cast<double>(amax[static_cast<size_t>(f)]) / (6.0 * static_cast<double>(st))));
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) {
+      const double d = static_cast<double>(e4m3_value(static_cast<const uint8_t*>(scales)[n * nb + k / 16])) *
+                       static_cast<double>(st);
+      put_code(codes, K, n, k, d > 0.0 ? e2m1_encode(static_cast<double>(v[n * K + k]) / d) : 0u);
+    }
+  return 0;
+}
 
 // ---- scalar access for the spec tests ------------------------------------------------------
 void oracle_nf4_levels_spec(float* out16) {
