@@ -14,6 +14,7 @@
 #include "qlora_fused.cuh"
 #include "qlora_lora.cuh"
 #include "qlora_stream.cuh"
+#include "qlora_quant.cuh"
 
 namespace qlora {
 namespace {
@@ -877,6 +878,76 @@ qlora_status_t qlora_debug_dequant(const qlora_weight_t* W, int transposed, void
     default: qlora_debug_dequant_kernel<kFmtNF4DQ, true><<<grid, 128, 0, s>>>(p); break;
   }
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status_t qlora_quantize(const qlora_weight_t* W, const void* v, int v_is_bf16,
+                              qlora_stream_t stream) {
+  const qlora_status_t st = check_weight(W);
+  if (st != QLORA_OK) return st;
+  if (!v || (reinterpret_cast<uintptr_t>(v) & 3u)) return QLORA_ERR_INVALID_ARG;
+  if (W->fmt == QLORA_FMT_NF4_DQ && W->N * (W->K / 64) > (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  QuantParams p{};
+  p.v = v;
+  p.v_bf16 = v_is_bf16 ? 1 : 0;
+  p.codes = const_cast<uint8_t*>(W->codes);
+  p.scales = const_cast<void*>(W->scales);
+  p.scales2 = const_cast<float*>(W->scales2);
+  p.tensor_scale = const_cast<float*>(W->tensor_scale);
+  p.N = int(W->N);
+  p.K = int(W->K);
+  const int bs = quant::block_size(W->fmt == QLORA_FMT_NF4 ? kFmtNF4
+                                   : W->fmt == QLORA_FMT_MXFP4 ? kFmtMXFP4
+                                   : W->fmt == QLORA_FMT_NVFP4 ? kFmtNVFP4 : kFmtNF4DQ);
+  const int64_t blocks = W->N * (W->K / bs);
+  const unsigned grid = unsigned((blocks + quant::kBlocksPerCta - 1) / quant::kBlocksPerCta);
+  if (W->fmt == QLORA_FMT_NVFP4) {
+    if (cudaMemsetAsync(p.tensor_scale, 0, sizeof(float), s) != cudaSuccess) return QLORA_ERR_CUDA;
+    qlora_quant_amax_kernel<<<unsigned(2 * num_sms()), 256, 0, s>>>(
+        p, reinterpret_cast<unsigned*>(p.tensor_scale));
+  }
+  switch (W->fmt) {
+    case QLORA_FMT_NF4: qlora_quant_encode_kernel<kFmtNF4><<<grid, quant::kBlocksPerCta, 0, s>>>(p); break;
+    case QLORA_FMT_MXFP4: qlora_quant_encode_kernel<kFmtMXFP4><<<grid, quant::kBlocksPerCta, 0, s>>>(p); break;
+    case QLORA_FMT_NVFP4: qlora_quant_encode_kernel<kFmtNVFP4><<<grid, quant::kBlocksPerCta, 0, s>>>(p); break;
+    default: qlora_quant_encode_kernel<kFmtNF4DQ><<<grid, quant::kBlocksPerCta, 0, s>>>(p); break;
+  }
+  if (W->fmt == QLORA_FMT_NVFP4) qlora_quant_tensor_scale_kernel<<<1, 1, 0, s>>>(p.tensor_scale);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status_t qlora_merge_requantize(const qlora_weight_t* W, const void* A, const void* B, int r,
+                                      float scale, const qlora_weight_t* W_out, float* merged,
+                                      qlora_stream_t stream) {
+  qlora_status_t st = check_weight(W);
+  if (st != QLORA_OK) return st;
+  st = check_weight(W_out);
+  if (st != QLORA_OK) return st;
+  if (W_out->N != W->N || W_out->K != W->K || r < 1 || r > 1024 || !ptr_ok(A) || !ptr_ok(B) ||
+      !ptr_ok(merged))
+    return QLORA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MergeParams p{};
+  p.codes = W->codes;
+  p.scales = W->scales;
+  p.scales2 = W->scales2;
+  p.tensor_scale = W->tensor_scale;
+  p.A = static_cast<const __nv_bfloat16*>(A);
+  p.B = static_cast<const __nv_bfloat16*>(B);
+  p.out = merged;
+  p.N = int(W->N);
+  p.K = int(W->K);
+  p.r = r;
+  p.s = scale;
+  const unsigned grid = unsigned(4 * num_sms());
+  switch (W->fmt) {
+    case QLORA_FMT_NF4: qlora_merge_values_kernel<kFmtNF4><<<grid, 256, 0, s>>>(p); break;
+    case QLORA_FMT_MXFP4: qlora_merge_values_kernel<kFmtMXFP4><<<grid, 256, 0, s>>>(p); break;
+    case QLORA_FMT_NVFP4: qlora_merge_values_kernel<kFmtNVFP4><<<grid, 256, 0, s>>>(p); break;
+    default: qlora_merge_values_kernel<kFmtNF4DQ><<<grid, 256, 0, s>>>(p); break;
+  }
+  if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
+  return qlora_quantize(W_out, merged, 0, stream);
 }
 
 qlora_status_t qlora_debug_decode_rate(int fmt, int iters, double* weights_per_clock_per_sm) {

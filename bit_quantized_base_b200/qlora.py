@@ -28,7 +28,7 @@ EXPORTS = ("qlora_workspace_size", "qlora_workspace_init", "qlora_linear_fwd", "
            "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_status_string",
            "qlora_build_info", "qlora_launch_count", "qlora_profile_enable",
            "qlora_profile_reset", "qlora_profile_read", "qlora_linear_fwd_noalloc",
-           "qlora_debug_decode_rate")
+           "qlora_debug_decode_rate", "qlora_quantize", "qlora_merge_requantize")
 
 
 class QLoraError(RuntimeError):
@@ -67,6 +67,8 @@ def _load():
     L.qlora_debug_dequant.argtypes = [W, c.c_int, P, P]
     L.qlora_debug_wait_timeout.argtypes = [P, c.c_size_t, c.c_int, P]
     L.qlora_debug_decode_rate.argtypes = [c.c_int, c.c_int, c.POINTER(c.c_double)]
+    L.qlora_quantize.argtypes = [W, P, c.c_int, P]
+    L.qlora_merge_requantize.argtypes = [W, P, P, c.c_int, c.c_float, W, P, P]
     L.qlora_status_string.argtypes = [c.c_int]
     L.qlora_status_string.restype = c.c_char_p
     L.qlora_build_info.restype = c.c_char_p
@@ -79,6 +81,7 @@ def _load():
     for name in ("qlora_workspace_init", "qlora_linear_fwd", "qlora_linear_bwd",
                  "qlora_grouped_fwd", "qlora_grouped_bwd", "qlora_get_device_status",
                  "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_debug_decode_rate",
+                 "qlora_quantize", "qlora_merge_requantize",
                  "qlora_profile_enable",
                  "qlora_profile_reset", "qlora_profile_read"):
         getattr(L, name).restype = c.c_int
@@ -191,6 +194,31 @@ def qlora_debug_dequant(W: Weight, transposed, out, stream=None):
 def qlora_debug_wait_timeout(ws, limit_us, stream=None):
     _check(lib.qlora_debug_wait_timeout(_p(ws), ws.numel(), int(limit_us), _stream(stream)),
            "qlora_debug_wait_timeout")
+
+
+def empty_weight(fmt, N, K, device="cuda"):
+    """Device storage for a weight of this format and shape (contents undefined)."""
+    fid = FMT[fmt]
+    bs = {0: 64, 1: 32, 2: 16, 3: 64}[fid]
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty((N, K // bs), dtype=torch.float32 if fid == 0 else torch.uint8,
+                         device=device)
+    ts = torch.empty(1, dtype=torch.float32, device=device) if fid == 2 else None
+    s2 = (torch.empty((N * (K // 64) + 255) // 256, dtype=torch.float32, device=device)
+          if fid == 3 else None)
+    return Weight(fmt, N, K, codes, scales, ts, s2)
+
+
+def qlora_quantize(W: Weight, v, stream=None):
+    """Quantise the float weight v [N,K] (fp32 or bf16 device tensor) into W's storage."""
+    _check(lib.qlora_quantize(W.ref, _p(v), 1 if v.dtype == torch.bfloat16 else 0, _stream(stream)),
+           "qlora_quantize")
+
+
+def qlora_merge_requantize(W: Weight, A, B, r, scale, W_out: Weight, merged, stream=None):
+    """W_out = Q(deq(W) + scale B A); the merged fp32 values land in `merged` [N,K]."""
+    _check(lib.qlora_merge_requantize(W.ref, _p(A), _p(B), int(r), float(scale), W_out.ref,
+                                      _p(merged), _stream(stream)), "qlora_merge_requantize")
 
 
 def qlora_debug_decode_rate(fmt, iters=2000):

@@ -205,6 +205,41 @@ QLORA_API qlora_status_t qlora_debug_dequant(const qlora_weight_t* W, int transp
 QLORA_API qlora_status_t qlora_debug_wait_timeout(void* ws, size_t ws_bytes, int limit_us,
                                         qlora_stream_t stream);
 
+/* Quantise a float weight once, before training ("Training LLMs on a Budget", §3 "The setup"):
+ * v [N,K] (row-major, device; fp32, or bf16 when v_is_bf16) into the
+ * storage W describes (fmt, N, K and device pointers codes, scales, tensor_scale for NVFP4,
+ * scales2 for NF4_DQ; the arrays are written although the struct declares them const).  One
+ * weight per call: an expert stack is quantised one expert at a time, each with its own slice of
+ * the arrays.  Errors: QLORA_ERR_INVALID_ARG for a shape or pointer outside the weight limits
+ * every entry point applies (N % 16, K % 64, 16-byte aligned codes and scales) or a v that is
+ * NULL or not 4-byte aligned; QLORA_ERR_CUDA for a failed launch.  The pages give no rounding rules; these are the
+ * library's (the oracle's `oracle_encode` states them the same way):
+ *   NF4    absmax = max |v| of the 64-block; code = the number of NF4 level midpoints below
+ *          v / absmax (binary64), ties to the lower code; an all-zero block is all code 7.
+ *   NF4_DQ as NF4 against the decoded absmax fp32(e4m3(c1) * s2), s2 = fp32(group max / 448) per
+ *          256 consecutive blocks (1 for an all-zero group), c1 = nearest E4M3 of absmax / s2.
+ *   MXFP4  e = clamp(floor(log2 amax) - 2 + 127, 0, 254) (0 for a zero block); code = nearest
+ *          E2M1 of v / 2^(e-127), ties to the even code, saturating at 6.
+ *   NVFP4  tensor_scale = fp32(max |v| / 2688) (1 for a zero tensor); block scale = nearest E4M3
+ *          of amax / (6 tensor_scale); code = nearest E2M1 of v / (e4m3(s_b) tensor_scale).
+ *   Quotients binary64, E4M3 ties to the even code, saturating at 448.  v must be finite.
+ * Async on stream (NVFP4: three launches, the tensor scale's slot used in between). */
+QLORA_API qlora_status_t qlora_quantize(const qlora_weight_t* W, const void* v, int v_is_bf16,
+                                        qlora_stream_t stream);
+
+/* Merge a trained adapter into a stored weight and requantise ("Training LLMs on a Budget",
+ * §2 "Deployment: keep or merge"; "Fine-Tuning 4-Bit Models", "Case 2" and "Case 3"):
+ * W_out = Q(deq(W) + scale B A),
+ * with Q the rules of qlora_quantize in W_out's format (any format, same N and K).  The merged
+ * value of (n,k) is fp32(deq(W)[n,k] + scale * sum_j B[n,j] A[j,k]), the sum over j = 0..r-1 in
+ * order, every product and sum in binary64; it is written to `merged` [N,K] fp32 (device,
+ * caller-owned scratch, kept as an output: the adapter signal lost to requantisation is
+ * deq(W_out) - merged).  A [r,K], B [N,r] bf16; 1 <= r <= 1024.  Async on stream. */
+QLORA_API qlora_status_t qlora_merge_requantize(const qlora_weight_t* W, const void* A,
+                                                const void* B, int r, float scale,
+                                                const qlora_weight_t* W_out, float* merged,
+                                                qlora_stream_t stream);
+
 /* Benchmark support: measure the decode throughput of the layer's own dequant stage (the code
  * every GEMM kernel decodes the 4-bit weight with) on every SM -- 256 threads per SM, each
  * decoding `iters` 64-element items into a shared-memory operand tile -- and return the mean

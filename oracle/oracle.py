@@ -200,5 +200,26 @@ def encode(fmt, v):
     return codes, scales, (float(ts[0]) if f == 2 else None), s2
 
 
+def merge(fmt, N, K, codes, scales, tensor_scale, A, B, s, scales2=None):
+    """The adapter merged into the stored weight before requantisation, fp32 [N,K]:
+    fp32(deq(W)[n,k] + s * sum_j B[n,j] A[j,k]).
+
+    "Training LLMs on a Budget: LoRA, QLoRA, and LoftQ", §2 "Deployment: keep or merge": a merge
+    adds the low-rank product B A, scaled, to the frozen weight; a quantised base is dequantised
+    first and the sum requantised afterwards (encode() of the result).  The sum over
+    j runs in order, in binary64 (each product of two bf16 values is exact), then s times it, then
+    the decoded weight plus that, rounded to fp32 once.  A [r,K], B [N,r] as bf16 bit patterns."""
+    A = np.ascontiguousarray(A, np.uint16)
+    B = np.ascontiguousarray(B, np.uint16)
+    r = A.shape[0]
+    wide = lambda h: (h.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    w = wide(dequant(fmt, N, K, codes, scales, tensor_scale, scales2=scales2))
+    Af, Bf = wide(A), wide(B)
+    acc = np.zeros((N, K))
+    for j in range(r):
+        acc = acc + Bf[:, j:j + 1] * Af[j:j + 1, :]
+    return (w + float(np.float32(s)) * acc).astype(np.float32)
+
+
 def num_threads():
     return lib().oracle_num_threads()

@@ -161,3 +161,20 @@ def test_encode_decode_error_bound(fmt):
     # scale rounding (amax <= 6 * scale * 2): < 2 / 6 + a bf16 ulp
     bound = {"nf4": 0.2, "nf4dq": 0.22, "mxfp4": 0.34, "nvfp4": 0.2}[fmt]
     assert np.all(np.abs(wf - v) <= bound * amax + 1e-12)
+
+
+def test_encode_mxfp4_round_trip_of_decoded_weight():
+    # an MXFP4-decoded weight is exactly representable again: encoding it and decoding the result
+    # gives it back bit for bit (the new block exponent may be finer when the block's largest
+    # code is small, but every E2M1 value times a power of two stays on the finer grid); equal as
+    # values: code 8 (-0) comes back as +0, the encoder gives the sign only to non-zero magnitudes
+    rng = np.random.default_rng(16)
+    N, K = 8, 256
+    codes = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    e = rng.integers(100, 150, size=(N, K // 32)).astype(np.uint8)
+    w = O.dequant("mxfp4", N, K, codes, e)
+    wf = (w.astype(np.uint32) << 16).view(np.float32)
+    c2, e2, _, _ = O.encode("mxfp4", wf)
+    w2 = (O.dequant("mxfp4", N, K, c2, e2).astype(np.uint32) << 16).view(np.float32)
+    assert np.array_equal(w2, wf)
+    assert not np.any(_unpack(c2, N, K) == 8)
