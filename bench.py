@@ -364,6 +364,69 @@ def nf4dq_step(Q, torch, p, Xs, dYs, A, B, ncopy, steps=60):
             "bits_per_weight": round(bits, 4), "data": "workload NF4 codes, random stored scales"}
 
 
+def quantize_merge(Q, torch, p, A, B, peaks, reps=10):
+    """The quantiser and the merge with requantisation on the workload's weight shape.
+
+    quantize: a float weight v ~ N(0, 0.02) (fp32, on the device, 235 MB > L2) encoded into each
+    format; algorithmic bytes = one read of v (two for NVFP4, whose tensor scale needs the whole
+    tensor's max before any block is encoded) + the stored bytes written.
+    merge: the workload's adapter (A, B, s) merged into the NF4 weight and requantised to NF4;
+    algorithmic bytes = stored weight read + A, B + merged fp32 written and read back + stored
+    weight written.  The merge computes every sum in binary64 (r products and sums per element),
+    so its bound is the fp64 pipe, reported beside the bytes.  adapter_retained: the share of the
+    adapter's change that the requantised weight keeps, <deq(W') - deq(W), d> / <d, d> with d the
+    merged values minus deq(W); lost_rel: ||deq(W') - merged|| / ||d||."""
+    N, K, r, s = p["N"], p["K"], p["r"], p["s"]
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    v = torch.randn((N, K), generator=g, device="cuda") * 0.02
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    hbm = peaks.get("hbm_gbs") or 6650.0
+    out = {"weight": f"{N}x{K}", "v": "fp32 N(0, 0.02), torch.randn on the device"}
+    for fmt in ("nf4", "nf4dq", "mxfp4", "nvfp4"):
+        W = Q.empty_weight(fmt, N, K)
+        for _ in range(2):
+            Q.qlora_quantize(W, v)
+        e0.record()
+        for _ in range(reps):
+            Q.qlora_quantize(W, v)
+        e1.record()
+        e1.synchronize()
+        t = e0.elapsed_time(e1) / reps * 1e-3
+        nbytes = (8 if fmt == "nvfp4" else 4) * N * K + W.nbytes()
+        out[f"quantize_{fmt}"] = {"ms": round(t * 1e3, 4), "gbs": round(nbytes / t / 1e9, 1),
+                                  "hbm_frac": round(nbytes / t / 1e9 / hbm, 3)}
+    W = Q.empty_weight("nf4", N, K)
+    Q.qlora_quantize(W, v)
+    del v
+    W_out = Q.empty_weight("nf4", N, K)
+    merged = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    Q.qlora_merge_requantize(W, A, B, r, s, W_out, merged)
+    e0.record()
+    for _ in range(reps):
+        Q.qlora_merge_requantize(W, A, B, r, s, W_out, merged)
+    e1.record()
+    e1.synchronize()
+    t = e0.elapsed_time(e1) / reps * 1e-3
+    nbytes = 2 * W.nbytes() + 2 * (A.numel() + B.numel()) + 8 * N * K
+    deq0 = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    deq1 = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    Q.qlora_debug_dequant(W, 0, deq0)
+    Q.qlora_debug_dequant(W_out, 0, deq1)
+    d = merged.double() - deq0.double()
+    moved = deq1.double() - deq0.double()
+    dd = float((d * d).sum())
+    out["merge_nf4_to_nf4"] = {
+        "r": r, "s": s, "ms": round(t * 1e3, 4), "gbs": round(nbytes / t / 1e9, 1),
+        "hbm_frac": round(nbytes / t / 1e9 / hbm, 3),
+        "fp64_ops_per_s": round(2.0 * r * N * K / t / 1e12, 2),
+        "fp64_unit": "T dmul+dadd per s",
+        "adapter_retained": round(float((moved * d).sum()) / dd, 4),
+        "lost_rel": round(float(((deq1.double() - merged.double()) ** 2).sum() / dd) ** 0.5, 4)}
+    return out
+
+
 def grouped_moe(Q, torch, synth, peaks):
     """One fwd+bwd of each MoE expert projection (64 experts, MXFP4, Zipf top-8 routing of 16384
     tokens): TFLOP/s.  Timing inputs: seeded random stored codes with a realistic E8M0 scale range
@@ -592,6 +655,11 @@ def run_own(args):
     if not args.no_sweep:
         dq = nf4dq_step(Q, torch, p, Xs, dYs, A, B, ncopy)
 
+    # ---- quantiser and merge with requantisation on the workload's weight shape
+    qm = None
+    if not args.no_sweep:
+        qm = quantize_merge(Q, torch, p, A, B, peaks)
+
     # ---- grouped (MoE) experts: 64 experts, 16384 tokens x top-8, one fwd+bwd per projection
     grouped = None
     if not args.no_sweep:
@@ -621,6 +689,7 @@ def run_own(args):
         "e2e": e2e,
         "weight_stream_small_m": sweep,
         "nf4_double_quant": dq,
+        "quantize_merge": qm,
         "grouped_moe": grouped,
         "cpu_baseline": cpu,
     }

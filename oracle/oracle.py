@@ -221,5 +221,53 @@ def merge(fmt, N, K, codes, scales, tensor_scale, A, B, s, scales2=None):
     return (w + float(np.float32(s)) * acc).astype(np.float32)
 
 
+def loftq(W, r, s, iters=5, fmt="nf4", quant=None):
+    """LoftQ initialisation of the adapter for a quantised base, in fp64.
+
+    "Training LLMs on a Budget: LoRA, QLoRA, and LoftQ", §4 "The algorithm: alternating
+    quantization and SVD": minimise ||W - Q - s B A||_F by alternating the two sub-problems --
+    Q = quantise(W - s B A) with the adapter fixed, then s B A = the best rank-r approximation of
+    R = W - Q (Eckart-Young: the top r singular triplets of R) with Q fixed -- starting from
+    B A = 0.  One iteration is one quantisation followed by one SVD, so a single iteration of the
+    page's 3x3 example already recovers W; the page's default is 5.  The split of the rank-r
+    factor follows the page, B = U_r sqrt(Sigma_r / s), A = sqrt(Sigma_r / s) V_r^T, the LoRA
+    scale s carried as in the layer (s B A = U_r Sigma_r V_r^T).
+
+    W: float array [N,K] (fp32 values; the quantiser reads W - s B A rounded to fp32).
+    quant: optional function v -> decoded array (float64) standing in for the format's encode +
+    decode (the page's worked example rounds to integers); default: encode() then dequant() in
+    `fmt`, the decoded weight being the bf16 values the layer multiplies by.
+    Returns dict: Q (decoded, float64), stored (codes, scales, ts, s2 of the last quantisation,
+    or None with `quant`), A [r,K] and B [N,r] (float64, before any rounding to bf16),
+    sigma (the top r singular values of the last residual), errs [iters+1]:
+    errs[0] = ||W - Q_1|| (the plain QLoRA start, B = 0), errs[t] = ||W - Q_t - s B_t A_t||."""
+    W = np.asarray(W, np.float64)
+    N, K = W.shape
+
+    def q(v):
+        if quant is not None:
+            return np.asarray(quant(v), np.float64), None
+        st = encode(fmt, v.astype(np.float32))
+        d = dequant(fmt, N, K, st[0], st[1], 1.0 if st[2] is None else st[2], scales2=st[3])
+        return (d.astype(np.uint32) << 16).view(np.float32).astype(np.float64), st
+
+    Q, stored = q(W)
+    errs = [float(np.linalg.norm(W - Q))]
+    A = np.zeros((r, K))
+    B = np.zeros((N, r))
+    sig = np.zeros(r)
+    for t in range(1, iters + 1):
+        if t > 1:
+            Q, stored = q(W - s * (B @ A))
+        R = W - Q
+        U, S, Vt = np.linalg.svd(R, full_matrices=False)
+        sig = S[:r].copy()
+        root = np.sqrt(sig / s)
+        B = U[:, :r] * root[None, :]
+        A = root[:, None] * Vt[:r, :]
+        errs.append(float(np.linalg.norm(R - s * (B @ A))))
+    return {"Q": Q, "stored": stored, "A": A, "B": B, "sigma": sig, "errs": errs}
+
+
 def num_threads():
     return lib().oracle_num_threads()

@@ -1,0 +1,104 @@
+"""Pins of the oracle's LoftQ initialisation (CPU only).
+
+"Training LLMs on a Budget: LoRA, QLoRA, and LoftQ", §4: alternate Q = quantise(W - s B A) and
+s B A = best rank-r approximation of W - Q.  Pinned by the page's worked 3x3 example (integer
+rounding for the quantiser), by Eckart-Young (the error of each SVD step equals the energy of the
+discarded singular values, computed here by an independent eigen-solver on R R^T), and by a
+planted case whose answer is known in closed form: a weight that is an NF4 grid point plus a
+rank-2 matrix too small to move any code, which LoftQ recovers exactly after one iteration."""
+import os
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden", "loftq_3x3.txt")
+
+
+def _golden():
+    lines = [l.split("#")[0].strip() for l in open(GOLD)]
+    lines = [l for l in lines if l]
+    out, i = {}, 0
+    while i < len(lines):
+        head = lines[i].split()
+        if len(head) == 2:
+            out[head[0]] = float(head[1])
+            i += 1
+        elif head[0] in ("u", "v"):
+            out[head[0]] = np.array([float(x) for x in lines[i + 1].split()])
+            i += 2
+        else:
+            out[head[0]] = np.array([[float(x) for x in lines[i + j].split()] for j in (1, 2, 3)])
+            i += 4
+    return out
+
+
+@pytest.mark.parametrize("s", [1.0, 2.0])
+def test_loftq_worked_example(s):
+    g = _golden()
+    res = O.loftq(g["W"], r=1, s=s, iters=1, quant=np.rint)
+    assert np.array_equal(np.rint(g["W"]), g["Q0"])
+    assert np.allclose(g["W"] - g["Q0"], g["R0"], atol=1e-12)
+    assert np.allclose(np.outer(g["u"], g["v"]), g["R0"], atol=1e-12)     # R0 is rank 1
+    assert abs(res["errs"][0] - g["err_qlora"]) < 1e-12
+    assert abs(res["errs"][1] - g["err_loftq_1"]) < 1e-12
+    assert np.allclose(s * res["B"] @ res["A"], g["R0"], atol=1e-12)
+    # B = U sqrt(sigma / s), A = sqrt(sigma / s) V^T: both factors carry half of sigma
+    assert np.allclose(np.linalg.norm(res["B"]), np.linalg.norm(res["A"]), atol=1e-12)
+    more = O.loftq(g["W"], r=1, s=s, iters=5, quant=np.rint)
+    assert all(abs(e - g["err_loftq_more"]) < 1e-12 for e in more["errs"][1:])
+    assert np.array_equal(more["Q"], g["Q0"])
+
+
+def test_loftq_svd_step_is_eckart_young():
+    # each iteration's error is the energy of R_t's discarded spectrum; the spectrum here comes
+    # from numpy's symmetric eigen-solver on R R^T, not from the SVD the oracle uses
+    rng = np.random.default_rng(3)
+    N, K, r = 40, 96, 5
+    W = rng.standard_normal((N, K)) * 0.7
+    res = O.loftq(W, r=r, s=0.5, iters=1, quant=lambda v: np.round(v * 2) / 2)
+    R = W - np.round(W * 2) / 2
+    lam = np.sort(np.linalg.eigvalsh(R @ R.T))[::-1]
+    assert abs(res["errs"][1] - np.sqrt(lam[r:].sum())) < 1e-9
+    assert np.allclose(res["sigma"] ** 2, lam[:r], rtol=1e-9)
+    assert res["errs"][1] < res["errs"][0]
+
+
+def _planted(N, K, rank, seed):
+    """W = D + L: D an NF4 grid point (every 64-block's column 0 at level +1 with a bf16-exact
+    absmax, the other codes strictly inside), L rank-`rank`, zero on column 0 of every block and
+    below 1/64 of the block's absmax -- too small to move a code or the absmax."""
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(1, 15, size=(N, K), dtype=np.uint8)
+    codes[:, ::64] = 15
+    a = rng.uniform(0.01, 0.04, size=(N, K // 64)).astype(np.float32)
+    a = ((a.view(np.uint32) + 0x8000) & 0xFFFF0000).view(np.float32)      # bf16-exact absmax
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    D = O.dequant("nf4", N, K, packed, a)
+    Df = (D.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    U = rng.standard_normal((N, rank))
+    V = rng.standard_normal((K, rank))
+    V[::64] = 0.0
+    L = U @ V.T
+    L *= (0.01 / 64) / np.abs(L).max()            # |L| < amin / 64 <= a / 64
+    W = (Df + L).astype(np.float32)
+    return W, packed, a, Df, L
+
+
+def test_loftq_planted_nf4_is_recovered():
+    N, K, rank = 32, 256, 2
+    W, packed, a, Df, L = _planted(N, K, rank, 7)
+    res = O.loftq(W, r=rank, s=2.0, iters=3, fmt="nf4")
+    codes, scales, _, _ = res["stored"]
+    assert np.array_equal(codes, packed) and np.array_equal(scales, a)
+    assert np.array_equal(res["Q"], Df)
+    assert abs(res["errs"][0] - np.linalg.norm(W.astype(np.float64) - Df)) < 1e-12
+    # what is left is W's own fp32 rounding of D + L: L is a rank-2 candidate, so the best rank-2
+    # fit leaves at most ||(W - D) - L||, and that is below 1e-4 of the start
+    resid = np.linalg.norm(W.astype(np.float64) - Df - L)
+    assert res["errs"][1] <= resid * (1 + 1e-9) and resid < 1e-4 * res["errs"][0]
+    assert np.allclose(2.0 * res["B"] @ res["A"], L, rtol=0, atol=1e-4 * np.abs(L).max())
+    # a rank below the planted one cannot recover it: the error stays at the dropped factor
+    low = O.loftq(W, r=rank - 1, s=2.0, iters=1, fmt="nf4")
+    assert low["errs"][1] > 1e-3 * low["errs"][0]
