@@ -424,6 +424,23 @@ def quantize_merge(Q, torch, p, A, B, peaks, reps=10):
         "fp64_unit": "T dmul+dadd per s",
         "adapter_retained": round(float((moved * d).sum()) / dd, 4),
         "lost_rel": round(float(((deq1.double() - merged.double()) ** 2).sum() / dd) ** 0.5, 4)}
+    del d, moved, deq0, deq1, merged
+    # LoftQ initialisation on the same weight: 5 iterations, rank r, 4 power iterations
+    v = torch.randn((N, K), generator=g, device="cuda") * 0.02
+    Wl = Q.empty_weight("nf4", N, K)
+    work = torch.empty(Q.qlora_loftq_workspace_size(N, K, r), dtype=torch.uint8, device="cuda")
+    Q.qlora_loftq(v, Wl, r, s, iters=1, power_iters=4, work=work)
+    e0.record()
+    _, _, errs, sig = Q.qlora_loftq(v, Wl, r, s, iters=5, power_iters=4, work=work)
+    e1.record()
+    e1.synchronize()
+    errs = errs.cpu().tolist()
+    out["loftq_nf4"] = {"r": r, "iters": 5, "power_iters": 4,
+                        "ms": round(e0.elapsed_time(e1), 2),
+                        "err_qlora": round(errs[0], 4), "err_loftq": round(errs[-1], 4),
+                        "err_ratio": round(errs[-1] / errs[0], 4),
+                        "note": "N(0, 0.02) weight: a flat residual spectrum, so the rank-r "
+                                "part of the quantisation error is small"}
     return out
 
 

@@ -14,7 +14,10 @@
 #include "qlora_fused.cuh"
 #include "qlora_lora.cuh"
 #include "qlora_stream.cuh"
+#include <algorithm>
+#include <utility>
 #include "qlora_quant.cuh"
+#include "qlora_loftq.cuh"
 
 namespace qlora {
 namespace {
@@ -928,10 +931,7 @@ qlora_status_t qlora_merge_requantize(const qlora_weight_t* W, const void* A, co
     return QLORA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   MergeParams p{};
-  p.codes = W->codes;
-  p.scales = W->scales;
-  p.scales2 = W->scales2;
-  p.tensor_scale = W->tensor_scale;
+  p.w = StoredView{W->codes, W->scales, W->scales2, W->tensor_scale, int(W->K)};
   p.A = static_cast<const __nv_bfloat16*>(A);
   p.B = static_cast<const __nv_bfloat16*>(B);
   p.out = merged;
@@ -948,6 +948,227 @@ qlora_status_t qlora_merge_requantize(const qlora_weight_t* W, const void* A, co
   }
   if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
   return qlora_quantize(W_out, merged, 0, stream);
+}
+
+}  // extern "C"
+
+namespace {
+// ------------------------------------------------------------------------------------- LoftQ
+// Split of a tall-product's reduction: up to 296 CTAs, one wave of a 148-SM part at the GEMM's
+// two CTAs per SM (a constant, so that the workspace size does not depend on the device), at
+// least 512 of the reduction per split.
+constexpr int64_t kLoftqTargetCtas = 296;
+
+int loftq_splits(int64_t M, int64_t Nn, int64_t Kk) {
+  const int64_t tiles = ((M + loftq::kBM - 1) / loftq::kBM) * ((Nn + loftq::kBN - 1) / loftq::kBN);
+  int64_t z = kLoftqTargetCtas / tiles;   // at most one wave at two CTAs per SM
+  if (z > Kk / 512) z = Kk / 512;
+  if (z > 256) z = 256;
+  return int(z < 1 ? 1 : z);
+}
+
+int loftq_width(int64_t N, int64_t K, int r) {
+  int64_t l = r + loftq::kOversample;
+  if (l > loftq::kMaxL) l = loftq::kMaxL;
+  if (l > N) l = N;
+  if (l > K) l = K;
+  return int(l);
+}
+
+struct LoftqLayout {
+  size_t R, Y, Y2, Z, Z2, omega, part, G, Mx, Cb, Ca, sig, Bf, Af, norm, total;
+};
+
+LoftqLayout loftq_layout(int64_t N, int64_t K, int r) {
+  const int64_t l = loftq_width(N, K, r);
+  int64_t part = 0;
+  auto need = [&](int64_t M, int64_t Nn, int64_t Kk, bool always) {
+    const int z = loftq_splits(M, Nn, Kk);
+    if (z > 1 || always) part = std::max(part, int64_t(z) * M * Nn);
+  };
+  need(N, l, K, false);   // Y = R Omega, Y = R Z
+  need(K, l, N, false);   // Z = R^T Y
+  need(l, l, N, true);    // Y^T Y
+  need(l, l, K, true);    // Z^T Z
+  LoftqLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~size_t(255);
+    return o;
+  };
+  L.R = take(size_t(N) * K * 4);
+  L.Y = take(size_t(N) * l * 4);
+  L.Y2 = take(size_t(N) * l * 4);
+  L.Z = take(size_t(K) * l * 4);
+  L.Z2 = take(size_t(K) * l * 4);
+  L.omega = take(size_t(K) * l * 4);
+  L.part = take(size_t(part) * 4);
+  L.G = take(size_t(l) * l * 8);
+  L.Mx = take(size_t(l) * l * 4);
+  L.Cb = take(size_t(l) * r * 4);
+  L.Ca = take(size_t(r) * l * 4);
+  L.sig = take(size_t(r) * 4);
+  L.Bf = take(size_t(N) * r * 4);
+  L.Af = take(size_t(r) * K * 4);
+  L.norm = take(size_t(loftq::kNormBlocks) * 8);
+  L.total = off;
+  return L;
+}
+
+// C = opA(A) opB(B) [M, Nn] (dense, ldc = Nn when split); out64: the result as fp64 instead.
+template <bool TA, bool TB>
+void loftq_gemm(const float* A, int64_t lda, const float* B, int64_t ldb, float* C, int64_t ldc,
+                int M, int Nn, int64_t Kk, float* part, double* out64, cudaStream_t s) {
+  const int z = loftq_splits(M, Nn, Kk);
+  const dim3 grid(unsigned((M + loftq::kBM - 1) / loftq::kBM),
+                  unsigned((Nn + loftq::kBN - 1) / loftq::kBN), unsigned(z));
+  if (z == 1 && !out64) {
+    loftq_gemm_kernel<TA, TB><<<grid, 256, 0, s>>>(A, lda, B, ldb, C, ldc, 0, M, Nn, Kk, Kk);
+    return;
+  }
+  const int64_t kchunk = ((Kk + z - 1) / z + loftq::kBK - 1) / loftq::kBK * loftq::kBK;
+  const int64_t count = int64_t(M) * Nn;
+  loftq_gemm_kernel<TA, TB><<<grid, 256, 0, s>>>(A, lda, B, ldb, part, Nn, count, M, Nn, Kk, kchunk);
+  const unsigned rb = unsigned(std::min<int64_t>((count + 255) / 256, 1184));
+  loftq_reduce_kernel<<<rb, 256, 0, s>>>(part, count, z, count, out64 ? nullptr : C, out64);
+}
+
+struct LoftqRun {
+  const LoftqLayout& L;
+  char* ws;
+  int64_t N, K;
+  int r, l;
+  float s;
+  cudaStream_t st;
+  template <typename T>
+  T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
+
+  void jacobi(int mode) const {
+    JacobiParams p{};
+    p.G = at<double>(L.G);
+    p.l = l;
+    p.mode = mode;
+    p.M = at<float>(L.Mx);
+    p.Cb = at<float>(L.Cb);
+    p.Ca = at<float>(L.Ca);
+    p.sigma = at<float>(L.sig);
+    p.r = r;
+    p.s = s;
+    loftq_jacobi_kernel<<<1, loftq::kJacobiThreads, loftq::jacobi_smem(l), st>>>(p);
+  }
+  // X [rows, l] <- a basis of its column space by SVQB; X and X2 swap.  Two passes make it
+  // orthonormal to fp32 precision (the basis Rayleigh-Ritz uses); one keeps the power iteration's
+  // intermediate bases well conditioned, which is all they need.
+  void orth(float*& X, float*& X2, int64_t rows, int passes) const {
+    for (int pass = 0; pass < passes; ++pass) {
+      loftq_gemm<true, false>(X, l, X, l, nullptr, l, l, l, rows, at<float>(L.part),
+                              at<double>(L.G), st);
+      jacobi(0);
+      loftq_gemm<false, false>(X, l, at<float>(L.Mx), l, X2, l, int(rows), l, l, nullptr, nullptr,
+                               st);
+      std::swap(X, X2);
+    }
+  }
+  // Top-r SVD of R [N, K] into Bf [N, r], Af [r, K] (s Bf Af = U_r S_r V_r^T), sigma [r].
+  void svd(int power_iters) const {
+    const float* R = at<float>(L.R);
+    float* Y = at<float>(L.Y);
+    float* Y2 = at<float>(L.Y2);
+    float* Z = at<float>(L.Z);
+    float* Z2 = at<float>(L.Z2);
+    float* part = at<float>(L.part);
+    loftq_gemm<false, false>(R, K, at<float>(L.omega), l, Y, l, int(N), l, K, part, nullptr, st);
+    orth(Y, Y2, N, power_iters == 0 ? 2 : 1);
+    for (int q = 0; q < power_iters; ++q) {
+      loftq_gemm<true, false>(R, K, Y, l, Z, l, int(K), l, N, part, nullptr, st);
+      orth(Z, Z2, K, 1);
+      loftq_gemm<false, false>(R, K, Z, l, Y, l, int(N), l, K, part, nullptr, st);
+      orth(Y, Y2, N, q + 1 == power_iters ? 2 : 1);
+    }
+    loftq_gemm<true, false>(R, K, Y, l, Z, l, int(K), l, N, part, nullptr, st);
+    loftq_gemm<true, false>(Z, l, Z, l, nullptr, l, l, l, K, part, at<double>(L.G), st);
+    jacobi(1);
+    loftq_gemm<false, false>(Y, l, at<float>(L.Cb), r, at<float>(L.Bf), r, int(N), r, l, nullptr,
+                             nullptr, st);
+    loftq_gemm<false, true>(at<float>(L.Ca), l, Z, l, at<float>(L.Af), K, r, int(K), l, nullptr,
+                            nullptr, st);
+  }
+};
+
+void loftq_residual(const qlora_weight_t* Q, const float* W, float* R, double* part, cudaStream_t s) {
+  const StoredView v{Q->codes, Q->scales, Q->scales2, Q->tensor_scale, int(Q->K)};
+  const int N = int(Q->N), K = int(Q->K);
+  const unsigned g = loftq::kNormBlocks;
+  switch (Q->fmt) {
+    case QLORA_FMT_NF4: loftq_residual_kernel<kFmtNF4><<<g, 256, 0, s>>>(W, v, R, N, K, part); break;
+    case QLORA_FMT_MXFP4: loftq_residual_kernel<kFmtMXFP4><<<g, 256, 0, s>>>(W, v, R, N, K, part); break;
+    case QLORA_FMT_NVFP4: loftq_residual_kernel<kFmtNVFP4><<<g, 256, 0, s>>>(W, v, R, N, K, part); break;
+    default: loftq_residual_kernel<kFmtNF4DQ><<<g, 256, 0, s>>>(W, v, R, N, K, part); break;
+  }
+}
+}  // namespace
+
+extern "C" {
+
+size_t qlora_loftq_workspace_size(int64_t N, int64_t K, int r) {
+  if (N < 1 || K < 1 || r < 1 || r > loftq::kMaxL || r > N || r > K) return 0;
+  return loftq_layout(N, K, r).total;
+}
+
+qlora_status_t qlora_loftq(const float* W, const qlora_weight_t* Q, int r, float scale, int iters,
+                           int power_iters, uint64_t seed, void* A_out, void* B_out, float* errs,
+                           float* sigma, void* work, size_t work_bytes, qlora_stream_t stream) {
+  qlora_status_t st = check_weight(Q);
+  if (st != QLORA_OK) return st;
+  const int64_t N = Q->N, K = Q->K;
+  if (r < 1 || r > loftq::kMaxL || r > N || r > K || !(scale > 0.0f) || !(scale < 3.0e38f) ||
+      iters < 1 || iters > 64 || power_iters < 0 || power_iters > 16 || !ptr_ok(W) ||
+      !ptr_ok(A_out) || !ptr_ok(B_out) || !errs || (reinterpret_cast<uintptr_t>(errs) & 3u) ||
+      (sigma && (reinterpret_cast<uintptr_t>(sigma) & 3u)) || !work ||
+      (reinterpret_cast<uintptr_t>(work) & 255u) || N * K > (int64_t(1) << 31))
+    return QLORA_ERR_INVALID_ARG;
+  const LoftqLayout L = loftq_layout(N, K, r);
+  if (work_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  static bool attr_done[kMaxDevices] = {false};
+  const int dev = current_device();
+  if (dev >= 0 && dev < kMaxDevices && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(loftq_jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(loftq::jacobi_smem(loftq::kMaxL))) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  const LoftqRun run{L, static_cast<char*>(work), N, K, r, loftq_width(N, K, r), scale, s};
+  float* R = run.at<float>(L.R);
+  double* norm = run.at<double>(L.norm);
+  const int64_t n_omega = K * run.l;
+  loftq_omega_kernel<<<unsigned(std::min<int64_t>((n_omega + 255) / 256, 1184)), 256, 0, s>>>(
+      run.at<float>(L.omega), n_omega, seed);
+  st = qlora_quantize(Q, W, 0, stream);                     // Q_1 = quantise(W)
+  if (st != QLORA_OK) return st;
+  for (int t = 1; t <= iters; ++t) {
+    loftq_residual(Q, W, R, norm, s);                       // R_t = W - deq(Q_t)
+    if (t == 1) loftq_norm_kernel<<<1, 32, 0, s>>>(norm, loftq::kNormBlocks, errs);
+    run.svd(power_iters);                                   // s B_t A_t = top-r part of R_t
+    const int more = t < iters;
+    loftq_shift_kernel<<<loftq::kNormBlocks, 256, 0, s>>>(W, R, run.at<float>(L.Bf),
+                                                          run.at<float>(L.Af), int(N), int(K), r,
+                                                          scale, more, norm);
+    loftq_norm_kernel<<<1, 32, 0, s>>>(norm, loftq::kNormBlocks, errs + t);
+    if (more) {
+      st = qlora_quantize(Q, R, 0, stream);                 // Q_{t+1} = quantise(W - s B_t A_t)
+      if (st != QLORA_OK) return st;
+    }
+  }
+  loftq_to_bf16_kernel<<<256, 256, 0, s>>>(run.at<float>(L.Af),
+                                           static_cast<__nv_bfloat16*>(A_out), int64_t(r) * K);
+  loftq_to_bf16_kernel<<<256, 256, 0, s>>>(run.at<float>(L.Bf),
+                                           static_cast<__nv_bfloat16*>(B_out), N * r);
+  if (sigma && cudaMemcpyAsync(sigma, run.at<float>(L.sig), size_t(r) * 4,
+                               cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 qlora_status_t qlora_debug_decode_rate(int fmt, int iters, double* weights_per_clock_per_sm) {

@@ -197,11 +197,17 @@ qlora_quant_encode_kernel(const QuantParams p) {
 // j = 0..r-1 in that order in binary64 (each bf16 product exact), plus and times in binary64
 // without contraction, one rounding to binary32 at the end.  deq(W) is the weight's full decode
 // (for NVFP4 including the tensor scale).
-struct MergeParams {
+// A stored weight as the element decode reads it.
+struct StoredView {
   const uint8_t* codes;
   const void* scales;
   const float* scales2;
   const float* tensor_scale;
+  int K;
+};
+
+struct MergeParams {
+  StoredView w;
   const __nv_bfloat16* A;   // [r, K]
   const __nv_bfloat16* B;   // [N, r]
   float* out;               // [N, K]
@@ -209,25 +215,30 @@ struct MergeParams {
   float s;
 };
 
+// Element (n, k) of the decoded weight as the layer's GEMMs see it: the bf16 value of the format's
+// decode chain (NVFP4 including the tensor scale), widened to fp32.
 template <int FMT>
-__device__ __forceinline__ float decode_element(const MergeParams& p, int n, int k) {
-  const uint8_t byte = p.codes[size_t(n) * (p.K / 2) + k / 2];
+__device__ __forceinline__ float decode_element(const StoredView& w, int n, int k) {
+  const uint8_t byte = w.codes[size_t(n) * (w.K / 2) + k / 2];
   const uint32_t c = (k & 1) ? uint32_t(byte >> 4) : uint32_t(byte & 15u);
   if constexpr (FMT == kFmtNF4 || FMT == kFmtNF4DQ) {
-    const size_t fb = size_t(n) * (p.K / 64) + k / 64;
+    const size_t fb = size_t(n) * (w.K / 64) + k / 64;
     const float a = FMT == kFmtNF4
-                        ? static_cast<const float*>(p.scales)[fb]
-                        : __fmul_rn(e4m3_f32(static_cast<const uint8_t*>(p.scales)[fb]),
-                                    p.scales2[fb / 256]);
-    return __bfloat162float(__float2bfloat16_rn(__fmul_rn(nf4_level_dev(int(c)), a)));
+                        ? static_cast<const float*>(w.scales)[fb]
+                        : __fmul_rn(e4m3_f32(static_cast<const uint8_t*>(w.scales)[fb]),
+                                    w.scales2[fb / 256]);
+    float lv = 0.0f;                       // select, not an indexed local array
+#pragma unroll
+    for (int i = 0; i < 16; ++i) lv = c == uint32_t(i) ? nf4_level_dev(i) : lv;
+    return __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv, a)));
   } else if constexpr (FMT == kFmtMXFP4) {
-    const uint32_t e = static_cast<const uint8_t*>(p.scales)[size_t(n) * (p.K / 32) + k / 32];
+    const uint32_t e = static_cast<const uint8_t*>(w.scales)[size_t(n) * (w.K / 32) + k / 32];
     const float sc = e == 255u ? __uint_as_float(0x7FC00000u)
                                : (e == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(e << 23));
     return __bfloat162float(__float2bfloat16_rn(__fmul_rn(e2m1_f32(c), sc)));
   } else {
-    const uint32_t sb = static_cast<const uint8_t*>(p.scales)[size_t(n) * (p.K / 16) + k / 16];
-    const float prod = __fmul_rn(__fmul_rn(e2m1_f32(c), e4m3_f32(sb)), *p.tensor_scale);
+    const uint32_t sb = static_cast<const uint8_t*>(w.scales)[size_t(n) * (w.K / 16) + k / 16];
+    const float prod = __fmul_rn(__fmul_rn(e2m1_f32(c), e4m3_f32(sb)), *w.tensor_scale);
     return __bfloat162float(__float2bfloat16_rn(prod));
   }
 }
@@ -242,7 +253,7 @@ __global__ void __launch_bounds__(256) qlora_merge_values_kernel(const MergePara
     for (int j = 0; j < p.r; ++j)
       lora = __dadd_rn(lora, __dmul_rn(double(__bfloat162float(p.B[size_t(n) * p.r + j])),
                                        double(__bfloat162float(p.A[size_t(j) * p.K + k]))));
-    const double v = __dadd_rn(double(decode_element<FMT>(p, n, k)), __dmul_rn(double(p.s), lora));
+    const double v = __dadd_rn(double(decode_element<FMT>(p.w, n, k)), __dmul_rn(double(p.s), lora));
     p.out[i] = __double2float_rn(v);
   }
 }

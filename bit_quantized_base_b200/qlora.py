@@ -28,7 +28,8 @@ EXPORTS = ("qlora_workspace_size", "qlora_workspace_init", "qlora_linear_fwd", "
            "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_status_string",
            "qlora_build_info", "qlora_launch_count", "qlora_profile_enable",
            "qlora_profile_reset", "qlora_profile_read", "qlora_linear_fwd_noalloc",
-           "qlora_debug_decode_rate", "qlora_quantize", "qlora_merge_requantize")
+           "qlora_debug_decode_rate", "qlora_quantize", "qlora_merge_requantize",
+           "qlora_loftq_workspace_size", "qlora_loftq")
 
 
 class QLoraError(RuntimeError):
@@ -69,6 +70,10 @@ def _load():
     L.qlora_debug_decode_rate.argtypes = [c.c_int, c.c_int, c.POINTER(c.c_double)]
     L.qlora_quantize.argtypes = [W, P, c.c_int, P]
     L.qlora_merge_requantize.argtypes = [W, P, P, c.c_int, c.c_float, W, P, P]
+    L.qlora_loftq_workspace_size.argtypes = [c.c_int64, c.c_int64, c.c_int]
+    L.qlora_loftq_workspace_size.restype = c.c_size_t
+    L.qlora_loftq.argtypes = [P, W, c.c_int, c.c_float, c.c_int, c.c_int, c.c_uint64, P, P, P, P,
+                              P, c.c_size_t, P]
     L.qlora_status_string.argtypes = [c.c_int]
     L.qlora_status_string.restype = c.c_char_p
     L.qlora_build_info.restype = c.c_char_p
@@ -81,7 +86,7 @@ def _load():
     for name in ("qlora_workspace_init", "qlora_linear_fwd", "qlora_linear_bwd",
                  "qlora_grouped_fwd", "qlora_grouped_bwd", "qlora_get_device_status",
                  "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_debug_decode_rate",
-                 "qlora_quantize", "qlora_merge_requantize",
+                 "qlora_quantize", "qlora_merge_requantize", "qlora_loftq",
                  "qlora_profile_enable",
                  "qlora_profile_reset", "qlora_profile_read"):
         getattr(L, name).restype = c.c_int
@@ -219,6 +224,29 @@ def qlora_merge_requantize(W: Weight, A, B, r, scale, W_out: Weight, merged, str
     """W_out = Q(deq(W) + scale B A); the merged fp32 values land in `merged` [N,K]."""
     _check(lib.qlora_merge_requantize(W.ref, _p(A), _p(B), int(r), float(scale), W_out.ref,
                                       _p(merged), _stream(stream)), "qlora_merge_requantize")
+
+
+def qlora_loftq_workspace_size(N, K, r):
+    return int(lib.qlora_loftq_workspace_size(int(N), int(K), int(r)))
+
+
+def qlora_loftq(W_float, Q: Weight, r, scale, iters=5, power_iters=4, seed=0, A=None, B=None,
+                errs=None, sigma=None, work=None, stream=None):
+    """LoftQ initialisation: Q receives the last quantisation; returns (A [r,K] bf16, B [N,r]
+    bf16, errs [iters+1] fp32, sigma [r] fp32), all device tensors."""
+    N, K = Q.N, Q.K
+    dev = W_float.device
+    A = torch.empty((r, K), dtype=torch.bfloat16, device=dev) if A is None else A
+    B = torch.empty((N, r), dtype=torch.bfloat16, device=dev) if B is None else B
+    errs = torch.empty(iters + 1, dtype=torch.float32, device=dev) if errs is None else errs
+    sigma = torch.empty(r, dtype=torch.float32, device=dev) if sigma is None else sigma
+    if work is None:
+        work = torch.empty(max(1, qlora_loftq_workspace_size(N, K, r)), dtype=torch.uint8,
+                           device=dev)
+    _check(lib.qlora_loftq(_p(W_float), Q.ref, int(r), float(scale), int(iters), int(power_iters),
+                           int(seed), _p(A), _p(B), _p(errs), _p(sigma), _p(work), work.numel(),
+                           _stream(stream)), "qlora_loftq")
+    return A, B, errs, sigma
 
 
 def qlora_debug_decode_rate(fmt, iters=2000):

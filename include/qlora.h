@@ -240,6 +240,31 @@ QLORA_API qlora_status_t qlora_merge_requantize(const qlora_weight_t* W, const v
                                                 const qlora_weight_t* W_out, float* merged,
                                                 qlora_stream_t stream);
 
+/* LoftQ initialisation of the adapter for a quantised base ("Training LLMs on a Budget: LoRA,
+ * QLoRA, and LoftQ", §4 "The algorithm: alternating quantization and SVD"): starting from
+ * B A = 0, `iters` rounds of  Q_t = quantise(W - scale B_{t-1} A_{t-1})  (the rules of
+ * qlora_quantize, in Q's format)  then  scale B_t A_t = the rank-r truncated SVD U_r S_r V_r^T of
+ * R_t = W - deq(Q_t), split as B_t = U_r sqrt(S_r / scale), A_t = sqrt(S_r / scale) V_r^T.
+ *   W       [N,K] fp32, device (N, K from Q); not modified.
+ *   Q       receives the last quantisation Q_iters (its storage is written).
+ *   A_out   [r,K] bf16, B_out [N,r] bf16 (device): A_iters, B_iters rounded to bf16 once at the end.
+ *   errs    [iters+1] fp32, device: errs[0] = ||W - deq(Q_1)||_F (the plain QLoRA start, B = 0),
+ *           errs[t] = ||W - deq(Q_t) - scale B_t A_t||_F with the unrounded factors.
+ *   sigma   [r] fp32, device, or NULL: the top r singular values of the last residual.
+ *   1 <= r <= min(96, N, K); 1 <= iters <= 64; scale > 0; N*K <= 2^31.
+ * The SVD is randomized subspace iteration (l = min(r + 16, 96, N, K) columns, a Rademacher test
+ * matrix from SplitMix64(seed), `power_iters` in [0, 16] rounds of R R^T, Rayleigh-Ritz) in fp32
+ * with fp64 l x l eigenproblems: exact for a residual of rank <= l, and within the usual
+ * randomized-SVD bound otherwise (more power iterations bring it closer to the truncated SVD).
+ * Deterministic for a given seed.  work: device scratch of qlora_loftq_workspace_size(N, K, r)
+ * bytes (256-byte aligned; about 4 N K bytes).  Async on stream.  Errors as qlora_quantize, plus
+ * QLORA_ERR_WORKSPACE for a short workspace. */
+QLORA_API size_t qlora_loftq_workspace_size(int64_t N, int64_t K, int r);
+QLORA_API qlora_status_t qlora_loftq(const float* W, const qlora_weight_t* Q, int r, float scale,
+                                     int iters, int power_iters, uint64_t seed, void* A_out,
+                                     void* B_out, float* errs, float* sigma, void* work,
+                                     size_t work_bytes, qlora_stream_t stream);
+
 /* Benchmark support: measure the decode throughput of the layer's own dequant stage (the code
  * every GEMM kernel decodes the 4-bit weight with) on every SM -- 256 threads per SM, each
  * decoding `iters` 64-element items into a shared-memory operand tile -- and return the mean

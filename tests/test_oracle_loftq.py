@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 
 from oracle import oracle as O
+from loftq_cases import planted
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden", "loftq_3x3.txt")
 
@@ -65,30 +66,9 @@ def test_loftq_svd_step_is_eckart_young():
     assert res["errs"][1] < res["errs"][0]
 
 
-def _planted(N, K, rank, seed):
-    """W = D + L: D an NF4 grid point (every 64-block's column 0 at level +1 with a bf16-exact
-    absmax, the other codes strictly inside), L rank-`rank`, zero on column 0 of every block and
-    below 1/64 of the block's absmax -- too small to move a code or the absmax."""
-    rng = np.random.default_rng(seed)
-    codes = rng.integers(1, 15, size=(N, K), dtype=np.uint8)
-    codes[:, ::64] = 15
-    a = rng.uniform(0.01, 0.04, size=(N, K // 64)).astype(np.float32)
-    a = ((a.view(np.uint32) + 0x8000) & 0xFFFF0000).view(np.float32)      # bf16-exact absmax
-    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
-    D = O.dequant("nf4", N, K, packed, a)
-    Df = (D.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    U = rng.standard_normal((N, rank))
-    V = rng.standard_normal((K, rank))
-    V[::64] = 0.0
-    L = U @ V.T
-    L *= (0.01 / 64) / np.abs(L).max()            # |L| < amin / 64 <= a / 64
-    W = (Df + L).astype(np.float32)
-    return W, packed, a, Df, L
-
-
 def test_loftq_planted_nf4_is_recovered():
     N, K, rank = 32, 256, 2
-    W, packed, a, Df, L = _planted(N, K, rank, 7)
+    W, packed, a, Df, L = planted(N, K, rank, 7)
     res = O.loftq(W, r=rank, s=2.0, iters=3, fmt="nf4")
     codes, scales, _, _ = res["stored"]
     assert np.array_equal(codes, packed) and np.array_equal(scales, a)
