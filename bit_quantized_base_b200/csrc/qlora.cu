@@ -887,7 +887,7 @@ qlora_status_t qlora_quantize(const qlora_weight_t* W, const void* v, int v_is_b
                               qlora_stream_t stream) {
   const qlora_status_t st = check_weight(W);
   if (st != QLORA_OK) return st;
-  if (!v || (reinterpret_cast<uintptr_t>(v) & 3u)) return QLORA_ERR_INVALID_ARG;
+  if (!ptr_ok(v)) return QLORA_ERR_INVALID_ARG;
   if (W->fmt == QLORA_FMT_NF4_DQ && W->N * (W->K / 64) > (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   QuantParams p{};
@@ -906,7 +906,7 @@ qlora_status_t qlora_quantize(const qlora_weight_t* W, const void* v, int v_is_b
   const unsigned grid = unsigned((blocks + quant::kBlocksPerCta - 1) / quant::kBlocksPerCta);
   if (W->fmt == QLORA_FMT_NVFP4) {
     if (cudaMemsetAsync(p.tensor_scale, 0, sizeof(float), s) != cudaSuccess) return QLORA_ERR_CUDA;
-    qlora_quant_amax_kernel<<<unsigned(2 * num_sms()), 256, 0, s>>>(
+    qlora_quant_amax_kernel<<<unsigned(8 * num_sms()), 256, 0, s>>>(
         p, reinterpret_cast<unsigned*>(p.tensor_scale));
   }
   switch (W->fmt) {

@@ -41,42 +41,52 @@ __device__ __forceinline__ float e2m1_f32(uint32_t c) {
   return (c & 8u) ? -mag : mag;
 }
 
-// Nearest E2M1 code of x: ties to the even code (mantissa bit 0), magnitude saturating at 6,
-// sign bit only on a non-zero magnitude.
-__device__ __forceinline__ uint32_t e2m1_encode(double x) {
-  const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
-  const double a = fabs(x) < 6.0 ? fabs(x) : 6.0;
+// Division-free comparisons.  The rules compare a binary64 quotient x = fl64(v / d) (d > 0)
+// with the midpoint m of two neighbouring grid values.  In every use v has at most 24
+// significant bits, d at most 28 and m at most 25, so the product m d is exact in binary64; and
+// fl64(v / d) cannot round onto m unless v / d equals m, because a non-zero v - m d is at least
+// 2^-49 of m d in magnitude, while rounding moves a quotient by at most 2^-53 of it.  So
+// "x > m" has the outcome of "v > m d", and "x == m" that of "v == m d".
+
+// Nearest E2M1 code of v / d (d > 0, at most 28 significant bits): ties to the even code
+// (mantissa bit 0), magnitude saturating at 6, sign bit only on a non-zero magnitude.
+__device__ __forceinline__ uint32_t e2m1_encode_scaled(float v, double d) {
+  constexpr double mids[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
+  const double a = fabs(double(v));
   uint32_t c = 0;
 #pragma unroll
   for (uint32_t i = 0; i < 7; ++i) {
-    const double mid = __dmul_rn(0.5, __dadd_rn(mag[i], mag[i + 1]));
-    if (a > mid || (a == mid && (i & 1u))) c = i + 1;
+    const double t = mids[i] * d;
+    if (a > t || (a == t && (i & 1u))) c = i + 1;
   }
-  return (c != 0u && signbit(x)) ? (c | 8u) : c;
+  return (c != 0u && signbit(v)) ? (c | 8u) : c;
 }
 
-// Nearest positive E4M3 code of q >= 0, ties to the even code, saturating at 448.
+// Nearest positive E4M3 code of q >= 0, ties to the even code, saturating at 448.  "q is past
+// the midpoint below code c" (strictly, or on it with c even) holds for c = 1..best and for no
+// larger c, so a binary search over c finds best in 7 steps.
 __device__ __forceinline__ uint32_t e4m3_encode_pos(double q) {
-  uint32_t best = 0;
-  double lo = 0.0;
-  for (uint32_t c = 1; c <= 0x7Eu; ++c) {
-    const double hi = double(e4m3_f32(c));
-    const double mid = __dmul_rn(0.5, __dadd_rn(lo, hi));
-    if (q > mid || (q == mid && (c & 1u) == 0u)) best = c;
-    lo = hi;
+  uint32_t lo = 0, hi = 0x7Fu;
+#pragma unroll
+  for (int it = 0; it < 7; ++it) {
+    const uint32_t c = (lo + hi) >> 1;
+    const double mid = 0.5 * (double(e4m3_f32(c - 1u)) + double(e4m3_f32(c)));
+    if (q > mid || (q == mid && (c & 1u) == 0u)) lo = c;
+    else hi = c;
   }
-  return best;
+  return lo;
 }
 
-// NF4 code of v against absmax a > 0.
+// NF4 code of v against absmax a > 0: the number of level midpoints m with m < v / a, as
+// m a < v (exact, see above).  The midpoints are compile-time constants (the sum of two
+// neighbouring binary32 levels is exact in binary64).
 __device__ __forceinline__ uint32_t nf4_encode(float v, float a) {
-  const double x = __ddiv_rn(double(v), double(a));
+  const double vv = double(v), aa = double(a);
   uint32_t c = 0;
 #pragma unroll
   for (int i = 0; i < 15; ++i) {
-    const double mid =
-        __dmul_rn(0.5, __dadd_rn(double(nf4_level_dev(i)), double(nf4_level_dev(i + 1))));
-    if (mid < x) c = uint32_t(i + 1);
+    const double mid = 0.5 * (double(nf4_level_dev(i)) + double(nf4_level_dev(i + 1)));
+    if (mid * aa < vv) c = uint32_t(i + 1);
   }
   return c;
 }
@@ -91,17 +101,30 @@ struct QuantParams {
   int N, K;
 };
 
-__device__ __forceinline__ float quant_load(const QuantParams& p, size_t i) {
-  return p.v_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.v)[i])
-                  : reinterpret_cast<const float*>(p.v)[i];
-}
 
-// max |v| over the tensor into *bits (non-negative binary32 values order like their bit patterns)
+// max |v| over the tensor into *bits (non-negative binary32 values order like their bit
+// patterns); 16-byte loads (N K is a multiple of 64, v 16-byte aligned).
 __global__ void __launch_bounds__(256) qlora_quant_amax_kernel(const QuantParams p, unsigned* bits) {
   const size_t n = size_t(p.N) * size_t(p.K);
+  const size_t stride = size_t(gridDim.x) * blockDim.x;
   float a = 0.0f;
-  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += size_t(gridDim.x) * blockDim.x)
-    a = fmaxf(a, fabsf(quant_load(p, i)));
+  if (p.v_bf16) {
+    const uint4* src = reinterpret_cast<const uint4*>(p.v);
+    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n / 8; i += stride) {
+      const uint4 q = src[i];
+      const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h)
+        a = fmaxf(a, fmaxf(fabsf(__uint_as_float(u[h] << 16)),
+                           fabsf(__uint_as_float(u[h] & 0xFFFF0000u))));
+    }
+  } else {
+    const float4* src = reinterpret_cast<const float4*>(p.v);
+    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n / 4; i += stride) {
+      const float4 q = src[i];
+      a = fmaxf(a, fmaxf(fmaxf(fabsf(q.x), fabsf(q.y)), fmaxf(fabsf(q.z), fabsf(q.w))));
+    }
+  }
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
   if ((threadIdx.x & 31) == 0) atomicMax(bits, __float_as_uint(a));
 }
@@ -127,11 +150,37 @@ qlora_quant_encode_kernel(const QuantParams p) {
   const size_t base = n * size_t(p.K) + size_t(b) * BS;
   float v[BS];
   float amax = 0.0f;
+  if (have) {
+    if (p.v_bf16) {                          // 8 bf16 per 16-byte load
+      const uint4* src = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const __nv_bfloat16*>(p.v) + base);
 #pragma unroll
-  for (int i = 0; i < BS; ++i) {
-    v[i] = have ? quant_load(p, base + i) : 0.0f;
-    amax = fmaxf(amax, fabsf(v[i]));
+      for (int w = 0; w < BS / 8; ++w) {
+        const uint4 q = src[w];
+        const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          v[8 * w + 2 * h] = __uint_as_float(u[h] << 16);
+          v[8 * w + 2 * h + 1] = __uint_as_float(u[h] & 0xFFFF0000u);
+        }
+      }
+    } else {                                 // 4 fp32 per 16-byte load
+      const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.v) + base);
+#pragma unroll
+      for (int w = 0; w < BS / 4; ++w) {
+        const float4 q = src[w];
+        v[4 * w] = q.x;
+        v[4 * w + 1] = q.y;
+        v[4 * w + 2] = q.z;
+        v[4 * w + 3] = q.w;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < BS; ++i) v[i] = 0.0f;
   }
+#pragma unroll
+  for (int i = 0; i < BS; ++i) amax = fmaxf(amax, fabsf(v[i]));
   uint32_t packed[BS / 8];
 #pragma unroll
   for (int w = 0; w < BS / 8; ++w) packed[w] = 0u;
@@ -169,15 +218,15 @@ qlora_quant_encode_kernel(const QuantParams p) {
     if (have) static_cast<uint8_t*>(p.scales)[f] = uint8_t(e);
     const double sc = ldexp(1.0, int(e) - 127);
 #pragma unroll
-    for (int i = 0; i < BS; ++i) put(i, e2m1_encode(__ddiv_rn(double(v[i]), sc)));
+    for (int i = 0; i < BS; ++i) put(i, e2m1_encode_scaled(v[i], sc));
   } else {
     const float T = *p.tensor_scale;
     const float st = T > 0.0f ? __double2float_rn(__ddiv_rn(double(T), 2688.0)) : 1.0f;
     const uint32_t sb = e4m3_encode_pos(__ddiv_rn(double(amax), __dmul_rn(6.0, double(st))));
     if (have) static_cast<uint8_t*>(p.scales)[f] = uint8_t(sb);
-    const double d = __dmul_rn(double(e4m3_f32(sb)), double(st));
+    const double d = double(e4m3_f32(sb)) * double(st);   // exact: 4 x 24 significant bits
 #pragma unroll
-    for (int i = 0; i < BS; ++i) put(i, d > 0.0 ? e2m1_encode(__ddiv_rn(double(v[i]), d)) : 0u);
+    for (int i = 0; i < BS; ++i) put(i, d > 0.0 ? e2m1_encode_scaled(v[i], d) : 0u);
   }
   if (have) {
     uint8_t* dst = p.codes + n * size_t(p.K / 2) + size_t(b) * (BS / 2);

@@ -212,7 +212,7 @@ QLORA_API qlora_status_t qlora_debug_wait_timeout(void* ws, size_t ws_bytes, int
  * weight per call: an expert stack is quantised one expert at a time, each with its own slice of
  * the arrays.  Errors: QLORA_ERR_INVALID_ARG for a shape or pointer outside the weight limits
  * every entry point applies (N % 16, K % 64, 16-byte aligned codes and scales) or a v that is
- * NULL or not 4-byte aligned; QLORA_ERR_CUDA for a failed launch.  The pages give no rounding rules; these are the
+ * NULL or not 16-byte aligned; QLORA_ERR_CUDA for a failed launch.  The pages give no rounding rules; these are the
  * library's (the oracle's `oracle_encode` states them the same way):
  *   NF4    absmax = max |v| of the 64-block; code = the number of NF4 level midpoints below
  *          v / absmax (binary64), ties to the lower code; an all-zero block is all code 7.

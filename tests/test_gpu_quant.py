@@ -26,7 +26,8 @@ def _Q():
 
 def _weight_v(N, K, seed):
     """Seeded float weight: N(0, 0.02) rows at scales 2^-3..2^3, with the special blocks the
-    encoders treat apart (a zero block, a zero row, fp32 subnormals, E2M1 midpoints)."""
+    encoders treat apart (a zero block, a zero row, fp32 subnormals, exact NF4 and E2M1
+    midpoints under MXFP4 and NVFP4 scales)."""
     rng = np.random.default_rng(seed)
     v = (rng.standard_normal((N, K)) * 0.02 * np.exp2(rng.integers(-3, 4, size=(N, 1)))).astype(np.float32)
     v[1, 64:128] = 0.0                                        # one zero block in every format
@@ -35,6 +36,20 @@ def _weight_v(N, K, seed):
     v[4, :32] = 0.0                                           # MXFP4 block with amax 4 (e = 127)
     v[4, 0] = 4.0
     v[4, 1:13] = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.75, -2.5, -0.25, 7.0, -7.5]
+    # NF4 block with absmax 1 holding the four NF4 level midpoints that binary32 represents
+    # exactly: each is a tie, which goes to the lower code
+    v[5, :64] = 0.0
+    v[5, 0] = 1.0
+    v[5, 1:5] = [-0.45999518036842346, -0.04552498832345009, 0.03979015722870827,
+                 0.861478328704834]
+    # NVFP4: the tensor max 1344 (s_t = 1344 / 2688 = 0.5) and a 16-block with amax 3 (block
+    # scale exactly 1, element step d = 0.5) holding every E2M1 midpoint times d: ties to even
+    v[7, 32:48] = 0.0
+    v[7, 32] = 1344.0
+    v[6, :16] = 0.0
+    v[6, 0] = 3.0
+    v[6, 1:15] = [0.125, 0.375, 0.625, 0.875, 1.25, 1.75, 2.5,
+                  -0.125, -0.375, -0.625, -0.875, -1.25, -1.75, -2.5]
     return v
 
 
@@ -78,6 +93,14 @@ def test_quantize_matches_oracle(fmt, shape):
     _assert_same_encoding(fmt, _stored(W), want)
     if fmt == "nf4dq" and shape == (64, 1024):
         assert want[3][1] == 1.0
+    c = want[0]
+    lo, hi = c & 15, c >> 4
+    if fmt == "nf4":          # ties to the lower code: levels 2, 6, 7, 14 (not 3, 7, 8, 15)
+        assert [int(x) for x in (hi[5, 0], lo[5, 1], hi[5, 1], lo[5, 2])] == [2, 6, 7, 14]
+    if fmt == "nvfp4":        # ties to the even E2M1 code; -0.125 rounds to magnitude 0: +0
+        assert want[2] == 0.5 and int(want[1][6, 0]) == 0x38
+        got = [int(x) for x in np.stack([lo[6, :8], hi[6, :8]], 1).reshape(-1)[1:15]]
+        assert got == [0, 2, 2, 4, 4, 6, 6, 0, 10, 10, 12, 12, 14, 14]
 
 
 @pytest.mark.parametrize("fmt", FMTS)
