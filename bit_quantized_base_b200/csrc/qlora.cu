@@ -1057,14 +1057,18 @@ struct LoftqRun {
     p.s = s;
     loftq_jacobi_kernel<<<1, loftq::kJacobiThreads, loftq::jacobi_smem(l), st>>>(p);
   }
-  // X [rows, l] <- a basis of its column space by SVQB; X and X2 swap.  Two passes make it
-  // orthonormal to fp32 precision (the basis Rayleigh-Ritz uses); one keeps the power iteration's
-  // intermediate bases well conditioned, which is all they need.
-  void orth(float*& X, float*& X2, int64_t rows, int passes) const {
-    for (int pass = 0; pass < passes; ++pass) {
+  // X [rows, l] <- a basis of its column space; X and X2 swap.  orthonormal: two SVQB passes
+  // (orthonormal to fp32 precision, rank deficiency dropped: the basis Rayleigh-Ritz uses);
+  // otherwise one shifted Cholesky QR step (a well-conditioned intermediate basis).
+  void orth(float*& X, float*& X2, int64_t rows, bool orthonormal) const {
+    for (int pass = 0; pass < (orthonormal ? 2 : 1); ++pass) {
       loftq_gemm<true, false>(X, l, X, l, nullptr, l, l, l, rows, at<float>(L.part),
                               at<double>(L.G), st);
-      jacobi(0);
+      if (orthonormal)
+        jacobi(0);
+      else
+        loftq_chol_kernel<<<1, loftq::kJacobiThreads, loftq::chol_smem(l), st>>>(
+            at<double>(L.G), l, at<float>(L.Mx));
       loftq_gemm<false, false>(X, l, at<float>(L.Mx), l, X2, l, int(rows), l, l, nullptr, nullptr,
                                st);
       std::swap(X, X2);
@@ -1079,12 +1083,12 @@ struct LoftqRun {
     float* Z2 = at<float>(L.Z2);
     float* part = at<float>(L.part);
     loftq_gemm<false, false>(R, K, at<float>(L.omega), l, Y, l, int(N), l, K, part, nullptr, st);
-    orth(Y, Y2, N, power_iters == 0 ? 2 : 1);
+    orth(Y, Y2, N, power_iters == 0);
     for (int q = 0; q < power_iters; ++q) {
       loftq_gemm<true, false>(R, K, Y, l, Z, l, int(K), l, N, part, nullptr, st);
-      orth(Z, Z2, K, 1);
+      orth(Z, Z2, K, false);
       loftq_gemm<false, false>(R, K, Z, l, Y, l, int(N), l, K, part, nullptr, st);
-      orth(Y, Y2, N, q + 1 == power_iters ? 2 : 1);
+      orth(Y, Y2, N, q + 1 == power_iters);
     }
     loftq_gemm<true, false>(R, K, Y, l, Z, l, int(K), l, N, part, nullptr, st);
     loftq_gemm<true, false>(Z, l, Z, l, nullptr, l, l, l, K, part, at<double>(L.G), st);
@@ -1135,7 +1139,9 @@ qlora_status_t qlora_loftq(const float* W, const qlora_weight_t* Q, int r, float
   const int dev = current_device();
   if (dev >= 0 && dev < kMaxDevices && !attr_done[dev]) {
     if (cudaFuncSetAttribute(loftq_jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(loftq::jacobi_smem(loftq::kMaxL))) != cudaSuccess)
+                             int(loftq::jacobi_smem(loftq::kMaxL))) != cudaSuccess ||
+        cudaFuncSetAttribute(loftq_chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(loftq::chol_smem(loftq::kMaxL))) != cudaSuccess)
       return QLORA_ERR_CUDA;
     attr_done[dev] = true;
   }

@@ -11,8 +11,9 @@
 // of l = r + 16 columns, `power_iters` rounds of R R^T with the basis re-orthonormalised between
 // products, then the small l x l eigenproblem of Z^T Z (Z = R^T Qb).  Every basis is made
 // orthonormal by SVQB (Stathopoulos and Wu, 2002): X <- X P diag(lambda^-1/2) from the eigen-pairs
-// of X^T X, columns whose lambda is below 1e-10 of the largest dropped (set to zero); twice for
-// the basis Rayleigh-Ritz uses, once for the power iteration's intermediate bases.
+// of X^T X, columns whose lambda is below 1e-10 of the largest dropped (set to zero), twice; the
+// power iteration's intermediate bases only need to stay well conditioned and take one shifted
+// Cholesky QR step instead.
 // The l x l symmetric eigenproblems are cyclic Jacobi (Golub and Van Loan, "Matrix
 // Computations", §8.5) in fp64 in one CTA, with round-robin pairs so that l/2 rotations run at
 // once.  The tall products are fp32 SIMT GEMMs (64 x 128 tiles, fixed-order split reductions);
@@ -31,6 +32,7 @@ constexpr int kNormBlocks = 592;
 constexpr double kDropRel = 1e-10;   // SVQB / Ritz: eigenvalues below this share of the largest
 __host__ __device__ constexpr int jacobi_pad(int l) { return (l + 1) & ~1; }
 // Row stride L + 1 (odd): a warp walking down a column of doubles touches distinct banks.
+__host__ __device__ constexpr size_t chol_smem(int l) { return size_t(l) * (l + 1) * sizeof(double); }
 __host__ __device__ constexpr size_t jacobi_smem(int l) {
   return size_t(2) * jacobi_pad(l) * (jacobi_pad(l) + 1) * sizeof(double);
 }
@@ -286,6 +288,71 @@ __global__ void __launch_bounds__(loftq::kJacobiThreads) loftq_jacobi_kernel(con
       p.Ca[j * l + row] = keep ? float(x / sqrt(double(p.s) * sig)) : 0.0f;
       if (row == 0) p.sigma[j] = float(sig);
     }
+  }
+}
+
+// Shifted Cholesky QR step for the power iteration's intermediate bases (Fukaya, Kannan,
+// Nakatsukasa, Yamamoto, Yanagisawa, "Shifted Cholesky QR for computing the QR factorization of
+// ill-conditioned matrices", 2020): G + delta I = L L^T with delta = 1e-5 of G's largest
+// diagonal entry, M = L^-T, so that X M has nearly orthonormal columns; directions of X whose
+// energy is below delta come out damped, which an intermediate basis can afford (the basis that
+// Rayleigh-Ritz uses is made by SVQB).  A pivot that the shift does not keep positive drops its
+// column (M's column zero); an all-zero G gives M = 0.  fp64, one CTA: the factorisation is
+// column by column, then each thread solves L x = e_c for one column c.
+__global__ void __launch_bounds__(loftq::kJacobiThreads) loftq_chol_kernel(const double* G, int l,
+                                                                          float* M) {
+  using namespace loftq;
+  extern __shared__ double csm[];
+  const int S = l + 1;                    // padded stride: column walks spread over banks
+  double* Lm = csm;                       // [l, S], lower triangle
+  __shared__ double delta;
+  __shared__ int dropped[kMaxL];
+  for (int i = threadIdx.x; i < l * l; i += blockDim.x) Lm[(i / l) * S + i % l] = G[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double dmax = 0.0;
+    for (int i = 0; i < l; ++i) dmax = fmax(dmax, Lm[i * S + i]);
+    delta = 1e-5 * dmax;
+  }
+  __syncthreads();
+  if (!(delta > 0.0)) {
+    for (int i = threadIdx.x; i < l * l; i += blockDim.x) M[i] = 0.0f;
+    return;
+  }
+  for (int i = threadIdx.x; i < l; i += blockDim.x) Lm[i * S + i] += delta;
+  __syncthreads();
+  for (int j = 0; j < l; ++j) {
+    const double d = Lm[j * S + j];
+    const bool drop = !(d > 0.5 * delta);
+    const double piv = drop ? 0.0 : sqrt(d);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      dropped[j] = drop;
+      Lm[j * S + j] = drop ? 1.0 : piv;
+    }
+    for (int i = j + 1 + threadIdx.x; i < l; i += blockDim.x)
+      Lm[i * S + j] = drop ? 0.0 : Lm[i * S + j] / piv;
+    __syncthreads();
+    const int m = l - j - 1;              // trailing update of the lower triangle
+    for (int t = threadIdx.x; t < m * m; t += blockDim.x) {
+      const int i = j + 1 + t / m, k = j + 1 + t % m;
+      if (k <= i) Lm[i * S + k] -= Lm[i * S + j] * Lm[k * S + j];
+    }
+    __syncthreads();
+  }
+  // column c of L^-1 by forward substitution; M = L^-T, i.e. M[i][c] = (L^-1)[c][i]
+  for (int c = threadIdx.x; c < l; c += blockDim.x) {
+    double x[kMaxL];
+    for (int i = 0; i < l; ++i) {
+      if (i < c || dropped[i]) {
+        x[i] = 0.0;
+        continue;
+      }
+      double acc = i == c ? 1.0 : 0.0;
+      for (int k = c; k < i; ++k) acc -= Lm[i * S + k] * x[k];
+      x[i] = acc / Lm[i * S + i];
+    }
+    for (int i = 0; i < l; ++i) M[c * l + i] = float(x[i]);
   }
 }
 
