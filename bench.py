@@ -224,7 +224,10 @@ class NvmlSampler:
 
 
 # ------------------------------------------------------------------------------- own arm
-def dist_setup(args):
+def dist_setup(args, backend="nccl"):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE).  The ranks are
+    independent replicas: the process group carries only the barrier and the max-over-ranks of the
+    timings.  backend "gloo" runs the same host logic without a GPU."""
     import torch
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -232,10 +235,13 @@ def dist_setup(args):
     if ws > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return ws, rank, local
 
@@ -247,13 +253,21 @@ def barrier(ws):
 
 
 def max_over_ranks(ws, x):
+    """The largest x over all ranks (timings: the job ends when its slowest rank does)."""
     if ws == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(ws_n, flops_per_step, steps, ms_max):
+    """Whole-job TFLOP/s: every rank runs `steps` steps of `flops_per_step`; the time is the
+    slowest rank's."""
+    return ws_n * flops_per_step * steps / (ms_max * 1e-3) / 1e12
 
 
 def short_batch_sweep(Q, torch, p, Ws, X, dY, A, B, peaks):
@@ -578,7 +592,7 @@ def run_own(args):
     Q.qlora_profile_enable(False)
     ms_step = ms_total / args.steps
     fl = flops(M, N, K, r)
-    value = ws_n * fl * args.steps / (ms_total * 1e-3) / 1e12
+    value = job_value(ws_n, fl, args.steps, ms_total)
 
     if Q.qlora_get_device_status(ws) != 0:
         raise RuntimeError("device status after the timed region: %d" % Q.qlora_get_device_status(ws))
@@ -656,7 +670,7 @@ def run_own(args):
     e1.record()
     e1.synchronize()
     e2e_ms = max_over_ranks(ws_n, e0.elapsed_time(e1))
-    e2e = {"value": round(ws_n * fl * e2e_steps / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+    e2e = {"value": round(job_value(ws_n, fl, e2e_steps, e2e_ms), 2), "unit": "TFLOP/s",
            "h2d_bytes_per_step": int((hX.numel() + hdY.numel()) * 2),
            "d2h_bytes_per_step": int((hdA.numel() + hdB.numel()) * 2),
            "ms_per_step": round(e2e_ms / e2e_steps, 4),

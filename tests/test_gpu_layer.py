@@ -184,6 +184,7 @@ CASES = [
     ("nvfp4", 200, 768, 4096, 8),
     ("nf4", 128, 4096, 512, 32),
     ("mxfp4", 2, 16, 64, 8),
+    ("nvfp4", 96, 528, 704, 32),
     # 76 pair tiles on 74 pairs: the last wave's tiles run split in two 256-row tiles (fwd, dX)
     ("nf4", 1000, 9728, 128, 8),
     ("mxfp4", 1024, 128, 9728, 16),
