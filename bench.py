@@ -467,7 +467,7 @@ def grouped_moe(Q, torch, synth, peaks):
     """One fwd+bwd of each MoE expert projection (64 experts, MXFP4, Zipf top-8 routing of 16384
     tokens): TFLOP/s.  Timing inputs: seeded random stored codes with a realistic E8M0 scale range
     and seeded normal activations generated on the device (values do not change the timing)."""
-    cfg = synth.CONFIGS[5]
+    cfg = synth.WORKLOADS["moe64_mxfp4"]
     offs = synth.moe_routing(cfg)
     E, r, s = cfg.experts, cfg.r, cfg.scale
     M = int(offs[-1])
@@ -530,8 +530,8 @@ def run_own(args):
     from bit_quantized_base_b200 import synth
 
     ws_n, rank, local = dist_setup(args)
-    cfg = synth.CONFIGS[2]
-    p = synth.layer_inputs(2)
+    cfg = synth.WORKLOADS["llama3_8b_up_nf4"]
+    p = synth.layer_inputs("llama3_8b_up_nf4")
     fmt, M, N, K, r, s = p["fmt"], p["M"], p["N"], p["K"], p["r"], p["s"]
     ncopy = 3
     Ws = [Q.weight_from_numpy(fmt, p["codes"], p["scales"], p["tensor_scale"]) for _ in range(ncopy)]
@@ -691,7 +691,7 @@ def run_own(args):
     sweep = None
     if not args.no_sweep:
         sweep = {"nf4_up_14336x4096": short_batch_sweep(Q, torch, p, Ws, Xs[0], dYs[0], A, B, peaks)}
-        p3 = synth.layer_inputs(3, M=256)
+        p3 = synth.layer_inputs("llama3_70b_gate_mxfp4", M=256)
         sweep["mxfp4_gate_28672x8192"] = short_batch_sweep(Q, torch, p3, None, None, None, None, None,
                                                            peaks)
         del p3
@@ -782,7 +782,7 @@ def run_reference(args):
         return
     from bit_quantized_base_b200 import synth
     from oracle import oracle as O
-    p = synth.layer_inputs(2)
+    p = synth.layer_inputs("llama3_8b_up_nf4")
     N, K, r = p["N"], p["K"], p["r"]
     # each step: the oracle on a bounded sample of the batch, sized so that warm-up + steps stay
     # within a few minutes

@@ -5,9 +5,11 @@ their stored 4-bit form (packed codes + block scales).  It holds none of the lay
 it never decodes a weight and never computes an output, so no expected value can come from here.
 To turn a float weight matrix into stored codes it carries simple encoders (quantisers); those sit
 outside the layer (the layer only ever decodes), and whatever codes they pick are valid inputs
-that the CUDA path and the oracle then decode independently.
+that the CUDA path and the oracle then decode independently.  These encoders are not the
+library's quantiser (qlora_quantize, tested against the oracle's own encoder) and need not agree
+with it.
 
-All draws use numpy PCG64 with seed = 1000*cfg + 10*proj + tensor_id
+All draws use numpy PCG64 with seed = 1000*seed_id + 10*proj + tensor_id (seed_id: the workload's)
 (tensor ids: X=1, W=2, A=3, B=4, dY=5, routing=6), then round to bf16 (round-to-nearest-even).
 
 Layouts (row-major, K contiguous):
@@ -33,8 +35,8 @@ BLOCK = {"nf4": 64, "mxfp4": 32, "nvfp4": 16}
 TID = {"X": 1, "W": 2, "A": 3, "B": 4, "dY": 5, "routing": 6}
 
 
-def rng_for(cfg: int, tensor: str, proj: int = 0) -> np.random.Generator:
-    return np.random.Generator(np.random.PCG64(1000 * cfg + 10 * proj + TID[tensor]))
+def rng_for(seed_id: int, tensor: str, proj: int = 0) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(1000 * seed_id + 10 * proj + TID[tensor]))
 
 
 # ---------------------------------------------------------------------------------------------
@@ -250,7 +252,7 @@ class Proj:
 
 @dataclass
 class Config:
-    cfg: int
+    seed_id: int
     fmt: str
     M: int
     projs: list
@@ -272,19 +274,19 @@ class Config:
         return self.alpha / self.r
 
 
-CONFIGS = {
-    1: Config(1, "nf4", 256, [Proj("proj", 1024, 1024)], 16, 32.0, dy_std=1.0,
+WORKLOADS = {
+    "nf4_1024x1024": Config(1, "nf4", 256, [Proj("proj", 1024, 1024)], 16, 32.0, dy_std=1.0,
               desc="single LoRA linear, NF4, M=256, N=K=1024, r=16"),
-    2: Config(2, "nf4", 4096, [Proj("up", 14336, 4096)], 64, 128.0,
+    "llama3_8b_up_nf4": Config(2, "nf4", 4096, [Proj("up", 14336, 4096)], 64, 128.0,
               desc="Llama-3-8B-shaped MLP up-proj, NF4, M=4096, N=14336, K=4096, r=64"),
-    3: Config(3, "mxfp4", 8192, [Proj("gate", 28672, 8192)], 16, 32.0, w_dist="t5",
+    "llama3_70b_gate_mxfp4": Config(3, "mxfp4", 8192, [Proj("gate", 28672, 8192)], 16, 32.0, w_dist="t5",
               desc="Llama-3-70B-shaped MLP gate-proj, MXFP4, M=8192, N=28672, K=8192, r=16"),
-    4: Config(4, "nvfp4", 4096,
+    "llama3_70b_layer_nvfp4": Config(4, "nvfp4", 4096,
               [Proj("q", 8192, 8192), Proj("k", 1024, 8192), Proj("v", 1024, 8192),
                Proj("o", 8192, 8192), Proj("gate", 28672, 8192), Proj("up", 28672, 8192),
                Proj("down", 8192, 28672)], 16, 32.0,
               desc="Llama-3-70B-shaped decoder layer, 7 NVFP4 projections, M=4096, r=16"),
-    5: Config(5, "mxfp4", 131072,
+    "moe64_mxfp4": Config(5, "mxfp4", 131072,
               [Proj("gate", 2048, 7168), Proj("up", 2048, 7168), Proj("down", 7168, 2048)],
               8, 16.0, experts=64, tokens=16384, topk=8,
               desc="MoE grouped experts, 64 x {gate,up 2048x7168; down 7168x2048}, MXFP4, "
@@ -298,7 +300,7 @@ def _normal(rng, shape, std):
 
 def make_weight(cfg: Config, proj: int, N: int, K: int, experts: int = 0):
     """Stored weight of projection `proj` ([E,...] stacked when experts > 0)."""
-    rng = rng_for(cfg.cfg, "W", proj)
+    rng = rng_for(cfg.seed_id, "W", proj)
     E = max(experts, 1)
     codes = np.empty((E, N, K // 2), np.uint8)
     scales = None
@@ -322,7 +324,7 @@ def make_weight(cfg: Config, proj: int, N: int, K: int, experts: int = 0):
 
 def make_adapters(cfg: Config, proj: int, N: int, K: int, experts: int = 0):
     E = max(experts, 1)
-    ra, rb = rng_for(cfg.cfg, "A", proj), rng_for(cfg.cfg, "B", proj)
+    ra, rb = rng_for(cfg.seed_id, "A", proj), rng_for(cfg.seed_id, "B", proj)
     bound = 1.0 / math.sqrt(K)   # Kaiming-uniform (a = sqrt 5) bound for fan-in K
     A = to_bf16_bits(ra.uniform(-bound, bound, size=(E, cfg.r, K)).astype(np.float32))
     B = to_bf16_bits(_normal(rb, (E, N, cfg.r), cfg.b_std))
@@ -330,8 +332,8 @@ def make_adapters(cfg: Config, proj: int, N: int, K: int, experts: int = 0):
 
 
 def make_activations(cfg: Config, proj: int, M: int, N: int, K: int):
-    X = to_bf16_bits(_normal(rng_for(cfg.cfg, "X", proj), (M, K), cfg.x_std))
-    dY = to_bf16_bits(_normal(rng_for(cfg.cfg, "dY", proj), (M, N), cfg.dy_std))
+    X = to_bf16_bits(_normal(rng_for(cfg.seed_id, "X", proj), (M, K), cfg.x_std))
+    dY = to_bf16_bits(_normal(rng_for(cfg.seed_id, "dY", proj), (M, N), cfg.dy_std))
     return X, dY
 
 
@@ -339,7 +341,7 @@ def moe_routing(cfg: Config):
     """Per-expert token counts: each token takes `topk` distinct experts by Gumbel-top-k over
     Zipf(s) weights p_e ~ rank_e^-s, ranks assigned by a seeded random permutation.
     Returns int64 offsets [E+1] (exclusive prefix sum, offsets[E] = tokens * topk)."""
-    rng = rng_for(cfg.cfg, "routing")
+    rng = rng_for(cfg.seed_id, "routing")
     E = cfg.experts
     ranks = rng.permutation(E) + 1
     logp = -cfg.zipf * np.log(ranks.astype(np.float64))
@@ -355,10 +357,10 @@ def moe_routing(cfg: Config):
     return offsets
 
 
-def layer_inputs(cfg_id: int, proj: int = 0, M: int | None = None):
+def layer_inputs(name: str, proj: int = 0, M: int | None = None):
     """Inputs of one (non-grouped) projection: dict with fmt, M, N, K, r, s, codes, scales,
     tensor_scale, X, A, B, dY."""
-    cfg = CONFIGS[cfg_id]
+    cfg = WORKLOADS[name]
     p = cfg.projs[proj]
     M = cfg.M if M is None else M
     codes, scales, ts = make_weight(cfg, proj, p.N, p.K)

@@ -25,22 +25,23 @@ def sample_rows(M, n, seed):
     return rows.astype(np.int64)
 
 
-DENSE = [(2, 0), (3, 0)] + [(4, i) for i in range(7)]
+DENSE = ([("llama3_8b_up_nf4", 0), ("llama3_70b_gate_mxfp4", 0)] +
+         [("llama3_70b_layer_nvfp4", i) for i in range(7)])
 
 
-@pytest.mark.parametrize("cfg_id,proj", DENSE,
-                         ids=[f"{synth.CONFIGS[c].fmt}-{synth.CONFIGS[c].projs[p].name}-"
-                              f"{synth.CONFIGS[c].projs[p].N}x{synth.CONFIGS[c].projs[p].K}"
+@pytest.mark.parametrize("name,proj", DENSE,
+                         ids=[f"{synth.WORKLOADS[c].fmt}-{synth.WORKLOADS[c].projs[p].name}-"
+                              f"{synth.WORKLOADS[c].projs[p].N}x{synth.WORKLOADS[c].projs[p].K}"
                               for c, p in DENSE])
-def test_full_size_layer_sampled(cfg_id, proj):
+def test_full_size_layer_sampled(name, proj):
     from oracle import oracle
-    p = synth.layer_inputs(cfg_id, proj)
+    p = synth.layer_inputs(name, proj)
     g = GpuLayer(p)
     Y, T = g.fwd()
     dX, dA, dB = g.bwd(T)
     torch.cuda.synchronize()
     assert g.status() == 0
-    rows = sample_rows(p["M"], 128, 7 + 100 * cfg_id + proj)
+    rows = sample_rows(p["M"], 128, 7 + 100 * synth.WORKLOADS[name].seed_id + proj)
     ref = oracle.layer(p["fmt"], p["M"], p["N"], p["K"], p["r"], p["s"], p["codes"], p["scales"],
                        p["tensor_scale"], p["X"], p["A"], p["B"], p["dY"], rows=rows,
                        want=("Y", "dX", "T", "dA", "dB"))
@@ -52,15 +53,15 @@ def test_full_size_layer_sampled(cfg_id, proj):
     assert_close(to_f64(dB), ref["dB"], "dB")
 
 
-SHORT = [(2, 16), (2, 256), (3, 64)]
+SHORT = [("llama3_8b_up_nf4", 16), ("llama3_8b_up_nf4", 256), ("llama3_70b_gate_mxfp4", 64)]
 
 
-@pytest.mark.parametrize("cfg_id,M", SHORT, ids=[f"{synth.CONFIGS[c].fmt}-M{m}" for c, m in SHORT])
-def test_full_size_weight_short_batch(cfg_id, M):
+@pytest.mark.parametrize("name,M", SHORT, ids=[f"{synth.WORKLOADS[c].fmt}-M{m}" for c, m in SHORT])
+def test_full_size_weight_short_batch(name, M):
     # the full-size weights of the NF4 up-proj and the MXFP4 gate-proj under the short batches of
     # the weight-stream sweep: every output row is checked
     from oracle import oracle
-    p = synth.layer_inputs(cfg_id, 0, M=M)
+    p = synth.layer_inputs(name, 0, M=M)
     g = GpuLayer(p)
     Y, T = g.fwd()
     dX, dA, dB = g.bwd(T)
@@ -77,7 +78,7 @@ def test_full_size_weight_short_batch(cfg_id, M):
 def test_full_size_grouped_sampled(proj):
     from oracle import oracle
     from bit_quantized_base_b200 import qlora as Q
-    cfg = synth.CONFIGS[5]
+    cfg = synth.WORKLOADS["moe64_mxfp4"]
     pr = cfg.projs[proj]
     E, N, K, r, s = cfg.experts, pr.N, pr.K, cfg.r, cfg.scale
     offsets = synth.moe_routing(cfg)
