@@ -791,9 +791,9 @@ def run_reference(args):
     per_step = budget_s / max(1, args.steps + args.warmup)
     rows, cols = 1, N
     if per_step > t1:
-        t4 = _oracle_sample(p, 4)
-        per_row = max((t4 - t1) / 3, 1e-4)
-        rows = int(max(1, min(p["M"], 1 + (per_step - t1) / per_row)))
+        t64 = _oracle_sample(p, 64)
+        per_row = max((t64 - t1) / 63, 1e-4)
+        rows = int(max(1, min(p["M"], 1 + 0.8 * (per_step - t1) / per_row)))
     else:
         # one row costs about the decode of W: narrow the sample to the first output features
         cols = int(max(16, min(N, N * per_step / t1 * 0.8)) // 16 * 16)
