@@ -1,5 +1,7 @@
 """Seeded LoftQ inputs whose answer is known in closed form (shared by the oracle pins and the GPU
-tests; inputs only, no expected value of the method is computed here)."""
+tests).  The planted weight is built with the oracle's decode of seeded codes; the answer a test
+checks -- the seeded codes and absmax, and the seeded low-rank matrix -- is fixed by the seeds,
+not computed by either side."""
 import numpy as np
 
 from oracle import oracle as O
