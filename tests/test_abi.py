@@ -110,3 +110,48 @@ def test_workspace_init_and_status_reject_null(Q):
     assert Q.STATUS[Q.lib.qlora_workspace_init(None, 1 << 20, None)] == "QLORA_ERR_WORKSPACE"
     assert Q.STATUS[Q.lib.qlora_get_device_status(None, None)] == "QLORA_ERR_WORKSPACE"
     assert Q.STATUS[Q.lib.qlora_debug_wait_timeout(0x1000, 1 << 20, 0, None)] == "QLORA_ERR_INVALID_ARG"
+
+
+def test_quantize_rejects_bad_arguments(Q):
+    def rc(W, v):
+        return Q.STATUS[Q.lib.qlora_quantize(W.ref, v, 0, None)]
+    assert rc(_w(Q), 0x1004) == "QLORA_ERR_INVALID_ARG"            # v not 16-byte aligned
+    assert rc(_w(Q), None) == "QLORA_ERR_INVALID_ARG"
+    assert rc(_w(Q, K=100), 0x10000) == "QLORA_ERR_INVALID_ARG"     # K % 64
+    assert rc(_w(Q, fmt="nvfp4"), 0x10000) == "QLORA_ERR_INVALID_ARG"   # no tensor-scale slot
+    assert rc(_w(Q, fmt="nf4dq"), 0x10000) == "QLORA_ERR_INVALID_ARG"   # no second-level scales
+
+
+def test_merge_rejects_bad_arguments(Q):
+    W, Wo = _w(Q), _w(Q, codes=0x3000, scales=0x4000)
+
+    def rc(W_out=Wo, A=0x10000, B=0x20000, r=16, merged=0x30000):
+        return Q.STATUS[Q.lib.qlora_merge_requantize(W.ref, A, B, r, 2.0, W_out.ref, merged, None)]
+    assert rc(r=0) == "QLORA_ERR_INVALID_ARG"
+    assert rc(r=1025) == "QLORA_ERR_INVALID_ARG"
+    assert rc(A=None) == "QLORA_ERR_INVALID_ARG"
+    assert rc(merged=0x30004) == "QLORA_ERR_INVALID_ARG"
+    assert rc(W_out=_w(Q, N=512, codes=0x3000, scales=0x4000)) == "QLORA_ERR_INVALID_ARG"
+
+
+def test_loftq_arguments(Q):
+    N, K = 256, 512
+    assert Q.qlora_loftq_workspace_size(N, K, 0) == 0
+    assert Q.qlora_loftq_workspace_size(N, K, 97) == 0              # above the subspace limit
+    assert Q.qlora_loftq_workspace_size(16, K, 32) == 0             # r > N
+    need = Q.qlora_loftq_workspace_size(N, K, 16)
+    assert need >= 4 * N * K
+    W = _w(Q, N=N, K=K)
+
+    def rc(r=16, scale=2.0, iters=5, power=4, work=0x100000, nbytes=need, errs=0x60000, v=0x70000):
+        return Q.STATUS[Q.lib.qlora_loftq(v, W.ref, r, scale, iters, power, 0, 0x80000, 0x90000,
+                                          errs, None, work, nbytes, None)]
+    assert rc(r=0) == "QLORA_ERR_INVALID_ARG"
+    assert rc(scale=0.0) == "QLORA_ERR_INVALID_ARG"
+    assert rc(scale=float("nan")) == "QLORA_ERR_INVALID_ARG"
+    assert rc(iters=0) == "QLORA_ERR_INVALID_ARG"
+    assert rc(power=17) == "QLORA_ERR_INVALID_ARG"
+    assert rc(work=0x100010) == "QLORA_ERR_INVALID_ARG"             # not 256-byte aligned
+    assert rc(errs=None) == "QLORA_ERR_INVALID_ARG"
+    assert rc(v=0x70008) == "QLORA_ERR_INVALID_ARG"
+    assert rc(nbytes=need - 1) == "QLORA_ERR_WORKSPACE"
