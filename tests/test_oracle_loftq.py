@@ -82,3 +82,29 @@ def test_loftq_planted_nf4_is_recovered():
     # a rank below the planted one cannot recover it: the error stays at the dropped factor
     low = O.loftq(W, r=rank - 1, s=2.0, iters=1, fmt="nf4")
     assert low["errs"][1] > 1e-3 * low["errs"][0]
+
+
+def test_loftq_planted_mxfp4_is_recovered():
+    # the same construction on the MXFP4 grid: every 32-block holds +6 (code 7) in column 0 at
+    # scale 2^(e-127), so its exponent stays e; the other codes lie in +-{0.5 .. 4} and L, zero on
+    # column 0, stays below a quarter of the smallest step (0.5 x scale): quantising W gives D back
+    rng = np.random.default_rng(8)
+    N, K, rank = 16, 256, 3
+    mag = rng.integers(1, 7, size=(N, K))                   # E2M1 magnitude codes 1..6
+    sign = rng.integers(0, 2, size=(N, K)) << 3
+    codes = (mag | sign).astype(np.uint8)
+    codes[:, ::32] = 7
+    e = rng.integers(118, 124, size=(N, K // 32)).astype(np.uint8)
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    D = (O.dequant("mxfp4", N, K, packed, e).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    V = rng.standard_normal((K, rank))
+    V[::32] = 0.0
+    L = rng.standard_normal((N, rank)) @ V.T
+    L *= 0.1 * np.exp2(float(e.min()) - 127) / np.abs(L).max()  # < 0.125 x the smallest scale
+    W = (D + L).astype(np.float32)
+    res = O.loftq(W, r=rank, s=1.0, iters=2, fmt="mxfp4")
+    c, sc, _, _ = res["stored"]
+    assert np.array_equal(c, packed) and np.array_equal(sc, e)
+    resid = np.linalg.norm(W.astype(np.float64) - D - L)
+    assert res["errs"][1] <= resid * (1 + 1e-9) and res["errs"][2] <= resid * (1 + 1e-9)
+    assert np.allclose(res["B"] @ res["A"], L, rtol=0, atol=1e-4 * np.abs(L).max())
