@@ -269,5 +269,69 @@ def loftq(W, r, s, iters=5, fmt="nf4", quant=None):
     return {"Q": Q, "stored": stored, "A": A, "B": B, "sigma": sig, "errs": errs}
 
 
+def _e4m3_table():
+    return np.array([decode_e4m3(c) for c in range(0x7F)], np.float64)   # codes 0..126, ascending
+
+
+def mxfp8_quantize(x):
+    """Activations [M, K] (float) to MXFP8: E4M3 elements with one E8M0 scale per 32 along K.
+
+    For the opt-in native block-scaled MMA forward ("Fine-Tuning 4-Bit Models", "Case 3": a
+    W4AFP8 variant of a 4-bit checkpoint), which multiplies 4-bit weight codes by 8-bit
+    activations.  The pages fix no rule; this follows the OCP MX shared-exponent rule as the
+    weight encoder does for MXFP4: e = clamp(floor(log2 amax) - 8 + 127, 0, 254) (8 = E4M3's
+    largest normal exponent; 0 for an all-zero block), elements = nearest E4M3 of x / 2^(e-127),
+    ties to the even code, magnitudes saturating at 448, the sign kept only on a non-zero
+    magnitude.  Returns (codes uint8 [M, K], scales uint8 [M, K/32])."""
+    x = np.asarray(x, np.float64)
+    M, K = x.shape
+    xb = x.reshape(M, K // 32, 32)
+    amax = np.abs(xb).max(axis=2)
+    e = np.zeros((M, K // 32), np.int64)
+    nz = amax > 0
+    e[nz] = np.clip(np.floor(np.log2(amax[nz])).astype(np.int64) - 8 + 127, 0, 254)
+    q = xb / np.exp2(e - 127.0)[:, :, None]
+    t = _e4m3_table()
+    mids = 0.5 * (t[:-1] + t[1:])
+    a = np.minimum(np.abs(q), 448.0)
+    c = np.searchsorted(mids, a, side="left")          # midpoints strictly below a
+    tie = (c < len(mids)) & (a == mids[np.minimum(c, len(mids) - 1)])
+    c = np.where(tie & (c % 2 == 1), c + 1, c)         # on a midpoint: the even code
+    codes = np.where((c != 0) & (q < 0), c | 0x80, c).astype(np.uint8)
+    return codes.reshape(M, K), e.astype(np.uint8)
+
+
+def mxfp8_dequant(codes, scales):
+    """Values of MXFP8 activations (fp64, exact)."""
+    codes = np.asarray(codes, np.uint8)
+    M, K = codes.shape
+    t = _e4m3_table()
+    mag = t[(codes & 0x7F).astype(np.int64)]
+    v = np.where(codes & 0x80, -mag, mag)
+    return (v.reshape(M, K // 32, 32) * np.exp2(np.asarray(scales, np.float64) - 127.0)[:, :, None]
+            ).reshape(M, K)
+
+
+def layer_w4a8_forward(fmt, M, N, K, r, s, codes, scales, tensor_scale, X, A, B):
+    """Forward of the opt-in native block-scaled MMA variant, fp64: the base product takes X
+    quantised to MXFP8 (mxfp8_quantize of the bf16 X) against the exact weight decode (E2M1 times
+    its block scale, times the NVFP4 tensor scale, not rounded to bf16: the block-scaled MMA
+    multiplies the codes themselves); the LoRA path is unchanged, T = X A^T from the bf16 X.
+    Y = deq8(X) deq(W)^T + s T B^T.  Only MXFP4 and NVFP4 weights (E2M1 codes) apply."""
+    if fmt not in ("mxfp4", "nvfp4"):
+        raise ValueError("the native FP4 MMA takes E2M1 weight codes (MXFP4, NVFP4)")
+    wide = lambda h: (np.asarray(h, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    Xf = wide(X)
+    xc, xs = mxfp8_quantize(Xf)
+    Xq = mxfp8_dequant(xc, xs)
+    # E2M1 x E8M0 and E2M1 x E4M3 are exact in bf16, so the bf16 decode without the tensor scale
+    # is the exact block product; the tensor scale is applied in fp64
+    Wd = wide(dequant(fmt, N, K, codes, scales, 1.0, with_tensor_scale=False))
+    if fmt == "nvfp4":
+        Wd = Wd * float(tensor_scale)
+    T = Xf @ wide(A).T
+    return Xq @ Wd.T + float(np.float32(s)) * (T @ wide(B).T)
+
+
 def num_threads():
     return lib().oracle_num_threads()
