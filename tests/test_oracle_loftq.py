@@ -108,3 +108,22 @@ def test_loftq_planted_mxfp4_is_recovered():
     resid = np.linalg.norm(W.astype(np.float64) - D - L)
     assert res["errs"][1] <= resid * (1 + 1e-9) and res["errs"][2] <= resid * (1 + 1e-9)
     assert np.allclose(res["B"] @ res["A"], L, rtol=0, atol=1e-4 * np.abs(L).max())
+
+
+def test_loftq_alternation_is_monotone_with_an_exact_projection():
+    # with rounding to a fixed grid as the quantiser, each sub-problem is solved exactly (rounding
+    # is the nearest grid point element by element; the truncated SVD is the best rank-r fit), so
+    # the objective ||W - Q - s B A|| can only fall from one iteration to the next -- and on a
+    # generic weight the requantisation of iteration 2 strictly lowers it
+    rng = np.random.default_rng(21)
+    W = rng.standard_normal((30, 50))
+    grid = lambda v: np.round(v * 2.0) / 2.0
+    res = O.loftq(W, r=4, s=1.5, iters=6, quant=grid)
+    e = res["errs"]
+    assert all(e[t + 1] <= e[t] * (1 + 1e-12) for t in range(len(e) - 1))
+    assert e[2] < e[1] * (1 - 1e-6)
+    # the returned Q is the quantisation of W - s B A with the factors before the last SVD: it
+    # is a grid point, and the final factors are the best rank-r fit of W - Q
+    assert np.array_equal(res["Q"], grid(res["Q"]))
+    S = np.linalg.svd(W - res["Q"], compute_uv=False)
+    assert abs(e[-1] - np.sqrt((S[4:] ** 2).sum())) < 1e-9
