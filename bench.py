@@ -383,6 +383,60 @@ def nf4dq_step(Q, torch, p, Xs, dYs, A, B, ncopy, steps=60):
             "bits_per_weight": round(bits, 4), "data": "workload NF4 codes, random stored scales"}
 
 
+def _pct(xs):
+    xs = sorted(xs)
+    pick = lambda q: xs[min(len(xs) - 1, int(round(q * (len(xs) - 1))))]
+    return {"median": round(pick(0.5), 2), "p10": round(pick(0.1), 2), "p90": round(pick(0.9), 2)}
+
+
+def phase_times(Q, torch, fwd, bwd, n, flush=None):
+    """Per-step device times (us) of the forward, the backward and the pair, each launch group
+    between its own event pair (so the backward does not start beside the forward's last kernel
+    here, unlike in the timed region), median / p10 / p90 over n steps.  flush(): called before
+    each step outside the events (an L2 flush for inputs that fit in L2)."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    for i in range(n):
+        if flush:
+            flush()
+        ev[i][0].record()
+        fwd(i)
+        ev[i][1].record()
+        bwd(i)
+        ev[i][2].record()
+    torch.cuda.synchronize()
+    f = [1e3 * e[0].elapsed_time(e[1]) for e in ev]
+    b = [1e3 * e[1].elapsed_time(e[2]) for e in ev]
+    return {"fwd_us": _pct(f), "bwd_us": _pct(b), "fwd_bwd_us": _pct([x + y for x, y in zip(f, b)]),
+            "steps": n}
+
+
+def small_layer_latency(Q, torch, synth, n=200):
+    """The 1024x1024 NF4 layer at M = 256 (microseconds per step; launch latency binds it): plain
+    launches, L2 flushed between steps by writing a 256 MB buffer outside the events."""
+    p = synth.layer_inputs("nf4_1024x1024")
+    M, N, K, r, s = p["M"], p["N"], p["K"], p["r"], p["s"]
+    W = Q.weight_from_numpy(p["fmt"], p["codes"], p["scales"], p["tensor_scale"])
+    X, A, B, dY = (Q.bf16_from_bits(p[k]) for k in ("X", "A", "B", "dY"))
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    T = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty((r, K), dtype=torch.bfloat16, device="cuda")
+    dB = torch.empty((N, r), dtype=torch.bfloat16, device="cuda")
+    ws = Q.alloc_workspace(Q.OP_BWD, W, M, r)
+    Q.qlora_workspace_init(ws)
+    junk = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    fwd = lambda i: Q.qlora_linear_fwd(W, X, A, B, Y, T, M, r, s, ws)
+    bwd = lambda i: Q.qlora_linear_bwd(W, X, A, B, T, dY, dX, dA, dB, M, r, s, ws)
+    for i in range(10):
+        fwd(i)
+        bwd(i)
+    out = phase_times(Q, torch, fwd, bwd, n, flush=lambda: junk.fill_(1))
+    if Q.qlora_get_device_status(ws) != 0:
+        raise RuntimeError("device status in the small-layer leg")
+    out["workload"] = "NF4 1024x1024, M=256, r=16 (plain launches, L2 flushed)"
+    return out
+
+
 def quantize_merge(Q, torch, p, A, B, peaks, reps=10):
     """The quantiser and the merge with requantisation on the workload's weight shape.
 
@@ -687,6 +741,19 @@ def run_own(args):
            "note": "host->device copies of each step's X and dY on a copy stream overlap the "
                    "previous step's compute; all of them inside the timed region"}
 
+    # ---- fwd, bwd and fwd+bwd separately (median / p10 / p90), and the microsecond-scale layer
+    phases = None
+    if not args.no_sweep:
+        try:
+            phases = {"bench_workload": phase_times(
+                Q, torch,
+                lambda i: Q.qlora_linear_fwd(Ws[i % ncopy], Xs[i % ncopy], A, B, Y, T, M, r, s, ws),
+                lambda i: Q.qlora_linear_bwd(Ws[i % ncopy], Xs[i % ncopy], A, B, T, dYs[i % ncopy],
+                                             dX, dA, dB, M, r, s, ws), 50)}
+            phases["small_layer"] = small_layer_latency(Q, torch, synth)
+        except Exception as exc:          # a side leg never takes the main line down
+            phases = {"error": f"{type(exc).__name__}: {exc}"}
+
     # ---- short-batch weight-stream sweeps: the NF4 up-proj weight and the MXFP4 gate-proj weight
     sweep = None
     if not args.no_sweep:
@@ -733,6 +800,7 @@ def run_own(args):
         "kernel_breakdown_method": f"separate pass of {prof_steps} steps after the timed region, "
                                    "CUDA events around every launch (launches serialised)",
         "e2e": e2e,
+        "phase_times": phases,
         "weight_stream_small_m": sweep,
         "nf4_double_quant": dq,
         "quantize_merge": qm,
