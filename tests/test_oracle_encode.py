@@ -178,3 +178,39 @@ def test_encode_mxfp4_round_trip_of_decoded_weight():
     w2 = (O.dequant("mxfp4", N, K, c2, e2).astype(np.uint32) << 16).view(np.float32)
     assert np.array_equal(w2, wf)
     assert not np.any(_unpack(c2, N, K) == 8)
+
+
+try:
+    from hypothesis import given, settings, strategies as st
+except ImportError:                                  # pragma: no cover
+    given = None
+
+
+if given is not None:
+    @settings(max_examples=25, deadline=None, derandomize=True)
+    @given(fmt=st.sampled_from(["nf4", "mxfp4", "nvfp4"]), rows=st.integers(1, 3),
+           blocks=st.integers(1, 3), log_scale=st.integers(-40, 40), seed=st.integers(0, 2**31))
+    def test_encode_random_shapes_and_scales(fmt, rows, blocks, log_scale, seed):
+        # random shapes (K a multiple of 64) and magnitudes from 2^-40 to 2^40: every code is the
+        # brute-force nearest value under the format's block scale
+        rng = np.random.default_rng(seed)
+        N, K = rows, 64 * blocks
+        v = (rng.standard_normal((N, K)) * math.ldexp(1.0, log_scale)).astype(np.float32)
+        codes, scales, ts, _ = O.encode(fmt, v)
+        c = _unpack(codes, N, K)
+        if fmt == "nf4":
+            L = O.nf4_levels_spec().astype(np.float64)
+            for n in range(N):
+                for k in range(K):
+                    a = float(scales[n, k // 64])
+                    assert c[n, k] == (_argmin_ties(L * a, float(v[n, k]), lambda b: b[0]) if a > 0 else 7)
+        elif fmt == "mxfp4":
+            for n in range(N):
+                for k in range(K):
+                    sc = math.ldexp(1.0, int(scales[n, k // 32]) - 127)
+                    assert c[n, k] == _e2m1_code(float(v[n, k]) / sc)
+        else:
+            for n in range(N):
+                for k in range(K):
+                    d = float(E4M3_POS[scales[n, k // 16]]) * ts
+                    assert c[n, k] == (_e2m1_code(float(v[n, k]) / d) if d > 0 else 0)
