@@ -1135,16 +1135,9 @@ qlora_status_t qlora_loftq(const float* W, const qlora_weight_t* Q, int r, float
   const LoftqLayout L = loftq_layout(N, K, r);
   if (work_bytes < L.total) return QLORA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  static bool attr_done[kMaxDevices] = {false};
-  const int dev = current_device();
-  if (dev >= 0 && dev < kMaxDevices && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(loftq_jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(loftq::jacobi_smem(loftq::kMaxL))) != cudaSuccess ||
-        cudaFuncSetAttribute(loftq_chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(loftq::chol_smem(loftq::kMaxL))) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    attr_done[dev] = true;
-  }
+  if (!set_smem(loftq_jacobi_kernel, loftq::jacobi_smem(loftq::kMaxL)) ||
+      !set_smem(loftq_chol_kernel, loftq::chol_smem(loftq::kMaxL)))
+    return QLORA_ERR_CUDA;
   const LoftqRun run{L, static_cast<char*>(work), N, K, r, loftq_width(N, K, r), scale, s};
   float* R = run.at<float>(L.R);
   double* norm = run.at<double>(L.norm);

@@ -155,3 +155,18 @@ def test_loftq_arguments(Q):
     assert rc(errs=None) == "QLORA_ERR_INVALID_ARG"
     assert rc(v=0x70008) == "QLORA_ERR_INVALID_ARG"
     assert rc(nbytes=need - 1) == "QLORA_ERR_WORKSPACE"
+
+
+def test_valid_offline_calls_reach_cuda_without_a_gpu(Q):
+    # arguments that pass every check: on a machine without a GPU driver the first CUDA call
+    # fails and the entry point reports QLORA_ERR_CUDA (nothing is left half-done on the host)
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    N, K = 256, 512
+    W = _w(Q, N=N, K=K)
+    need = Q.qlora_loftq_workspace_size(N, K, 16)
+    rc = Q.lib.qlora_loftq(0x70000, W.ref, 16, 2.0, 5, 4, 0, 0x80000, 0x90000, 0x60000, None,
+                           0x100000, need, None)
+    assert Q.STATUS[rc] == "QLORA_ERR_CUDA"
+    assert Q.STATUS[Q.lib.qlora_quantize(W.ref, 0x10000, 0, None)] == "QLORA_ERR_CUDA"
