@@ -45,15 +45,15 @@ int current_device() {
 }
 
 int num_sms() {
-  static int cache[kMaxDevices] = {0};
+  static std::atomic<int> cache[kMaxDevices] = {};   // threads may race to fill it: same value
   const int d = current_device();
   if (d < 0 || d >= kMaxDevices) return 148;
-  if (cache[d] == 0) {
-    int v = 0;
+  int v = cache[d].load(std::memory_order_relaxed);
+  if (v == 0) {
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || v <= 0) v = 148;
-    cache[d] = v;
+    cache[d].store(v, std::memory_order_relaxed);
   }
-  return cache[d];
+  return v;
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
