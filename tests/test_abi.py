@@ -170,3 +170,19 @@ def test_valid_offline_calls_reach_cuda_without_a_gpu(Q):
                            0x100000, need, None)
     assert Q.STATUS[rc] == "QLORA_ERR_CUDA"
     assert Q.STATUS[Q.lib.qlora_quantize(W.ref, 0x10000, 0, None)] == "QLORA_ERR_CUDA"
+
+
+@pytest.mark.parametrize("fmt,bs,sdt", [("nf4", 64, "float32"), ("nf4dq", 64, "uint8"),
+                                        ("mxfp4", 32, "uint8"), ("nvfp4", 16, "uint8")])
+def test_empty_weight_storage_shapes(Q, fmt, bs, sdt):
+    # the binding's storage for a weight matches the layouts include/qlora.h states
+    N, K = 48, 704
+    W = Q.empty_weight(fmt, N, K, device="cpu")
+    assert tuple(W.codes.shape) == (N, K // 2) and str(W.codes.dtype) == "torch.uint8"
+    assert tuple(W.scales.shape) == (N, K // bs) and str(W.scales.dtype) == f"torch.{sdt}"
+    assert (W.tensor_scale is not None) == (fmt == "nvfp4")
+    if fmt == "nf4dq":
+        assert W.scales2.numel() == -(-N * (K // 64) // 256)       # one per 256 first-level codes
+    else:
+        assert W.scales2 is None
+    assert W.c.fmt == Q.FMT[fmt] and W.c.N == N and W.c.K == K
