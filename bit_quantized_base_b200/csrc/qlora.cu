@@ -786,7 +786,7 @@ qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const void* X, 
                                         float scale, qlora_stream_t stream) {
   qlora_status_t st = check_common(W, M, r);
   if (st != QLORA_OK) return st;
-  if (!ptr_ok(X) || !ptr_ok(A) || !ptr_ok(B) || !ptr_ok(Y) || (T_save && !aligned16(T_save)))
+  if (!act_ok(X, M) || !ptr_ok(A) || !ptr_ok(B) || !act_ok(Y, M) || (T_save && !aligned16(T_save)))
     return QLORA_ERR_INVALID_ARG;
   const size_t mr = align_up(size_t(M) * size_t(r) * 2, 256);
   const size_t need = kHeaderBytes + mr + (T_save ? 0 : mr);
@@ -804,6 +804,17 @@ qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const void* X, 
                         kDownCtasBesidePair, s);
   if (st != QLORA_OK) return st;
   return launch_fused(W, false, X, Zs, B, Y, M, r, status, nullptr, 1, false, s);
+}
+
+qlora_status_t qlora_linear_fwd_noalloc_status(qlora_stream_t stream) {
+  uint8_t* w = static_cast<uint8_t*>(noalloc_scratch_address());
+  if (!w) return QLORA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, w, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return static_cast<qlora_status_t>(v);
 }
 
 qlora_status_t qlora_linear_bwd(const qlora_weight_t* W, const void* X, const void* A,

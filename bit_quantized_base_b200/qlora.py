@@ -28,6 +28,7 @@ EXPORTS = ("qlora_workspace_size", "qlora_workspace_init", "qlora_linear_fwd", "
            "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_status_string",
            "qlora_build_info", "qlora_launch_count", "qlora_profile_enable",
            "qlora_profile_reset", "qlora_profile_read", "qlora_linear_fwd_noalloc",
+           "qlora_linear_fwd_noalloc_status",
            "qlora_debug_decode_rate", "qlora_quantize", "qlora_merge_requantize",
            "qlora_loftq_workspace_size", "qlora_loftq")
 
@@ -80,6 +81,8 @@ def _load():
     L.qlora_launch_count.restype = c.c_int64
     L.qlora_linear_fwd_noalloc.argtypes = [W, P, P, P, P, P, c.c_int64, c.c_int, c.c_float, P]
     L.qlora_linear_fwd_noalloc.restype = c.c_int
+    L.qlora_linear_fwd_noalloc_status.argtypes = [P]
+    L.qlora_linear_fwd_noalloc_status.restype = c.c_int
     L.qlora_profile_enable.argtypes = [c.c_int]
     L.qlora_profile_read.argtypes = [c.c_int, c.POINTER(c.c_int), c.POINTER(c.c_char_p),
                                      c.POINTER(c.c_int), c.POINTER(c.c_double)]
@@ -162,6 +165,11 @@ def qlora_linear_fwd_noalloc(W: Weight, X, A, B, Y, T_save, M, r, scale, stream=
     _check(lib.qlora_linear_fwd_noalloc(W.ref, _p(X), _p(A), _p(B), _p(Y), _p(T_save), int(M),
                                         int(r), float(scale), _stream(stream)),
            "qlora_linear_fwd_noalloc")
+
+
+def qlora_linear_fwd_noalloc_status(stream=None):
+    """Synchronise the stream and return the no-alloc scratch's device status word (an int)."""
+    return int(lib.qlora_linear_fwd_noalloc_status(_stream(stream)))
 
 
 def qlora_linear_bwd(W: Weight, X, A, B, T, dY, dX, dA, dB, M, r, scale, ws, stream=None):

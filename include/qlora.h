@@ -174,22 +174,30 @@ QLORA_API qlora_status_t qlora_grouped_bwd(const qlora_weight_t* W, int E, const
  *   until the process exits): 256 bytes of status, the [M,r] bf16 operand Zs and, when T_save is
  *   NULL, an [M,r] bf16 T.  It always runs the tiled kernels, so for M > 256 its results are
  *   bitwise those of qlora_linear_fwd; shorter batches, which qlora_linear_fwd runs through the
- *   weight-streaming kernel, differ from them in rounding only.  Sizes that do not fit
- *   -- M*r > 2,097,024 with T_save, or
- *   M*r > 1,048,512 without -- are rejected with QLORA_ERR_WORKSPACE before anything is enqueued.
+ *   weight-streaming kernel, differ from them in rounding only.  A call fits when
+ *   256 + Z <= 4 MiB with T_save, or 256 + 2 Z <= 4 MiB without, where Z = 2*M*r bytes rounded up
+ *   to a multiple of 256: M*r <= 2,097,024 with T_save, or M*r <= 1,048,448 without (for r = 64:
+ *   M <= 32766 and M <= 16382).  Larger sizes are rejected with QLORA_ERR_WORKSPACE before
+ *   anything is enqueued.
  *   The call allocates nothing (no cudaMalloc/cudaFree, no allocating library routine); it clears
  *   the status word on `stream` each call.
  *   The first call on each device looks up the array's device address (cudaGetSymbolAddress) with
  *   that device current; make that first call before any stream capture.
  *   Every call uses the same array and leaves its contents behind: calls whose work overlaps on
  *   the GPU (other streams, other threads) race on it, so order them on one stream.
- *   A device-side wait that gives up ends the kernel early; its status word lives in the array and
- *   is not visible through qlora_get_device_status.
- * Arguments and their checks are those of qlora_linear_fwd, minus the workspace. */
+ *   A device-side wait that gives up ends the kernel early and records QLORA_ERR_DEVICE_TIMEOUT
+ *   in the array's status word; read it with qlora_linear_fwd_noalloc_status.
+ * Arguments and their checks are those of qlora_linear_fwd, minus the workspace (M = 0 is a
+ * no-op returning QLORA_OK and accepts NULL X and Y). */
 QLORA_API qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const void* X,
                                                   const void* A, const void* B, void* Y,
                                                   void* T_save, int64_t M, int r, float scale,
                                                   qlora_stream_t stream);
+
+/* Synchronise `stream` and read the status word of qlora_linear_fwd_noalloc's fixed scratch on
+ * the current device: QLORA_OK, or the device-side error of the last no-alloc call (each call
+ * clears it when it starts).  Allocates nothing.  Not for the compute path. */
+QLORA_API qlora_status_t qlora_linear_fwd_noalloc_status(qlora_stream_t stream);
 
 /* Synchronise `stream` and read the workspace's device status word (QLORA_OK or the first
  * device-side error recorded since qlora_workspace_init).  Not for the compute path. */

@@ -186,3 +186,29 @@ def test_empty_weight_storage_shapes(Q, fmt, bs, sdt):
     else:
         assert W.scales2 is None
     assert W.c.fmt == Q.FMT[fmt] and W.c.N == N and W.c.K == K
+
+
+def test_noalloc_empty_batch_accepts_null_activations(Q):
+    # M = 0 is a no-op, as for qlora_linear_fwd: NULL X and Y are accepted and nothing is enqueued
+    rc = Q.lib.qlora_linear_fwd_noalloc(_w(Q).ref, None, 0x20000, 0x30000, None, None, 0, 16, 2.0,
+                                        None)
+    assert Q.STATUS[rc] == "QLORA_OK"
+    rc = Q.lib.qlora_linear_fwd_noalloc(_w(Q).ref, None, 0x20000, 0x30000, None, None, 4, 16, 2.0,
+                                        None)
+    assert Q.STATUS[rc] == "QLORA_ERR_INVALID_ARG"
+
+
+@pytest.mark.parametrize("keep_t,m_max", [(False, 16382), (True, 32766)])
+def test_noalloc_size_limit_boundary(Q, keep_t, m_max):
+    # r = 64: the largest batch that fits the fixed scratch passes the size check (on a machine
+    # without a GPU it then fails at the first CUDA call); one row more is refused before any
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present: the accepted size would run")
+    T = 0x60000 if keep_t else None
+
+    def rc(M):
+        return Q.STATUS[Q.lib.qlora_linear_fwd_noalloc(_w(Q).ref, 0x10000, 0x20000, 0x30000,
+                                                       0x40000, T, M, 64, 2.0, None)]
+    assert rc(m_max + 1) == "QLORA_ERR_WORKSPACE"
+    assert rc(m_max) == "QLORA_ERR_CUDA"
