@@ -577,6 +577,132 @@ def grouped_moe(Q, torch, synth, peaks):
     return res
 
 
+def _device_weight(Q, torch, fmt, N, K, dist, gen):
+    """A stored weight made on the device: v ~ N(0, 0.02) (or 0.02 x Student-t(5), as
+    z0 sqrt(5 / sum of 5 squared normals)) in fp32, encoded by the library's own quantiser
+    (qlora_quantize, bit-exact against the oracle's encoder rules)."""
+    v = torch.randn((N, K), device="cuda", generator=gen)
+    if dist == "t5":
+        chi = sum(torch.randn((N, K), device="cuda", generator=gen) ** 2 for _ in range(5))
+        v.mul_(torch.sqrt(5.0 / chi))
+        del chi
+    v.mul_(0.02)
+    W = Q.empty_weight(fmt, N, K)
+    Q.qlora_quantize(W, v)
+    del v
+    return W
+
+
+def layer_leg(Q, torch, peaks, fmt, M, N, K, r, s, dist, seed, steps=30):
+    """fwd+bwd of one full-size layer at its own batch M, as in the headline loop (no per-kernel
+    events in the timed loop; rotating device copies of W, X, dY whose total exceeds 2.5x L2),
+    with its own clock record; then fwd / bwd / fwd+bwd separately (median, p10, p90) and the
+    dominant kernel's roofline from a profiled pass (an event pair around every launch)."""
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed)
+    per_copy = weight_bytes(fmt, N, K) + 2 * M * (K + N)
+    ncopy = max(3, int(math.ceil(2.5 * 126e6 / per_copy)))
+    Ws = [_device_weight(Q, torch, fmt, N, K, dist, gen) for _ in range(ncopy)]
+    Xs = [torch.randn((M, K), device="cuda", generator=gen).bfloat16() for _ in range(ncopy)]
+    dYs = [(torch.randn((M, N), device="cuda", generator=gen) * 0.01).bfloat16()
+           for _ in range(ncopy)]
+    bound = 1.0 / math.sqrt(K)
+    A = ((torch.rand((r, K), device="cuda", generator=gen) * 2 - 1) * bound).bfloat16()
+    B = (torch.randn((N, r), device="cuda", generator=gen) * 0.01).bfloat16()
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    T = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty((r, K), dtype=torch.bfloat16, device="cuda")
+    dB = torch.empty((N, r), dtype=torch.bfloat16, device="cuda")
+    ws = Q.alloc_workspace(Q.OP_BWD, Ws[0], M, r)
+    Q.qlora_workspace_init(ws)
+    fwd = lambda i: Q.qlora_linear_fwd(Ws[i % ncopy], Xs[i % ncopy], A, B, Y, T, M, r, s, ws)
+    bwd = lambda i: Q.qlora_linear_bwd(Ws[i % ncopy], Xs[i % ncopy], A, B, T, dYs[i % ncopy], dX,
+                                       dA, dB, M, r, s, ws)
+    for i in range(5):
+        fwd(i)
+        bwd(i)
+    torch.cuda.synchronize()
+    clk = NvmlSampler(torch.cuda.current_device())
+    clk.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        fwd(i)
+        bwd(i)
+    e1.record()
+    e1.synchronize()
+    clocks = clk.stop()
+    t = e0.elapsed_time(e1) / steps * 1e-3
+    phases = phase_times(Q, torch, fwd, bwd, 20)
+    time.sleep(1.0)
+    pclk = NvmlSampler(torch.cuda.current_device())
+    pclk.start()
+    Q.qlora_profile_enable(True)
+    Q.qlora_profile_reset()
+    for i in range(10):
+        fwd(i)
+        bwd(i)
+    torch.cuda.synchronize()
+    prof_clocks = pclk.stop()
+    prof = Q.qlora_profile_read()
+    Q.qlora_profile_enable(False)
+    if Q.qlora_get_device_status(ws) != 0:
+        raise RuntimeError("device status in a large-batch leg")
+    kflops = {"fused_fwd": 2.0 * M * N * K + 2.0 * M * N * r,
+              "fused_dx": 2.0 * M * N * K + 2.0 * M * K * r,
+              "stream_fwd": 2.0 * M * N * K + 2.0 * M * N * r,
+              "stream_dx": 2.0 * M * N * K + 2.0 * M * K * r}
+    dom = max((k for k in prof if k in kflops), key=lambda k: prof[k][1])
+    cnt, tot = prof[dom]
+    capped = "sw_power_cap" in prof_clocks.get("reasons", [])
+    peak = peaks["bf16_tflops_sustained"] if capped else peaks["bf16_tflops"]
+    achieved = kflops[dom] / (tot / cnt * 1e-3) / 1e12
+    fl = flops(M, N, K, r)
+    res = {"M": M, "N": N, "K": K, "r": r, "fmt": fmt, "ms_per_step": round(t * 1e3, 4),
+           "tflops": round(fl / t / 1e12, 1), "frac_of_bf16_peak": round(fl / t / 1e12 / peak, 4),
+           "peak_source": "sustained" if capped else "burst",
+           "phase_us": phases, "clocks": {k: clocks.get(k) for k in ("sm_mhz", "sm_mhz_min",
+                                                                      "reasons", "samples")},
+           "roofline": {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
+                        "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                        "avg_launch_ms": round(tot / cnt, 4),
+                        "clocks_while_timed": {k: prof_clocks.get(k)
+                                               for k in ("sm_mhz", "reasons", "samples")}},
+           "l2": f"{ncopy} rotating device copies of W, X, dY ({ncopy * per_copy / 1e6:.0f} MB)",
+           "data": "W ~ " + ("0.02 t(5)" if dist == "t5" else "N(0, 0.02)") +
+                   " made on the device and encoded by qlora_quantize; X ~ N(0,1), dY ~ N(0,0.01)"}
+    del Ws, Xs, dYs, Y, T, dX, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def large_batch_legs(Q, torch, synth, peaks):
+    """The two other dense workloads at their own batch sizes: the MXFP4 Llama-3-70B-shaped
+    gate-proj (M=8192, 28672x8192, r=16) and the seven NVFP4 Llama-3-70B-shaped decoder-layer
+    projections (M=4096, r=16), each timed as its own layer, plus the layer's sum."""
+    out = {}
+    c3 = synth.WORKLOADS["llama3_70b_gate_mxfp4"]
+    pr = c3.projs[0]
+    out["llama3_70b_gate_mxfp4"] = layer_leg(Q, torch, peaks, c3.fmt, c3.M, pr.N, pr.K, c3.r,
+                                             c3.scale, "t5", 3000)
+    c4 = synth.WORKLOADS["llama3_70b_layer_nvfp4"]
+    legs, tot_fl, tot_t = {}, 0.0, 0.0
+    for i, pr in enumerate(c4.projs):
+        leg = layer_leg(Q, torch, peaks, c4.fmt, c4.M, pr.N, pr.K, c4.r, c4.scale, "normal",
+                        4000 + i, steps=20)
+        legs[pr.name] = leg
+        tot_fl += flops(c4.M, pr.N, pr.K, c4.r)
+        tot_t += leg["ms_per_step"] * 1e-3
+    out["llama3_70b_layer_nvfp4"] = {
+        "projections": legs, "ms_per_layer": round(tot_t * 1e3, 4),
+        "tflops": round(tot_fl / tot_t / 1e12, 1),
+        "frac_of_bf16_burst_peak": round(tot_fl / tot_t / 1e12 / peaks["bf16_tflops"], 4),
+        "frac_of_bf16_sustained_peak": round(tot_fl / tot_t / 1e12 / peaks["bf16_tflops_sustained"], 4)}
+    return out
+
+
 def run_own(args):
     import numpy as np
     import torch
@@ -778,10 +904,23 @@ def run_own(args):
     if not args.no_sweep:
         grouped = grouped_moe(Q, torch, synth, peaks)
 
+    # ---- the MXFP4 gate-proj at M = 8192 and the seven NVFP4 decoder-layer projections at M = 4096
+    large = None
+    if not args.no_sweep:
+        try:
+            large = large_batch_legs(Q, torch, synth, peaks)
+        except Exception as exc:          # a side leg never takes the main line down
+            large = {"error": f"{type(exc).__name__}: {exc}"}
+
     # ---- CPU baseline: the oracle on a bounded sample of the same workload
     cpu = None
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(p, args.cpu_seconds)
+        if not args.no_sweep:
+            try:
+                cpu["per_config"] = cpu_baseline_per_config(synth, cpu)
+            except Exception as exc:
+                cpu["per_config"] = {"error": f"{type(exc).__name__}: {exc}"}
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws_n,
@@ -805,6 +944,7 @@ def run_own(args):
         "nf4_double_quant": dq,
         "quantize_merge": qm,
         "grouped_moe": grouped,
+        "large_batch": large,
         "cpu_baseline": cpu,
     }
     if rank == 0:
@@ -828,6 +968,17 @@ def _oracle_sample(p, rows, cols=None):
     return time.perf_counter() - t0
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(p, target_s):
     from oracle import oracle as O
     N, K, r = p["N"], p["K"], p["r"]
@@ -838,9 +989,76 @@ def cpu_baseline(p, target_s):
     t = _oracle_sample(p, rows)
     v = flops(rows, N, K, r) / t / 1e12
     return {"value": round(v, 6), "unit": "TFLOP/s", "cores": O.num_threads(), "kind": "oracle",
-            "seconds": round(t, 2),
+            "seconds": round(t, 2), "nproc": os.cpu_count(), "cpu_model": cpu_model(),
             "sample": f"full fp64 fwd+bwd of the same layer on the first {rows} of the "
                       f"{p['M']} rows (W decode included), OpenMP"}
+
+
+def _recipe_slice(synth, name, proj, n_out, m_rows):
+    """A problem drawn from a workload's recipe (format, K, distributions, rank) with n_out output
+    features and m_rows batch rows: the oracle's cost per flop on it stands for the full layer's."""
+    cfg = synth.WORKLOADS[name]
+    pr = cfg.projs[proj]
+    p = synth.small_layer(cfg.fmt, m_rows, min(n_out, pr.N), pr.K, cfg.r, s=cfg.scale,
+                          seed=9000 + 10 * cfg.seed_id + proj, dy_std=cfg.dy_std, b_std=cfg.b_std)
+    return p
+
+
+def cpu_baseline_per_config(synth, p2_result, seconds_each=4.0):
+    """The oracle per workload: in full for the 1024x1024 layer (M = 256) and, from the headline
+    baseline, the bench workload; for the three large workloads, timed on a sample drawn from the
+    recipe (the first output features and rows of the layer, all of K) and extrapolated to the
+    workload's flops at the sample's fp64 rate -- labelled as extrapolated."""
+    from oracle import oracle as O
+    out = {"nproc": os.cpu_count(), "threads": O.num_threads(), "cpu_model": cpu_model()}
+    p1 = synth.layer_inputs("nf4_1024x1024")
+    t0 = time.perf_counter()
+    O.layer(p1["fmt"], p1["M"], p1["N"], p1["K"], p1["r"], p1["s"], p1["codes"], p1["scales"],
+            p1["tensor_scale"], p1["X"], p1["A"], p1["B"], p1["dY"])
+    t = time.perf_counter() - t0
+    fl = flops(p1["M"], p1["N"], p1["K"], p1["r"])
+    out["nf4_1024x1024"] = {"seconds": round(t, 4), "tflops": round(fl / t / 1e12, 6),
+                            "how": "full oracle, every output"}
+    if p2_result is not None:
+        out["llama3_8b_up_nf4"] = {"seconds": p2_result["seconds"], "tflops": p2_result["value"],
+                                   "how": p2_result["sample"]}
+
+    n_slice = 2048
+    thr = max(1, O.num_threads())
+
+    def cost_model(name, proj):
+        # seconds = fixed (the weight decode) + rows x per-row, on an n_slice-output slice; both
+        # grow with the number of output features, so the full layer scales them by N / n_slice
+        p = _recipe_slice(synth, name, proj, n_slice, 8 * thr)
+        m1, m2 = 2 * thr, 4 * thr
+        t1 = _oracle_sample(p, m1)
+        if t1 * 2 < seconds_each:
+            m2 = 8 * thr
+        t2 = _oracle_sample(p, m2)
+        per_row = max((t2 - t1) / (m2 - m1), 1e-6)
+        fixed = max(t1 - m1 * per_row, 0.0)
+        return fixed, per_row, p["N"], (m1, m2)
+
+    for name in ("llama3_70b_gate_mxfp4", "llama3_70b_layer_nvfp4", "moe64_mxfp4"):
+        cfg = synth.WORKLOADS[name]
+        tot_fl, tot_s, how = 0.0, 0.0, []
+        models = {}
+        for i, pr in enumerate(cfg.projs):
+            key = (pr.K, cfg.fmt)
+            if key not in models:
+                models[key] = cost_model(name, i)
+            fixed, per_row, n_out, ms = models[key]
+            scale = pr.N / n_out
+            E = max(cfg.experts, 1)
+            # grouped: every expert decodes its own weight; the rows add up to cfg.M
+            tot_s += scale * (E * fixed + cfg.M * per_row)
+            tot_fl += flops(cfg.M, pr.N, pr.K, cfg.r)
+            how.append(f"{pr.name} (K={pr.K}): fixed {fixed:.3f} s + {per_row * 1e3:.2f} ms/row "
+                       f"timed at {ms[0]} and {ms[1]} rows x {n_out} outputs")
+        out[name] = {"seconds_extrapolated": round(tot_s, 1),
+                     "tflops": round(tot_fl / tot_s / 1e12, 6), "extrapolated": True,
+                     "how": "; ".join(how)}
+    return out
 
 
 def run_reference(args):

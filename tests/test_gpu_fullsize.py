@@ -53,10 +53,13 @@ def test_full_size_layer_sampled(name, proj):
     assert_close(to_f64(dB), ref["dB"], "dB")
 
 
-SHORT = [("llama3_8b_up_nf4", 16), ("llama3_8b_up_nf4", 256), ("llama3_70b_gate_mxfp4", 64)]
+# the single NF4 layer N = K = 1024 at its own batch of 256 rows (every output checked), then
+# the full-size weights of the NF4 up-proj and the MXFP4 gate-proj under short batches
+SHORT = [("nf4_1024x1024", 256), ("llama3_8b_up_nf4", 16), ("llama3_8b_up_nf4", 256),
+         ("llama3_70b_gate_mxfp4", 64)]
 
 
-@pytest.mark.parametrize("name,M", SHORT, ids=[f"{synth.WORKLOADS[c].fmt}-M{m}" for c, m in SHORT])
+@pytest.mark.parametrize("name,M", SHORT, ids=[f"{c}-M{m}" for c, m in SHORT])
 def test_full_size_weight_short_batch(name, M):
     # the full-size weights of the NF4 up-proj and the MXFP4 gate-proj under the short batches of
     # the weight-stream sweep: every output row is checked
