@@ -14,6 +14,7 @@
 #include "qlora_fused.cuh"
 #include "qlora_lora.cuh"
 #include "qlora_stream.cuh"
+#include "qlora_short.cuh"
 #include <algorithm>
 #include <utility>
 #include "qlora_quant.cuh"
@@ -23,7 +24,13 @@ namespace qlora {
 namespace {
 
 // ------------------------------------------------------------------------------------ helpers
-constexpr size_t kHeaderBytes = 256;        // [0]: device status word, [1]: pair-kernel ticket
+// Workspace header, cleared by qlora_workspace_init: [0] device status word, [1] pair-kernel
+// ticket, bytes [256, 8192) the short-batch kernels' arrival counters, 4 per tile (each launch
+// leaves them at zero).
+constexpr size_t kHeaderBytes = 8192;
+constexpr size_t kCounterOffset = 256;
+// The no-alloc forward's scratch holds only the status word and the ticket in its header.
+constexpr size_t kNoAllocHeaderBytes = 256;
 constexpr int kMaxClusterSplits = 8;        // split-K CTAs of one LoRA tile (one portable cluster)
 // CTAs of a lora_down launch that feeds the pair kernel: the pair kernel starts beside it on the
 // other SMs and waits for its output only at the end of its first tile
@@ -241,6 +248,48 @@ bool stream_fits(const qlora_weight_t* W, int64_t M, int E, bool dx, size_t regi
          stream_plan(W->N, W->K, M, dx, num_sms()).partial_bytes <= region;
 }
 
+// Batches of at most 64 rows (one weight, NF4 / MXFP4 / NVFP4) use the short-batch kernels: the
+// flat space of (output tile, 64-deep step) iterations plus one LoRA step per tile, cut into equal
+// contiguous ranges, one per CTA; pieces of split tiles go to fp32 partials [tiles][pieces][M][tile
+// columns].  The SMs the launch leaves free run lora_down beside it.
+struct ShortPlan {
+  int tiles, nk, iters, grid, max_pieces, tile_cols;
+  size_t partial_bytes;
+};
+
+ShortPlan short_plan(int64_t N, int64_t K, int64_t M, bool dx, int sms) {
+  ShortPlan p{};
+  if (sms > 4 * kDownCtasBesideStream) sms -= kDownCtasBesideStream;
+  p.tile_cols = dx ? shortk::D_TILE : shortk::F_TILE;
+  p.tiles = int(((dx ? K : N) + p.tile_cols - 1) / p.tile_cols);
+  // contraction iterations: 256 weight columns (forward) or 128 weight rows (dX)
+  p.nk = int(dx ? (N + 127) / 128 : (K + 255) / 256);
+  const int64_t nk1 = p.nk + 1;
+  const int64_t total = int64_t(p.tiles) * nk1;
+  int64_t L = (total + sms - 1) / sms;
+  if (L < 2) L = 2;
+  p.iters = int(L);
+  p.grid = int((total + L - 1) / L);
+  int mp = 1;
+  for (int64_t t = 0; t < p.tiles; ++t) {
+    const int64_t first = t * nk1 / L, last = (t * nk1 + nk1 - 1) / L;
+    if (last - first + 1 > mp) mp = int(last - first + 1);
+  }
+  p.max_pieces = mp;
+  p.partial_bytes = size_t(p.tiles) * size_t(mp) * size_t(M) * size_t(p.tile_cols) * 4;
+  return p;
+}
+
+bool use_short(const qlora_weight_t* W, int64_t M, int E) {
+  return E == 1 && M > 0 && M <= shortk::kMaxRows && W->fmt != QLORA_FMT_NF4_DQ;
+}
+
+bool short_fits(const qlora_weight_t* W, int64_t M, int E, bool dx, size_t region) {
+  if (!use_short(W, M, E)) return false;
+  const ShortPlan sp = short_plan(W->N, W->K, M, dx, num_sms());
+  return sp.tiles <= shortk::kMaxTiles && sp.partial_bytes <= region;
+}
+
 struct WsLayout {
   size_t zs, t, u, partial, partial_bytes, total;
 };
@@ -255,6 +304,14 @@ WsLayout ws_layout(int64_t N, int64_t K, int64_t M, int r, bool bwd, int E, int 
   L.partial = off;
   // fp32 partials of the short-batch weight-streaming kernels
   size_t pb = 0;
+  if (E == 1 && M > 0 && M <= shortk::kMaxRows) {
+    const size_t sf = short_plan(N, K, M, false, sms).partial_bytes;
+    pb = sf > pb ? sf : pb;
+    if (bwd) {
+      const size_t sd = short_plan(N, K, M, true, sms).partial_bytes;
+      pb = sd > pb ? sd : pb;
+    }
+  }
   if (use_stream(M, E)) {
     const size_t sf = stream_plan(N, K, M, false, sms).partial_bytes;
     pb = sf > pb ? sf : pb;
@@ -275,12 +332,12 @@ int* ws_status(void* ws) { return reinterpret_cast<int*>(ws); }
 enum Kind : int {
   kKindFusedFwd = 0, kKindFusedDx, kKindDownT, kKindDownU, kKindWgrad,
   kKindGFusedFwd, kKindGFusedDx, kKindGDownT, kKindGDownU, kKindGWgrad,
-  kKindStreamFwd, kKindStreamDx, kKindStreamReduce, kNumKinds
+  kKindStreamFwd, kKindStreamDx, kKindStreamReduce, kKindShortFwd, kKindShortDx, kNumKinds
 };
 const char* const kKindNames[kNumKinds] = {
     "fused_fwd", "fused_dx", "lora_down_T", "lora_down_U", "lora_wgrad",
     "grouped_fused_fwd", "grouped_fused_dx", "grouped_lora_down_T", "grouped_lora_down_U",
-    "grouped_lora_wgrad", "stream_fwd", "stream_dx", "stream_reduce"};
+    "grouped_lora_wgrad", "stream_fwd", "stream_dx", "stream_reduce", "short_fwd", "short_dx"};
 constexpr int kMaxProfiled = 65536;
 
 std::atomic<int64_t> g_launches{0};
@@ -330,7 +387,7 @@ bool tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_
 qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t Kc, const void* R,
                                 int r, float s, const float* ts, void* z, void* zs, int* status,
                                 const int32_t* offsets, int E, bool grouped, int max_ctas,
-                                cudaStream_t st) {
+                                cudaStream_t st, float zs_mul = 1.0f) {
   DownParams p{};
   const int rpad = rank_pad(r);
   const DownPlan dp = down_plan(M, Kc, E, max_ctas > 0 ? max_ctas : num_sms());
@@ -356,6 +413,7 @@ qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t K
   p.steps_per_split = dp.sps;
   p.E = E;
   p.s = s;
+  p.zs_mul = zs_mul;
   const dim3 grid(unsigned(dp.tiles * dp.S));
   const size_t smem = lora::smem_bytes(E);
   LaunchScope scope(grouped ? (r_mn ? kKindGDownU : kKindGDownT) : (r_mn ? kKindDownU : kKindDownT), st);
@@ -533,6 +591,72 @@ qlora_status_t launch_stream(const qlora_weight_t* W, bool dx, const void* act, 
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// NVFP4 runs the short-batch kernels with its elements decoded times 2^-8: Zs carries the same
+// factor and the kernels' epilogue multiplies by 2^8 times the tensor scale.
+constexpr float kShortNvZsMul = 1.0f / 256.0f;
+float short_zs_mul(const qlora_weight_t* W) { return W->fmt == QLORA_FMT_NVFP4 ? kShortNvZsMul : 1.0f; }
+
+template <int FMT, bool DX>
+qlora_status_t launch_short_t(const ShortParams& p, int grid, cudaStream_t st) {
+  const size_t smem = DX ? shortk::dx_smem_bytes() : shortk::fwd_smem_bytes(p.xrows);
+  auto kern = DX ? qlora_short_dx_kernel<FMT> : qlora_short_fwd_kernel<FMT>;
+  if (!set_smem(kern, smem)) return QLORA_ERR_CUDA;
+  LaunchScope scope(DX ? kKindShortDx : kKindShortFwd, st);
+  if (launch_pdl(kern, dim3(grid), dim3(shortk::kThreads), smem, st, p) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// Short-batch path of the fused GEMM (same operands and result as launch_fused with one expert,
+// Zs written by lora_down with zs_mul = short_zs_mul(W)).
+qlora_status_t launch_short(const qlora_weight_t* W, bool dx, const void* act, const void* zs,
+                            const void* lora_up, void* out, int64_t M, int r, void* ws,
+                            float* partial, size_t partial_bytes, cudaStream_t st) {
+  const int64_t N = W->N, K = W->K;
+  const int64_t Kc = dx ? N : K;
+  const ShortPlan sp = short_plan(N, K, M, dx, num_sms());
+  if (sp.partial_bytes > partial_bytes || sp.tiles > shortk::kMaxTiles) return QLORA_ERR_WORKSPACE;
+  ShortParams p{};
+  p.xrows = int((M + 15) / 16 * 16);
+  if (!tmap_2d(&p.tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, uint64_t(Kc), uint64_t(M),
+               uint64_t(Kc) * 2, 64, uint32_t(p.xrows), CU_TENSOR_MAP_SWIZZLE_128B))
+    return QLORA_ERR_CUDA;
+  if (!tmap_2d(&p.tm_zs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, zs, uint64_t(r), uint64_t(M),
+               uint64_t(r) * 2, 64, uint32_t(p.xrows), CU_TENSOR_MAP_SWIZZLE_128B))
+    return QLORA_ERR_CUDA;
+  if (!tmap_2d(&p.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, uint64_t(K / 2), uint64_t(N),
+               uint64_t(K / 2), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return QLORA_ERR_CUDA;
+  p.codes = static_cast<const uint8_t*>(W->codes);
+  p.scales = W->scales;
+  p.tensor_scale = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
+  p.lora_up = static_cast<const __nv_bfloat16*>(lora_up);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.partial = partial;
+  p.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + kCounterOffset);
+  p.status = ws_status(ws);
+  p.M = int(M);
+  p.N = int(N);
+  p.K = int(K);
+  p.r = r;
+  p.rpad = rank_pad(r);
+  p.num_k = sp.nk;
+  p.num_tiles = sp.tiles;
+  p.iters = sp.iters;
+  p.max_pieces = sp.max_pieces;
+  p.ts_mul = 1.0f / short_zs_mul(W);
+  p.one = 1u;
+  p.zero = 0u;
+  switch (W->fmt * 2 + (dx ? 1 : 0)) {
+    case 0: return launch_short_t<kFmtNF4, false>(p, sp.grid, st);
+    case 1: return launch_short_t<kFmtNF4, true>(p, sp.grid, st);
+    case 2: return launch_short_t<kFmtMXFP4, false>(p, sp.grid, st);
+    case 3: return launch_short_t<kFmtMXFP4, true>(p, sp.grid, st);
+    case 4: return launch_short_t<kFmtNVFP4, false>(p, sp.grid, st);
+    default: return launch_short_t<kFmtNVFP4, true>(p, sp.grid, st);
+  }
+}
+
 // dB [E, N, r] = s dY_e^T T_e and dA [E, r, K] = s U_e^T X_e over each expert's rows.
 qlora_status_t launch_wgrad(const void* X, const void* dY, const void* T, const void* U, int64_t M,
                             int64_t N, int64_t K, int r, float s, void* dA, void* dB, void* ws,
@@ -685,14 +809,18 @@ qlora_status_t run_fwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   void* T = T_save ? T_save : w + L.t;
   void* Zs = w + L.zs;
   const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
-  const bool short_fwd = stream_fits(W, M, E, false, ws_bytes - L.partial);
+  float* part = reinterpret_cast<float*>(w + L.partial);
+  const size_t region = ws_bytes - L.partial;
+  const bool short_fwd = short_fits(W, M, E, false, region);
+  const bool stream_fwd = !short_fwd && stream_fits(W, M, E, false, region);
   qlora_status_t st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, T, Zs, ws_status(ws),
                                        offsets, E, grouped,
-                                       short_fwd ? kDownCtasBesideStream : kDownCtasBesidePair, s);
+                                       (short_fwd || stream_fwd) ? kDownCtasBesideStream
+                                                                 : kDownCtasBesidePair,
+                                       s, short_fwd ? short_zs_mul(W) : 1.0f);
   if (st != QLORA_OK) return st;
-  if (short_fwd)
-    return launch_stream(W, false, X, Zs, B, Y, M, r, ws_status(ws),
-                         reinterpret_cast<float*>(w + L.partial), ws_bytes - L.partial, s);
+  if (short_fwd) return launch_short(W, false, X, Zs, B, Y, M, r, ws, part, region, s);
+  if (stream_fwd) return launch_stream(W, false, X, Zs, B, Y, M, r, ws_status(ws), part, region, s);
   return launch_fused(W, false, X, Zs, B, Y, M, r, ws_status(ws), offsets, E, grouped, s);
 }
 
@@ -717,19 +845,28 @@ qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   void* Zs = w + L.zs;
   void* U = w + L.u;
   float* part = reinterpret_cast<float*>(w + L.partial);
+  const size_t region = ws_bytes - L.partial;
   qlora_status_t st;
   if (!T) {  // recompute T = X A^T (its scaled copy lands in Zs and is overwritten below) with
              // the forward's split plan, so it equals the forward's T bit for bit
-    const bool short_fwd = stream_fits(W, M, E, false, ws_bytes - L.partial);
+    const bool beside = short_fits(W, M, E, false, region) || stream_fits(W, M, E, false, region);
     st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, w + L.t, Zs, ws_status(ws), offsets,
-                          E, grouped, short_fwd ? kDownCtasBesideStream : kDownCtasBesidePair, s);
+                          E, grouped, beside ? kDownCtasBesideStream : kDownCtasBesidePair, s);
     if (st != QLORA_OK) return st;
     T = w + L.t;
   }
-  const bool short_dx = dX && stream_fits(W, M, E, true, ws_bytes - L.partial);
+  const bool short_dx = dX && short_fits(W, M, E, true, region);
+  const bool stream_dx = dX && !short_dx && stream_fits(W, M, E, true, region);
   st = launch_lora_down(true, dY, M, W->N, B, r, scale, ts, U, Zs, ws_status(ws), offsets, E,
-                        grouped, !dX ? 0 : (short_dx ? kDownCtasBesideStream : kDownCtasBesidePair), s);
+                        grouped,
+                        !dX ? 0 : ((short_dx || stream_dx) ? kDownCtasBesideStream : kDownCtasBesidePair),
+                        s, short_dx ? short_zs_mul(W) : 1.0f);
   if (st != QLORA_OK) return st;
+  auto run_dx = [&]() {
+    if (short_dx) return launch_short(W, true, dY, Zs, A, dX, M, r, ws, part, region, s);
+    if (stream_dx) return launch_stream(W, true, dY, Zs, A, dX, M, r, ws_status(ws), part, region, s);
+    return launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), offsets, E, grouped, s);
+  };
   if (dX) {
     // The adapter gradients need only T, U, X and dY, so they run on a side stream beside the dX
     // kernel, on the SMs it leaves idle (the tiled kernel's last wave of tiles; the SMs the
@@ -745,17 +882,13 @@ qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
                         side->stream);
       if (st != QLORA_OK) return st;
       if (cudaEventRecord(side->join[slot], side->stream) != cudaSuccess) return QLORA_ERR_CUDA;
-      st = short_dx ? launch_stream(W, true, dY, Zs, A, dX, M, r, ws_status(ws), part,
-                                    ws_bytes - L.partial, s)
-                    : launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), offsets, E, grouped, s);
+      st = run_dx();
       if (cudaStreamWaitEvent(s, side->join[slot], 0) != cudaSuccess) return QLORA_ERR_CUDA;
       return st;
     }
   }
   if (dX) {
-    st = short_dx ? launch_stream(W, true, dY, Zs, A, dX, M, r, ws_status(ws), part,
-                                  ws_bytes - L.partial, s)
-                  : launch_fused(W, true, dY, Zs, A, dX, M, r, ws_status(ws), offsets, E, grouped, s);
+    st = run_dx();
     if (st != QLORA_OK) return st;
   }
   return launch_wgrad(X, dY, T, U, M, W->N, W->K, r, scale, dA, dB, ws, L, offsets, E, grouped, s);
@@ -789,16 +922,16 @@ qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const void* X, 
   if (!act_ok(X, M) || !ptr_ok(A) || !ptr_ok(B) || !act_ok(Y, M) || (T_save && !aligned16(T_save)))
     return QLORA_ERR_INVALID_ARG;
   const size_t mr = align_up(size_t(M) * size_t(r) * 2, 256);
-  const size_t need = kHeaderBytes + mr + (T_save ? 0 : mr);
+  const size_t need = kNoAllocHeaderBytes + mr + (T_save ? 0 : mr);
   if (need > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
   if (M == 0) return QLORA_OK;
   uint8_t* w = static_cast<uint8_t*>(noalloc_scratch_address());
   if (!w) return QLORA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(w, 0, kHeaderBytes, s) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaMemsetAsync(w, 0, kNoAllocHeaderBytes, s) != cudaSuccess) return QLORA_ERR_CUDA;
   int* status = reinterpret_cast<int*>(w);
-  void* Zs = w + kHeaderBytes;
-  void* T = T_save ? T_save : w + kHeaderBytes + mr;
+  void* Zs = w + kNoAllocHeaderBytes;
+  void* T = T_save ? T_save : w + kNoAllocHeaderBytes + mr;
   const float* ts = W->fmt == QLORA_FMT_NVFP4 ? W->tensor_scale : nullptr;
   st = launch_lora_down(false, X, M, W->K, A, r, scale, ts, T, Zs, status, nullptr, 1, false,
                         kDownCtasBesidePair, s);
@@ -865,6 +998,29 @@ qlora_status_t qlora_debug_dequant(const qlora_weight_t* W, int transposed, void
   qlora_status_t st = check_weight(W);
   if (st != QLORA_OK) return st;
   if (!ptr_ok(out)) return QLORA_ERR_INVALID_ARG;
+  if (transposed < 0 || transposed > 3) return QLORA_ERR_INVALID_ARG;
+  if (transposed >= 2) {   // the short-batch kernels' decoders
+    if (W->fmt == QLORA_FMT_NF4_DQ) return QLORA_ERR_UNSUPPORTED;
+    ShortParams sp{};
+    sp.codes = static_cast<const uint8_t*>(W->codes);
+    sp.scales = W->scales;
+    sp.out = static_cast<__nv_bfloat16*>(out);
+    sp.N = int(W->N);
+    sp.K = int(W->K);
+    sp.one = 1u;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const unsigned grid = unsigned((W->N * (W->K / 64) + 127) / 128);
+    const bool regs = transposed == 2;
+    switch (W->fmt * 2 + (regs ? 1 : 0)) {
+      case 0: qlora_debug_short_decode_kernel<kFmtNF4, false><<<grid, 128, 0, s>>>(sp); break;
+      case 1: qlora_debug_short_decode_kernel<kFmtNF4, true><<<grid, 128, 0, s>>>(sp); break;
+      case 2: qlora_debug_short_decode_kernel<kFmtMXFP4, false><<<grid, 128, 0, s>>>(sp); break;
+      case 3: qlora_debug_short_decode_kernel<kFmtMXFP4, true><<<grid, 128, 0, s>>>(sp); break;
+      case 4: qlora_debug_short_decode_kernel<kFmtNVFP4, false><<<grid, 128, 0, s>>>(sp); break;
+      default: qlora_debug_short_decode_kernel<kFmtNVFP4, true><<<grid, 128, 0, s>>>(sp); break;
+    }
+    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  }
   DebugDequantParams p{};
   const bool dx = transposed != 0;
   const int64_t N = W->N, K = W->K;
@@ -1194,9 +1350,9 @@ qlora_status_t qlora_debug_decode_rate(int fmt, int iters, double* weights_per_c
     cudaFree(cyc);
     return QLORA_ERR_CUDA;
   }
-  if (fmt == QLORA_FMT_NF4) qlora_debug_decode_rate_kernel<kFmtNF4><<<sms, 256>>>(iters, cyc, sink);
-  else if (fmt == QLORA_FMT_MXFP4) qlora_debug_decode_rate_kernel<kFmtMXFP4><<<sms, 256>>>(iters, cyc, sink);
-  else qlora_debug_decode_rate_kernel<kFmtNVFP4><<<sms, 256>>>(iters, cyc, sink);
+  if (fmt == QLORA_FMT_NF4) qlora_debug_decode_rate_kernel<kFmtNF4><<<sms, 512>>>(iters, cyc, sink, 1u);
+  else if (fmt == QLORA_FMT_MXFP4) qlora_debug_decode_rate_kernel<kFmtMXFP4><<<sms, 512>>>(iters, cyc, sink, 1u);
+  else qlora_debug_decode_rate_kernel<kFmtNVFP4><<<sms, 512>>>(iters, cyc, sink, 1u);
   std::vector<unsigned long long> h(sms);
   const bool ok = cudaGetLastError() == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess &&
                   cudaMemcpy(h.data(), cyc, sizeof(unsigned long long) * sms,
@@ -1207,7 +1363,7 @@ qlora_status_t qlora_debug_decode_rate(int fmt, int iters, double* weights_per_c
   double c = 0;
   for (int i = 0; i < sms; ++i) c += double(h[i]);
   c /= sms;
-  *weights_per_clock_per_sm = c > 0 ? double(iters) * 256.0 * 64.0 / c : 0.0;
+  *weights_per_clock_per_sm = c > 0 ? double(iters) * 512.0 * 64.0 / c : 0.0;
   return QLORA_OK;
 }
 

@@ -3,6 +3,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include "qlora_fused.cuh"
+#include "qlora_short.cuh"
 
 namespace qlora {
 
@@ -71,18 +72,51 @@ qlora_debug_dequant_kernel(const __grid_constant__ DebugDequantParams p) {
   }
 }
 
-// Decode throughput of the layer's own dequant stage on one SM, the bound of the short-batch
-// (weight-streaming) path: 256 threads (the two dequant groups' worth) each decode `iters`
-// 64-element items with dequant_item_store into a swizzled operand tile, fresh codes every item
-// (updated with a multiply-add, so the integer pipe does only decode work).  cycles[b] = the CTA's
-// clock cycles for the loop.
+// The short-batch kernels' decoders run on their own: one thread per 64-element item (row n,
+// columns [64 c, 64 c + 64)), with the item's codes and block scale.
+// REGS = true: decode_item_regs (the forward's tensor-memory form), written straight out;
+// REGS = false: decode_item_store into a swizzled shared-memory row, read back through the swizzle.
+// NVFP4 elements come out times 2^-8, as those kernels use them.
+template <int FMT, bool REGS>
+__global__ void __launch_bounds__(128)
+qlora_debug_short_decode_kernel(const __grid_constant__ ShortParams p) {
+  __shared__ __align__(1024) uint8_t rows[128 * 128];
+  const int item = int(blockIdx.x) * 128 + int(threadIdx.x);
+  const int per_row = p.K / 64;
+  if (item >= p.N * per_row) return;
+  const int n = item / per_row, kcol = (item - n * per_row) * 64;
+  const uint4* cp = reinterpret_cast<const uint4*>(p.codes + size_t(n) * size_t(p.K / 2) + size_t(kcol / 2));
+  const uint4 c0 = cp[0], c1 = cp[1];
+  const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  ItemScale sc = load_item_scale<FMT>(p.scales, n, kcol, p.K);
+  const DecodeMul km = decode_mul(p.one);
+  uint4* dst = reinterpret_cast<uint4*>(p.out + size_t(n) * p.K + kcol);
+  if constexpr (REGS) {
+    uint32_t o[32];
+    decode_item_regs<FMT>(cw, sc, km, o);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+  } else {
+    const uint32_t rb = ptx::smem_u32(rows) + threadIdx.x * 128u;
+    const uint32_t swz = threadIdx.x & 7u;
+    decode_item_store<FMT>(cw, sc, km, rb, swz);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) dst[j] = ptx::ld_shared_v4(rb + ((uint32_t(j) ^ swz) << 4));
+  }
+}
+
+// Decode throughput of the short-batch kernels' dequant stage on one SM, the bound of the
+// short-batch path: 512 threads (the short-batch kernels' 16 dequant warps) each decode `iters`
+// 64-element items with decode_item_store into a swizzled operand tile, fresh codes every item
+// (one xor per code word).  cycles[b] = the CTA's clock cycles for the loop.
 template <int FMT>
-__global__ void __launch_bounds__(256, 1)
-qlora_debug_decode_rate_kernel(int iters, unsigned long long* cycles, uint32_t* sink) {
+__global__ void __launch_bounds__(512, 1)
+qlora_debug_decode_rate_kernel(int iters, unsigned long long* cycles, uint32_t* sink, uint32_t one) {
   __shared__ __align__(1024) uint8_t tile[2][fused::W_BYTES];
   const int tg = threadIdx.x & 127;
   const ItemGeom<false> geo(tg);
-  const uint32_t rb = geo.op_row_base(ptx::smem_u32(tile[threadIdx.x >> 7]));
+  const uint32_t rb = geo.op_row_base(ptx::smem_u32(tile[(threadIdx.x >> 7) & 1]));
+  const DecodeMul km = decode_mul(one);
   uint32_t cw[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) cw[j] = (threadIdx.x * 8u + j + blockIdx.x * 7919u) * 0x9E3779B1u;
@@ -92,9 +126,9 @@ qlora_debug_decode_rate_kernel(int iters, unsigned long long* cycles, uint32_t* 
   __syncthreads();
   const unsigned long long t0 = clock64();
   for (int it = 0; it < iters; ++it) {
-    dequant_item_store<FMT>(cw, sc, rb, geo.swz());
+    decode_item_store<FMT>(cw, sc, km, rb, geo.swz());
 #pragma unroll
-    for (int j = 0; j < 8; ++j) cw[j] = cw[j] * 0x9E3779B1u + 0x7F4A7C15u;
+    for (int j = 0; j < 8; ++j) cw[j] ^= 0x9E3779B1u + uint32_t(it);
   }
   __syncthreads();
   const unsigned long long t1 = clock64();

@@ -177,6 +177,188 @@ __device__ __forceinline__ void dequant_item_store(const uint32_t (&cw)[8], Item
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Short-batch decoders.  On sm_100a the byte-permute, logic and shift instructions share one
+// 64-lane-per-clock pipe, while integer multiply-add and packed bf16 multiplies share another of
+// the same width, so the decoders below move shifts onto the multiply pipe: a right shift by n is
+// the high word of a multiply by 2^(32-n), a left shift a multiply by 2^n.  The multipliers come
+// from a run-time 1 (a kernel argument) so the compiler cannot turn them back into shifts.
+struct DecodeMul {
+  uint32_t hi16, hi28, hi29;   // 2^16, 2^28, 2^29: high words give >> 16, >> 4, >> 3
+  uint32_t x63, x64;           // 63, 64
+};
+__device__ __forceinline__ DecodeMul decode_mul(uint32_t one) {
+  DecodeMul k;
+  k.hi16 = one << 16;
+  k.hi28 = one << 28;
+  k.hi29 = one << 29;
+  k.x63 = one * 63u;
+  k.x64 = one << 6;
+  return k;
+}
+
+// NF4: 8 codes of w through the item's 16-entry table; out[i] = {t[code 2i], t[code 2i+1]}.
+// Same selection as lut16_lookup8, with the selector shifts done as multiply-high.
+__device__ __forceinline__ void nf4_lookup8_mul(const Lut16& t, uint32_t w, const DecodeMul& k,
+                                                uint32_t (&out)[4]) {
+  const uint32_t b3 = w & 0x88888888u;                 // bit 3 of each code
+  const uint32_t sel3 = w ^ b3;                        // low 3 bits of each code
+  const uint32_t msel = __umulhi(b3, k.hi29) + b3;     // b3 | (b3 >> 3): 9 where code >= 8
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t s = h ? __umulhi(sel3, k.hi16) : sel3;
+    const uint32_t ms = h ? __umulhi(msel, k.hi16) : msel;
+    const uint32_t m = ptx::prmt(0x00008000u, 0u, ms);  // byte i = 0xFF where code i >= 8
+    const uint32_t lo0 = ptx::prmt(t.lo[0], t.lo[1], s);
+    const uint32_t lo1 = ptx::prmt(t.lo[2], t.lo[3], s);
+    const uint32_t hi0 = ptx::prmt(t.hi[0], t.hi[1], s);
+    const uint32_t hi1 = ptx::prmt(t.hi[2], t.hi[3], s);
+    const uint32_t lo = (lo0 & ~m) | (lo1 & m);
+    const uint32_t hi = (hi0 & ~m) | (hi1 & m);
+    out[2 * h] = ptx::prmt(lo, hi, 0x5140u);
+    out[2 * h + 1] = ptx::prmt(lo, hi, 0x7362u);
+  }
+}
+
+// E2M1 bit placement: for a code c = s e1 e0 m the bf16 pattern (c & 7) << 6 | (c & 8) << 12 puts
+// e1 e0 in the two lowest exponent bits and m in the top mantissa bit, which is exactly
+// e2m1(c) * 2^-126 (e1 e0 = 0 lands on the bf16 subnormals 0 and 2^-127, matching E2M1's own
+// subnormal 0.5 m), with the sign in place.  One packed bf16 multiply by (block scale * 2^126)
+// then gives e2m1(c) * scale exactly whenever that product is representable.
+// out[i] = {pattern(code 2i), pattern(code 2i+1)}.
+__device__ __forceinline__ void e2m1_pattern8(uint32_t w, const DecodeMul& k, uint32_t (&out)[4]) {
+  const uint32_t lo = w & 0x0F0F0F0Fu;                        // codes 2i in byte i
+  const uint32_t hi = __umulhi(w, k.hi28) & 0x0F0F0F0Fu;      // codes 2i+1 in byte i
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    // byte 0 <- code 2i, byte 2 <- code 2i+1, bytes 1 and 3 <- the sign of a byte whose top bit
+    // is 0, i.e. zero: each 16-bit lane holds one bare code
+    const uint32_t x = ptx::prmt(lo, hi, uint32_t(i) | 0x80u | (uint32_t(4 + i) << 8) | 0x8000u);
+    const uint32_t sg = x & 0x00080008u;
+    out[i] = (x + sg * k.x63) * k.x64;                        // mag << 6 | sign << 12
+  }
+}
+
+// Packed bf16 scale operands for the bit-placement decode.
+//   MXFP4: 2^(e-1) (= 2^(e-127) * 2^126), exact for e <= 128; bit 0 of *slow* is set when an
+//          E8M0 exponent is above 128 (the product no longer fits: decode in two multiplies).
+//   NVFP4: e4m3(s) * 2^118, exact for every E4M3 byte (NaN stays NaN): the decoded element is
+//          e2m1 * e4m3 * 2^-8, and the kernel multiplies its accumulator by 2^8 * tensor scale.
+__device__ __forceinline__ uint32_t mx_fast_scale(uint32_t e) {
+  const uint32_t v = ((e & 0xFFu) + 126u) << 7;
+  return v | (v << 16);
+}
+__device__ __forceinline__ uint32_t nv_shifted_scale(uint32_t b) {
+  const uint32_t v = __float_as_uint(__fmul_rn(e4m3_f32(b), 3.3230699894622896e+35f)) >> 16;  // 2^118
+  return v | (v << 16);
+}
+// 2^126 in both halves, and the exact E8M0 scale in both halves.
+constexpr uint32_t kBf16x2Pow126 = 0x7E807E80u;
+__device__ __forceinline__ uint32_t mx_exact_scale(uint32_t e) {
+  const uint32_t v = e8m0_bf16(e);
+  return v | (v << 16);
+}
+
+// Decode one 64-element item into 32 packed words (word j = elements 2j, 2j+1), for operands kept
+// in tensor memory.  NVFP4 elements come out times 2^-8 (see nv_shifted_scale).
+template <int FMT>
+__device__ __forceinline__ void decode_item_regs(const uint32_t (&cw)[8], ItemScale sc,
+                                                 const DecodeMul& k, uint32_t (&o)[32]) {
+  if constexpr (FMT == kFmtNF4 || FMT == kFmtNF4DQ) {
+    const Lut16 t = nf4_lut(__uint_as_float(sc.raw));
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint32_t q[4];
+      nf4_lookup8_mul(t, cw[j], k, q);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[4 * j + i] = q[i];
+    }
+  } else if constexpr (FMT == kFmtMXFP4) {
+    const uint32_t e0 = sc.raw & 0xFFu, e1 = (sc.raw >> 8) & 0xFFu;
+    if (e0 <= 128u && e1 <= 128u) {
+      const uint32_t s0 = mx_fast_scale(e0), s1 = mx_fast_scale(e1);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t q[4];
+        e2m1_pattern8(cw[j], k, q);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[4 * j + i] = ptx::mul_bf16x2(q[i], j < 4 ? s0 : s1);
+      }
+    } else {
+      const uint32_t s0 = mx_exact_scale(e0), s1 = mx_exact_scale(e1);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t q[4];
+        e2m1_pattern8(cw[j], k, q);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          o[4 * j + i] = ptx::mul_bf16x2(ptx::mul_bf16x2(q[i], kBf16x2Pow126), j < 4 ? s0 : s1);
+      }
+    }
+  } else {
+    uint32_t s[4];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) s[q4] = nv_shifted_scale((sc.raw >> (8 * q4)) & 0xFFu);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint32_t q[4];
+      e2m1_pattern8(cw[j], k, q);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[4 * j + i] = ptx::mul_bf16x2(q[i], s[j >> 1]);
+    }
+  }
+}
+
+// The same decode stored as eight swizzled 16-byte chunks (chunk j at row_base + ((j ^ swz) << 4)),
+// for operands kept in shared memory.  NVFP4 elements come out times 2^-8.
+template <int FMT>
+__device__ __forceinline__ void decode_item_store(const uint32_t (&cw)[8], ItemScale sc,
+                                                  const DecodeMul& k, uint32_t row_base,
+                                                  uint32_t swz) {
+  if constexpr (FMT == kFmtNF4 || FMT == kFmtNF4DQ) {
+    const Lut16 t = nf4_lut(__uint_as_float(sc.raw));
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint32_t q[4];
+      nf4_lookup8_mul(t, cw[j], k, q);
+      ptx::st_shared_v4(row_base + ((uint32_t(j) ^ swz) << 4), q[0], q[1], q[2], q[3]);
+    }
+  } else {
+    uint32_t s[4];
+    bool slow = false;
+    if constexpr (FMT == kFmtMXFP4) {
+      const uint32_t e0 = sc.raw & 0xFFu, e1 = (sc.raw >> 8) & 0xFFu;
+      slow = e0 > 128u || e1 > 128u;
+      s[0] = s[1] = slow ? mx_exact_scale(e0) : mx_fast_scale(e0);
+      s[2] = s[3] = slow ? mx_exact_scale(e1) : mx_fast_scale(e1);
+    } else {
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) s[q4] = nv_shifted_scale((sc.raw >> (8 * q4)) & 0xFFu);
+    }
+    if (!slow) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t q[4];
+        e2m1_pattern8(cw[j], k, q);
+        const uint32_t sj = s[j >> 1];
+        ptx::st_shared_v4(row_base + ((uint32_t(j) ^ swz) << 4), ptx::mul_bf16x2(q[0], sj),
+                          ptx::mul_bf16x2(q[1], sj), ptx::mul_bf16x2(q[2], sj),
+                          ptx::mul_bf16x2(q[3], sj));
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t q[4];
+        e2m1_pattern8(cw[j], k, q);
+        const uint32_t sj = s[j >> 1];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) q[i] = ptx::mul_bf16x2(ptx::mul_bf16x2(q[i], kBf16x2Pow126), sj);
+        ptx::st_shared_v4(row_base + ((uint32_t(j) ^ swz) << 4), q[0], q[1], q[2], q[3]);
+      }
+    }
+  }
+}
+
 // Store 64 zeros (an item outside the weight).
 __device__ __forceinline__ void zero_item_store(uint32_t row_base) {
 #pragma unroll

@@ -89,6 +89,7 @@ struct FusedParams {
   int M, N, K, r, E;                 // M: all rows (packed over experts)
   int num_n, num_k;                  // pair tiles over output columns; contraction steps
   int tail_split;                    // the last tail_split 512-row tiles run as 2 x 256-row tiles
+  uint32_t zero;                     // 0 (see zero_after)
 };
 
 __device__ __forceinline__ void fused_tile_coords(int t, int num_m, int num_n, int& mt, int& nt) {
@@ -531,8 +532,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
         // release the code stage only once the loaded code words have been consumed: the
         // producer's next TMA into this stage must not overtake the loads above
         const uint32_t used = (c_lo.x ^ c_lo.y ^ c_lo.z ^ c_lo.w) ^ (c_hi.x ^ c_hi.y ^ c_hi.z ^ c_hi.w);
-        uint32_t dep;
-        asm volatile("and.b32 %0, %1, 0;" : "=r"(dep) : "r"(used));
+        const uint32_t dep = ptx::zero_after(used, p.zero);
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(empty_c(scs) + dep);
       } else {

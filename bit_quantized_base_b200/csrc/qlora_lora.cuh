@@ -132,6 +132,8 @@ struct DownParams {
   int* status;
   int M, r, rpad, num_k, S, steps_per_split, E;
   float s;
+  float zs_mul;        // an exact power of two folded into Zs (2^-8 when the next kernel decodes
+                       // NVFP4 elements times 2^-8), else 1
 };
 
 template <bool R_MN>
@@ -186,7 +188,7 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
   const uint32_t rowb = uint32_t(p.rpad) * 2u;
   const uint32_t r_bytes = uint32_t(p.rpad) * 128u;
   const float ts = p.tensor_scale ? __ldg(p.tensor_scale + e) : 1.0f;
-  const float zscale = p.s / ts;
+  const float zscale = p.s / ts * p.zs_mul;
   // Z and Zs = bf16(Z * s / ts) for columns c .. c+7 of row rw
   auto write8 = [&](int rw, int c, const float (&v)[8]) {
     if (c >= p.r) return;

@@ -78,6 +78,7 @@ struct StreamParams {
   int iters;                         // L: (tile, step) iterations per CTA
   long long lcm;                     // lcm(L, num_k + 1)
   int xrows;                         // M rounded up to 16: activation rows per stage, MMA N
+  uint32_t zero;                     // 0 (see zero_after)
 };
 
 // Segments are the pieces of the iteration space between consecutive CTA-range starts (multiples
@@ -409,8 +410,7 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
         }
         if (!ok) break;
         // release the code stage only once the loaded words have been consumed
-        uint32_t dep;
-        asm volatile("and.b32 %0, %1, 0;" : "=r"(dep) : "r"(used));
+        const uint32_t dep = ptx::zero_after(used, p.zero);
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(empty_c(scs) + dep);
       } else {
@@ -442,7 +442,7 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
         }
         if (!ok) break;
       }
-      asm volatile("and.b32 %0, %1, 0;" : "=r"(sdep) : "r"(sdep));
+      sdep = ptx::zero_after(sdep, p.zero);
       scale_fetch(pf, slot, sdep);
       ptx::fence_proxy_async_smem();
       __syncwarp();

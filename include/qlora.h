@@ -206,7 +206,10 @@ QLORA_API qlora_status_t qlora_get_device_status(void* ws, qlora_stream_t stream
 /* Test-only: decode the whole weight through the kernels' own dequant stage (TMA code loads,
  * register decode, swizzled shared-memory tile) and write it un-swizzled as bf16 [N,K] to `out`
  * (N*K*2 bytes).  transposed = 0 uses the forward tiling (K-major operand tile), 1 the dX tiling
- * (MN-major operand tile).  NVFP4 is written WITHOUT the tensor scale (the kernels apply it in the
+ * (MN-major operand tile); 2 and 3 run the short-batch kernels' decoders (batches of up to 64
+ * rows: 2 the forward's register / tensor-memory form, 3 the dX shared-memory form; not for
+ * NF4_DQ, which those kernels do not take) -- their NVFP4 elements are written times 2^-8, as
+ * those kernels use them.  NVFP4 is written WITHOUT the tensor scale (the kernels apply it in the
  * epilogue).  This is the one call that writes a bf16 weight to memory: it exists to check the
  * decode bit for bit and is never used by the layer. */
 QLORA_API qlora_status_t qlora_debug_dequant(const qlora_weight_t* W, int transposed, void* out,
@@ -278,10 +281,10 @@ QLORA_API qlora_status_t qlora_loftq(const float* W, const qlora_weight_t* Q, in
                                      void* B_out, float* errs, float* sigma, void* work,
                                      size_t work_bytes, qlora_stream_t stream);
 
-/* Benchmark support: measure the decode throughput of the layer's own dequant stage (the code
- * every GEMM kernel decodes the 4-bit weight with) on every SM -- 256 threads per SM, each
- * decoding `iters` 64-element items into a shared-memory operand tile -- and return the mean
- * decoded weights per SM clock cycle in *weights_per_clock_per_sm.  fmt: QLORA_FMT_*; 1 <= iters
+/* Benchmark support: measure the decode throughput of the short-batch kernels' dequant stage
+ * (the decoder that streams the 4-bit weight at batches of up to 64 rows) on every SM -- 512
+ * threads per SM, each decoding `iters` 64-element items into a shared-memory operand tile -- and
+ * return the mean decoded weights per SM clock cycle in *weights_per_clock_per_sm.  fmt: QLORA_FMT_*; 1 <= iters
  * <= 2^20.  Synchronises the device and allocates two small device buffers; not for the compute
  * path.  The result is the ceiling of the short-batch path, where every weight is decoded for a
  * few activation rows. */
@@ -293,7 +296,9 @@ QLORA_API qlora_status_t qlora_debug_decode_rate(int fmt, int iters,
  * bracketed by two CUDA events recorded on its stream (up to 65536 launches; events are created by
  * qlora_profile_enable, never on the compute path); qlora_profile_read synchronises on them and
  * returns, per kernel kind, the launch count and total milliseconds.  Kinds: "fused_fwd",
- * "fused_dx", "lora_down_T", "lora_down_U", "lora_wgrad" (grouped variants add "grouped_").
+ * "fused_dx", "lora_down_T", "lora_down_U", "lora_wgrad" (grouped variants add "grouped_"),
+ * "stream_fwd", "stream_dx", "stream_reduce" (batches of 65-256 rows), "short_fwd", "short_dx"
+ * (batches of up to 64 rows).
  * Host-side bookkeeping only; the compute path is unchanged when profiling is off. */
 QLORA_API int64_t qlora_launch_count(void);
 QLORA_API qlora_status_t qlora_profile_enable(int enable);
