@@ -272,8 +272,10 @@ def job_value(ws_n, flops_per_step, steps, ms_max):
 
 def short_batch_sweep(Q, torch, p, Ws, X, dY, A, B, peaks):
     """fwd+bwd at M in {16, 32, 64, 128, 256} on one weight (rotating device copies whose total
-    exceeds 3x L2): weight bytes read per step (two passes) / time, TFLOP/s, and the fraction of
-    the binding roofline max(flops / bf16 peak, bytes / HBM peak, decoded weights / decode peak).
+    exceeds 3x L2): weight bytes read per step (two passes) / time and that rate as a fraction of
+    the measured HBM bandwidth (hbm_frac), TFLOP/s, the fraction of the binding roofline
+    max(flops / bf16 peak, bytes / HBM peak, decoded weights / decode peak), and the clock record
+    of each point's own timed region (at least ~50 ms of steps).
     The decode peak is the library's own dequant stage measured on every SM of this GPU
     (qlora_debug_decode_rate: decoded weights per SM clock) x SMs x the maximum SM clock; it binds
     the short batches, where each decoded weight meets only M activation rows."""
@@ -306,17 +308,23 @@ def short_batch_sweep(Q, torch, p, Ws, X, dY, A, B, peaks):
             Q.qlora_linear_fwd(w, Xm, A, B, Ym, Tm, Ms, r, s, wsm)
             Q.qlora_linear_bwd(w, Xm, A, B, Tm, dYm, dXm, dA, dB, Ms, r, s, wsm)
 
-        for i in range(5):
-            sstep(i)
-        torch.cuda.synchronize()
-        n_it = 60
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for i in range(5):
+            sstep(i)
+        a1.record()
+        a1.synchronize()
+        # at least ~50 ms of timed steps, so the clock record holds several samples
+        n_it = max(60, int(0.05 / max(a0.elapsed_time(a1) / 5 * 1e-3, 1e-6)))
+        clk = NvmlSampler(torch.cuda.current_device())
+        clk.start()
         a0.record()
         for i in range(n_it):
             sstep(i)
         a1.record()
         a1.synchronize()
+        crec = clk.stop()
         if Q.qlora_get_device_status(wsm) != 0:
             raise RuntimeError("device status in the short-batch sweep")
         t = a0.elapsed_time(a1) / n_it * 1e-3
@@ -328,9 +336,11 @@ def short_batch_sweep(Q, torch, p, Ws, X, dY, A, B, peaks):
         bound = max(bounds, key=bounds.get)
         out[str(Ms)] = {"us_per_step": round(t * 1e6, 1),
                         "weight_gbs": round(2 * wbytes / t / 1e9, 1),
+                        "hbm_frac": round(2 * wbytes / t / (peaks["hbm_gbs"] * 1e9), 4),
                         "tflops": round(fl / t / 1e12, 1),
                         "roofline_frac": round(bounds[bound] / t, 4),
-                        "bound": bound}
+                        "bound": bound, "steps": n_it,
+                        "clocks": {k: crec.get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")}}
     out["decode_peak"] = {"weights_per_clk_per_sm": round(per_clk, 2), "sms": sms,
                           "sm_mhz": clk_hz / 1e6, "weights_per_s": round(decode_peak / 1e12, 3),
                           "unit": "T weights/s", "source": "qlora_debug_decode_rate (measured)"}

@@ -552,6 +552,7 @@ qlora_status_t launch_stream(const qlora_weight_t* W, bool dx, const void* act, 
   p.num_tiles = sp.tiles;
   p.iters = sp.iters;
   p.lcm = sp.lcm;
+  p.segments = sp.segments;
   qlora_status_t rc;
   switch ((W->fmt * 2 + (dx ? 1 : 0)) * 2 + (mt - 1)) {
     case 0: rc = launch_stream_t<kFmtNF4, false, 1>(p, sp.grid, st); break;
@@ -1392,7 +1393,11 @@ const char* qlora_status_string(qlora_status_t status) {
   return "unknown status";
 }
 
+#ifdef QLORA_DEBUG
+const char* qlora_build_info(void) { return "qlora-b200 0.1 sm_100a debug (device bounds checks)"; }
+#else
 const char* qlora_build_info(void) { return "qlora-b200 0.1 sm_100a"; }
+#endif
 
 int64_t qlora_launch_count(void) { return g_launches.load(); }
 

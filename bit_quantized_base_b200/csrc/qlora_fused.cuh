@@ -311,8 +311,12 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
           const uint32_t fx = ptx::mapa(full_s(sx), 0);
           for (int blk = 0; blk < pt.nb; ++blk) {
             const uint32_t xd = ptx::smem_u32(xs + (sx * MB + blk) * X_BYTES);
-            if (ks < nk) ptx::tma_load_2d_pair(xd, &p.tm_act, fx, ks * BK, m0 + blk * 2 * HM);
-            else ptx::tma_load_2d_pair(xd, &p.tm_zs, fx, 0, m0 + blk * 2 * HM);
+            if (ks < nk) {
+              if (ptx::dcheck(ptx::tma_x_ok(ks * BK, 2), p.status))
+                ptx::tma_load_2d_pair(xd, &p.tm_act, fx, ks * BK, m0 + blk * 2 * HM);
+            } else {
+              ptx::tma_load_2d_pair(xd, &p.tm_zs, fx, 0, m0 + blk * 2 * HM);
+            }
           }
         }
         if (!ok) break;
@@ -332,8 +336,10 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
           if (!ptx::mbar_wait(empty_c(sc), pc ^ 1u, p.status, abort_flag)) { ok = false; break; }
           ptx::mbar_arrive_expect_tx(full_c(sc), C_BYTES);
           const uint32_t cd = ptx::smem_u32(cs + sc * C_BYTES);
-          if (!DX) ptx::tma_load_2d(cd, &p.tm_codes, full_c(sc), ks * (BK / 2), wrow0 + h0);
-          else ptx::tma_load_2d(cd, &p.tm_codes, full_c(sc), h0 / 2, wrow0 + ks * BK);
+          const int cx = !DX ? ks * (BK / 2) : h0 / 2;
+          if (!ptx::dcheck(ptx::tma_x_ok(cx, 1) && pt.e < p.E, p.status)) continue;
+          if (!DX) ptx::tma_load_2d(cd, &p.tm_codes, full_c(sc), cx, wrow0 + h0);
+          else ptx::tma_load_2d(cd, &p.tm_codes, full_c(sc), cx, wrow0 + ks * BK);
         }
         if (!ok) break;
       }
@@ -455,7 +461,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
 #pragma unroll
           for (int it = 0; it < 4; ++it) {
             const int row = rbase + it * 8 + rr0;
-            if (row < pt.row_end && col < ncols)
+            if (row < pt.row_end && col < ncols && ptx::dcheck(row >= 0 && pt.row_end <= p.M, p.status))
               *reinterpret_cast<uint4*>(p.out + size_t(row) * ncols + col) = o[it];
           }
         }

@@ -192,6 +192,7 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
   // Z and Zs = bf16(Z * s / ts) for columns c .. c+7 of row rw
   auto write8 = [&](int rw, int c, const float (&v)[8]) {
     if (c >= p.r) return;
+    if (!ptx::dcheck(rw >= 0 && rw < p.M, p.status)) return;
     uint4 z, zs;
     z.x = ptx::cvt_bf16x2(v[0], v[1]); z.y = ptx::cvt_bf16x2(v[2], v[3]);
     z.z = ptx::cvt_bf16x2(v[4], v[5]); z.w = ptx::cvt_bf16x2(v[6], v[7]);
@@ -210,6 +211,7 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
         const uint32_t s = it % NS, ph = (it / NS) & 1;
         if (!ptx::mbar_wait(empty(s), ph ^ 1u, p.status, abort_flag)) break;
         ptx::mbar_arrive_expect_tx(full(s), A_BYTES + r_bytes);
+        if (!ptx::dcheck(ptx::tma_x_ok(ks * BK, 2) && e < p.E, p.status)) break;
         ptx::tma_load_2d(ptx::smem_u32(as + s * A_BYTES), &p.tm_act, full(s), ks * BK, m0);
         if (!R_MN) ptx::tma_load_3d(ptx::smem_u32(rs + s * R_BYTES), &p.tm_r, full(s), ks * BK, 0, e);
         else ptx::tma_load_3d(ptx::smem_u32(rs + s * R_BYTES), &p.tm_r, full(s), 0, ks * BK, e);
@@ -351,6 +353,7 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
   // s * the reduction for columns c .. c+7 of output row pr (dB row-major, dA transposed)
   auto write8 = [&](int pr, int c, const float (&v)[8]) {
     if (c >= p.r) return;
+    if (!ptx::dcheck(pr >= 0 && pr < (prob == 0 ? p.P0 : p.P1) && e < p.E, p.status)) return;
     if (prob == 0) {
       uint4 o;
       o.x = ptx::cvt_bf16x2(v[0] * p.s, v[1] * p.s);
@@ -373,6 +376,7 @@ qlora_lora_wgrad_kernel(const __grid_constant__ WgradParams p) {
         ptx::mbar_arrive_expect_tx(full(s), A_BYTES + r_bytes);
         const uint32_t ad = ptx::smem_u32(as + s * A_BYTES);
         const int m = row_begin + ks * BK;
+        if (!ptx::dcheck(ptx::tma_x_ok(p0, 2) && m >= 0 && m < p.M, p.status)) break;
         ptx::tma_load_2d(ad, tml, full(s), p0, m);
         ptx::tma_load_2d(ad + A_BYTES / 2, tml, full(s), p0 + 64, m);
         ptx::tma_load_2d(ptx::smem_u32(rs + s * R_BYTES), tmr, full(s), 0, m);

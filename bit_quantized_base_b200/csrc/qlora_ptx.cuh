@@ -87,6 +87,26 @@ __device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity, in
   }
 }
 
+// Debug build (compiled with -DQLORA_DEBUG into libqlora_debug.so): the kernels check their own
+// index arithmetic before the accesses it computes.  dcheck(ok, status) returns ok; when ok is
+// false it records QLORA_ERR_INVALID_ARG in the launch's status word (the first error wins) and
+// the caller skips the access instead of faulting.  A skipped TMA copy leaves its barrier short of
+// bytes, and the bounded wait on that barrier then ends the launch.  In the release build dcheck
+// is `true` and the checks compile away.
+#ifdef QLORA_DEBUG
+__device__ __forceinline__ bool dcheck(bool ok, int* status) {
+  if (!ok && status) atomicCAS(status, 0, 1 /* QLORA_ERR_INVALID_ARG */);
+  return ok;
+}
+#else
+__device__ __forceinline__ bool dcheck(bool, int*) { return true; }
+#endif
+// The innermost coordinate of a tiled TMA copy: not below zero, and its byte offset a multiple of
+// 16 (an unaligned start is an illegal instruction).
+__device__ __forceinline__ bool tma_x_ok(int x, int elem_bytes) {
+  return x >= 0 && ((x * elem_bytes) & 15) == 0;
+}
+
 // Zero, computed from v: `zero` is a kernel argument the host sets to 0, which the compiler cannot
 // see, so the AND is not folded away and an instruction that takes the result issues only once v
 // has arrived.  Used to hold a slot-release arrive (or a refill of the slot) behind the shared-

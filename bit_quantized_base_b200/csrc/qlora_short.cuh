@@ -226,7 +226,8 @@ qlora_short_fwd_kernel(const __grid_constant__ ShortParams p) {
           ptx::mbar_arrive_expect_tx(full(s), uint32_t(IW) * XB);
 #pragma unroll
           for (int kb = 0; kb < IW; ++kb)
-            ptx::tma_load_2d(xs(s) + uint32_t(kb) * XB, &p.tm_act, full(s), (st * IW + kb) * KB, 0);
+            if (ptx::dcheck(ptx::tma_x_ok((st * IW + kb) * KB, 2), p.status))
+              ptx::tma_load_2d(xs(s) + uint32_t(kb) * XB, &p.tm_act, full(s), (st * IW + kb) * KB, 0);
         } else {
           ptx::mbar_arrive_expect_tx(full(s), XB);
           ptx::tma_load_2d(xs(s), &p.tm_zs, full(s), 0, 0);
@@ -244,7 +245,8 @@ qlora_short_fwd_kernel(const __grid_constant__ ShortParams p) {
         if (st < nk) {
           if (!ptx::mbar_wait_idle(cempty(c), ph ^ 1u, p.status, abort_flag)) break;
           ptx::mbar_arrive_expect_tx(cfull(c), C_BYTES);
-          ptx::tma_load_2d(cs(c), &p.tm_codes, cfull(c), st * (IW * KB / 2), t * F_TILE);
+          if (ptx::dcheck(ptx::tma_x_ok(st * (IW * KB / 2), 1) && t < p.num_tiles, p.status))
+            ptx::tma_load_2d(cs(c), &p.tm_codes, cfull(c), st * (IW * KB / 2), t * F_TILE);
           if (++c == uint32_t(NC)) { c = 0; ph ^= 1u; }
         }
         if (++st == nk1) { st = 0; ++t; }
@@ -346,6 +348,10 @@ qlora_short_fwd_kernel(const __grid_constant__ ShortParams p) {
       tile_pieces(tile, nk1, p.iters, first, last);
       const int n = tile * F_TILE + nl;
       const uint32_t tbase = tmem + (uint32_t(q * 32) << 16) + b * uint32_t(F_ACC_COLS);
+      // this CTA's piece of the tile and the tile's arrival counter lie inside their regions
+      const bool seg_ok = ptx::dcheck(tile < p.num_tiles && p.num_tiles <= kMaxTiles &&
+                                      int(blockIdx.x) >= first &&
+                                      int(blockIdx.x) - first < p.max_pieces, p.status);
       float* piece = p.partial + (size_t(tile) * p.max_pieces + size_t(int(blockIdx.x) - first)) * piece_elems;
 #pragma unroll 1
       for (int c0 = 0; c0 < p.xrows; c0 += 16) {
@@ -362,7 +368,7 @@ qlora_short_fwd_kernel(const __grid_constant__ ShortParams p) {
         } else {
 #pragma unroll
           for (int u = 0; u < 16; ++u)
-            if (c0 + u < p.M) __stcg(piece + size_t(c0 + u) * F_TILE + nl, __uint_as_float(v[u]));
+            if (seg_ok && c0 + u < p.M) __stcg(piece + size_t(c0 + u) * F_TILE + nl, __uint_as_float(v[u]));
         }
       }
       ptx::tc_fence_before();
@@ -370,7 +376,7 @@ qlora_short_fwd_kernel(const __grid_constant__ ShortParams p) {
       if (lane == 0) ptx::mbar_arrive(acc_empty(b));
       b ^= 1u;
       if (b == 0u) bph ^= 1u;
-      if (first != last && arrive_piece(p.counters + tile * 4 + q, last - first + 1)) {
+      if (seg_ok && first != last && arrive_piece(p.counters + tile * 4 + q, last - first + 1)) {
         // add the pieces in piece order, 16 batch rows at a time, two pieces' loads in flight
         // before their sums
         const float* p0 = p.partial + size_t(tile) * p.max_pieces * piece_elems + nl;
@@ -568,8 +574,10 @@ qlora_short_dx_kernel(const __grid_constant__ ShortParams p) {
         if (!ptx::mbar_wait_idle(done(s), ph ^ 1u, p.status, abort_flag)) break;
         if (st < nk) {
           ptx::mbar_arrive_expect_tx(full(s), 2u * XB);
-          ptx::tma_load_2d(xs(s), &p.tm_act, full(s), st * 128, 0);
-          ptx::tma_load_2d(xs(s) + D_A_SLAB, &p.tm_act, full(s), st * 128 + 64, 0);
+          if (ptx::dcheck(ptx::tma_x_ok(st * 128, 2), p.status)) {
+            ptx::tma_load_2d(xs(s), &p.tm_act, full(s), st * 128, 0);
+            ptx::tma_load_2d(xs(s) + D_A_SLAB, &p.tm_act, full(s), st * 128 + 64, 0);
+          }
         } else {
           ptx::mbar_arrive_expect_tx(full(s), XB);
           ptx::tma_load_2d(xs(s), &p.tm_zs, full(s), 0, 0);
@@ -587,7 +595,8 @@ qlora_short_dx_kernel(const __grid_constant__ ShortParams p) {
         if (st < nk) {
           if (!ptx::mbar_wait_idle(cempty(c), ph ^ 1u, p.status, abort_flag)) break;
           ptx::mbar_arrive_expect_tx(cfull(c), C_BYTES);
-          ptx::tma_load_2d(cs(c), &p.tm_codes, cfull(c), t * (D_TILE / 2), st * 128);
+          if (ptx::dcheck(ptx::tma_x_ok(t * (D_TILE / 2), 1) && t < p.num_tiles, p.status))
+            ptx::tma_load_2d(cs(c), &p.tm_codes, cfull(c), t * (D_TILE / 2), st * 128);
           if (++c == uint32_t(NC)) { c = 0; ph ^= 1u; }
         }
         if (++st == nk1) { st = 0; ++t; }
@@ -683,6 +692,9 @@ qlora_short_dx_kernel(const __grid_constant__ ShortParams p) {
       int first, last;
       tile_pieces(tile, nk1, p.iters, first, last);
       const int k0 = tile * D_TILE;
+      const bool seg_ok = ptx::dcheck(tile < p.num_tiles && p.num_tiles <= kMaxTiles &&
+                                      int(blockIdx.x) >= first &&
+                                      int(blockIdx.x) - first < p.max_pieces, p.status);
       float* piece = p.partial + (size_t(tile) * p.max_pieces + size_t(int(blockIdx.x) - first)) * piece_elems;
       if (active) {
         const uint32_t tbase = tmem + (uint32_t(q * 32) << 16) + b * uint32_t(D_TILE);
@@ -691,7 +703,7 @@ qlora_short_dx_kernel(const __grid_constant__ ShortParams p) {
           uint32_t v[32];
           ptx::tmem_ld_32x32b_x32(tbase + uint32_t(c * 32), v);
           ptx::tmem_ld_wait(v);
-          if (m < p.M && k0 + c * 32 < p.K) {
+          if (seg_ok && m < p.M && k0 + c * 32 < p.K) {
             if (first == last) {
               uint4* dst = reinterpret_cast<uint4*>(p.out + size_t(m) * p.K + k0 + c * 32);
 #pragma unroll
@@ -718,7 +730,7 @@ qlora_short_dx_kernel(const __grid_constant__ ShortParams p) {
       if (lane == 0) ptx::mbar_arrive(acc_empty(b));
       b ^= 1u;
       if (b == 0u) bph ^= 1u;
-      if (first != last) {
+      if (seg_ok && first != last) {
         // Split tile: the 4 warps' row slices of this piece are stored; count the CTA's piece
         // once (thread 0), and if it was the last to arrive, all 128 epilogue threads add the
         // tile's pieces in piece order (each thread 4 columns of every other batch row).  The

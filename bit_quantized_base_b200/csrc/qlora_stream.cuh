@@ -79,6 +79,7 @@ struct StreamParams {
   long long lcm;                     // lcm(L, num_k + 1)
   int xrows;                         // M rounded up to 16: activation rows per stage, MMA N
   uint32_t zero;                     // 0 (see zero_after)
+  int segments;                      // partial segments the workspace holds
 };
 
 // Segments are the pieces of the iteration space between consecutive CTA-range starts (multiples
@@ -174,8 +175,12 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
         }
         if (!ptx::mbar_wait_idle(empty_s(s), ph ^ 1u, p.status, abort_flag)) break;
         ptx::mbar_arrive_expect_tx(full_s(s), XSTAGE);
-        if (ks < nk) ptx::tma_load_2d(xs(s), &p.tm_act, full_s(s), ks * BK, 0);
-        else ptx::tma_load_2d(xs(s), &p.tm_zs, full_s(s), 0, 0);
+        if (ks < nk) {
+          if (ptx::dcheck(ptx::tma_x_ok(ks * BK, 2), p.status))
+            ptx::tma_load_2d(xs(s), &p.tm_act, full_s(s), ks * BK, 0);
+        } else {
+          ptx::tma_load_2d(xs(s), &p.tm_zs, full_s(s), 0, 0);
+        }
         if (++s == uint32_t(NS)) { s = 0; ph ^= 1u; }
         if (++ks == rg.nk1) ks = 0;
       }
@@ -192,8 +197,10 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
           const uint32_t cd = ptx::smem_u32(cs + sc * C_BYTES);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            if (!DX) ptx::tma_load_2d(cd + h * HC_BYTES, &p.tm_codes, full_c(sc), ks * (BK / 2), c0 + h * HN);
-            else ptx::tma_load_2d(cd + h * HC_BYTES, &p.tm_codes, full_c(sc), (c0 + h * HN) / 2, ks * BK);
+            const int cx = !DX ? ks * (BK / 2) : (c0 + h * HN) / 2;
+            if (!ptx::dcheck(ptx::tma_x_ok(cx, 1), p.status)) continue;
+            if (!DX) ptx::tma_load_2d(cd + h * HC_BYTES, &p.tm_codes, full_c(sc), cx, c0 + h * HN);
+            else ptx::tma_load_2d(cd + h * HC_BYTES, &p.tm_codes, full_c(sc), cx, ks * BK);
           }
           if (++sc == uint32_t(NC)) { sc = 0; ph ^= 1u; }
         }
@@ -280,7 +287,9 @@ qlora_stream_gemm_kernel(const __grid_constant__ StreamParams p) {
       if (!ptx::mbar_wait_idle(acc_full(b), bph, p.status, abort_flag)) break;
       ptx::tc_fence_after();
       const long long st = max((long long)rg.g0, (long long)rg.tile(g) * rg.nk1);
-      float* base = p.partial + size_t(stream_segment(st, p.iters, rg.nk1, p.lcm)) * size_t(p.M) * BN;
+      const int seg = stream_segment(st, p.iters, rg.nk1, p.lcm);
+      if (!ptx::dcheck(seg >= 0 && seg < p.segments, p.status)) break;
+      float* base = p.partial + size_t(seg) * size_t(p.M) * BN;
       if constexpr (MT == 1) {
         // Tensor-memory lane 32q + lane holds batch row 32q + lane; its 256 columns are the tile's
         // output columns.  Warps whose rows are all past the batch have nothing to store.
@@ -489,6 +498,7 @@ qlora_stream_reduce_kernel(const __grid_constant__ StreamReduceParams p) {
   const int seg0 = stream_rank32(t * p.nk1, p.iters, p.nk1, p.lcm);
   const int seg1 = t + 1 == p.num_tiles ? p.segments
                                         : stream_rank32((t + 1) * p.nk1, p.iters, p.nk1, p.lcm);
+  if (!ptx::dcheck(seg0 >= 0 && seg1 <= p.segments && seg0 <= seg1, nullptr)) return;
   const float* src = p.partial + (size_t(seg0) * p.M + m) * BN + col;
   const size_t sstride = size_t(p.M) * BN;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);

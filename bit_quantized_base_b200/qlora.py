@@ -13,7 +13,9 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libqlora.so")
+# QLORA_LIBRARY=debug selects the bounds-checked debug build (libqlora_debug.so, -DQLORA_DEBUG)
+LIB_PATH = os.path.join(_PKG, "libqlora_debug.so" if os.environ.get("QLORA_LIBRARY") == "debug"
+                        else "libqlora.so")
 
 FMT = {"nf4": 0, "mxfp4": 1, "nvfp4": 2, "nf4dq": 3}
 BLOCK = {"nf4": 64, "mxfp4": 32, "nvfp4": 16}
