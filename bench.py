@@ -713,6 +713,80 @@ def large_batch_legs(Q, torch, synth, peaks):
     return out
 
 
+def w4a8_leg(Q, torch, synth, peaks, steps=20):
+    """The opt-in native block-scaled forward (W4A8: X quantised to MXFP8 on the fly, MXFP4 codes
+    straight into tcgen05 kind::mxf8f6f4 block-scaled MMAs) on the MXFP4 Llama-3-70B-shaped
+    gate-proj at its own batch (M=8192, 28672x8192, r=16), beside the bf16 forward of the same
+    inputs: ms per forward, TFLOP/s, and the GEMM kernel's roofline against the FP8 dense peak
+    (the measured bf16 peak x 2, the nominal FP8:bf16 ratio)."""
+    c3 = synth.WORKLOADS["llama3_70b_gate_mxfp4"]
+    pr = c3.projs[0]
+    M, N, K, r, s = c3.M, pr.N, pr.K, c3.r, c3.scale
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5000)
+    per_copy = weight_bytes("mxfp4", N, K) + 2 * M * K
+    ncopy = max(2, int(math.ceil(2.5 * 126e6 / per_copy)))
+    Ws = [_device_weight(Q, torch, "mxfp4", N, K, "t5", gen) for _ in range(ncopy)]
+    Xs = [torch.randn((M, K), device="cuda", generator=gen).bfloat16() for _ in range(ncopy)]
+    bound = 1.0 / math.sqrt(K)
+    A = ((torch.rand((r, K), device="cuda", generator=gen) * 2 - 1) * bound).bfloat16()
+    B = (torch.randn((N, r), device="cuda", generator=gen) * 0.01).bfloat16()
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    T = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    ws8 = Q.alloc_workspace(Q.OP_FWD_W4A8, Ws[0], M, r)
+    wsb = Q.alloc_workspace(Q.OP_FWD, Ws[0], M, r)
+    Q.qlora_workspace_init(ws8)
+    Q.qlora_workspace_init(wsb)
+    f8 = lambda i: Q.qlora_linear_fwd_w4a8(Ws[i % ncopy], Xs[i % ncopy], A, B, Y, T, M, r, s, ws8)
+    fb = lambda i: Q.qlora_linear_fwd(Ws[i % ncopy], Xs[i % ncopy], A, B, Y, T, M, r, s, wsb)
+
+    def timed(f):
+        for i in range(3):
+            f(i)
+        torch.cuda.synchronize()
+        clk = NvmlSampler(torch.cuda.current_device())
+        clk.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            f(i)
+        e1.record()
+        e1.synchronize()
+        return e0.elapsed_time(e1) / steps * 1e-3, clk.stop()
+
+    t8, c8 = timed(f8)
+    tb, cb = timed(fb)
+    Q.qlora_profile_enable(True)
+    Q.qlora_profile_reset()
+    for i in range(5):
+        f8(i)
+    torch.cuda.synchronize()
+    prof = Q.qlora_profile_read()
+    Q.qlora_profile_enable(False)
+    if Q.qlora_get_device_status(ws8) != 0 or Q.qlora_get_device_status(wsb) != 0:
+        raise RuntimeError("device status in the W4A8 leg")
+    fl = 2.0 * M * N * K + 2.0 * M * N * r + 2.0 * M * K * r
+    gflops = 2.0 * M * N * K + 2.0 * M * N * r
+    cnt, tot = prof["w4a8_gemm"]
+    capped = "sw_power_cap" in c8.get("reasons", [])
+    peak8 = 2.0 * (peaks["bf16_tflops_sustained"] if capped else peaks["bf16_tflops"])
+    achieved = gflops / (tot / cnt * 1e-3) / 1e12
+    res = {"M": M, "N": N, "K": K, "r": r, "fmt": "mxfp4 weights, MXFP8 activations",
+           "ms_per_fwd": round(t8 * 1e3, 4), "tflops": round(fl / t8 / 1e12, 1),
+           "bf16_fwd_ms": round(tb * 1e3, 4), "speedup_vs_bf16_fwd": round(tb / t8, 3),
+           "kernels_ms": {k: round(v[1] / v[0], 4) for k, v in prof.items()},
+           "roofline": {"kernel": "w4a8_gemm", "bound": "tensor", "achieved": round(achieved, 1),
+                        "peak": round(peak8, 1), "unit": "TFLOP/s", "frac": round(achieved / peak8, 4),
+                        "peak_source": ("sustained" if capped else "burst") +
+                                       " bf16 measured x 2 (nominal FP8:bf16 ratio)"},
+           "clocks": {k: c8.get(k) for k in ("sm_mhz", "sm_mhz_min", "reasons", "samples")},
+           "bf16_clocks": {k: cb.get(k) for k in ("sm_mhz", "reasons", "samples")},
+           "l2": f"{ncopy} rotating device copies of W and X ({ncopy * per_copy / 1e6:.0f} MB)"}
+    del Ws, Xs, Y, T, ws8, wsb
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_own(args):
     import numpy as np
     import torch
@@ -922,6 +996,14 @@ def run_own(args):
         except Exception as exc:          # a side leg never takes the main line down
             large = {"error": f"{type(exc).__name__}: {exc}"}
 
+    # ---- the opt-in native block-scaled (W4A8) forward on the MXFP4 gate-proj at M = 8192
+    w4a8 = None
+    if not args.no_sweep:
+        try:
+            w4a8 = w4a8_leg(Q, torch, synth, peaks)
+        except Exception as exc:
+            w4a8 = {"error": f"{type(exc).__name__}: {exc}"}
+
     # ---- CPU baseline: the oracle on a bounded sample of the same workload
     cpu = None
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
@@ -955,6 +1037,7 @@ def run_own(args):
         "quantize_merge": qm,
         "grouped_moe": grouped,
         "large_batch": large,
+        "w4a8_forward": w4a8,
         "cpu_baseline": cpu,
     }
     if rank == 0:

@@ -15,6 +15,7 @@
 #include "qlora_lora.cuh"
 #include "qlora_stream.cuh"
 #include "qlora_short.cuh"
+#include "qlora_w4a8.cuh"
 #include <algorithm>
 #include <utility>
 #include "qlora_quant.cuh"
@@ -332,12 +333,14 @@ int* ws_status(void* ws) { return reinterpret_cast<int*>(ws); }
 enum Kind : int {
   kKindFusedFwd = 0, kKindFusedDx, kKindDownT, kKindDownU, kKindWgrad,
   kKindGFusedFwd, kKindGFusedDx, kKindGDownT, kKindGDownU, kKindGWgrad,
-  kKindStreamFwd, kKindStreamDx, kKindStreamReduce, kKindShortFwd, kKindShortDx, kNumKinds
+  kKindStreamFwd, kKindStreamDx, kKindStreamReduce, kKindShortFwd, kKindShortDx,
+  kKindW4a8Quant, kKindW4a8Gemm, kNumKinds
 };
 const char* const kKindNames[kNumKinds] = {
     "fused_fwd", "fused_dx", "lora_down_T", "lora_down_U", "lora_wgrad",
     "grouped_fused_fwd", "grouped_fused_dx", "grouped_lora_down_T", "grouped_lora_down_U",
-    "grouped_lora_wgrad", "stream_fwd", "stream_dx", "stream_reduce", "short_fwd", "short_dx"};
+    "grouped_lora_wgrad", "stream_fwd", "stream_dx", "stream_reduce", "short_fwd", "short_dx",
+    "w4a8_quant", "w4a8_gemm"};
 constexpr int kMaxProfiled = 65536;
 
 std::atomic<int64_t> g_launches{0};
@@ -758,12 +761,93 @@ void* noalloc_scratch_address() {
 }  // namespace
 }  // namespace qlora
 
+namespace qlora {
+namespace {
+
+// Workspace of the native W4A8 forward: header | Zs [M, r] | T [M, r] (when T_save is NULL) |
+// quantised X [M, K] E4M3 | its scales [M, K/32] E8M0.
+struct W4a8Layout {
+  size_t zs, t, xq, xs, total;
+};
+
+W4a8Layout w4a8_layout(int64_t K, int64_t M, int r) {
+  W4a8Layout L{};
+  const size_t m = size_t(M > 0 ? M : 0);
+  size_t off = kHeaderBytes;
+  L.zs = off;
+  off += align_up(m * size_t(r) * 2, 256);
+  L.t = off;
+  off += align_up(m * size_t(r) * 2, 256);
+  L.xq = off;
+  off += align_up(m * size_t(K), 256);
+  L.xs = off;
+  off += align_up(m * size_t(K / 32), 256);
+  L.total = off;
+  return L;
+}
+
+qlora_status_t launch_mxfp8_quant(const void* X, int64_t M, int64_t K, void* codes, void* scales,
+                                  cudaStream_t st) {
+  Mxfp8Params p{};
+  p.x = static_cast<const __nv_bfloat16*>(X);
+  p.codes = static_cast<uint8_t*>(codes);
+  p.scales = static_cast<uint8_t*>(scales);
+  p.blocks = (long long)(M * (K / 32));
+  if (p.blocks == 0) return QLORA_OK;
+  const unsigned grid = unsigned((p.blocks + 255) / 256);
+  LaunchScope scope(kKindW4a8Quant, st);
+  if (launch_pdl(qlora_mxfp8_quant_kernel, dim3(grid), dim3(256), 0, st, p) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status_t launch_w4a8_gemm(const qlora_weight_t* W, const void* xq, const void* xs,
+                                const void* zs, const void* B, void* Y, int64_t M, int r,
+                                int* status, cudaStream_t st) {
+  using namespace w4a8;
+  const int64_t N = W->N, K = W->K;
+  W4a8Params p{};
+  const uint64_t rows = uint64_t(M);
+  if (!tmap_2d(&p.tm_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, uint64_t(K), rows, uint64_t(K), BK, BM,
+               CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tmap_2d(&p.tm_w, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, W->codes, uint64_t(K), uint64_t(N),
+               uint64_t(K / 2), BK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tmap_2d(&p.tm_zs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, zs, uint64_t(r), rows, uint64_t(r) * 2,
+               64, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tmap_2d(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, uint64_t(r), uint64_t(N),
+               uint64_t(r) * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return QLORA_ERR_CUDA;
+  p.xs = static_cast<const uint8_t*>(xs);
+  p.wsc = static_cast<const uint8_t*>(W->scales);
+  p.out = static_cast<__nv_bfloat16*>(Y);
+  p.status = status;
+  p.M = int(M);
+  p.N = int(N);
+  p.K = int(K);
+  p.rpad = rank_pad(r);
+  p.num_m = int((M + BM - 1) / BM);
+  p.num_n = int((N + BN - 1) / BN);
+  p.num_k = int(K / BK);
+  const int tiles = p.num_m * p.num_n;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  const size_t smem = smem_bytes();
+  if (!set_smem(qlora_w4a8_gemm_kernel, smem)) return QLORA_ERR_CUDA;
+  LaunchScope scope(kKindW4a8Gemm, st);
+  if (launch_pdl(qlora_w4a8_gemm_kernel, dim3(grid), dim3(kThreads), smem, st, p) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace qlora
+
 using namespace qlora;
 
 extern "C" {
 
 size_t qlora_workspace_size(int op, const qlora_weight_t* W, int64_t M, int r, int E) {
   if (check_weight(W) != QLORA_OK || M < 0 || !rank_ok(r)) return 0;
+  if (op == QLORA_OP_FWD_W4A8) return w4a8_layout(W->K, M, r).total;
   const bool grouped = op == QLORA_OP_GROUPED_FWD || op == QLORA_OP_GROUPED_BWD;
   if (!grouped && op != QLORA_OP_FWD && op != QLORA_OP_BWD) return 0;
   if (grouped && (E < 1 || E > kMaxExperts)) return 0;
@@ -913,6 +997,37 @@ qlora_status_t qlora_linear_fwd(const qlora_weight_t* W, const void* X, const vo
   if (st != QLORA_OK) return st;
   return run_fwd(W, 1, nullptr, false, X, A, B, Y, T_save, M, r, scale, ws, ws_bytes,
                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+qlora_status_t qlora_mxfp8_quantize(const void* X, int64_t M, int64_t K, void* codes, void* scales,
+                                    qlora_stream_t stream) {
+  if (M < 0 || K <= 0 || K % 128 != 0 || M > (int64_t(1) << 31) - 512) return QLORA_ERR_INVALID_ARG;
+  if (M > 0 && (!ptr_ok(X) || !ptr_ok(codes) || !ptr_ok(scales))) return QLORA_ERR_INVALID_ARG;
+  return launch_mxfp8_quant(X, M, K, codes, scales, reinterpret_cast<cudaStream_t>(stream));
+}
+
+qlora_status_t qlora_linear_fwd_w4a8(const qlora_weight_t* W, const void* X, const void* A,
+                                     const void* B, void* Y, void* T_save, int64_t M, int r,
+                                     float scale, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  qlora_status_t st = check_common(W, M, r);
+  if (st != QLORA_OK) return st;
+  if (W->fmt != QLORA_FMT_MXFP4 || W->K % 128 != 0) return QLORA_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(W->codes) & 31u) != 0 || !act_ok(X, M) || !ptr_ok(A) ||
+      !ptr_ok(B) || !act_ok(Y, M) || (T_save && !aligned16(T_save)))
+    return QLORA_ERR_INVALID_ARG;
+  const W4a8Layout L = w4a8_layout(W->K, M, r);
+  if (!ws || !aligned16(ws) || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (M == 0) return QLORA_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  void* T = T_save ? T_save : w + L.t;
+  st = launch_mxfp8_quant(X, M, W->K, w + L.xq, w + L.xs, s);
+  if (st != QLORA_OK) return st;
+  // T = X A^T from the bf16 X and Zs = bf16(s T), as in the bf16 forward
+  st = launch_lora_down(false, X, M, W->K, A, r, scale, nullptr, T, w + L.zs, ws_status(ws),
+                        nullptr, 1, false, kDownCtasBesidePair, s);
+  if (st != QLORA_OK) return st;
+  return launch_w4a8_gemm(W, w + L.xq, w + L.xs, w + L.zs, B, Y, M, r, ws_status(ws), s);
 }
 
 qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const void* X, const void* A,

@@ -434,6 +434,28 @@ __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t M, uint32_t N, uint32
          ((M >> 4) << 24);
 }
 
+// Instruction descriptor of kind::mxf8f6f4 with block scaling: A E4M3, B E2M1 (4-bit codes in the
+// 16-bytes-per-16-elements shared-memory layout), both K-major, fp32 accumulator, E8M0 scale
+// factors (bit 23), one per 32 elements along K; sf_id (bits 4-5 for B, 29-30 for A) selects the
+// byte of each 32-bit scale cell in tensor memory that this MMA's 32-deep step uses.
+//   bits 7-9 A format (0 = E4M3), 10-12 B format (5 = E2M1), 17-22 N >> 3, 24-28 M >> 4.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3_e2m1(uint32_t M, uint32_t N, uint32_t sf_id) {
+  return (sf_id << 4) | (0u << 7) | (5u << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24) |
+         (sf_id << 29);
+}
+// D (+)= (A x 2^(sfa-127)) (B x 2^(sfb-127))^T over one 32-deep step, block-scaled: sfa_tmem /
+// sfb_tmem are the tensor-memory columns of the scale factors (row m of a 128-row block at lane
+// 32 q + m % 32 of every lane quarter q, column base + m / 32; rows 128..255 of B at base + 4..7).
+__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate, uint32_t sfa_tmem,
+                                       uint32_t sfb_tmem) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+        "r"(sfb_tmem) : "memory");
+}
+
 // ---------------------------------------------------------------------------- misc
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;

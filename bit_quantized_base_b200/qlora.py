@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libqlora_debug.so" if os.environ.get("QLORA_LIBRA
 
 FMT = {"nf4": 0, "mxfp4": 1, "nvfp4": 2, "nf4dq": 3}
 BLOCK = {"nf4": 64, "mxfp4": 32, "nvfp4": 16}
-OP_FWD, OP_BWD, OP_GROUPED_FWD, OP_GROUPED_BWD = 0, 1, 2, 3
+OP_FWD, OP_BWD, OP_GROUPED_FWD, OP_GROUPED_BWD, OP_FWD_W4A8 = 0, 1, 2, 3, 4
 
 STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED",
           3: "QLORA_ERR_WORKSPACE", 4: "QLORA_ERR_CUDA", 5: "QLORA_ERR_DEVICE_TIMEOUT"}
@@ -30,7 +30,7 @@ EXPORTS = ("qlora_workspace_size", "qlora_workspace_init", "qlora_linear_fwd", "
            "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_status_string",
            "qlora_build_info", "qlora_launch_count", "qlora_profile_enable",
            "qlora_profile_reset", "qlora_profile_read", "qlora_linear_fwd_noalloc",
-           "qlora_linear_fwd_noalloc_status",
+           "qlora_linear_fwd_noalloc_status", "qlora_linear_fwd_w4a8", "qlora_mxfp8_quantize",
            "qlora_debug_decode_rate", "qlora_quantize", "qlora_merge_requantize",
            "qlora_loftq_workspace_size", "qlora_loftq")
 
@@ -81,6 +81,9 @@ def _load():
     L.qlora_status_string.restype = c.c_char_p
     L.qlora_build_info.restype = c.c_char_p
     L.qlora_launch_count.restype = c.c_int64
+    L.qlora_linear_fwd_w4a8.argtypes = [W, P, P, P, P, P, c.c_int64, c.c_int, c.c_float, P,
+                                        c.c_size_t, P]
+    L.qlora_mxfp8_quantize.argtypes = [P, c.c_int64, c.c_int64, P, P, P]
     L.qlora_linear_fwd_noalloc.argtypes = [W, P, P, P, P, P, c.c_int64, c.c_int, c.c_float, P]
     L.qlora_linear_fwd_noalloc.restype = c.c_int
     L.qlora_linear_fwd_noalloc_status.argtypes = [P]
@@ -92,6 +95,7 @@ def _load():
                  "qlora_grouped_fwd", "qlora_grouped_bwd", "qlora_get_device_status",
                  "qlora_debug_dequant", "qlora_debug_wait_timeout", "qlora_debug_decode_rate",
                  "qlora_quantize", "qlora_merge_requantize", "qlora_loftq",
+                 "qlora_linear_fwd_w4a8", "qlora_mxfp8_quantize",
                  "qlora_profile_enable",
                  "qlora_profile_reset", "qlora_profile_read"):
         getattr(L, name).restype = c.c_int
@@ -160,6 +164,19 @@ def qlora_linear_fwd(W: Weight, X, A, B, Y, T_save, M, r, scale, ws, stream=None
     _check(lib.qlora_linear_fwd(W.ref, _p(X), _p(A), _p(B), _p(Y), _p(T_save), int(M), int(r),
                                 float(scale), _p(ws), 0 if ws is None else ws.numel(),
                                 _stream(stream)), "qlora_linear_fwd")
+
+
+def qlora_linear_fwd_w4a8(W: Weight, X, A, B, Y, T_save, M, r, scale, ws, stream=None):
+    """Opt-in native block-scaled forward (MXFP4 weight, activations quantised to MXFP8)."""
+    _check(lib.qlora_linear_fwd_w4a8(W.ref, _p(X), _p(A), _p(B), _p(Y), _p(T_save), int(M), int(r),
+                                     float(scale), _p(ws), 0 if ws is None else ws.numel(),
+                                     _stream(stream)), "qlora_linear_fwd_w4a8")
+
+
+def qlora_mxfp8_quantize(X, M, K, codes, scales, stream=None):
+    """X [M,K] bf16 -> codes [M,K] uint8 (E4M3) and scales [M,K/32] uint8 (E8M0)."""
+    _check(lib.qlora_mxfp8_quantize(_p(X), int(M), int(K), _p(codes), _p(scales), _stream(stream)),
+           "qlora_mxfp8_quantize")
 
 
 def qlora_linear_fwd_noalloc(W: Weight, X, A, B, Y, T_save, M, r, scale, stream=None):

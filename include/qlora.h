@@ -115,7 +115,8 @@ typedef enum {
   QLORA_OP_FWD = 0,
   QLORA_OP_BWD = 1,
   QLORA_OP_GROUPED_FWD = 2,
-  QLORA_OP_GROUPED_BWD = 3
+  QLORA_OP_GROUPED_BWD = 3,
+  QLORA_OP_FWD_W4A8 = 4       /* qlora_linear_fwd_w4a8 */
 } qlora_op_t;
 
 /* Bytes of device workspace `op` needs for these shapes (E = number of experts for the grouped
@@ -193,6 +194,37 @@ QLORA_API qlora_status_t qlora_linear_fwd_noalloc(const qlora_weight_t* W, const
                                                   const void* A, const void* B, void* Y,
                                                   void* T_save, int64_t M, int r, float scale,
                                                   qlora_stream_t stream);
+
+/* Opt-in native block-scaled forward for MXFP4 weights (W4A8), an inference-style variant of
+ * qlora_linear_fwd ("Quantized weights, full precision", "LoRA operations and quantization":
+ * Blackwell's mxfp4-native ops; "Fine-Tuning 4-Bit Models", "Case 3": a W4AFP8 variant):
+ *   Y = deq8(X) deq(W)^T + s (X A^T) B^T
+ * deq8(X) is X quantised to MXFP8 as qlora_mxfp8_quantize does; deq(W) is the exact product of
+ * each E2M1 code and its E8M0 block scale (not rounded to bf16).  The tensor cores multiply the
+ * stored 4-bit codes by the 8-bit activation codes with both block scales, accumulating in fp32
+ * (tcgen05.mma kind::mxf8f6f4 block_scale); the LoRA term is the bf16 one of qlora_linear_fwd
+ * (T = X A^T from the bf16 X, written to T_save when not NULL).  Y therefore differs from
+ * qlora_linear_fwd by the activation quantisation (each element of X moves by up to 2^-4 of its
+ * magnitude); the backward pass stays qlora_linear_bwd.  Three launches: quantise X, T, GEMM.
+ *   W: MXFP4 only, K % 128 == 0 (others: QLORA_ERR_UNSUPPORTED); W->codes 32-byte aligned.
+ *   Other arguments and limits as qlora_linear_fwd; ws >= qlora_workspace_size(
+ *   QLORA_OP_FWD_W4A8), which holds Zs, T (when T_save is NULL), the E4M3 codes of X [M,K] and
+ *   their scales [M,K/32].  M = 0 is a no-op. */
+QLORA_API qlora_status_t qlora_linear_fwd_w4a8(const qlora_weight_t* W, const void* X,
+                                               const void* A, const void* B, void* Y,
+                                               void* T_save, int64_t M, int r, float scale,
+                                               void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* Quantise X [M,K] bf16 to MXFP8: codes [M,K] uint8 E4M3 and scales [M,K/32] uint8 E8M0, one per
+ * 32 consecutive elements along K.  The pages fix no activation format or rule; this is the OCP MX
+ * shared-exponent rule, as the weight encoder uses for MXFP4: per block e = clamp(floor(log2 amax)
+ * - 8 + 127, 0, 254) (8 = E4M3's largest normal exponent; 0 for an all-zero block), element =
+ * the nearest E4M3 value of x / 2^(e-127), ties to the even code, magnitudes saturating at 448,
+ * the sign dropped when the magnitude rounds to zero.  Requires K % 128 == 0 and 16-byte aligned
+ * pointers (M = 0 is a no-op).  X must be finite.  Async on stream; used by qlora_linear_fwd_w4a8
+ * and exported for testing. */
+QLORA_API qlora_status_t qlora_mxfp8_quantize(const void* X, int64_t M, int64_t K, void* codes,
+                                              void* scales, qlora_stream_t stream);
 
 /* Synchronise `stream` and read the status word of qlora_linear_fwd_noalloc's fixed scratch on
  * the current device: QLORA_OK, or the device-side error of the last no-alloc call (each call

@@ -212,3 +212,40 @@ def test_noalloc_size_limit_boundary(Q, keep_t, m_max):
                                                        0x40000, T, M, 64, 2.0, None)]
     assert rc(m_max + 1) == "QLORA_ERR_WORKSPACE"
     assert rc(m_max) == "QLORA_ERR_CUDA"
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(W=dict(fmt="nf4")), "QLORA_ERR_UNSUPPORTED"),             # E2M1 codes only: MXFP4
+    (dict(W=dict(fmt="mxfp4", K=192)), "QLORA_ERR_UNSUPPORTED"),    # K % 128
+    (dict(W=dict(fmt="mxfp4", codes=0x1010)), "QLORA_ERR_INVALID_ARG"),   # codes not 32-aligned
+    (dict(M=-1), "QLORA_ERR_INVALID_ARG"),
+    (dict(r=12), "QLORA_ERR_UNSUPPORTED"),
+    (dict(X=0x1004), "QLORA_ERR_INVALID_ARG"),
+    (dict(ws=0), "QLORA_ERR_WORKSPACE"),
+    (dict(ws_bytes=64), "QLORA_ERR_WORKSPACE"),
+])
+def test_w4a8_forward_rejects_bad_arguments(Q, bad, status):
+    wargs = dict(fmt="mxfp4")
+    wargs.update(bad.get("W", {}))
+    W = _w(Q, **wargs)
+    args = dict(X=0x10000, A=0x20000, B=0x30000, Y=0x40000, M=64, r=16, ws=0x50000,
+                ws_bytes=1 << 30)
+    args.update({k: v for k, v in bad.items() if k != "W"})
+    rc = Q.lib.qlora_linear_fwd_w4a8(W.ref, args["X"], args["A"], args["B"], args["Y"], None,
+                                     args["M"], args["r"], 2.0, args["ws"] or None,
+                                     args["ws_bytes"], None)
+    assert Q.STATUS[rc] == status
+
+
+def test_w4a8_workspace_and_quantizer_rules(Q):
+    W = _w(Q, fmt="mxfp4", N=256, K=512)
+    M, r = 300, 16
+    n = Q.qlora_workspace_size(Q.OP_FWD_W4A8, W, M, r)
+    # header + Zs + T + codes [M,K] + scales [M,K/32], each rounded up to 256 bytes
+    up = lambda x: (x + 255) // 256 * 256
+    assert n == 8192 + 2 * up(M * r * 2) + up(M * 512) + up(M * 512 // 32)
+    assert Q.STATUS[Q.lib.qlora_mxfp8_quantize(0x10000, 4, 192, 0x20000, 0x30000, None)] == \
+        "QLORA_ERR_INVALID_ARG"                                      # K % 128
+    assert Q.STATUS[Q.lib.qlora_mxfp8_quantize(0x10008, 4, 256, 0x20000, 0x30000, None)] == \
+        "QLORA_ERR_INVALID_ARG"                                      # misaligned X
+    assert Q.STATUS[Q.lib.qlora_mxfp8_quantize(None, 0, 256, None, None, None)] == "QLORA_OK"
