@@ -49,7 +49,18 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None,
+                    help="run only one small workload (--warmup + --steps passes, for ncu) and exit")
     return ap.parse_args()
+
+
+# Small single-workload runs for profiler captures (a few hundred MB on the device, inputs larger
+# than L2, one or two kernels of interest): name -> (what, fmt, M, N, K, r)
+PROFILE_CASES = {
+    "short_nf4_m16": ("fwd+bwd", "nf4", 16, 14336, 4096, 64),
+    "short_mxfp4_m16": ("fwd+bwd", "mxfp4", 16, 28672, 8192, 16),
+    "w4a8_mxfp4_m2048": ("w4a8 fwd", "mxfp4", 2048, 28672, 8192, 16),
+}
 
 
 def flops(M, N, K, r):
@@ -1200,8 +1211,47 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_profile_case(args):
+    """One small workload for a profiler capture: two rotating weight copies (each larger than
+    half of L2), --warmup + --steps passes, then a one-line summary.  Not a bench number."""
+    import torch
+    from bit_quantized_base_b200 import qlora as Q
+    what, fmt, M, N, K, r = PROFILE_CASES[args.profile_case]
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7)
+    Ws = [_device_weight(Q, torch, fmt, N, K, "normal", gen) for _ in range(2)]
+    X = torch.randn((M, K), device="cuda", generator=gen).bfloat16()
+    dY = (torch.randn((M, N), device="cuda", generator=gen) * 0.01).bfloat16()
+    A = ((torch.rand((r, K), device="cuda", generator=gen) * 2 - 1) / math.sqrt(K)).bfloat16()
+    B = (torch.randn((N, r), device="cuda", generator=gen) * 0.01).bfloat16()
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    T = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty((r, K), dtype=torch.bfloat16, device="cuda")
+    dB = torch.empty((N, r), dtype=torch.bfloat16, device="cuda")
+    op = Q.OP_FWD_W4A8 if what == "w4a8 fwd" else Q.OP_BWD
+    ws = Q.alloc_workspace(op, Ws[0], M, r)
+    Q.qlora_workspace_init(ws)
+    for i in range(args.warmup + args.steps):
+        W = Ws[i % 2]
+        if what == "w4a8 fwd":
+            Q.qlora_linear_fwd_w4a8(W, X, A, B, Y, T, M, r, 2.0, ws)
+        else:
+            Q.qlora_linear_fwd(W, X, A, B, Y, T, M, r, 2.0, ws)
+            Q.qlora_linear_bwd(W, X, A, B, T, dY, dX, dA, dB, M, r, 2.0, ws)
+    torch.cuda.synchronize()
+    st = Q.qlora_get_device_status(ws)
+    print(json.dumps({"profile_case": args.profile_case, "what": what, "fmt": fmt, "M": M, "N": N,
+                      "K": K, "r": r, "passes": args.warmup + args.steps, "status": st}))
+    if st != 0:
+        raise SystemExit(1)
+
+
 def main():
     args = parse()
+    if args.profile_case:
+        run_profile_case(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

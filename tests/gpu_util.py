@@ -1,12 +1,15 @@
 """Shared helpers of the GPU parity tests: upload seeded inputs, run the library through its C ABI
 (the Python binding), and compare against the oracle with the stated tolerance."""
+import os
+
 import numpy as np
 import torch
 
 from bit_quantized_base_b200 import synth
 
 # Output tolerance for bf16 outputs against the fp64 oracle: relative Frobenius error and
-# max-abs error relative to the largest reference magnitude.
+# max-abs error relative to the largest reference magnitude.  With QLORA_PRINT_ERRORS=1 every
+# comparison prints its two errors (run pytest with -s to see them).
 REL_FRO = 4e-3
 MAX_ABS_REL = 2e-2
 
@@ -30,6 +33,9 @@ def assert_close(got, ref, name, rel_fro=REL_FRO, max_abs_rel=MAX_ABS_REL):
     if nref == 0.0:
         assert err == 0.0, f"{name}: expected exact zeros, |err|={err}"
         return
+    if os.environ.get("QLORA_PRINT_ERRORS"):
+        print(f"[parity] {os.environ.get('PYTEST_CURRENT_TEST', '').split(' ')[0]} {name}: "
+              f"rel_fro={err / nref:.3e} max_abs_rel={np.abs(got - ref).max() / mx:.3e}")
     assert err / nref <= rel_fro, f"{name}: rel Frobenius error {err / nref:.3e} > {rel_fro}"
     assert np.abs(got - ref).max() <= max_abs_rel * mx, \
         f"{name}: max abs error {np.abs(got - ref).max():.3e} > {max_abs_rel} * {mx:.3e}"
