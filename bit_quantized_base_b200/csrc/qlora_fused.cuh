@@ -92,12 +92,18 @@ struct FusedParams {
   uint32_t zero;                     // 0 (see zero_after)
 };
 
-__device__ __forceinline__ void fused_tile_coords(int t, int num_m, int num_n, int& mt, int& nt) {
-  const int per_group = fused::GM * num_n;
+// Tile t of an expert's (m-tile, n-tile) grid, in raster groups of `group_m` m-tiles.  The
+// forward takes groups of GM: a wave then shares each weight tile among several row blocks.  dX
+// takes groups of 1 (the n-tiles of one row block consecutive): the num_n tiles that read the same
+// dY row block (up to 15 MB) run in the same wave and share it through L2, instead of reading it
+// again a wave later.
+__device__ __forceinline__ void fused_tile_coords(int t, int num_m, int num_n, int group_m, int& mt,
+                                                  int& nt) {
+  const int per_group = group_m * num_n;
   const int g = t / per_group;
   const int within = t - g * per_group;
-  const int m_base = g * fused::GM;
-  const int gm = min(fused::GM, num_m - m_base);
+  const int m_base = g * group_m;
+  const int gm = min(group_m, num_m - m_base);
   mt = m_base + within % gm;
   nt = within / gm;
 }
@@ -159,6 +165,7 @@ struct PairTile {
 // Tiles [0, total - tail) are the 512-row tiles of the table; when the last wave of tiles would
 // leave most pairs idle, the host asks for the last `tail` of them to be split in two 256-row
 // tiles each, scheduled after all others (indices total - tail .. total + tail - 1).
+template <bool DX>
 __device__ __forceinline__ PairTile pair_tile_at(const GroupView& g, int t, int num_n, int tail) {
   PairTile pt;
   int half = -1;
@@ -172,7 +179,7 @@ __device__ __forceinline__ PairTile pair_tile_at(const GroupView& g, int t, int 
   const int rows = g.off[pt.e + 1] - g.off[pt.e];
   const int mtiles = (rows + fused::BM - 1) / fused::BM;
   int mt, nt;
-  fused_tile_coords(local, mtiles, num_n, mt, nt);
+  fused_tile_coords(local, mtiles, num_n, DX ? 1 : fused::GM, mt, nt);
   pt.row0 = g.off[pt.e] + mt * fused::BM;
   pt.row_end = g.off[pt.e + 1];
   pt.nt = nt;
@@ -297,7 +304,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
       uint32_t i = 0;
       bool waited = false;
       for (int t = pair; t < num_tiles; t += npairs) {
-        const PairTile pt = pair_tile_at(grp_view, t, p.num_n, p.tail_split);
+        const PairTile pt = pair_tile_at<DX>(grp_view, t, p.num_n, p.tail_split);
         const int m0 = pt.row0 + int(rank) * HM;      // this CTA's rows of block 0 (+256: block 1)
         bool ok = true;
         for (int ks = 0; ks <= nk; ++ks, ++i) {
@@ -327,7 +334,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     if (lane == 0) {
       uint32_t j = 0;
       for (int t = pair; t < num_tiles; t += npairs) {
-        const PairTile pt = pair_tile_at(grp_view, t, p.num_n, p.tail_split);
+        const PairTile pt = pair_tile_at<DX>(grp_view, t, p.num_n, p.tail_split);
         const int h0 = pt.nt * BN + int(rank) * HN;   // this CTA's weight half
         const int wrow0 = pt.e * p.N;                 // the expert's first row of the codes
         bool ok = true;
@@ -361,7 +368,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
       constexpr uint64_t kABlk = X_BYTES >> 4, kAkk = 32 >> 4, kBkk = DX ? (2048 >> 4) : (32 >> 4);
       uint32_t i = 0, tc = 0;
       for (int t = pair; t < num_tiles; t += npairs, ++tc) {
-        const int nb = pair_tile_at(grp_view, t, p.num_n, p.tail_split).nb;
+        const int nb = pair_tile_at<DX>(grp_view, t, p.num_n, p.tail_split).nb;
         if (!ptx::mbar_wait_cluster(acc_empty, (tc & 1u) ^ 1u, p.status, abort_flag)) break;
         ptx::tc_fence_after();
         bool ok = true;
@@ -423,7 +430,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     const int rr0 = lane >> 2, rc = lane & 3;                     // read: row rr0 + 8 it, chunk rc
     uint32_t tc = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++tc) {
-      const PairTile pt = pair_tile_at(grp_view, t, p.num_n, p.tail_split);
+      const PairTile pt = pair_tile_at<DX>(grp_view, t, p.num_n, p.tail_split);
       const int c0 = pt.nt * BN;
       const float ts = (FMT == kFmtNVFP4 && p.tensor_scale) ? __ldg(p.tensor_scale + pt.e) : 1.0f;
       if (!ptx::mbar_wait(acc_full, tc & 1u, p.status, abort_flag)) break;
@@ -483,7 +490,7 @@ qlora_fused_gemm_kernel(const __grid_constant__ FusedParams p) {
     };
     auto set_tile = [&](Cursor& c) {
       if (c.t < num_tiles) {
-        const PairTile pt = pair_tile_at(grp_view, c.t, p.num_n, p.tail_split);
+        const PairTile pt = pair_tile_at<DX>(grp_view, c.t, p.num_n, p.tail_split);
         c.h0 = pt.nt * BN + int(rank) * HN;
         c.e = pt.e;
       }
