@@ -102,12 +102,33 @@ CUtensorMapSwizzle swizzle_for_bytes(uint32_t b) {
 
 template <typename K>
 bool set_smem(K kernel, size_t bytes) {
-  // every kernel of the library asks for the largest shared-memory carveout, so that consecutive
-  // launches never make the SMs switch their L1 / shared-memory split
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(bytes)) == cudaSuccess &&
-         cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                              cudaSharedmemCarveoutMaxShared) == cudaSuccess;
+  // Both attributes persist per kernel and device, so each (kernel, device) is set once, to the
+  // largest size asked for so far; later launches that ask no more make no driver call.  Every
+  // kernel of the library asks for the largest shared-memory carveout, so that consecutive
+  // launches never make the SMs switch their L1 / shared-memory split.
+  struct Entry {
+    const void* fn;
+    int dev;
+    size_t bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const void* fn = reinterpret_cast<const void*>(kernel);
+  std::lock_guard<std::mutex> lk(mu);
+  Entry* hit = nullptr;
+  for (Entry& e : done)
+    if (e.fn == fn && e.dev == dev) hit = &e;
+  if (hit && hit->bytes >= bytes) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes)) != cudaSuccess ||
+      cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+    return false;
+  if (hit) hit->bytes = bytes;
+  else done.push_back(Entry{fn, dev, bytes});
+  return true;
 }
 
 // Launch with programmatic stream serialization: the kernel may begin while the previous kernel of

@@ -35,7 +35,9 @@
  *     caller's job).  Results are deterministic: the same inputs give bitwise-identical outputs.
  *   - Calls that share a workspace must be ordered on one stream.
  *   - Host threads may call the library concurrently.  Its process-wide state is small: per-device
- *     caches filled once (SM count, kernel shared-memory attributes), a pool of events and a side
+ *     caches filled once (SM count, kernel shared-memory attributes, set on a kernel's first launch
+ *     on a device and not again: a cudaDeviceReset discards them, so do not reset a device that
+ *     the library has run on and use it again in the same process), a pool of events and a side
  *     stream per device used to order the backward pass's dA/dB launch (mutex-guarded), the launch
  *     counter (atomic) and the opt-in profiling record (qlora_profile_*, mutex-guarded); the
  *     fixed scratch of qlora_linear_fwd_noalloc is shared by all its callers (see there).
