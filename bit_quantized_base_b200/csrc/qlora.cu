@@ -26,10 +26,13 @@ namespace {
 
 // ------------------------------------------------------------------------------------ helpers
 // Workspace header, cleared by qlora_workspace_init: [0] device status word, [1] pair-kernel
-// ticket, bytes [256, 8192) the short-batch kernels' arrival counters, 4 per tile (each launch
-// leaves them at zero).
+// ticket, bytes [64, 192) lora_down's arrival counters of a multi-cluster split, bytes
+// [256, 8192) the short-batch kernels' arrival counters, 4 per tile (each launch leaves all
+// counters at zero).
 constexpr size_t kHeaderBytes = 8192;
 constexpr size_t kCounterOffset = 256;
+constexpr size_t kDownCountOffset = 64;
+constexpr int kDownCounters = 32;
 // The no-alloc forward's scratch holds only the status word and the ticket in its header.
 constexpr size_t kNoAllocHeaderBytes = 256;
 constexpr int kMaxClusterSplits = 8;        // split-K CTAs of one LoRA tile (one portable cluster)
@@ -39,6 +42,13 @@ constexpr int kDownCtasBesidePair = 32;
 // The same for the short-batch streaming kernel, which up to 64 rows also leaves that many SMs to
 // lora_down (its ranges are equal, so a late CTA would delay the whole launch)
 constexpr int kDownCtasBesideStream = 16;
+// U = dY B ahead of the short-batch dX kernel: the whole contraction (N deep) on one 128-row
+// tile, which one cluster of 8 CTAs takes ~0.35 us per 64-deep step to stream; up to this many
+// CTAs (clusters of 8) split it, their sums added through the workspace.  The dX kernel's CTAs
+// that find no free SM start when these end, a few microseconds later.
+constexpr int kDownWideCtas = 64;
+constexpr int kMaxDownClusters = kDownWideCtas / kMaxClusterSplits;
+static_assert(kMaxClusterSplits <= kDownCounters, "one tile's counters fit the header");
 constexpr int kMaxDevices = 64;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -213,11 +223,13 @@ WgradPlan wgrad_plan(int64_t N, int64_t K, int64_t M, int E, int sms) {
 
 // Split plan of the lora_down kernel: 128-row tiles (at most ceil(M/128) + E - 1 over all
 // experts), the contraction (Kc) split into S ranges of whole 64-deep steps, >= 2 steps each.
+// wide > 0 (one layer of one tile, S = 8): C = min(wide / 8, steps / 16) clusters of S CTAs
+// split it S * C ways (trailing splits may be empty), C * 128 * rpad fp32 sums in the workspace.
 struct DownPlan {
-  int tiles, S, sps, num_k;
+  int tiles, S, C, sps, num_k;
 };
 
-DownPlan down_plan(int64_t M, int64_t Kc, int E, int ctas) {
+DownPlan down_plan(int64_t M, int64_t Kc, int E, int ctas, int wide) {
   DownPlan p{};
   p.tiles = int((M + 127) / 128) + (E > 1 ? E - 1 : 0);
   p.num_k = int((Kc + 63) / 64);
@@ -225,9 +237,27 @@ DownPlan down_plan(int64_t M, int64_t Kc, int E, int ctas) {
   S = S < 1 ? 1 : (S > kMaxClusterSplits ? kMaxClusterSplits : S);
   const int max_s = p.num_k / 2 > 0 ? p.num_k / 2 : 1;
   if (S > max_s) S = max_s;
-  p.sps = (p.num_k + S - 1) / S;
-  p.S = (p.num_k + p.sps - 1) / p.sps;
+  p.C = 1;
+  if (wide > 0 && E == 1 && p.tiles == 1 && S == kMaxClusterSplits) {
+    int C = wide / S;
+    const int max_c = p.num_k / (2 * S);
+    C = C > max_c ? max_c : C;
+    C = C > kMaxDownClusters ? kMaxDownClusters : C;
+    p.C = C < 1 ? 1 : C;
+  }
+  if (p.C > 1) {
+    p.sps = (p.num_k + S * p.C - 1) / (S * p.C);
+    p.S = S;
+  } else {
+    p.sps = (p.num_k + S - 1) / S;
+    p.S = (p.num_k + p.sps - 1) / p.sps;
+  }
   return p;
+}
+
+// Workspace bytes of lora_down's cluster sums for a multi-cluster U of rank r (and any M).
+size_t down_sum_bytes(int r) {
+  return size_t(kMaxDownClusters) * 128 * size_t(rank_pad(r)) * 4;
 }
 
 // Short batches (M <= 256 rows, one weight) use the weight-streaming kernels: the flat space of
@@ -313,7 +343,7 @@ bool short_fits(const qlora_weight_t* W, int64_t M, int E, bool dx, size_t regio
 }
 
 struct WsLayout {
-  size_t zs, t, u, partial, partial_bytes, total;
+  size_t zs, t, u, dsum, partial, partial_bytes, total;
 };
 
 WsLayout ws_layout(int64_t N, int64_t K, int64_t M, int r, bool bwd, int E, int sms) {
@@ -323,6 +353,7 @@ WsLayout ws_layout(int64_t N, int64_t K, int64_t M, int r, bool bwd, int E, int 
   L.zs = off; off += mr;
   L.t = off; off += mr;
   L.u = off; off += bwd ? mr : 0;
+  L.dsum = off; off += (bwd && E == 1) ? down_sum_bytes(r) : 0;   // independent of M
   L.partial = off;
   // fp32 partials of the short-batch weight-streaming kernels
   size_t pb = 0;
@@ -407,14 +438,18 @@ bool tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_
 // Z = Act . R for every expert's rows: R is A [E, r, Kc] (r_mn false, T = X A^T) or
 // B [E, Kc, r] (r_mn true, U = dY B).  offsets == nullptr: one expert of M rows.  beside_pair:
 // max_ctas > 0: the next launch of the stream (pair or streaming kernel) runs beside this one,
-// which then uses at most that many CTAs.
+// which then uses at most that many CTAs.  wide > 0: a one-tile layer may use up to `wide` CTAs
+// in several clusters, whose sums go to `sums` (down_sum_bytes) and whose arrival counters are
+// the workspace header's (`header`).
 qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t Kc, const void* R,
                                 int r, float s, const float* ts, void* z, void* zs, int* status,
                                 const int32_t* offsets, int E, bool grouped, int max_ctas,
-                                cudaStream_t st, float zs_mul = 1.0f) {
+                                cudaStream_t st, float zs_mul = 1.0f, int wide = 0,
+                                void* sums = nullptr, void* header = nullptr) {
   DownParams p{};
   const int rpad = rank_pad(r);
-  const DownPlan dp = down_plan(M, Kc, E, max_ctas > 0 ? max_ctas : num_sms());
+  const DownPlan dp = down_plan(M, Kc, E, max_ctas > 0 ? max_ctas : num_sms(),
+                                sums && header ? wide : 0);
   if (!tmap_2d(&p.tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, uint64_t(Kc), uint64_t(M),
                uint64_t(Kc) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
@@ -434,11 +469,16 @@ qlora_status_t launch_lora_down(bool r_mn, const void* act, int64_t M, int64_t K
   p.rpad = rpad;
   p.num_k = dp.num_k;
   p.S = dp.S;
+  p.C = dp.C;
   p.steps_per_split = dp.sps;
   p.E = E;
   p.s = s;
   p.zs_mul = zs_mul;
-  const dim3 grid(unsigned(dp.tiles * dp.S));
+  if (dp.C > 1) {
+    p.cpart = static_cast<float*>(sums);
+    p.ccount = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(header) + kDownCountOffset);
+  }
+  const dim3 grid(unsigned(dp.tiles * dp.S * dp.C));
   const size_t smem = lora::smem_bytes(E);
   LaunchScope scope(grouped ? (r_mn ? kKindGDownU : kKindGDownT) : (r_mn ? kKindDownU : kKindDownT), st);
   if (r_mn) {
@@ -966,7 +1006,8 @@ qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   st = launch_lora_down(true, dY, M, W->N, B, r, scale, ts, U, Zs, ws_status(ws), offsets, E,
                         grouped,
                         !dX ? 0 : ((short_dx || stream_dx) ? kDownCtasBesideStream : kDownCtasBesidePair),
-                        s, short_dx ? short_zs_mul(W) : 1.0f);
+                        s, short_dx ? short_zs_mul(W) : 1.0f, short_dx ? kDownWideCtas : 0,
+                        w + L.dsum, ws);
   if (st != QLORA_OK) return st;
   auto run_dx = [&]() {
     if (short_dx) return launch_short(W, true, dY, Zs, A, dX, M, r, ws, part, region, s);

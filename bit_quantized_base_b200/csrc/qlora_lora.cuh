@@ -23,7 +23,11 @@
 // Both kernels are memory bound (they stream an activation once) and have few output tiles, so
 // the contraction is split over S CTAs per tile to fill the GPU.  The S CTAs of a tile run as one
 // thread-block cluster and add their fp32 partial tiles through distributed shared memory, in
-// split order 0..S-1, so the result is bitwise deterministic.
+// split order 0..S-1, so the result is bitwise deterministic.  A short batch (one tile) has too
+// few splits for that: lora_down may then run C clusters per tile over consecutive ranges of the
+// contraction; each cluster stores its sum as fp32 in the workspace and the last cluster to
+// arrive (an arrival counter per row slice, reset by that cluster) adds the C sums in cluster
+// order 0..C-1, again a fixed order.
 #pragma once
 #include <cuda_bf16.h>
 #include "qlora_ptx.cuh"
@@ -36,6 +40,7 @@ constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int R_BYTES = 64 * 128;     // up to 64 x 128 B
 constexpr int kThreads = 6 * 32;      // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int kTmemCols = 64;
+constexpr int kMaxClusters = 8;       // C > 1: the workspace holds the sums of 8 clusters of one tile
 constexpr size_t kSmemBase = 1024 + size_t(NS) * (A_BYTES + R_BYTES) + 512;
 __host__ __device__ constexpr size_t smem_bytes(int E) { return kSmemBase + size_t(2) * (E + 1) * 4; }
 }  // namespace lora
@@ -130,7 +135,9 @@ struct DownParams {
   __nv_bfloat16* zs;   // [M, r]
   const int32_t* offsets;      // grouped: device [E+1]; nullptr: one expert
   int* status;
-  int M, r, rpad, num_k, S, steps_per_split, E;
+  float* cpart;        // C > 1: the clusters' sums [tiles][C][128][rpad] fp32
+  unsigned* ccount;    // C > 1: arrival counters [tiles][S], zero between launches
+  int M, r, rpad, num_k, S, C, steps_per_split, E;
   float s;
   float zs_mul;        // an exact power of two folded into Zs (2^-8 when the next kernel decodes
                        // NVFP4 elements times 2^-8), else 1
@@ -148,6 +155,7 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(rs + NS * R_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile unsigned* s_ticket = reinterpret_cast<volatile unsigned*>(tmem_slot + 2);
   int* s_off = reinterpret_cast<int*>(smem + (kSmemBase - 1024));
   int* s_first = s_off + (p.E + 1);
   const uint32_t b0 = ptx::smem_u32(bars);
@@ -158,14 +166,20 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
   // (expert, 128-row tile, split) of this CTA; CTAs beyond the table's last tile have no work.
   // The table's tile count and the grid are multiples of S, so the S CTAs of a cluster either
   // all leave here or all stay.
-  const GroupView gv = build_group_view(p.offsets, p.E, p.M, BM, p.S, s_off, s_first, p.status);
+  // With C clusters per tile the table repeats each tile S * C times: global split gs = cg * S +
+  // split covers steps [gs * steps_per_split, ...), cluster cg of the tile holds splits
+  // cg * S .. cg * S + S - 1 (consecutive CTAs, so one cluster).
+  const int per_tile = p.S * p.C;
+  const GroupView gv = build_group_view(p.offsets, p.E, p.M, BM, per_tile, s_off, s_first, p.status);
   if (int(blockIdx.x) >= gv.total()) return;
   const int e = gv.expert_of(blockIdx.x);
   const int local = int(blockIdx.x) - gv.first[e];
-  const int mt = local / p.S, split = local % p.S;
+  const int mt = local / per_tile, gs = local % per_tile;
+  const int split = gs % p.S, cg = gs / p.S;
+  const int tidx = int(blockIdx.x) / per_tile;          // the tile's index in the table
   const int m0 = gv.off[e] + mt * BM;
   const int row_end = gv.off[e + 1];
-  const int ks0 = split * p.steps_per_split;
+  const int ks0 = min(gs * p.steps_per_split, p.num_k);
   const int ks1 = min(ks0 + p.steps_per_split, p.num_k);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -270,11 +284,57 @@ qlora_lora_down_kernel(const __grid_constant__ DownParams p) {
     }
   }
   if (p.S > 1) {
+    const int nrows = min(BM, row_end - m0);
+    // C > 1: this cluster's sum of row lr, columns c .. c+7 (the sums of one tile's clusters and
+    // its S counters are what the workspace holds)
+    float* const csum = p.cpart + (size_t(tidx) * p.C + cg) * BM * p.rpad;
+    const bool wide_ok = p.C == 1 || ptx::dcheck(tidx == 0 && p.C <= kMaxClusters, p.status);
     ptx::cluster_sync();
-    if (warp >= 2 && *abort_flag == 0)
-      cluster_sum(ptx::smem_u32(as), p.rpad, p.S, split, min(BM, row_end - m0), threadIdx.x - 64,
-                  [&](int lr, int c, const float (&v)[8]) { write8(m0 + lr, c, v); });
+    if (warp >= 2 && *abort_flag == 0 && wide_ok) {
+      if (p.C == 1)
+        cluster_sum(ptx::smem_u32(as), p.rpad, p.S, split, nrows, threadIdx.x - 64,
+                    [&](int lr, int c, const float (&v)[8]) { write8(m0 + lr, c, v); });
+      else
+        cluster_sum(ptx::smem_u32(as), p.rpad, p.S, split, nrows, threadIdx.x - 64,
+                    [&](int lr, int c, const float (&v)[8]) {
+                      float4* d = reinterpret_cast<float4*>(csum + size_t(lr) * p.rpad + c);
+                      __stcg(d, make_float4(v[0], v[1], v[2], v[3]));
+                      __stcg(d + 1, make_float4(v[4], v[5], v[6], v[7]));
+                    });
+    }
     ptx::cluster_sync();
+    if (p.C > 1 && warp >= 2 && wide_ok) {
+      // Count this cluster's slice in (also after an abort, so the counter stays consistent);
+      // the last of the C clusters adds the slice's C sums in cluster order.
+      const int et = int(threadIdx.x) - 64;
+      unsigned* const counter = p.ccount + tidx * p.S + split;
+      __threadfence();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (et == 0) *s_ticket = atomicAdd(counter, 1u);
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (*s_ticket == unsigned(p.C - 1)) {
+        __threadfence();
+        const int rows_per = (BM + p.S - 1) / p.S;
+        const int r0 = split * rows_per, r1 = min(nrows, r0 + rows_per);
+        const int g8 = p.rpad / 8;
+        const int items = r1 > r0 ? (r1 - r0) * g8 : 0;
+        const float* const c0 = p.cpart + size_t(tidx) * p.C * BM * p.rpad;
+        for (int it = et; it < items && *abort_flag == 0; it += 128) {
+          const int lr = r0 + it / g8, c = (it % g8) * 8;
+          float v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) v[u] = 0.0f;
+          for (int k = 0; k < p.C; ++k) {
+            const float4* src = reinterpret_cast<const float4*>(c0 + (size_t(k) * BM + lr) * p.rpad + c);
+            const float4 a = __ldcg(src), b = __ldcg(src + 1);
+            v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+            v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+          }
+          write8(m0 + lr, c, v);
+        }
+        if (et == 0) *counter = 0u;
+      }
+    }
   }
   ptx::tc_fence_before();
   __syncthreads();

@@ -126,9 +126,10 @@ typedef enum {
  * arguments.  A workspace sized for an op and shapes also serves smaller M. */
 QLORA_API size_t qlora_workspace_size(int op, const qlora_weight_t* W, int64_t M, int r, int E);
 
-/* Zero the workspace's 256-byte header (device status word and the tiled kernel's tile ticket,
- * which every launch leaves where it found it).  Call once after allocating a workspace (or zero
- * it yourself), and again after a QLORA_ERR_DEVICE_TIMEOUT.  Async on stream. */
+/* Zero the workspace's 8192-byte header (device status word, the tiled kernel's tile ticket and
+ * the arrival counters of the split reductions, which every launch leaves at zero).  Call once
+ * after allocating a workspace (or zero its first 8192 bytes yourself), and again after a
+ * QLORA_ERR_DEVICE_TIMEOUT.  Async on stream. */
 QLORA_API qlora_status_t qlora_workspace_init(void* ws, size_t ws_bytes, qlora_stream_t stream);
 
 /* Forward: Y = X deq(W)^T + s (X A^T) B^T.  Two launches: T = X A^T (written to T_save when not

@@ -127,7 +127,9 @@ def test_short_layer_parity(fmt, M, N, K, r):
     assert_close(to_f64(dX), ref["dX"], "dX")
     assert_close(to_f64(dA), ref["dA"], "dA")
     assert_close(to_f64(dB), ref["dB"], "dB")
-    # every launch leaves the per-tile arrival counters (workspace bytes 256..8191) at zero
+    # every launch leaves the arrival counters (workspace bytes 64..191: lora_down's multi-cluster
+    # U; 256..8191: the short-batch kernels' tiles) at zero
+    assert int(torch.count_nonzero(g.ws[64:192])) == 0
     assert int(torch.count_nonzero(g.ws[256:8192])) == 0
 
 
