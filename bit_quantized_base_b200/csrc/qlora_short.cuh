@@ -507,6 +507,7 @@ qlora_short_dx_kernel(const __grid_constant__ ShortParams p) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 2 * NC + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  volatile int* s_defer = reinterpret_cast<volatile int*>(tmem_slot + 3);   // tile reduced at the end
   const uint32_t b0 = ptx::smem_u32(bars);
   auto full = [&](uint32_t s) { return b0 + 8u * s; };
   auto done = [&](uint32_t s) { return b0 + 8u * (NS + s); };
@@ -543,6 +544,7 @@ qlora_short_dx_kernel(const __grid_constant__ ShortParams p) {
     ptx::mbar_init(epi_a, kEpiWarps);
     ptx::mbar_init(epi_b, 1);
     *abort_flag = 0;
+    *s_defer = -1;
     ptx::fence_mbarrier_init();
   }
   if (warp == kXWarp && lane == 0) {
@@ -747,7 +749,11 @@ qlora_short_dx_kernel(const __grid_constant__ ShortParams p) {
         }
         if (!ptx::mbar_wait(epi_b, ephase, p.status, abort_flag)) break;
         ephase ^= 1u;
-        if (*s_last) {
+        if (*s_last && g + 1 == g1) {
+          // the tile of the range's last segment: every thread of the CTA adds it once all roles
+          // are done (below), with 5.75 times the epilogue warps' loads in flight
+          if (threadIdx.x == 0) *s_defer = tile;
+        } else if (*s_last) {
           __threadfence();
           const int e = int(threadIdx.x);                     // 0..127
           const int c0 = (e & 63) * 4, rh = e >> 6;
@@ -856,6 +862,65 @@ qlora_short_dx_kernel(const __grid_constant__ ShortParams p) {
   __syncthreads();
   ptx::tc_fence_after();
   if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, kTmemCols);
+
+  // This CTA was the last to arrive at the tile of its final segment: add the tile's pieces in
+  // piece order (the order of the epilogue's own reduction, so the result is the same bit for
+  // bit) with all threads, two 4-column groups of a row per thread and four pieces of each in
+  // flight, then reset the tile's counter.
+  const int dtile = *s_defer;
+  if (dtile >= 0) {
+    int first, last;
+    tile_pieces(dtile, nk1, p.iters, first, last);
+    const int np = last - first + 1;
+    if (*abort_flag == 0 && ptx::dcheck(dtile < p.num_tiles && np <= p.max_pieces, p.status)) {
+      __threadfence();
+      const int k0 = dtile * D_TILE;
+      const float tse = (p.tensor_scale ? __ldg(p.tensor_scale) : 1.0f) * p.ts_mul;
+      const size_t piece_elems = size_t(p.M) * D_TILE;
+      const float* base = p.partial + size_t(dtile) * p.max_pieces * piece_elems;
+      const int items = p.M * (D_TILE / 4);              // (batch row, 4-column group)
+      const int T = int(blockDim.x);
+      auto item_ptr = [&](int i) { return base + size_t(i >> 6) * D_TILE + (i & 63) * 4; };
+      auto write4 = [&](int i, const float4& a) {
+        const int mm = i >> 6, c0 = (i & 63) * 4;
+        if (k0 + c0 < p.K) {
+          uint2 w;
+          w.x = ptx::cvt_bf16x2(a.x * tse, a.y * tse);
+          w.y = ptx::cvt_bf16x2(a.z * tse, a.w * tse);
+          *reinterpret_cast<uint2*>(p.out + size_t(mm) * p.K + k0 + c0) = w;
+        }
+      };
+#pragma unroll 1
+      for (int i0 = int(threadIdx.x); i0 < items; i0 += 2 * T) {
+        const int i1 = i0 + T;
+        const bool two = i1 < items;
+        const float* q0 = item_ptr(i0);
+        const float* q1 = item_ptr(two ? i1 : i0);
+        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+#pragma unroll 1
+        for (int j = 0; j < np; j += 4) {
+          float4 v0[4], v1[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const bool ok = j + u < np;
+            v0[u] = ok ? __ldcg(reinterpret_cast<const float4*>(q0 + size_t(j + u) * piece_elems))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+            v1[u] = ok && two ? __ldcg(reinterpret_cast<const float4*>(q1 + size_t(j + u) * piece_elems))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (j + u < np) {
+              a0.x += v0[u].x; a0.y += v0[u].y; a0.z += v0[u].z; a0.w += v0[u].w;
+              a1.x += v1[u].x; a1.y += v1[u].y; a1.z += v1[u].z; a1.w += v1[u].w;
+            }
+        }
+        write4(i0, a0);
+        if (two) write4(i1, a1);
+      }
+    }
+    if (threadIdx.x == 0) p.counters[dtile * 4] = 0u;
+  }
 }
 
 }  // namespace qlora
