@@ -949,7 +949,9 @@ qlora_status_t run_fwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
   if (!act_ok(X, M) || !ptr_ok(A) || !ptr_ok(B) || !act_ok(Y, M) || (T_save && !aligned16(T_save)))
     return QLORA_ERR_INVALID_ARG;
   const WsLayout L = ws_layout(W->N, W->K, M, r, false, E, num_sms());
-  if (!ws || !aligned16(ws) || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  // The split partials are optional: without room for them the tiled kernels run (so that a
+  // workspace sized for a larger batch serves every smaller one).
+  if (!ws || !aligned16(ws) || ws_bytes < L.partial) return QLORA_ERR_WORKSPACE;
   if (M == 0) return QLORA_OK;
   uint8_t* w = static_cast<uint8_t*>(ws);
   void* T = T_save ? T_save : w + L.t;
@@ -979,7 +981,7 @@ qlora_status_t run_bwd(const qlora_weight_t* W, int E, const int32_t* offsets, b
       (T && !aligned16(T)) || (dX && !aligned16(dX)))
     return QLORA_ERR_INVALID_ARG;
   const WsLayout L = ws_layout(W->N, W->K, M, r, true, E, num_sms());
-  if (!ws || !aligned16(ws) || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (!ws || !aligned16(ws) || ws_bytes < L.partial) return QLORA_ERR_WORKSPACE;   // as run_fwd
   if (M == 0) {
     if (cudaMemsetAsync(dA, 0, size_t(E) * r * W->K * 2, s) != cudaSuccess ||
         cudaMemsetAsync(dB, 0, size_t(E) * W->N * r * 2, s) != cudaSuccess)

@@ -32,7 +32,8 @@
  *     still overwrites dA and dB with zeros), r in {8, 16, 32, 64}; every pointer 16-byte aligned
  *     (with M == 0 the [M, ...] activation pointers may be NULL).  Grouped ops: 1 <= E <= 1024.
  *   - Outputs are overwritten, never accumulated (gradient accumulation across micro-batches is the
- *     caller's job).  Results are deterministic: the same inputs give bitwise-identical outputs.
+ *     caller's job).  Results are deterministic: the same inputs (and workspace size) give
+ *     bitwise-identical outputs.
  *   - Calls that share a workspace must be ordered on one stream.
  *   - Host threads may call the library concurrently.  Its process-wide state is small: per-device
  *     caches filled once (SM count, kernel shared-memory attributes, set on a kernel's first launch
@@ -81,7 +82,7 @@ typedef enum {
   QLORA_OK = 0,
   QLORA_ERR_INVALID_ARG = 1,    /* a NULL/misaligned pointer or a shape outside the limits */
   QLORA_ERR_UNSUPPORTED = 2,    /* a valid request this build does not implement (e.g. rank) */
-  QLORA_ERR_WORKSPACE = 3,      /* workspace NULL or smaller than qlora_workspace_size() */
+  QLORA_ERR_WORKSPACE = 3,      /* workspace NULL, misaligned or too small (qlora_workspace_size) */
   QLORA_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed (launch, tensor map) */
   QLORA_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait gave up (kernel ended early) */
 } qlora_status_t;
@@ -123,7 +124,12 @@ typedef enum {
 
 /* Bytes of device workspace `op` needs for these shapes (E = number of experts for the grouped
  * ops, ignored otherwise; for the grouped ops M is the total row count).  Returns 0 for invalid
- * arguments.  A workspace sized for an op and shapes also serves smaller M. */
+ * arguments.  A workspace sized for an op and shapes also serves smaller M.  For one layer of at
+ * most 256 rows the size includes the fp32 split partials of the short-batch kernels (tens of MB
+ * for a 14336 x 4096 weight); a call whose workspace lacks room for them (e.g. one sized for
+ * more than 256 rows, which need none) runs the tiled kernels instead: the same results up to
+ * the order of fp32 additions.  The training calls reject only a workspace smaller than the
+ * part without those partials (QLORA_ERR_WORKSPACE). */
 QLORA_API size_t qlora_workspace_size(int op, const qlora_weight_t* W, int64_t M, int r, int E);
 
 /* Zero the workspace's 8192-byte header (device status word, the tiled kernel's tile ticket and

@@ -106,6 +106,45 @@ def test_backward_rejects_bad_arguments(Q):
     assert Q.STATUS[rc] == "QLORA_ERR_INVALID_ARG"
 
 
+def test_workspace_sized_for_more_rows_serves_fewer(Q):
+    # The workspace size is not monotone in M: one layer of at most 256 rows adds the short-batch
+    # kernels' fp32 split partials, which larger batches do not use.  A workspace sized for more
+    # rows is still accepted for fewer (the call then runs the tiled kernels); one without room
+    # for Zs, T and U is rejected.  Without a GPU driver an accepted call stops at its first CUDA
+    # call (QLORA_ERR_CUDA), before which nothing is enqueued.
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    W = _w(Q, N=14336, K=4096)
+    r = 16
+    for op in (Q.OP_FWD, Q.OP_BWD):
+        big = Q.qlora_workspace_size(op, W, 1024, r)
+        for M in (16, 64, 256):
+            assert Q.qlora_workspace_size(op, W, M, r) > big      # the partials of the short path
+            if op == Q.OP_FWD:
+                rc = Q.lib.qlora_linear_fwd(W.ref, 0x10000, 0x20000, 0x30000, 0x40000, None, M, r,
+                                            2.0, 0x50000, big, None)
+            else:
+                rc = Q.lib.qlora_linear_bwd(W.ref, 0x10000, 0x20000, 0x30000, None, 0x60000,
+                                            0x90000, 0x70000, 0x80000, M, r, 2.0, 0x50000, big,
+                                            None)
+            assert Q.STATUS[rc] == "QLORA_ERR_CUDA", (op, M)
+        # required: the 8192-byte header, Zs and T (and U) as 256-byte rounded [M, r] bf16 regions,
+        # and for the backward lora_down's cluster sums (8 x 128 x r fp32)
+        m = 256
+        z = -(-m * r * 2 // 256) * 256
+        need = 8192 + (3 * z + 8 * 128 * r * 4 if op == Q.OP_BWD else 2 * z)
+        for nbytes, want in ((need - 16, "QLORA_ERR_WORKSPACE"), (need, "QLORA_ERR_CUDA")):
+            if op == Q.OP_FWD:
+                rc = Q.lib.qlora_linear_fwd(W.ref, 0x10000, 0x20000, 0x30000, 0x40000, None, m, r,
+                                            2.0, 0x50000, nbytes, None)
+            else:
+                rc = Q.lib.qlora_linear_bwd(W.ref, 0x10000, 0x20000, 0x30000, None, 0x60000,
+                                            0x90000, 0x70000, 0x80000, m, r, 2.0, 0x50000, nbytes,
+                                            None)
+            assert Q.STATUS[rc] == want, (op, nbytes)
+
+
 def test_workspace_init_and_status_reject_null(Q):
     assert Q.STATUS[Q.lib.qlora_workspace_init(None, 1 << 20, None)] == "QLORA_ERR_WORKSPACE"
     assert Q.STATUS[Q.lib.qlora_get_device_status(None, None)] == "QLORA_ERR_WORKSPACE"

@@ -213,6 +213,30 @@ def test_layer_parity(fmt, M, N, K, r):
     assert_close(to_f64(dB), ref["dB"], "dB")
 
 
+@pytest.mark.parametrize("fmt,M", [("nf4", 16), ("mxfp4", 64), ("nvfp4", 200)])
+def test_workspace_without_partials_runs_the_tiled_kernels(fmt, M):
+    # a workspace holding only the header, Zs, T, U and lora_down's cluster sums -- what one sized
+    # for more than 256 rows offers a short batch -- has no room for the short-batch or streaming
+    # kernels' split partials: the calls run the tiled kernels and still match the oracle
+    from bit_quantized_base_b200 import qlora as Q
+    N, K, r = 2064, 1216, 16
+    p = synth.small_layer(fmt, M, N, K, r, s=2.0, seed=M + 5)
+    g = GpuLayer(p)
+    z = -(-M * r * 2 // 256) * 256
+    need = 8192 + 3 * z + 8 * 128 * r * 4
+    assert Q.qlora_workspace_size(Q.OP_BWD, g.W, M, r) > need
+    g.ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    Q.qlora_workspace_init(g.ws)
+    Y, T = g.fwd()
+    dX, dA, dB = g.bwd(T)
+    torch.cuda.synchronize()
+    assert g.status() == 0
+    ref = O.layer(fmt, M, N, K, r, p["s"], p["codes"], p["scales"], p["tensor_scale"], p["X"],
+                  p["A"], p["B"], p["dY"])
+    for name, got in (("T", T), ("Y", Y), ("dX", dX), ("dA", dA), ("dB", dB)):
+        assert_close(to_f64(got), ref[name], name)
+
+
 def test_backward_recomputes_T_and_skips_dx():
     p = synth.small_layer("mxfp4", 200, 256, 384, 16, seed=3)
     g = GpuLayer(p)
